@@ -1,0 +1,144 @@
+"""Seeded synthetic inputs shaped like the workloads on the pages.
+
+This module only draws random numbers and lays them out (tensor shapes, page
+permutation, block table); it contains none of the attention arithmetic. Both the
+CUDA path and the CPU oracle consume what it returns.
+
+Recipe (also stated in the design notes):
+* values: i.i.d. N(0, 1) * std drawn in float32 by a seeded torch generator on the
+  target device, then rounded to the storage dtype (bf16 round-to-nearest-even);
+* integer structure (sequence lengths, page permutation): numpy PCG64 seeded from
+  the same seed, drawn on the host so it does not depend on the device.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+PAGE_SIZE = 16
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    kind: str  # "prefill" | "decode" | "mla"
+    params: dict = field(default_factory=dict)
+
+
+# The five workloads, named by what they are.
+WORKLOADS = {
+    "mha_prefill_b1_h4_s256_d64_f32": Workload(
+        "mha_prefill_b1_h4_s256_d64_f32", "prefill",
+        dict(B=1, Hq=4, Hkv=4, S=256, D=64, dtype="f32", std=1.0, theta=1e4, scale=1.0 / 8.0)),
+    "gqa_prefill_b2_hq32_hkv8_s4096_d128": Workload(
+        "gqa_prefill_b2_hq32_hkv8_s4096_d128", "prefill",
+        dict(B=2, Hq=32, Hkv=8, S=4096, D=128, dtype="bf16", std=1.0, theta=1e4, scale=1.0 / math.sqrt(128))),
+    "gqa_prefill_b1_hq32_hkv8_s32768_d128": Workload(
+        "gqa_prefill_b1_hq32_hkv8_s32768_d128", "prefill",
+        dict(B=1, Hq=32, Hkv=8, S=32768, D=128, dtype="bf16", std=0.5, theta=1e6, scale=1.0 / math.sqrt(128))),
+    "paged_decode_b64_hq32_hkv8_d128": Workload(
+        "paged_decode_b64_hq32_hkv8_d128", "decode",
+        dict(B=64, Hq=32, Hkv=8, D=128, lmin=1024, lmax=32768, std=1.0, scale=1.0 / math.sqrt(128))),
+    "mla_decode_b32_h128_dc512_dr64": Workload(
+        "mla_decode_b32_h128_dc512_dr64", "mla",
+        dict(B=32, H=128, Dc=512, Dr=64, lmin=4096, lmax=32768, std=1.0, scale=1.0 / math.sqrt(192))),
+}
+
+_TORCH_DT = {"bf16": torch.bfloat16, "f32": torch.float32}
+
+
+def _gen(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return g
+
+
+def _randn(shape, std, dtype, g, device):
+    x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    if std != 1.0:
+        x.mul_(std)
+    return x.to(_TORCH_DT[dtype])
+
+
+def prefill_inputs(B, Hq, Hkv, S, D, dtype="bf16", std=1.0, seed=0, device="cpu"):
+    """q [B,Hq,S,D], k [B,Hkv,S,D], v [B,Hkv,S,D] (contiguous, BNHS order)."""
+    g = _gen(seed, device)
+    q = _randn((B, Hq, S, D), std, dtype, g, device)
+    k = _randn((B, Hkv, S, D), std, dtype, g, device)
+    v = _randn((B, Hkv, S, D), std, dtype, g, device)
+    return q, k, v
+
+
+def draw_lengths(B, lmin, lmax, seed):
+    """Integer lengths uniform in [lmin, lmax] (inclusive), numpy PCG64."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    return rng.integers(lmin, lmax + 1, size=B).astype(np.int32)
+
+
+def decode_inputs(B, Hq, Hkv, D, lmin=1024, lmax=32768, std=1.0, seed=0, device="cpu",
+                  seq_lens=None, max_pages_per_seq=None, page_size=PAGE_SIZE, dtype="bf16",
+                  extra_pages=0):
+    """Paged KV cache for one-token decode.
+
+    k_pages, v_pages: [num_pages, page_size, Hkv, D]; every slot is filled with
+    random values, including the unused tail of each sequence's last page.
+    block_table: [B, max_pages_per_seq] int32; logical page j of sequence b is at
+    physical page block_table[b, j]; the physical order is a seeded random
+    permutation; entries past the end of a sequence are -1.
+    extra_pages adds unreferenced pages to the pool (their content is never read).
+    """
+    if seq_lens is None:
+        seq_lens = draw_lengths(B, lmin, lmax, seed)
+    seq_lens = np.asarray(seq_lens, dtype=np.int32)
+    npages = [int(math.ceil(int(L) / page_size)) for L in seq_lens]
+    if max_pages_per_seq is None:
+        max_pages_per_seq = max(1, int(math.ceil(lmax / page_size)), max(npages) if npages else 1)
+    total = int(sum(npages)) + int(extra_pages)
+    rng = np.random.Generator(np.random.PCG64(seed + 7919))
+    perm = rng.permutation(max(total, 1)).astype(np.int32)
+    table = np.full((B, max_pages_per_seq), -1, dtype=np.int32)
+    off = 0
+    for b, n in enumerate(npages):
+        table[b, :n] = perm[off:off + n]
+        off += n
+    g = _gen(seed, device)
+    q = _randn((B, Hq, D), std, dtype, g, device)
+    num_pages = max(total, 1)
+    k_pages = _randn((num_pages, page_size, Hkv, D), std, dtype, g, device)
+    v_pages = _randn((num_pages, page_size, Hkv, D), std, dtype, g, device)
+    return dict(q=q, k_pages=k_pages, v_pages=v_pages,
+                block_table=torch.from_numpy(table).to(device),
+                seq_lens=torch.from_numpy(seq_lens).to(device),
+                max_pages_per_seq=max_pages_per_seq, num_pages=num_pages, page_size=page_size)
+
+
+def mla_inputs(B, H, Dc, Dr, lmin=4096, lmax=32768, std=1.0, seed=0, device="cpu", seq_lens=None,
+               T_max=None):
+    """Absorbed-MLA decode inputs: q_nope [B,1,H,Dc], q_pe [B,1,H,Dr],
+    kv_cache [B,T_max,Dc], pe_cache [B,T_max,Dr] (filled beyond each length too),
+    seq_lens [B] int32."""
+    if seq_lens is None:
+        seq_lens = draw_lengths(B, lmin, lmax, seed)
+    seq_lens = np.asarray(seq_lens, dtype=np.int32)
+    if T_max is None:
+        T_max = max(int(lmax), int(seq_lens.max()) if len(seq_lens) else 1)
+    g = _gen(seed, device)
+    q_nope = _randn((B, 1, H, Dc), std, "bf16", g, device)
+    q_pe = _randn((B, 1, H, Dr), std, "bf16", g, device)
+    kv = _randn((B, T_max, Dc), std, "bf16", g, device)
+    pe = _randn((B, T_max, Dr), std, "bf16", g, device)
+    return dict(q_nope=q_nope, q_pe=q_pe, kv_cache=kv, pe_cache=pe,
+                seq_lens=torch.from_numpy(seq_lens).to(device), T_max=T_max)
+
+
+def workload_inputs(name: str, seed: int = 20261202, device="cpu"):
+    w = WORKLOADS[name]
+    p = w.params
+    if w.kind == "prefill":
+        return prefill_inputs(p["B"], p["Hq"], p["Hkv"], p["S"], p["D"], p["dtype"], p["std"], seed, device)
+    if w.kind == "decode":
+        return decode_inputs(p["B"], p["Hq"], p["Hkv"], p["D"], p["lmin"], p["lmax"], p["std"], seed, device)
+    return mla_inputs(p["B"], p["H"], p["Dc"], p["Dr"], p["lmin"], p["lmax"], p["std"], seed, device)

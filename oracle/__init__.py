@@ -1,0 +1,18 @@
+"""CPU float64 oracle: test infrastructure, not part of the product.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference arm
+of ``bench.py`` may import this package. The CUDA library neither imports nor
+links it, and it shares no code with the CUDA path.
+"""
+from .attention import (  # noqa: F401
+    apply_rope,
+    decode_paged_ref,
+    gather_pages,
+    lse_merge,
+    mla_decode_ref,
+    mla_naive_ref,
+    online_softmax_merge,
+    prefill_ref,
+    rope_cache,
+    two_pass_softmax_rows,
+)
