@@ -1,0 +1,213 @@
+"""Thin ctypes binding over libattn_b200.so (argument marshalling only).
+
+Every step of the attention path runs in the CUDA library; this module only
+allocates outputs / workspace through torch (device memory plumbing), passes
+raw pointers and the current CUDA stream, and turns error codes into
+exceptions. There is no CPU fallback: if the library is missing, importing
+this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from .build import LIB
+
+ATTN_OK = 0
+ATTN_ERR_INVALID_ARG = 1
+ATTN_ERR_UNSUPPORTED = 2
+ATTN_ERR_WORKSPACE = 3
+ATTN_ERR_CUDA = 4
+ATTN_ERR_DEVICE = 5
+ATTN_DTYPE_F32 = 0
+ATTN_DTYPE_BF16 = 1
+ATTN_DEV_TIMEOUT = 1
+ATTN_DEV_BAD_PAGE = 2
+ATTN_DEV_BAD_LENGTH = 4
+
+EXPORTED = (
+    "attn_prefill_workspace_size", "attn_prefill",
+    "attn_decode_paged_workspace_size", "attn_decode_paged",
+    "mla_decode_workspace_size", "mla_decode",
+    "attn_last_error", "attn_read_status", "attn_selftest_wait_timeout",
+    "attn_profile_enable", "attn_profile_collect",
+)
+
+
+class AttnError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"attn_b200 error {code}: {msg}")
+        self.code = code
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB):
+        raise ImportError(f"CUDA library not built: {LIB} is missing (run attention_causal_gqa_b200.build)")
+    lib = ctypes.CDLL(LIB)
+    vp, i32, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.attn_prefill_workspace_size.restype = sz
+    lib.attn_prefill_workspace_size.argtypes = [i32] * 5
+    lib.attn_prefill.restype = i32
+    lib.attn_prefill.argtypes = [vp] * 5 + [i32] * 6 + [f32, f32, i32, vp, sz, vp]
+    lib.attn_decode_paged_workspace_size.restype = sz
+    lib.attn_decode_paged_workspace_size.argtypes = [i32] * 5
+    lib.attn_decode_paged.restype = i32
+    lib.attn_decode_paged.argtypes = [vp] * 7 + [i32] * 7 + [f32, i32, vp, sz, vp]
+    lib.mla_decode_workspace_size.restype = sz
+    lib.mla_decode_workspace_size.argtypes = [i32] * 5
+    lib.mla_decode.restype = i32
+    lib.mla_decode.argtypes = [vp] * 5 + [f32, vp, vp] + [i32] * 5 + [vp, sz, vp]
+    lib.attn_last_error.restype = ctypes.c_char_p
+    lib.attn_last_error.argtypes = []
+    lib.attn_read_status.restype = i32
+    lib.attn_read_status.argtypes = [vp, ctypes.POINTER(i32), vp]
+    lib.attn_selftest_wait_timeout.restype = i32
+    lib.attn_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_ulonglong, vp]
+    lib.attn_profile_enable.restype = i32
+    lib.attn_profile_enable.argtypes = [i32]
+    lib.attn_profile_collect.restype = i32
+    lib.attn_profile_collect.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i32)]
+    return lib
+
+
+lib = _load()
+
+
+def _check(rc: int):
+    if rc != ATTN_OK:
+        raise AttnError(rc, lib.attn_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("attn_b200 takes CUDA tensors (no CPU path)")
+        if not t.is_contiguous():
+            raise ValueError("attn_b200 takes contiguous tensors")
+
+
+def _workspace(nbytes: int, device, workspace):
+    if workspace is not None:
+        if workspace.numel() * workspace.element_size() < nbytes:
+            raise ValueError("workspace too small")
+        return workspace
+    return torch.empty(int(nbytes), dtype=torch.uint8, device=device)
+
+
+# ------------------------------------------------------------------ prefill
+def prefill_workspace_size(B, Hkv, S, D, dtype=torch.bfloat16) -> int:
+    dt = ATTN_DTYPE_F32 if dtype == torch.float32 else ATTN_DTYPE_BF16
+    return int(lib.attn_prefill_workspace_size(B, Hkv, S, D, dt))
+
+
+def attn_prefill(q, k, v, causal=True, rope_theta=10000.0, scale=None, out=None, lse=None, workspace=None,
+                 stream=None):
+    """Causal GQA prefill with RoPE. q [B,Hq,S,D], k/v [B,Hkv,S,D] (bf16 or fp32).
+    Returns (out [B,Hq,S,D] same dtype, lse [B,Hq,S] fp32)."""
+    _need_cuda(q, k, v)
+    B, Hq, S, D = q.shape
+    Hkv = k.shape[1]
+    dt = ATTN_DTYPE_F32 if q.dtype == torch.float32 else ATTN_DTYPE_BF16
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
+    ws_bytes = prefill_workspace_size(B, Hkv, S, D, q.dtype)
+    ws = _workspace(ws_bytes, q.device, workspace)
+    rc = lib.attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, S, D, int(bool(causal)),
+                          float(rope_theta if rope_theta else 0.0), float(scale or 0.0), dt, _ptr(ws),
+                          ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc)
+    return out, lse
+
+
+# ------------------------------------------------------------- paged decode
+def decode_workspace_size(B, Hq, D, max_pages_per_seq, page_size=16) -> int:
+    return int(lib.attn_decode_paged_workspace_size(B, Hq, D, max_pages_per_seq, page_size))
+
+
+def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale=None, out=None, lse=None, workspace=None,
+                      stream=None):
+    """Paged GQA decode. q [B,Hq,D] bf16, k/v_pages [P,16,Hkv,D] bf16, block_table [B,maxp] int32,
+    seq_lens [B] int32. Returns (out [B,Hq,D] bf16, lse [B,Hq] fp32)."""
+    _need_cuda(q, k_pages, v_pages, block_table, seq_lens)
+    B, Hq, D = q.shape
+    P, ps, Hkv, _ = k_pages.shape
+    maxp = block_table.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    ws = _workspace(decode_workspace_size(B, Hq, D, maxp, ps), q.device, workspace)
+    rc = lib.attn_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens), _ptr(out),
+                               _ptr(lse), B, Hq, Hkv, D, ps, maxp, P, float(scale or 0.0), ATTN_DTYPE_BF16, _ptr(ws),
+                               ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc)
+    return out, lse
+
+
+# --------------------------------------------------------------- MLA decode
+def mla_workspace_size(B, H, Dc, Dr, T_max) -> int:
+    return int(lib.mla_decode_workspace_size(B, H, Dc, Dr, T_max))
+
+
+def mla_decode(q_nope, q_pe, kv_cache, pe_cache, seq_lens, scale, out=None, lse=None, workspace=None,
+               stream=None):
+    """MLA absorbed decode. q_nope [B,1,H,Dc], q_pe [B,1,H,Dr], kv_cache [B,T,Dc], pe_cache [B,T,Dr] (bf16),
+    seq_lens [B] int32. Returns (out [B,1,H,Dc] bf16, lse [B,1,H] fp32)."""
+    _need_cuda(q_nope, q_pe, kv_cache, pe_cache, seq_lens)
+    B, _, H, Dc = q_nope.shape
+    Dr = q_pe.shape[-1]
+    T = kv_cache.shape[1]
+    if not scale or scale <= 0:
+        raise ValueError("mla_decode needs an explicit positive scale (DeepSeek-V3 shapes: 1/sqrt(192))")
+    if out is None:
+        out = torch.empty_like(q_nope)
+    if lse is None:
+        lse = torch.empty((B, 1, H), dtype=torch.float32, device=q_nope.device)
+    ws = _workspace(mla_workspace_size(B, H, Dc, Dr, T), q_nope.device, workspace)
+    rc = lib.mla_decode(_ptr(q_nope), _ptr(q_pe), _ptr(kv_cache), _ptr(pe_cache), _ptr(seq_lens), float(scale),
+                        _ptr(out), _ptr(lse), B, H, Dc, Dr, T, _ptr(ws), ws.numel() * ws.element_size(),
+                        _stream(stream))
+    _check(rc)
+    return out, lse
+
+
+# ------------------------------------------------------------------- status
+def read_status(workspace, stream=None) -> int:
+    flags = ctypes.c_int(0)
+    rc = lib.attn_read_status(_ptr(workspace), ctypes.byref(flags), _stream(stream))
+    if rc not in (ATTN_OK, ATTN_ERR_DEVICE):
+        _check(rc)
+    return flags.value
+
+
+def selftest_wait_timeout(timeout_ns: int, workspace=None, stream=None) -> int:
+    ws = workspace if workspace is not None else torch.zeros(256, dtype=torch.uint8, device="cuda")
+    _check(lib.attn_selftest_wait_timeout(_ptr(ws), ws.numel(), int(timeout_ns), _stream(stream)))
+    return read_status(ws, stream)
+
+
+# ------------------------------------------------------------ timing hook
+def profile_enable(on: bool = True):
+    _check(lib.attn_profile_enable(1 if on else 0))
+
+
+def profile_collect():
+    """(summed main-kernel milliseconds, number of recorded calls) since the last collect."""
+    ms = ctypes.c_double(0.0)
+    n = ctypes.c_int(0)
+    _check(lib.attn_profile_collect(ctypes.byref(ms), ctypes.byref(n)))
+    return ms.value, n.value

@@ -1,0 +1,454 @@
+// C-ABI layer: host-side validation, workspace carving, TMA tensor-map
+// encoding and kernel launches. No allocation, no synchronisation on the hot calls.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/attn_b200.h"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int ok() {
+  g_last_error.clear();
+  return ATTN_OK;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(ATTN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+constexpr size_t kHeader = 256;  // status word lives at offset 0
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Tiled tensor map with 128-byte swizzle; dims/strides innermost first, strides in bytes for dims 1..rank-1.
+int make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const cuuint64_t* dims,
+             const cuuint64_t* strides, const cuuint32_t* box, const char* what) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(m, dt, static_cast<cuuint32_t>(rank), const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(ATTN_ERR_CUDA, "tensor map encode failed for %s (CUresult %d)", what, (int)r);
+  return ATTN_OK;
+}
+
+int clear_status(void* ws, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int), st);
+  if (e != cudaSuccess) return cuda_fail(e, "status clear");
+  return ATTN_OK;
+}
+
+int decode_splits(int max_pages) {
+  return (max_pages + attn::kDecodePagesPerSplit - 1) / attn::kDecodePagesPerSplit;
+}
+int mla_splits(int T_max) {
+  const int tps = attn::kMlaTokensPerTile * attn::kMlaTilesPerSplit;
+  return (T_max + tps - 1) / tps;
+}
+
+// ----------------------------------------------------------- timing hook
+constexpr int kProfSlots = 4096;
+struct Profiler {
+  bool on = false;
+  bool created = false;
+  cudaEvent_t ev[2 * kProfSlots];
+  int used = 0;
+} g_prof;
+
+void prof_before(cudaStream_t st) {
+  if (g_prof.on && g_prof.used < kProfSlots) cudaEventRecord(g_prof.ev[2 * g_prof.used], st);
+}
+void prof_after(cudaStream_t st) {
+  if (g_prof.on && g_prof.used < kProfSlots) {
+    cudaEventRecord(g_prof.ev[2 * g_prof.used + 1], st);
+    ++g_prof.used;
+  }
+}
+
+}  // namespace
+
+namespace attn {
+__global__ void selftest_wait_kernel(int* status, unsigned long long timeout_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // Nothing ever arrives on `bar`: the wait must give up by itself.
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(&bar, 0)) {
+      if (globaltimer_ns() - t0 > timeout_ns) {
+        atomicOr(status, kDevErrTimeout);
+        break;
+      }
+    }
+  }
+  __syncthreads();
+}
+}  // namespace attn
+
+extern "C" {
+
+const char* attn_last_error(void) { return g_last_error.c_str(); }
+
+// Prefill workspace: [status | cos/sin table | key operand | value operand]
+//   bf16 input: key operand = rotated K in fp16 [B*Hkv, S, D]; no value operand.
+//   fp32 input: key and value operands = bf16 hi parts then lo parts [2*B*Hkv, S, D] each.
+size_t attn_prefill_workspace_size(int B, int Hkv, int S, int D, int dtype) {
+  if (B <= 0 || Hkv <= 0 || S <= 0 || D <= 0) return kHeader;
+  const size_t n = static_cast<size_t>(B) * Hkv * S * D;
+  const size_t table = round_up(static_cast<size_t>(S) * (D / 2) * sizeof(float2), 256);
+  if (dtype == ATTN_DTYPE_F32) return kHeader + table + 2 * round_up(2 * n * 2, 256);
+  return kHeader + table + round_up(n * 2, 256);
+}
+
+int attn_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv, int S,
+                 int D, int causal, float rope_theta, float scale, int dtype, void* workspace,
+                 size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !out || !lse || !workspace) return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || S <= 0 || D <= 0)
+    return fail(ATTN_ERR_INVALID_ARG, "sizes must be positive (B=%d Hq=%d Hkv=%d S=%d D=%d)", B, Hq, Hkv, S, D);
+  if (Hq % Hkv != 0) return fail(ATTN_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+  if (dtype != ATTN_DTYPE_BF16 && dtype != ATTN_DTYPE_F32) return fail(ATTN_ERR_UNSUPPORTED, "dtype %d", dtype);
+  const bool f32 = dtype == ATTN_DTYPE_F32;
+  if (!(f32 ? D == 64 : (D == 64 || D == 128)))
+    return fail(ATTN_ERR_UNSUPPORTED, "head dim %d unsupported for %s", D, f32 ? "fp32" : "bf16");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4) ||
+      !aligned(workspace, 256))
+    return fail(ATTN_ERR_INVALID_ARG, "misaligned pointer (tensors 16 B, lse 4 B, workspace 256 B)");
+  if (static_cast<long long>(B) * Hkv > (1LL << 30) || S > (1 << 24))
+    return fail(ATTN_ERR_UNSUPPORTED, "problem too large");
+  const size_t need = attn_prefill_workspace_size(B, Hkv, S, D, dtype);
+  if (workspace_bytes < need)
+    return fail(ATTN_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace_bytes, need);
+  if (!std::isfinite(scale)) return fail(ATTN_ERR_INVALID_ARG, "scale is not finite");
+  if (scale <= 0.f) scale = 1.0f / std::sqrt(static_cast<float>(D));
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* status = reinterpret_cast<int*>(ws);
+  float2* cs = reinterpret_cast<float2*>(ws + kHeader);
+  const size_t n = static_cast<size_t>(B) * Hkv * S * D;
+  uint8_t* kop = ws + kHeader + round_up(static_cast<size_t>(S) * (D / 2) * sizeof(float2), 256);
+  uint8_t* vop = kop + round_up(2 * n * 2, 256);  // fp32 input only
+  int rc = clear_status(ws, st);
+  if (rc) return rc;
+
+  const bool rope = rope_theta > 0.f;
+  if (rope) {
+    cudaError_t e = attn::launch_rope_table(cs, S, D, static_cast<double>(rope_theta), st);
+    if (e != cudaSuccess) return cuda_fail(e, "rope table launch");
+  }
+  const long long rows = static_cast<long long>(B) * Hkv * S;
+  const void* kbase = k;
+  const void* vbase = v;
+  CUtensorMapDataType kdt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  cuuint64_t zdim = static_cast<cuuint64_t>(B) * Hkv;
+  if (f32) {
+    cudaError_t e = attn::launch_split_f32(static_cast<const float*>(k), kop, rope ? cs : nullptr, rows, S, D, st);
+    if (e == cudaSuccess) e = attn::launch_split_f32(static_cast<const float*>(v), vop, nullptr, rows, S, D, st);
+    if (e != cudaSuccess) return cuda_fail(e, "operand split launch");
+    kbase = kop;
+    vbase = vop;
+    zdim *= 2;
+  } else if (rope) {
+    cudaError_t e = attn::launch_rope_k_f16(k, kop, cs, rows, S, D, status, st);
+    if (e != cudaSuccess) return cuda_fail(e, "rope K launch");
+    kbase = kop;
+    kdt = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  }
+  const int BN = attn::prefill_block_n(D, f32);
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S), zdim};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(S) * D * 2};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(BN), 1};
+  CUtensorMap tmK, tmV;
+  if ((rc = make_map(&tmK, kdt, 3, kbase, dims, strides, box, "K"))) return rc;
+  if ((rc = make_map(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, vbase, dims, strides, box, "V"))) return rc;
+
+  attn::PrefillParams p{};
+  p.q = q;
+  p.out = out;
+  p.lse = lse;
+  p.rope_cs = rope ? cs : nullptr;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.S = S;
+  p.G = Hq / Hkv;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.pair_heads = (p.G % 2 == 0) ? 1 : 0;
+  p.n_row_blocks = (S + 127) / 128;
+  p.status = status;
+  const long long grid = p.pair_heads ? static_cast<long long>(B) * (Hq / 2) * p.n_row_blocks
+                                      : static_cast<long long>(B) * Hq * ((p.n_row_blocks + 1) / 2);
+  if (grid > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "grid too large");
+  prof_before(st);
+  cudaError_t e = attn::launch_prefill(p, tmK, tmV, D, f32, rope, static_cast<int>(grid), st);
+  prof_after(st);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+  return ok();
+}
+
+size_t attn_decode_paged_workspace_size(int B, int Hq, int D, int max_pages_per_seq, int page_size) {
+  (void)page_size;
+  if (B <= 0 || Hq <= 0 || D <= 0 || max_pages_per_seq <= 0) return kHeader;
+  const size_t ns = decode_splits(max_pages_per_seq);
+  return kHeader + round_up(static_cast<size_t>(B) * ns * Hq * D * sizeof(float), 256) +
+         round_up(static_cast<size_t>(B) * ns * Hq * sizeof(float), 256);
+}
+
+int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
+                      const int32_t* seq_lens, void* out, float* lse, int B, int Hq, int Hkv, int D, int page_size,
+                      int max_pages_per_seq, int num_pages, float scale, int dtype, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !out || !lse || !workspace)
+    return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || max_pages_per_seq <= 0 || num_pages <= 0 || page_size <= 0)
+    return fail(ATTN_ERR_INVALID_ARG, "sizes must be positive");
+  if (Hq % Hkv != 0) return fail(ATTN_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+  if (dtype != ATTN_DTYPE_BF16) return fail(ATTN_ERR_UNSUPPORTED, "paged decode supports bf16 only");
+  if (page_size != 16) return fail(ATTN_ERR_UNSUPPORTED, "page_size %d (only 16)", page_size);
+  if (D != 64 && D != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d", D);
+  if (Hkv > 8) return fail(ATTN_ERR_UNSUPPORTED, "Hkv %d > 8", Hkv);
+  if (Hq / Hkv > 16) return fail(ATTN_ERR_UNSUPPORTED, "group size %d > 16", Hq / Hkv);
+  if (!aligned(q, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(out, 16) ||
+      !aligned(block_table, 4) || !aligned(seq_lens, 4) || !aligned(lse, 4) || !aligned(workspace, 256))
+    return fail(ATTN_ERR_INVALID_ARG, "misaligned pointer");
+  const size_t need = attn_decode_paged_workspace_size(B, Hq, D, max_pages_per_seq, page_size);
+  if (workspace_bytes < need)
+    return fail(ATTN_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace_bytes, need);
+  if (!std::isfinite(scale)) return fail(ATTN_ERR_INVALID_ARG, "scale is not finite");
+  if (scale <= 0.f) scale = 1.0f / std::sqrt(static_cast<float>(D));
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int ns = decode_splits(max_pages_per_seq);
+  float* part_o = reinterpret_cast<float*>(ws + kHeader);
+  float* part_lse =
+      reinterpret_cast<float*>(ws + kHeader + round_up(static_cast<size_t>(B) * ns * Hq * D * sizeof(float), 256));
+  int rc = clear_status(ws, st);
+  if (rc) return rc;
+
+  // 5-D view of a page pool [num_pages][16][Hkv][D]: (d%64, token, d/64, head, page);
+  // its shared-memory image is [head][d/64][token][64].
+  const cuuint64_t row = static_cast<cuuint64_t>(Hkv) * D * 2;
+  const cuuint64_t dims[5] = {64, 16, static_cast<cuuint64_t>(D / 64), static_cast<cuuint64_t>(Hkv),
+                              static_cast<cuuint64_t>(num_pages)};
+  const cuuint64_t strides[4] = {row, 128, static_cast<cuuint64_t>(D) * 2, 16 * row};
+  const cuuint32_t box[5] = {64, 16, static_cast<cuuint32_t>(D / 64), static_cast<cuuint32_t>(Hkv), 1};
+  CUtensorMap tmK, tmV;
+  if ((rc = make_map(&tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, k_pages, dims, strides, box, "k_pages"))) return rc;
+  if ((rc = make_map(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, v_pages, dims, strides, box, "v_pages"))) return rc;
+
+  attn::DecodeParams p{};
+  p.q = q;
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.part_o = part_o;
+  p.part_lse = part_lse;
+  p.out = out;
+  p.lse = lse;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.D = D;
+  p.G = Hq / Hkv;
+  p.max_pages = max_pages_per_seq;
+  p.num_pages = num_pages;
+  p.n_splits = ns;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.status = reinterpret_cast<int*>(ws);
+  prof_before(st);
+  cudaError_t e = attn::launch_decode(p, tmK, tmV, st);
+  prof_after(st);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  e = attn::launch_merge(part_o, part_lse, seq_lens, out, lse, B, Hq, D, ns, attn::kDecodePagesPerSplit * 16, st);
+  if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  return ok();
+}
+
+size_t mla_decode_workspace_size(int B, int H, int Dc, int Dr, int T_max) {
+  (void)Dr;
+  if (B <= 0 || H <= 0 || Dc <= 0 || T_max <= 0) return kHeader;
+  const size_t ns = mla_splits(T_max);
+  return kHeader + round_up(static_cast<size_t>(B) * ns * H * Dc * sizeof(float), 256) +
+         round_up(static_cast<size_t>(B) * ns * H * sizeof(float), 256);
+}
+
+int mla_decode(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
+               const int32_t* seq_lens, float scale, void* out, float* lse, int B, int H, int Dc, int Dr, int T_max,
+               void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q_nope || !q_pe || !kv_cache || !pe_cache || !seq_lens || !out || !lse || !workspace)
+    return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
+  if (B <= 0 || H <= 0 || Dc <= 0 || Dr <= 0 || T_max <= 0) return fail(ATTN_ERR_INVALID_ARG, "sizes must be positive");
+  if (H != 128 || Dc != 512 || Dr != 64)
+    return fail(ATTN_ERR_UNSUPPORTED, "MLA decode supports H=128, Dc=512, Dr=64 (got %d, %d, %d)", H, Dc, Dr);
+  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(ATTN_ERR_INVALID_ARG, "scale must be positive");
+  if (!aligned(q_nope, 16) || !aligned(q_pe, 16) || !aligned(kv_cache, 16) || !aligned(pe_cache, 16) ||
+      !aligned(out, 16) || !aligned(seq_lens, 4) || !aligned(lse, 4) || !aligned(workspace, 256))
+    return fail(ATTN_ERR_INVALID_ARG, "misaligned pointer");
+  if (T_max > (1 << 26)) return fail(ATTN_ERR_UNSUPPORTED, "T_max too large");
+  const size_t need = mla_decode_workspace_size(B, H, Dc, Dr, T_max);
+  if (workspace_bytes < need)
+    return fail(ATTN_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace_bytes, need);
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int ns = mla_splits(T_max);
+  float* part_o = reinterpret_cast<float*>(ws + kHeader);
+  float* part_lse =
+      reinterpret_cast<float*>(ws + kHeader + round_up(static_cast<size_t>(B) * ns * H * Dc * sizeof(float), 256));
+  int rc = clear_status(ws, st);
+  if (rc) return rc;
+
+  CUtensorMap tmQn, tmQp, tmKV, tmPE;
+  {
+    const cuuint64_t d[3] = {static_cast<cuuint64_t>(Dc), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
+    const cuuint64_t s[2] = {static_cast<cuuint64_t>(Dc) * 2, static_cast<cuuint64_t>(H) * Dc * 2};
+    const cuuint32_t bx[3] = {64, 128, 1};
+    if ((rc = make_map(&tmQn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, q_nope, d, s, bx, "q_nope"))) return rc;
+  }
+  {
+    const cuuint64_t d[3] = {static_cast<cuuint64_t>(Dr), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
+    const cuuint64_t s[2] = {static_cast<cuuint64_t>(Dr) * 2, static_cast<cuuint64_t>(H) * Dr * 2};
+    const cuuint32_t bx[3] = {64, 128, 1};
+    if ((rc = make_map(&tmQp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, q_pe, d, s, bx, "q_pe"))) return rc;
+  }
+  {
+    const cuuint64_t d[3] = {static_cast<cuuint64_t>(Dc), static_cast<cuuint64_t>(T_max), static_cast<cuuint64_t>(B)};
+    const cuuint64_t s[2] = {static_cast<cuuint64_t>(Dc) * 2, static_cast<cuuint64_t>(T_max) * Dc * 2};
+    const cuuint32_t bx[3] = {64, static_cast<cuuint32_t>(attn::kMlaTokensPerTile), 1};
+    if ((rc = make_map(&tmKV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, kv_cache, d, s, bx, "kv_cache"))) return rc;
+  }
+  {
+    const cuuint64_t d[3] = {static_cast<cuuint64_t>(Dr), static_cast<cuuint64_t>(T_max), static_cast<cuuint64_t>(B)};
+    const cuuint64_t s[2] = {static_cast<cuuint64_t>(Dr) * 2, static_cast<cuuint64_t>(T_max) * Dr * 2};
+    const cuuint32_t bx[3] = {64, static_cast<cuuint32_t>(attn::kMlaTokensPerTile), 1};
+    if ((rc = make_map(&tmPE, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, pe_cache, d, s, bx, "pe_cache"))) return rc;
+  }
+  attn::MlaParams p{};
+  p.seq_lens = seq_lens;
+  p.part_o = part_o;
+  p.part_lse = part_lse;
+  p.out = out;
+  p.lse = lse;
+  p.B = B;
+  p.H = H;
+  p.Dc = Dc;
+  p.Dr = Dr;
+  p.T_max = T_max;
+  p.n_splits = ns;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.status = reinterpret_cast<int*>(ws);
+  prof_before(st);
+  cudaError_t e = attn::launch_mla(p, tmQn, tmQp, tmKV, tmPE, st);
+  prof_after(st);
+  if (e != cudaSuccess) return cuda_fail(e, "mla launch");
+  e = attn::launch_merge(part_o, part_lse, seq_lens, out, lse, B, H, Dc, ns,
+                         attn::kMlaTokensPerTile * attn::kMlaTilesPerSplit, st);
+  if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  return ok();
+}
+
+int attn_read_status(const void* workspace, int* flags, void* stream) {
+  if (!workspace || !flags) return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  int v = 0;
+  e = cudaMemcpy(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "status copy");
+  *flags = v;
+  if (v) return fail(ATTN_ERR_DEVICE, "device status flags 0x%x", v);
+  return ok();
+}
+
+int attn_selftest_wait_timeout(void* workspace, size_t workspace_bytes, unsigned long long timeout_ns,
+                               void* stream) {
+  if (!workspace) return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
+  if (workspace_bytes < kHeader) return fail(ATTN_ERR_WORKSPACE, "workspace must hold at least 256 bytes");
+  if (timeout_ns < 1000ull || timeout_ns > 10000000000ull)
+    return fail(ATTN_ERR_INVALID_ARG, "timeout must be within 1e3 .. 1e10 ns");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int rc = clear_status(workspace, st);
+  if (rc) return rc;
+  attn::selftest_wait_kernel<<<1, 32, 0, st>>>(static_cast<int*>(workspace), timeout_ns);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "selftest launch");
+  return ok();
+}
+
+int attn_profile_enable(int on) {
+  if (on && !g_prof.created) {
+    for (int i = 0; i < 2 * kProfSlots; ++i) {
+      cudaError_t e = cudaEventCreate(&g_prof.ev[i]);
+      if (e != cudaSuccess) return cuda_fail(e, "event create");
+    }
+    g_prof.created = true;
+  }
+  g_prof.on = on != 0;
+  g_prof.used = 0;
+  return ok();
+}
+
+int attn_profile_collect(double* total_ms, int* count) {
+  if (!total_ms || !count) return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
+  double tot = 0.0;
+  for (int i = 0; i < g_prof.used; ++i) {
+    cudaError_t e = cudaEventSynchronize(g_prof.ev[2 * i + 1]);
+    if (e != cudaSuccess) return cuda_fail(e, "event synchronize");
+    float ms = 0.f;
+    e = cudaEventElapsedTime(&ms, g_prof.ev[2 * i], g_prof.ev[2 * i + 1]);
+    if (e != cudaSuccess) return cuda_fail(e, "event elapsed");
+    tot += ms;
+  }
+  *total_ms = tot;
+  *count = g_prof.used;
+  g_prof.used = 0;
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,79 @@
+// Launch interfaces between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace attn {
+
+struct PrefillParams {
+  const void* q;          // [B, Hq, S, D] (T)
+  void* out;              // [B, Hq, S, D] (T)
+  float* lse;             // [B, Hq, S]
+  const float2* rope_cs;  // [S, D/2] (cos, sin) or nullptr when RoPE is off
+  int B, Hq, Hkv, S, G;
+  int causal;
+  float scale_log2;       // scale * log2(e)
+  int pair_heads;         // 1: the CTA's two tiles are heads h, h+1; 0: row blocks r, r+1 of one head
+  int n_row_blocks;       // ceil(S / 128)
+  int* status;            // device status word
+};
+
+// RoPE prologue: cos/sin table (angles in fp64), then the key operand.
+cudaError_t launch_rope_table(float2* cs, int S, int D, double theta, cudaStream_t stream);
+// bf16 K [rows, D] -> rotated fp16 K (row r at position r % S); flags values outside fp16 range.
+cudaError_t launch_rope_k_f16(const void* k, void* k_f16, const float2* cs, long long rows, int S, int D,
+                              int* status, cudaStream_t stream);
+// fp32 X [rows, D] -> bf16 hi parts at out[0, rows) and lo parts at out[rows, 2 rows), rotating
+// first when cs is non-null.
+cudaError_t launch_split_f32(const float* x, void* out, const float2* cs, long long rows, int S, int D,
+                             cudaStream_t stream);
+
+int prefill_block_n(int D, bool f32);
+cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV, int D, bool f32,
+                           bool rope, int grid, cudaStream_t stream);
+
+// ----------------------------------------------------------- paged decode
+constexpr int kDecodePagesPerSplit = 32;  // pages (of 16 tokens) handled by one split
+
+struct DecodeParams {
+  const void* q;            // [B, Hq, D] bf16
+  const int32_t* block_table;  // [B, max_pages]
+  const int32_t* seq_lens;  // [B]
+  float* part_o;            // [B, n_splits, Hq, D] fp32 (normalised partial outputs)
+  float* part_lse;          // [B, n_splits, Hq]
+  void* out;                // [B, Hq, D] bf16
+  float* lse;               // [B, Hq]
+  int B, Hq, Hkv, D, G;
+  int max_pages, num_pages, n_splits;
+  float scale_log2;
+  int* status;
+};
+cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                          cudaStream_t stream);
+
+// ------------------------------------------------------------------ MLA
+constexpr int kMlaTokensPerTile = 32;
+constexpr int kMlaTilesPerSplit = 16;  // 512 tokens per split
+
+struct MlaParams {
+  const int32_t* seq_lens;  // [B]
+  float* part_o;            // [B, n_splits, H, Dc] fp32
+  float* part_lse;          // [B, n_splits, H]
+  void* out;                // [B, H, Dc] bf16
+  float* lse;               // [B, H]
+  int B, H, Dc, Dr, T_max, n_splits;
+  float scale_log2;
+  int* status;
+};
+cudaError_t launch_mla(const MlaParams& p, const CUtensorMap& tmQn, const CUtensorMap& tmQp,
+                       const CUtensorMap& tmKV, const CUtensorMap& tmPE, cudaStream_t stream);
+
+// ------------------------------------------------------------- LSE merge
+// Combines n_valid(b) normalised partials per (b, head) into bf16 out and fp32 lse.
+// n_valid(b) = ceil(len_b / tokens_per_split); len_b == 0 gives out = 0, lse = -inf.
+cudaError_t launch_merge(const float* part_o, const float* part_lse, const int32_t* seq_lens, void* out, float* lse,
+                         int B, int H, int D, int n_splits, int tokens_per_split, cudaStream_t stream);
+
+}  // namespace attn

@@ -1,0 +1,554 @@
+// Causal GQA prefill on tcgen05 tensor cores (sm_100a).
+//
+// Computes O = softmax(scale * rope(Q) rope(K)^T [causal mask]) V and the
+// natural-log LSE of every row, tile by tile with the online-softmax recurrence
+// ("attention study note", sections "FlashAttention的改进" and
+// "online-softmax 分块计算原理": running max m, running sum l, and the matching
+// rescale of the output accumulator). Query head h reads KV head h / (Hq/Hkv)
+// (same page, GQA worked table).
+//
+// One CTA owns two 128-row query tiles that share one KV head: two heads of
+// the same group over the same rows when the group size is even, otherwise two
+// consecutive row blocks of one head. Roles (320 threads):
+//   warps 0-3  softmax warpgroup of tile 0 (one thread per query row)
+//   warps 4-7  softmax warpgroup of tile 1
+//   warp  8    TMA producer: K/V tiles into a shared-memory ring
+//   warp  9    TMEM allocator and single-thread tcgen05.mma issuer
+// TMEM holds S_0, S_1 (BN fp32 columns each) and O_0, O_1 (D columns each).
+// Q is rotated (RoPE from the fp32 cos/sin table) by the softmax threads while
+// they stage it into shared memory; K arrives already rotated from the prologue
+// kernel. P goes back to shared memory as the A operand of O += P V.
+//
+// Operand precision (every shared-memory tile is 16-bit):
+//   kModeBF16   bf16 input, no RoPE: Q K^T and P V in bf16 (exact inputs).
+//   kModeF16QK  bf16 input with RoPE: the rotated Q and K are rounded to fp16
+//               (11-bit significand, same tensor-core rate as bf16) so the
+//               rotation costs 8x less rounding than a bf16 round trip; P V in bf16.
+//   kModeSplit  fp32 input: every operand x is carried as hi = bf16(x) plus
+//               lo = bf16(x - hi), and each product uses the three terms
+//               hi*hi + hi*lo + lo*hi (about 16 significant bits per operand).
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <type_traits>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace attn {
+
+enum { kModeBF16 = 0, kModeF16QK = 1, kModeSplit = 2 };
+
+template <int D, int BN, int MODE>
+struct PrefillShape {
+  static constexpr int BM = 128;
+  static constexpr bool SPLIT = MODE == kModeSplit;
+  static constexpr int NPART = SPLIT ? 2 : 1;  // hi (and lo) parts of each operand tile
+  static constexpr int Q_BOX = BM * 128;       // bytes of one 64-column block of a Q tile
+  static constexpr int Q_PART = BM * D * 2;
+  static constexpr int KV_BOX = BN * 128;
+  static constexpr int KV_PART = BN * D * 2;
+  static constexpr int KV_SLOT = NPART * KV_PART;
+  static constexpr int P_BOX = BM * 128;
+  static constexpr int P_PART = BM * BN * 2;
+  static constexpr int FIXED = 2 * NPART * Q_PART + 2 * NPART * P_PART;
+  static constexpr int NST_RAW = (232448 - 1024 - 256 - FIXED) / KV_SLOT;
+  static constexpr int NST = NST_RAW > 8 ? 8 : NST_RAW;
+  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + FIXED + NST * KV_SLOT + 256 /*barriers*/;
+  static constexpr int TMEM_NEEDED = 2 * BN + 2 * D;
+  static constexpr int TMEM_COLS = TMEM_NEEDED <= 256 ? 256 : 512;
+  static constexpr int S_COL0 = 0;
+  static constexpr int O_COL0 = 2 * BN;
+  static constexpr uint32_t QK_FMT = MODE == kModeF16QK ? 0u : 1u;  // f16 : bf16
+  static_assert(NST >= 2, "K/V ring needs at least two slots");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(TMEM_NEEDED <= 512, "TMEM budget");
+  static_assert(D % 64 == 0 && BN % 64 == 0, "tiles are whole 128-byte swizzle rows");
+};
+
+constexpr float kRescaleThreshold = 8.0f;  // log2 domain: rescale O only when the max grows by > 2^8
+constexpr float kF16Max = 65504.f;
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// 8 consecutive values -> one 16-byte chunk of 16-bit elements.
+template <bool kF16>
+__device__ __forceinline__ uint4 pack8(const float* f) {
+  if constexpr (kF16)
+    return make_uint4(pack_half2(f[0], f[1]), pack_half2(f[2], f[3]), pack_half2(f[4], f[5]),
+                      pack_half2(f[6], f[7]));
+  else
+    return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                      pack_bf16x2(f[6], f[7]));
+}
+
+// hi = bf16(x), lo = bf16(x - hi) for 8 values.
+__device__ __forceinline__ void split8(const float* f, uint4& hi, uint4& lo) {
+  float h[8], l[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    h[e] = __bfloat162float(__float2bfloat16_rn(f[e]));
+    l[e] = f[e] - h[e];
+  }
+  hi = pack8<false>(h);
+  lo = pack8<false>(l);
+}
+
+template <typename TIn>
+__device__ __forceinline__ void load8(const TIn* p, float* f);
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float* f) {
+  const uint4 raw = __ldg(reinterpret_cast<const uint4*>(p));
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+template <>
+__device__ __forceinline__ void load8<float>(const float* p, float* f) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
+template <typename TIn>
+__device__ __forceinline__ void store32(TIn* dst, const float* f);
+template <>
+__device__ __forceinline__ void store32<__nv_bfloat16>(__nv_bfloat16* dst, const float* f) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) reinterpret_cast<uint4*>(dst)[i] = pack8<false>(f + 8 * i);
+}
+template <>
+__device__ __forceinline__ void store32<float>(float* dst, const float* f) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    reinterpret_cast<float4*>(dst)[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
+}
+
+template <int D, int BN, int MODE>
+__global__ void __launch_bounds__(320, 1)
+    prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV) {
+  using Sh = PrefillShape<D, BN, MODE>;
+  using TIn = typename std::conditional<MODE == kModeSplit, float, __nv_bfloat16>::type;
+  constexpr int NP = Sh::NPART;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;                           // [2 tiles][NP parts][Q_PART]
+  uint8_t* sP = sQ + 2 * NP * Sh::Q_PART;       // [2 tiles][NP parts][P_PART]
+  uint8_t* sKV = sP + 2 * NP * Sh::P_PART;      // [NST][NP parts][KV_PART]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + Sh::NST * Sh::KV_SLOT);
+  uint64_t* kv_full = bars;                     // [NST]
+  uint64_t* kv_empty = bars + Sh::NST;          // [NST]
+  uint64_t* q_full = bars + 2 * Sh::NST;        // [1]
+  uint64_t* s_full = q_full + 1;                // [2]
+  uint64_t* p_full = s_full + 2;                // [2]
+  uint64_t* o_done = p_full + 2;                // [2]
+  uint64_t* mma_done = o_done + 2;              // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---------------------------------------------------------------- work item
+  int b, h0, h1, r0_0, r0_1;
+  {
+    const int w = blockIdx.x;
+    if (p.pair_heads) {
+      const int units = p.B * (p.Hq / 2);
+      const int rb = p.n_row_blocks - 1 - w / units;  // heaviest (last) row blocks first
+      const int bh = w % units;
+      b = bh / (p.Hq / 2);
+      h0 = 2 * (bh % (p.Hq / 2));
+      h1 = h0 + 1;
+      r0_0 = r0_1 = rb * Sh::BM;
+    } else {
+      const int units = p.B * p.Hq;
+      const int n_rp = (p.n_row_blocks + 1) / 2;
+      const int rp = n_rp - 1 - w / units;
+      const int bh = w % units;
+      b = bh / p.Hq;
+      h0 = h1 = bh % p.Hq;
+      r0_0 = 2 * rp * Sh::BM;
+      r0_1 = r0_0 + Sh::BM;
+    }
+  }
+  const int kvh = h0 / p.G;
+  const int n_kv_all = (p.S + BN - 1) / BN;
+  auto n_kv_for = [&](int r0) -> int {
+    if (r0 >= p.S) return 0;
+    if (!p.causal) return n_kv_all;
+    const int last = min(p.S, r0 + Sh::BM) - 1;
+    return last / BN + 1;
+  };
+  const int n_kv0 = n_kv_for(r0_0);
+  const int n_kv1 = n_kv_for(r0_1);
+  const int n_max = max(n_kv0, n_kv1);
+
+  // -------------------------------------------------------------------- setup
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < Sh::NST; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    mbar_init(q_full, 256);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 128);
+      mbar_init(&o_done[t], 1);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, Sh::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      const int zc = b * p.Hkv + kvh;
+      const int zlo = p.B * p.Hkv;  // the lo parts follow the hi parts in the split layout
+      for (int i = 0; i < 2 * n_max; ++i) {
+        const int j = i >> 1;
+        const int s = i % Sh::NST;
+        const uint32_t ph = (i / Sh::NST) & 1;
+        if (!mbar_wait(&kv_empty[s], ph ^ 1, abort_flag, p.status)) break;
+        uint8_t* dst = sKV + s * Sh::KV_SLOT;
+        mbar_arrive_expect_tx(&kv_full[s], Sh::KV_SLOT);
+        const CUtensorMap* map = (i & 1) ? &tmV : &tmK;
+#pragma unroll
+        for (int u = 0; u < NP; ++u)
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(dst + u * Sh::KV_PART + c * Sh::KV_BOX, map, &kv_full[s], c * 64, j * BN, zc + u * zlo);
+      }
+    }
+  } else if (warp == 9) {
+    // -------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_f32acc(Sh::QK_FMT, 128, BN, false, false);
+      constexpr uint32_t idesc_pv = idesc_f32acc(1, 128, D, false, true);
+      // (A part, B part) products: hi*hi, plus hi*lo and lo*hi for split operands
+      constexpr int NPROD = Sh::SPLIT ? 3 : 1;
+      const int n_kv[2] = {n_kv0, n_kv1};
+      bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
+      auto issue_qk = [&](int t, int slot) {
+        const uint32_t a0 = smem_u32(sQ + t * NP * Sh::Q_PART);
+        const uint32_t b0 = smem_u32(sKV + slot * Sh::KV_SLOT);
+        const uint32_t d = tmem_base + Sh::S_COL0 + t * BN;
+#pragma unroll
+        for (int kb = 0; kb < D / 16; ++kb) {
+          const uint32_t koff = (kb >> 2) * 0u + (kb & 3) * 32u;  // 32-byte K step inside a 128-byte row
+#pragma unroll
+          for (int x = 0; x < NPROD; ++x) {
+            const int pa = x == 2 ? 1 : 0, pb = x == 1 ? 1 : 0;
+            const uint64_t ad = sdesc_sw128(a0 + pa * Sh::Q_PART + (kb >> 2) * Sh::Q_BOX + koff, 16, 1024);
+            const uint64_t bd = sdesc_sw128(b0 + pb * Sh::KV_PART + (kb >> 2) * Sh::KV_BOX + koff, 16, 1024);
+            umma_ss<false>(d, ad, bd, idesc_qk, (kb > 0 || x > 0) ? 1u : 0u);
+          }
+        }
+      };
+      auto issue_pv = [&](int t, int slot, bool acc) {
+        const uint32_t a0 = smem_u32(sP + t * NP * Sh::P_PART);
+        const uint32_t b0 = smem_u32(sKV + slot * Sh::KV_SLOT);
+        const uint32_t d = tmem_base + Sh::O_COL0 + t * D;
+#pragma unroll
+        for (int kb = 0; kb < BN / 16; ++kb) {
+#pragma unroll
+          for (int x = 0; x < NPROD; ++x) {
+            const int pa = x == 2 ? 1 : 0, pb = x == 1 ? 1 : 0;
+            const uint64_t ad =
+                sdesc_sw128(a0 + pa * Sh::P_PART + (kb >> 2) * Sh::P_BOX + (kb & 3) * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(b0 + pb * Sh::KV_PART + kb * 16 * 128, Sh::KV_BOX, 1024);
+            umma_ss<false>(d, ad, bd, idesc_pv, (acc || kb > 0 || x > 0) ? 1u : 0u);
+          }
+        }
+      };
+      if (ok && n_max > 0) {
+        // K_0 sits in ring slot 0
+        ok = mbar_wait(&kv_full[0], 0, abort_flag, p.status);
+        if (ok) {
+          tc_fence_after();
+          for (int t = 0; t < 2; ++t)
+            if (n_kv[t] > 0) {
+              issue_qk(t, 0);
+              umma_commit(&s_full[t]);
+            }
+          umma_commit(&kv_empty[0]);
+        }
+        for (int j = 0; ok && j < n_max; ++j) {
+          const int iV = 2 * j + 1, sV = iV % Sh::NST;
+          const int iK = 2 * j + 2, sK = iK % Sh::NST;
+          if (!mbar_wait(&kv_full[sV], (iV / Sh::NST) & 1, abort_flag, p.status)) { ok = false; break; }
+          bool k_ready = false;
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (j >= n_kv[t]) continue;
+            if (!mbar_wait(&p_full[t], j & 1, abort_flag, p.status)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(t, sV, j > 0);
+            umma_commit(&o_done[t]);
+            if (j + 1 < n_kv[t]) {
+              if (!k_ready) {
+                if (!mbar_wait(&kv_full[sK], (iK / Sh::NST) & 1, abort_flag, p.status)) { ok = false; break; }
+                tc_fence_after();
+                k_ready = true;
+              }
+              issue_qk(t, sK);
+              umma_commit(&s_full[t]);
+            }
+          }
+          if (!ok) break;
+          umma_commit(&kv_empty[sV]);
+          if (k_ready) umma_commit(&kv_empty[sK]);
+        }
+      }
+      // drain: every MMA issued above has completed once this barrier flips
+      umma_commit(mma_done);
+      mbar_wait(mma_done, 0, abort_flag, p.status);
+    }
+  } else {
+    // ------------------------------------------------------- softmax warpgroups
+    const int t = warp >> 2;
+    const int wr = warp & 3;
+    const int row = wr * 32 + lane;  // TMEM lane == query row within the tile
+    const int h = t ? h1 : h0;
+    const int r0 = t ? r0_1 : r0_0;
+    const int n_kv = t ? n_kv1 : n_kv0;
+    const int grow = r0 + row;
+    const bool row_valid = grow < p.S;
+    const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(wr * 32) << 16);
+
+    // Stage Q (rotated) into the swizzled K-major tile(s).
+    {
+      uint8_t* qtile = sQ + t * NP * Sh::Q_PART;
+      const TIn* qrow = reinterpret_cast<const TIn*>(p.q) + ((static_cast<size_t>(b) * p.Hq + h) * p.S + grow) * D;
+      const float2* cs = p.rope_cs ? p.rope_cs + static_cast<size_t>(grow) * (D / 2) : nullptr;
+      bool range_ok = true;
+#pragma unroll 2
+      for (int c = 0; c < D / 8; ++c) {
+        float f[8];
+        if (row_valid && n_kv > 0) {
+          load8<TIn>(qrow + c * 8, f);
+          if (cs) {
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              const float2 r = __ldg(cs + (c * 8 + e) / 2);
+              const float x0 = f[e], x1 = f[e + 1];
+              f[e] = x0 * r.x - x1 * r.y;
+              f[e + 1] = x0 * r.y + x1 * r.x;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = 0.f;
+        }
+        const int box = c >> 3, ch = c & 7;
+        const int off = box * Sh::Q_BOX + row * 128 + ((ch ^ (row & 7)) << 4);
+        if constexpr (MODE == kModeSplit) {
+          uint4 hi, lo;
+          split8(f, hi, lo);
+          *reinterpret_cast<uint4*>(qtile + off) = hi;
+          *reinterpret_cast<uint4*>(qtile + Sh::Q_PART + off) = lo;
+        } else if constexpr (MODE == kModeF16QK) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) range_ok = range_ok && fabsf(f[e]) <= kF16Max;
+          *reinterpret_cast<uint4*>(qtile + off) = pack8<true>(f);
+        } else {
+          *reinterpret_cast<uint4*>(qtile + off) = pack8<false>(f);
+        }
+      }
+      if (!range_ok) atomicOr(p.status, kDevErrRange);
+      fence_proxy_async_smem();
+      mbar_arrive(q_full);
+    }
+
+    float m_run = -INFINITY;
+    float l_run = 0.f;
+    const float sl2 = p.scale_log2;
+    const int limit = p.causal ? min(grow, p.S - 1) : p.S - 1;  // last key this row may see
+    bool alive = true;
+    uint8_t* ptile = sP + t * NP * Sh::P_PART;
+
+    for (int j = 0; j < n_kv && alive; ++j) {
+      bool ok = mbar_wait(&s_full[t], j & 1, abort_flag, p.status);
+      if (__any_sync(0xffffffffu, !ok)) { alive = false; break; }
+      tc_fence_after();
+      // Pass 1: row max over the tile. The last KEEP 32-column chunks stay in
+      // registers; the others are read again from TMEM in pass 2 (S_t is not
+      // overwritten before this warpgroup arrives on p_full).
+      constexpr int NCH = BN / 32;
+      constexpr int KEEP = NCH > 2 ? 2 : NCH;
+      const int thr = limit - j * BN;  // columns > thr are masked
+      float keep[KEEP * 32];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) {
+        uint32_t r[32];
+        tmem_ld32(t_lane + Sh::S_COL0 + t * BN + c * 32, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float x = (c * 32 + e > thr) ? -INFINITY : __uint_as_float(r[e]);
+          mx = fmaxf(mx, x);
+          if (c >= NCH - KEEP) keep[(c - (NCH - KEEP)) * 32 + e] = x;
+        }
+      }
+      const float m_tile = mx * sl2;
+      const float m_new = fmaxf(m_run, m_tile);
+
+      // PV(j-1) must be complete before P is overwritten and before O is rescaled.
+      float alpha = 1.f;
+      bool rescale = false;
+      if (j > 0) {
+        ok = mbar_wait(&o_done[t], (j - 1) & 1, abort_flag, p.status);
+        if (__any_sync(0xffffffffu, !ok)) { alive = false; break; }
+        tc_fence_after();
+        rescale = __any_sync(0xffffffffu, m_new > m_run + kRescaleThreshold);
+        if (rescale) {
+          alpha = ex2_approx(m_run - m_new);
+          m_run = m_new;
+          l_run *= alpha;
+        }
+      } else {
+        m_run = m_new;
+      }
+
+      // Pass 2: P = exp2(s * scale * log2(e) - m), row sum, store swizzled (K-major) for P V.
+      const float neg_m = -m_run;
+      float lsum = 0.f;
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) {
+        float x[32];
+        if (c < NCH - KEEP) {
+          uint32_t r[32];
+          tmem_ld32(t_lane + Sh::S_COL0 + t * BN + c * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[e] = (c * 32 + e > thr) ? -INFINITY : __uint_as_float(r[e]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[e] = keep[(c - (NCH - KEEP)) * 32 + e];
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float f[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float pv = ex2_approx(fmaf(x[i * 8 + e], sl2, neg_m));
+            f[e] = pv;
+            lsum += pv;
+          }
+          const int gc = c * 4 + i;  // 16-byte chunk index within the row
+          const int off = (gc >> 3) * Sh::P_BOX + row * 128 + (((gc & 7) ^ (row & 7)) << 4);
+          if constexpr (Sh::SPLIT) {
+            uint4 hi, lo;
+            split8(f, hi, lo);
+            *reinterpret_cast<uint4*>(ptile + off) = hi;
+            *reinterpret_cast<uint4*>(ptile + Sh::P_PART + off) = lo;
+          } else {
+            *reinterpret_cast<uint4*>(ptile + off) = pack8<false>(f);
+          }
+        }
+      }
+      // O *= alpha (warp-uniform decision; exact because P and l use the same m)
+      if (rescale) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          const uint32_t ta = t_lane + Sh::O_COL0 + t * D + c * 32;
+          tmem_ld32(ta, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          tmem_st32(ta, r);
+        }
+        tmem_st_wait();
+      }
+      l_run += lsum;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_full[t]);
+    }
+
+    // Epilogue: O / l and LSE = (m + log2 l) * ln 2.
+    if (alive && n_kv > 0) {
+      bool ok = mbar_wait(&o_done[t], (n_kv - 1) & 1, abort_flag, p.status);
+      if (!__any_sync(0xffffffffu, !ok)) {
+        tc_fence_after();
+        const float inv_l = 1.f / l_run;
+        TIn* orow = reinterpret_cast<TIn*>(p.out) + ((static_cast<size_t>(b) * p.Hq + h) * p.S + grow) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(t_lane + Sh::O_COL0 + t * D + c * 32, r);
+          tmem_ld_wait();
+          if (row_valid) {
+            float f[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(r[e]) * inv_l;
+            store32<TIn>(orow + c * 32, f);
+          }
+        }
+        if (row_valid)
+          p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.S + grow] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Sh::TMEM_COLS);
+  }
+}
+
+template <int D, int BN, int MODE>
+static cudaError_t launch_prefill_t(const PrefillParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                    int grid, cudaStream_t stream) {
+  using Sh = PrefillShape<D, BN, MODE>;
+  auto kern = prefill_kernel<D, BN, MODE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sh::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, 320, Sh::SMEM_BYTES, stream>>>(p, tmK, tmV);
+  return cudaGetLastError();
+}
+
+int prefill_block_n(int D, bool f32) {
+  (void)D;
+  return f32 ? 64 : 128;
+}
+
+cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV, int D, bool f32,
+                           bool rope, int grid, cudaStream_t stream) {
+  if (f32) {
+    if (D == 64) return launch_prefill_t<64, 64, kModeSplit>(p, tmK, tmV, grid, stream);
+    return cudaErrorInvalidValue;
+  }
+  if (rope) {
+    if (D == 128) return launch_prefill_t<128, 128, kModeF16QK>(p, tmK, tmV, grid, stream);
+    if (D == 64) return launch_prefill_t<64, 128, kModeF16QK>(p, tmK, tmV, grid, stream);
+  } else {
+    if (D == 128) return launch_prefill_t<128, 128, kModeBF16>(p, tmK, tmV, grid, stream);
+    if (D == 64) return launch_prefill_t<64, 128, kModeBF16>(p, tmK, tmV, grid, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace attn

@@ -1,0 +1,431 @@
+#!/usr/bin/env python
+"""Benchmark: prefill attention TFLOP/s (headline) plus paged-decode and MLA-decode
+KV-read GB/s, each against the B200 roofline.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Headline step: one attn_prefill call (RoPE prologue + tcgen05 prefill kernel) on the
+causal GQA workload B=2, Hq=32, Hkv=8, S=4096, D=128, bf16; L2 is flushed between
+timed steps. The paged-decode (B=64, Hq=32, Hkv=8, D=128, lengths U[1024, 32768],
+16-token pages) and MLA-decode (B=32, H=128, Dc=512, Dr=64, T U[4096, 32768])
+workloads are timed the same way in their own regions and reported beside it.
+Under torchrun every rank runs its own replica (independent batches, no data-path
+collective): weak scaling; times are device times, max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+PREFILL = "gqa_prefill_b2_hq32_hkv8_s4096_d128"
+DECODE = "paged_decode_b64_hq32_hkv8_d128"
+MLA = "mla_decode_b32_h128_dc512_dr64"
+METRIC = "prefill attn TFLOP/s & decode KV-read GB/s, % of B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def prefill_flops(p):
+    # exact causal: Q K^T and P V over the lower triangle incl. the diagonal
+    return p["B"] * p["Hq"] * 4.0 * p["D"] * p["S"] * (p["S"] + 1) / 2.0
+
+
+# ------------------------------------------------------------------ clocks
+class Clocks:
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        q = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 7:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    mx = float(parts[1])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[3:7]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------- helpers
+def traffic_for(kernel: str, fingerprint: str):
+    """DRAM bytes per launch from a committed ncu summary, only if taken on this exact source."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 3 and not line.startswith("#") and parts[0] == kernel and parts[1] == fingerprint:
+                return float(parts[2])
+    return None
+
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def timed_region(fn, steps, warmup, world, flush=None):
+    """Runs warmup + steps calls of fn; returns (summed device ms of the steps, max over ranks)."""
+    import torch
+    for _ in range(warmup):
+        if flush is not None:
+            flush()
+        fn()
+    barrier(world)
+    evs = []
+    st = torch.cuda.current_stream()
+    for _ in range(steps):
+        if flush is not None:
+            flush()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        fn()
+        e1.record(st)
+        evs.append((e0, e1))
+    barrier(world)
+    ms = sum(a.elapsed_time(b) for a, b in evs)
+    return max_over_ranks(ms, world)
+
+
+# ----------------------------------------------------------- CPU oracle leg
+def oracle_prefill_sample(q, k, v, p, budget_s):
+    """Times the float64 oracle on whole heads of the workload until ~budget_s elapsed."""
+    import numpy as np
+    from oracle import prefill_ref
+    qn = q.float().cpu().numpy()
+    kn = k.float().cpu().numpy()
+    vn = v.float().cpu().numpy()
+    G = p["Hq"] // p["Hkv"]
+    heads, t0 = 0, time.perf_counter()
+    for b in range(p["B"]):
+        for h in range(p["Hq"]):
+            kvh = h // G
+            prefill_ref(qn[b:b + 1, h:h + 1], kn[b:b + 1, kvh:kvh + 1], vn[b:b + 1, kvh:kvh + 1], causal=True,
+                        rope_theta=p["theta"], scale=p["scale"])
+            heads += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    flops = heads * 4.0 * p["D"] * p["S"] * (p["S"] + 1) / 2.0
+    return flops / dt / 1e12, heads, dt
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def run_reference(args):
+    """Reference arm: the float64 CPU oracle, timed as it stands on the host cores."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import numpy as np
+    from attention_causal_gqa_b200.synthetic import WORKLOADS, prefill_inputs
+    from oracle import prefill_ref
+    p = WORKLOADS[PREFILL].params
+    q, k, v = prefill_inputs(p["B"], p["Hq"], p["Hkv"], p["S"], p["D"], p["dtype"], p["std"], seed=20261202,
+                             device="cpu")
+    qn, kn, vn = (x.float().numpy() for x in (q, k, v))
+    G = p["Hq"] // p["Hkv"]
+    per_head = 4.0 * p["D"] * p["S"] * (p["S"] + 1) / 2.0
+    times = []
+    for i in range(args.warmup + args.steps):
+        b, h = divmod(i % (p["B"] * p["Hq"]), p["Hq"])
+        t0 = time.perf_counter()
+        prefill_ref(qn[b:b + 1, h:h + 1], kn[b:b + 1, h // G:h // G + 1], vn[b:b + 1, h // G:h // G + 1],
+                    causal=True, rope_theta=p["theta"], scale=p["scale"])
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    tot = sum(times)
+    val = per_head * len(times) / tot / 1e12
+    sample = f"one (b, head) of the {PREFILL} workload per step: all {p['S']} causal rows, float64"
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": PREFILL, "sample": "one head per step"},
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+    world, rank, local = dist_setup()
+    from attention_causal_gqa_b200 import binding as B_
+    from attention_causal_gqa_b200.build import _fingerprint
+    from attention_causal_gqa_b200.synthetic import WORKLOADS, workload_inputs
+
+    pk, pk_kind = peaks()
+    fp = _fingerprint()[:16]
+    dev = torch.device("cuda", local if world > 1 else 0)
+    seed = 20261202 + 1000 * rank
+    flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def flush():
+        flush_buf.zero_()
+
+    # ------------------------------------------------------------ prefill
+    p = WORKLOADS[PREFILL].params
+    q, k, v = workload_inputs(PREFILL, seed=seed, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((p["B"], p["Hq"], p["S"]), dtype=torch.float32, device=dev)
+    ws = torch.empty(B_.prefill_workspace_size(p["B"], p["Hkv"], p["S"], p["D"]), dtype=torch.uint8, device=dev)
+
+    def step_prefill():
+        B_.attn_prefill(q, k, v, causal=True, rope_theta=p["theta"], scale=p["scale"], out=out, lse=lse,
+                        workspace=ws)
+
+    clocks = Clocks(local if world > 1 else int(os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0] or 0))
+    B_.profile_enable(True)
+    B_.profile_collect()
+    clocks.start()
+    # warm-up is excluded from the kernel timing hook by collecting after it
+    for _ in range(args.warmup):
+        flush()
+        step_prefill()
+    torch.cuda.synchronize()
+    B_.profile_collect()
+    ms = timed_region(step_prefill, args.steps, 0, world, flush=flush)
+    kern_ms, n_launch = B_.profile_collect()
+    clk = clocks.stop()
+    flops = prefill_flops(p)
+    value = world * flops * args.steps / (ms * 1e-3) / 1e12
+    kern_avg = kern_ms / max(n_launch, 1)
+    kern_avg = max_over_ranks(kern_avg, world)
+    achieved = flops / (kern_avg * 1e-3) / 1e12
+    peak = pk["bf16_tflops"]
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "traffic": traffic_for("prefill_kernel", fp), "kernel": "prefill_kernel",
+            "peak_kind": f"{pk_kind} dense bf16 (burst)", "kernel_ms": kern_avg,
+            "algorithmic": f"{flops:.4g} flop per launch = B*Hq*4*D*S(S+1)/2"}
+
+    # e2e: host (pinned) buffers, copies inside the timed region
+    qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
+    oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    lh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+    def step_e2e():
+        q.copy_(qh, non_blocking=True)
+        k.copy_(kh, non_blocking=True)
+        v.copy_(vh, non_blocking=True)
+        step_prefill()
+        oh.copy_(out, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+
+    e2e_steps = max(3, args.steps // 2)
+    ms_e2e = timed_region(step_e2e, e2e_steps, 2, world)
+    e2e_val = world * flops * e2e_steps / (ms_e2e * 1e-3) / 1e12
+    h2d = sum(x.numel() * x.element_size() for x in (qh, kh, vh))
+    d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
+    del qh, kh, vh, oh, lh
+
+    # ------------------------------------------------------------- decode
+    sub = {}
+    if not args.prefill_only:
+        dp = WORKLOADS[DECODE].params
+        d = workload_inputs(DECODE, seed=seed, device=dev)
+        dout = torch.empty_like(d["q"])
+        dlse = torch.empty((dp["B"], dp["Hq"]), dtype=torch.float32, device=dev)
+        dws = torch.empty(B_.decode_workspace_size(dp["B"], dp["Hq"], dp["D"], d["max_pages_per_seq"]),
+                          dtype=torch.uint8, device=dev)
+
+        def step_decode():
+            B_.attn_decode_paged(d["q"], d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"],
+                                 scale=dp["scale"], out=dout, lse=dlse, workspace=dws)
+
+        tokens = int(d["seq_lens"].sum().item())
+        kv_bytes = tokens * dp["Hkv"] * dp["D"] * 2 * 2
+        for _ in range(args.warmup):
+            step_decode()
+        torch.cuda.synchronize()
+        B_.profile_collect()
+        dms = timed_region(step_decode, args.steps, 0, world)
+        dk_ms, dn = B_.profile_collect()
+        dk_avg = max_over_ranks(dk_ms / max(dn, 1), world)
+        sub["decode"] = {
+            "workload": DECODE, "value": world * kv_bytes * args.steps / (dms * 1e-3) / 1e9, "unit": "GB/s",
+            "ms_per_step": dms / args.steps, "kv_tokens": tokens, "kv_bytes_per_step": kv_bytes,
+            "gpu_launches": 2 * args.steps,
+            "roofline": {"bound": "hbm", "achieved": kv_bytes / (dk_avg * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": kv_bytes / (dk_avg * 1e-3) / 1e9 / pk["hbm_gbs"],
+                         "traffic": traffic_for("decode_kernel", fp), "kernel": "decode_kernel",
+                         "kernel_ms": dk_avg, "peak_kind": f"{pk_kind} HBM copy",
+                         "algorithmic": "4096 B per cached token (K+V, 8 heads x 128 x bf16)"}}
+        del d, dout, dlse, dws
+        torch.cuda.empty_cache()
+
+        # ------------------------------------------------------------ MLA
+        mp = WORKLOADS[MLA].params
+        m = workload_inputs(MLA, seed=seed, device=dev)
+        mout = torch.empty_like(m["q_nope"])
+        mlse = torch.empty((mp["B"], 1, mp["H"]), dtype=torch.float32, device=dev)
+        mws = torch.empty(B_.mla_workspace_size(mp["B"], mp["H"], mp["Dc"], mp["Dr"], m["T_max"]),
+                          dtype=torch.uint8, device=dev)
+
+        def step_mla():
+            B_.mla_decode(m["q_nope"], m["q_pe"], m["kv_cache"], m["pe_cache"], m["seq_lens"], mp["scale"],
+                          out=mout, lse=mlse, workspace=mws)
+
+        mtok = int(m["seq_lens"].sum().item())
+        mbytes = mtok * (mp["Dc"] + mp["Dr"]) * 2
+        mflops = mtok * mp["H"] * (2.0 * (mp["Dc"] + mp["Dr"]) + 2.0 * mp["Dc"])
+        for _ in range(args.warmup):
+            step_mla()
+        torch.cuda.synchronize()
+        B_.profile_collect()
+        mms = timed_region(step_mla, args.steps, 0, world)
+        mk_ms, mn = B_.profile_collect()
+        mk_avg = max_over_ranks(mk_ms / max(mn, 1), world)
+        sub["mla"] = {
+            "workload": MLA, "value": world * mbytes * args.steps / (mms * 1e-3) / 1e9, "unit": "GB/s",
+            "ms_per_step": mms / args.steps, "kv_tokens": mtok, "kv_bytes_per_step": mbytes,
+            "tflops": world * mflops * args.steps / (mms * 1e-3) / 1e12, "gpu_launches": 2 * args.steps,
+            "roofline": {"bound": "hbm", "achieved": mbytes / (mk_avg * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": mbytes / (mk_avg * 1e-3) / 1e9 / pk["hbm_gbs"],
+                         "traffic": traffic_for("mla_kernel", fp), "kernel": "mla_kernel", "kernel_ms": mk_avg,
+                         "peak_kind": f"{pk_kind} HBM copy",
+                         "algorithmic": "1152 B per cached token (kv 512 + pe 64, bf16)",
+                         "tensor_frac": mflops / (mk_avg * 1e-3) / 1e12 / pk["bf16_tflops"]}}
+        del m, mout, mlse, mws
+    B_.profile_enable(False)
+
+    # -------------------------------------------------------- CPU baseline
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, heads, dt = oracle_prefill_sample(q, k, v, p, budget_s=args.cpu_budget)
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{heads} whole heads (all {p['S']} causal rows each) of {PREFILL}, float64, {dt:.1f} s"}
+
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": PREFILL, "B": p["B"], "Hq": p["Hq"], "Hkv": p["Hkv"], "S": p["S"], "D": p["D"],
+                       "causal": True, "rope_theta": p["theta"], "l2": "flushed (256 MB write) between steps",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": roof, "cpu_baseline": cpu,
+            "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": 3 * args.steps, "clocks": clk, "source_fingerprint": fp}
+    line.update(sub)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--prefill-only", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

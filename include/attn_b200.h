@@ -1,0 +1,153 @@
+/*
+ * attn_b200 — exact causal GQA attention, paged GQA decode and MLA absorbed decode
+ * for NVIDIA B200 (sm_100a). C ABI: plain pointers and sizes only.
+ *
+ * Conventions for every entry point
+ *  - All tensor pointers are DEVICE pointers, contiguous, 16-byte aligned
+ *    (lse arrays: 4-byte aligned). The caller owns every buffer (inputs, outputs,
+ *    workspace); the library allocates nothing on these calls and keeps no pointer
+ *    after it returns.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Work is enqueued asynchronously; buffers must stay alive until it completes.
+ *  - Return value: ATTN_OK, or an error code. Arguments are validated on the host
+ *    before anything is enqueued; on error nothing is launched and
+ *    attn_last_error() describes the problem (thread-local string).
+ *  - Device-side problems (a bounded wait that ran out, a block-table entry outside
+ *    the page pool, a length beyond the cache) are recorded as bit flags in a status
+ *    word at the start of the workspace; read it with attn_read_status() after the
+ *    call's work has completed. Each call clears it when it starts.
+ *  - LSE is the natural logarithm of the sum of exp(scaled scores), fp32.
+ *  - A sequence of length 0 yields out = 0 and lse = -inf.
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, Hq % Hkv != 0, misalignment */
+  ATTN_ERR_UNSUPPORTED = 2,  /* shape or dtype outside what the kernels implement */
+  ATTN_ERR_WORKSPACE = 3,    /* workspace smaller than the *_workspace_size() query */
+  ATTN_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed (message has details) */
+  ATTN_ERR_DEVICE = 5        /* returned by attn_read_status() when the device flagged a problem */
+};
+
+enum { ATTN_DTYPE_F32 = 0, ATTN_DTYPE_BF16 = 1 };
+
+/* Device status flags (attn_read_status). */
+enum { ATTN_DEV_TIMEOUT = 1, ATTN_DEV_BAD_PAGE = 2, ATTN_DEV_BAD_LENGTH = 4, ATTN_DEV_RANGE = 8 };
+
+/*
+ * Causal GQA/MQA/MHA prefill with RoPE.
+ * Defined by: "attention study note" (makinaruto.github.io, llm_learning/attention),
+ * sections "FlashAttention的改进" / "online-softmax 分块计算原理" (tiled exact attention
+ * with running max/sum) and the GQA worked table (query head h uses kv head
+ * h / (Hq/Hkv)); "From 32K to 256K: DeepSeek long-context" (tqpw.cn) section 2.1
+ * (RoPE on adjacent pairs, theta_i = rope_theta^(-2i/D)) and 2.5 (cos/sin cache).
+ *
+ *   q   [B, Hq,  S, D]   dtype (bf16, or fp32 computed as tf32)
+ *   k,v [B, Hkv, S, D]   dtype
+ *   out [B, Hq,  S, D]   dtype (written)
+ *   lse [B, Hq,  S]      fp32  (written)
+ * causal: 1 -> key j is visible to query i iff j <= i; 0 -> all keys.
+ * rope_theta: > 0 applies RoPE to q and k at positions 0..S-1; <= 0 disables it.
+ * scale: multiplies q.k before the softmax; <= 0 selects 1/sqrt(D).
+ * Supported: dtype BF16 with D in {64, 128}; dtype F32 with D = 64.
+ * Tensor-core operand precision: bf16 without RoPE multiplies the bf16 inputs as
+ * they are; bf16 with RoPE rounds the rotated q and k to fp16 for Q.K^T (so
+ * |rotated value| must stay <= 65504, else ATTN_DEV_RANGE is flagged); fp32 input
+ * carries every operand as a bf16 hi + lo pair (three products per MMA step).
+ * P.V always accumulates in fp32 from bf16 P (hi + lo for fp32 input).
+ * workspace: >= attn_prefill_workspace_size(B, Hkv, S, D, dtype) bytes of device memory,
+ * 256-byte aligned.
+ */
+size_t attn_prefill_workspace_size(int B, int Hkv, int S, int D, int dtype);
+int attn_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv, int S,
+                 int D, int causal, float rope_theta, float scale, int dtype, void* workspace,
+                 size_t workspace_bytes, void* stream);
+
+/*
+ * Paged split-KV GQA decode: one query token per sequence attends to all
+ * seq_lens[b] cached tokens (already rotated; no RoPE, no mask).
+ * Defined by: "attention study note", section "Page Attention" (fixed-size pages
+ * reached through a per-sequence table) and the online-softmax recurrence used to
+ * merge per-split partial results.
+ *
+ *   q            [B, Hq, D]                       bf16
+ *   k_pages      [num_pages, page_size, Hkv, D]   bf16
+ *   v_pages      [num_pages, page_size, Hkv, D]   bf16
+ *   block_table  [B, max_pages_per_seq]  int32: physical page of logical page j;
+ *                entries at or past ceil(seq_lens[b]/page_size) are never read
+ *   seq_lens     [B] int32, 0 <= seq_lens[b] <= max_pages_per_seq * page_size
+ *   out          [B, Hq, D] bf16 (written);  lse [B, Hq] fp32 (written)
+ * Supported: dtype BF16, page_size 16, D in {64, 128}, Hkv <= 8, Hq/Hkv <= 16.
+ * scale <= 0 selects 1/sqrt(D). Out-of-range table entries or lengths are clamped
+ * (no fault) and flagged in the status word.
+ */
+size_t attn_decode_paged_workspace_size(int B, int Hq, int D, int max_pages_per_seq, int page_size);
+int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
+                      const int32_t* seq_lens, void* out, float* lse, int B, int Hq, int Hkv, int D, int page_size,
+                      int max_pages_per_seq, int num_pages, float scale, int dtype, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
+/*
+ * DeepSeek MLA absorbed decode (one query token per sequence).
+ * Defined by: "DeepSeek-V3 attention: einsum vs hand-optimised" (dksg.cn), absorbed
+ * form: scores = (q_nope . kv_cache^T + q_pe . pe_cache^T) * scale,
+ * out = softmax(scores) . kv_cache; "attention study note", MLA absorption and
+ * decoupled-RoPE sections.
+ *
+ *   q_nope   [B, 1, H, Dc]   bf16      q_pe     [B, 1, H, Dr]  bf16
+ *   kv_cache [B, T_max, Dc]  bf16      pe_cache [B, T_max, Dr] bf16
+ *   seq_lens [B] int32, 0 <= seq_lens[b] <= T_max (tokens past it are never used)
+ *   out      [B, 1, H, Dc]   bf16 (written);  lse [B, 1, H] fp32 (written)
+ * Supported: H = 128, Dc = 512, Dr = 64. scale must be > 0.
+ */
+size_t mla_decode_workspace_size(int B, int H, int Dc, int Dr, int T_max);
+int mla_decode(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
+               const int32_t* seq_lens, float scale, void* out, float* lse, int B, int H, int Dc, int Dr, int T_max,
+               void* workspace, size_t workspace_bytes, void* stream);
+
+/* Thread-local description of the last error returned on this thread ("" if none). */
+const char* attn_last_error(void);
+
+/*
+ * Waits for `stream`, then copies the status word at the start of `workspace` into
+ * *flags (a bitwise OR of ATTN_DEV_*). Returns ATTN_OK when no flag is set,
+ * ATTN_ERR_DEVICE when one is, ATTN_ERR_CUDA when the copy fails.
+ */
+int attn_read_status(const void* workspace, int* flags, void* stream);
+
+/*
+ * Self-test of the bounded-wait mechanism every kernel uses: launches one CTA that
+ * waits on an mbarrier nothing ever arrives at, with the given limit in
+ * nanoseconds (1e3 .. 1e10). The wait gives up, the kernel records
+ * ATTN_DEV_TIMEOUT in the workspace status word and exits normally, so the CUDA
+ * context stays usable. workspace: >= 256 bytes.
+ */
+int attn_selftest_wait_timeout(void* workspace, size_t workspace_bytes, unsigned long long timeout_ns,
+                               void* stream);
+
+/*
+ * Kernel timing hook for benchmarks. While enabled (on != 0), every call above
+ * records a pair of CUDA events on its stream immediately around its main kernel
+ * (prefill_kernel, decode_kernel, mla_kernel), so the time excludes the RoPE
+ * prologue, the merge and host work. attn_profile_collect() waits for the recorded
+ * events, returns the summed milliseconds and the number of pairs, and forgets
+ * them. Enabling creates the events once (host-side resources, no device memory).
+ * Not thread-safe; intended for a single benchmarking thread.
+ */
+int attn_profile_enable(int on);
+int attn_profile_collect(double* total_ms, int* count);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */

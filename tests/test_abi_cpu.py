@@ -1,0 +1,98 @@
+"""Host-only checks of the C ABI: the library loads, exports every function the
+header declares, and rejects bad arguments before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn_b200.h")
+
+
+def _declared():
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b([a-z_][a-z0-9_]*)\s*\(", txt)) - {"defined"})
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from attention_causal_gqa_b200.build import build
+    build()
+    from attention_causal_gqa_b200 import binding
+    return binding.lib
+
+
+def test_header_declares_the_three_entry_points():
+    names = _declared()
+    for n in ("attn_prefill", "attn_decode_paged", "mla_decode"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for n in _declared():
+        assert hasattr(lib, n), n
+
+
+FAKE = 1 << 20  # non-null, 256-byte aligned; never dereferenced because validation fails first
+
+
+def _err(lib):
+    return lib.attn_last_error().decode()
+
+
+def test_prefill_validation_codes(lib):
+    f = lib.attn_prefill
+    P = ctypes.c_void_p(FAKE)
+    assert f(None, P, P, P, P, 1, 4, 2, 64, 128, 1, 1e4, 0.0, 1, P, 1 << 30, None) == 1
+    assert "null" in _err(lib)
+    assert f(P, P, P, P, P, 1, 6, 4, 64, 128, 1, 1e4, 0.0, 1, P, 1 << 30, None) == 1  # Hq % Hkv
+    assert f(P, P, P, P, P, 0, 4, 2, 64, 128, 1, 1e4, 0.0, 1, P, 1 << 30, None) == 1  # B = 0
+    assert f(P, P, P, P, P, 1, 4, 2, 64, 96, 1, 1e4, 0.0, 1, P, 1 << 30, None) == 2   # D = 96
+    assert f(P, P, P, P, P, 1, 4, 2, 64, 128, 1, 1e4, 0.0, 0, P, 1 << 30, None) == 2  # fp32 with D = 128
+    assert f(P, P, P, P, P, 1, 4, 2, 64, 128, 1, 1e4, 0.0, 7, P, 1 << 30, None) == 2  # unknown dtype
+    need = lib.attn_prefill_workspace_size(1, 2, 64, 128, 1)
+    assert f(P, P, P, P, P, 1, 4, 2, 64, 128, 1, 1e4, 0.0, 1, P, need - 1, None) == 3
+    Q = ctypes.c_void_p(FAKE + 8)  # misaligned q
+    assert f(Q, P, P, P, P, 1, 4, 2, 64, 128, 1, 1e4, 0.0, 1, P, need, None) == 1
+
+
+def test_decode_validation_codes(lib):
+    f = lib.attn_decode_paged
+    P = ctypes.c_void_p(FAKE)
+    need = lib.attn_decode_paged_workspace_size(2, 32, 128, 64, 16)
+    args = lambda **kw: dict(dict(B=2, Hq=32, Hkv=8, D=128, ps=16, maxp=64, npg=100, dt=1, ws=need), **kw)
+
+    def call(**kw):
+        a = args(**kw)
+        return f(P, P, P, P, P, P, P, a["B"], a["Hq"], a["Hkv"], a["D"], a["ps"], a["maxp"], a["npg"], 0.0, a["dt"],
+                 P, a["ws"], None)
+    assert call(Hq=30) == 1
+    assert call(ps=32) == 2
+    assert call(D=256) == 2
+    assert call(Hkv=16, Hq=32) == 2
+    assert call(dt=0) == 2
+    assert call(ws=need - 1) == 3
+    assert call(npg=0) == 1
+    assert f(None, P, P, P, P, P, P, 2, 32, 8, 128, 16, 64, 100, 0.0, 1, P, need, None) == 1
+
+
+def test_mla_validation_codes(lib):
+    f = lib.mla_decode
+    P = ctypes.c_void_p(FAKE)
+    need = lib.mla_decode_workspace_size(2, 128, 512, 64, 4096)
+    assert f(P, P, P, P, P, 0.07, P, P, 2, 64, 512, 64, 4096, P, need, None) == 2   # H = 64
+    assert f(P, P, P, P, P, 0.07, P, P, 2, 128, 256, 64, 4096, P, need, None) == 2  # Dc = 256
+    assert f(P, P, P, P, P, 0.0, P, P, 2, 128, 512, 64, 4096, P, need, None) == 1   # scale
+    assert f(P, P, P, P, P, 0.07, P, P, 2, 128, 512, 64, 4096, P, need - 1, None) == 3
+    assert f(P, None, P, P, P, 0.07, P, P, 2, 128, 512, 64, 4096, P, need, None) == 1
+
+
+def test_workspace_sizes_grow_with_problem(lib):
+    a = lib.attn_prefill_workspace_size(1, 8, 4096, 128, 1)
+    b = lib.attn_prefill_workspace_size(2, 8, 4096, 128, 1)
+    assert b > a > 256
+    assert lib.mla_decode_workspace_size(32, 128, 512, 64, 32768) > lib.mla_decode_workspace_size(1, 128, 512, 64, 512)
+    assert lib.attn_selftest_wait_timeout(ctypes.c_void_p(FAKE), 100, 10 ** 6, None) == 3
+    assert lib.attn_selftest_wait_timeout(ctypes.c_void_p(FAKE), 256, 10, None) == 1

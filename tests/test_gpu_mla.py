@@ -1,0 +1,85 @@
+"""GPU parity: mla_decode (C-ABI via the binding) against the float64 oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import mla_decode_ref
+from tests.parity import check, to_np
+
+pytestmark = pytest.mark.gpu
+cuda = pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA GPU")
+SCALE = 1.0 / math.sqrt(192)
+
+
+def _run(d, scale=SCALE):
+    from attention_causal_gqa_b200 import mla_decode
+    out, lse = mla_decode(d["q_nope"], d["q_pe"], d["kv_cache"], d["pe_cache"], d["seq_lens"], scale)
+    torch.cuda.synchronize()
+    return out, lse
+
+
+def _oracle(d, pairs=None, scale=SCALE):
+    sl = d["seq_lens"].cpu().numpy()
+    if pairs is None:
+        return mla_decode_ref(to_np(d["q_nope"]), to_np(d["q_pe"]), to_np(d["kv_cache"]), to_np(d["pe_cache"]), sl,
+                              scale)
+    outs, lses, order = [], [], []
+    for b in sorted({b for b, _ in pairs}):
+        L = int(sl[b])
+        hs = [h for bb, h in pairs if bb == b]
+        o, l = mla_decode_ref(to_np(d["q_nope"][b:b + 1]), to_np(d["q_pe"][b:b + 1]),
+                              to_np(d["kv_cache"][b:b + 1, :L]), to_np(d["pe_cache"][b:b + 1, :L]),
+                              sl[b:b + 1], scale, pairs=[(0, h) for h in hs])
+        outs.append(o)
+        lses.append(l)
+        order += [(b, h) for h in hs]
+    return np.concatenate(outs), np.concatenate(lses), order
+
+
+@cuda
+@pytest.mark.parametrize("lens,T_max", [([1, 31, 32, 33], 64), ([600, 1500, 513, 511, 512], 1536),
+                                        ([2048, 100], 2048)])
+def test_mla_matches_oracle_small(lens, T_max):
+    from attention_causal_gqa_b200.synthetic import mla_inputs
+    d = mla_inputs(len(lens), 128, 512, 64, seq_lens=lens, T_max=T_max, seed=T_max + len(lens), device="cuda")
+    out, lse = _run(d)
+    ro, rl = _oracle(d)
+    check(out, ro, lse, rl, what=f"mla {lens}")
+
+
+@cuda
+def test_mla_empty_sequence_and_poison_past_length():
+    from attention_causal_gqa_b200.synthetic import mla_inputs
+    lens = [0, 45, 700]
+    d = mla_inputs(3, 128, 512, 64, seq_lens=lens, T_max=1024, seed=9, device="cuda")
+    ro, rl = _oracle(d)
+    for b, L in enumerate(lens):
+        d["kv_cache"][b, L:] = float("nan")
+        d["pe_cache"][b, L:] = float("inf")
+    out, lse = _run(d)
+    check(out, ro, lse, rl, what="mla poison")
+    assert torch.all(out[0] == 0) and torch.all(torch.isneginf(lse[0]))
+
+
+@cuda
+def test_mla_full_size_sampled():
+    from attention_causal_gqa_b200.synthetic import workload_inputs
+    d = workload_inputs("mla_decode_b32_h128_dc512_dr64", device="cuda")
+    out, lse = _run(d)
+    rng = np.random.default_rng(8)
+    pairs = sorted({(int(rng.integers(32)), int(rng.integers(128))) for _ in range(40)} | {(0, 0), (31, 127)})
+    ro, rl, order = _oracle(d, pairs)
+    idx = torch.tensor(order, device="cuda")
+    check(out[idx[:, 0], 0, idx[:, 1]], ro, lse[idx[:, 0], 0, idx[:, 1]], rl, what="mla full")
+    assert torch.isfinite(out).all() and torch.isfinite(lse).all()
+
+
+@cuda
+def test_mla_deterministic():
+    from attention_causal_gqa_b200.synthetic import mla_inputs
+    d = mla_inputs(2, 128, 512, 64, seq_lens=[3000, 777], T_max=3072, seed=1, device="cuda")
+    o1, l1 = _run(d)
+    o2, l2 = _run(d)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
