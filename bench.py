@@ -243,12 +243,153 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------- our arm
+def bench_prefill(args, world, dev, seed, flush, pk, pk_kind, fp):
+    import torch
+    from attention_causal_gqa_b200 import binding as B_
+    from attention_causal_gqa_b200.synthetic import WORKLOADS, workload_inputs
+    p = WORKLOADS[PREFILL].params
+    q, k, v = workload_inputs(PREFILL, seed=seed, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((p["B"], p["Hq"], p["S"]), dtype=torch.float32, device=dev)
+    ws = torch.empty(B_.prefill_workspace_size(p["B"], p["Hkv"], p["S"], p["D"]), dtype=torch.uint8, device=dev)
+
+    def step():
+        B_.attn_prefill(q, k, v, causal=True, rope_theta=p["theta"], scale=p["scale"], out=out, lse=lse,
+                        workspace=ws)
+
+    for _ in range(args.warmup):
+        flush()
+        step()
+    torch.cuda.synchronize()
+    B_.profile_collect()
+    ms = timed_region(step, args.steps, 0, world, flush=flush)
+    kern_ms, n_launch = B_.profile_collect()
+    flops = prefill_flops(p)
+    value = world * flops * args.steps / (ms * 1e-3) / 1e12
+    kern_avg = max_over_ranks(kern_ms / max(n_launch, 1), world)
+    achieved = flops / (kern_avg * 1e-3) / 1e12
+    roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": achieved / pk["bf16_tflops"], "traffic": traffic_for("prefill_kernel", fp),
+            "kernel": "prefill_kernel", "kernel_ms": kern_avg, "peak_kind": f"{pk_kind} dense bf16 (burst)",
+            "algorithmic": f"{flops:.4g} flop per launch = B*Hq*4*D*S(S+1)/2 (exact causal)"}
+    res = {"value": value, "ms": ms, "roofline": roof, "flops": flops, "p": p}
+    if not args.no_e2e:
+        # end to end through the public call: pinned host buffers, copies inside the timed region
+        qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
+        oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        lh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+        def step_e2e():
+            q.copy_(qh, non_blocking=True)
+            k.copy_(kh, non_blocking=True)
+            v.copy_(vh, non_blocking=True)
+            step()
+            oh.copy_(out, non_blocking=True)
+            lh.copy_(lse, non_blocking=True)
+
+        n = max(3, args.steps // 2)
+        ms_e2e = timed_region(step_e2e, n, 2, world)
+        B_.profile_collect()
+        res["e2e"] = {"value": world * flops * n / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+                      "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in (qh, kh, vh)),
+                      "d2h_bytes_per_step": oh.numel() * oh.element_size() + lh.numel() * lh.element_size()}
+    res["inputs"] = (q, k, v)
+    return res
+
+
+def bench_decode(args, world, dev, seed, pk, pk_kind, fp):
+    import torch
+    from attention_causal_gqa_b200 import binding as B_
+    from attention_causal_gqa_b200.synthetic import WORKLOADS, workload_inputs
+    dp = dict(WORKLOADS[DECODE].params)
+    if args.small:
+        from attention_causal_gqa_b200.synthetic import decode_inputs
+        dp["B"] = 8
+        d = decode_inputs(8, dp["Hq"], dp["Hkv"], dp["D"], dp["lmin"], dp["lmax"], dp["std"], seed, dev)
+    else:
+        d = workload_inputs(DECODE, seed=seed, device=dev)
+    out = torch.empty_like(d["q"])
+    lse = torch.empty((dp["B"], dp["Hq"]), dtype=torch.float32, device=dev)
+    ws = torch.empty(B_.decode_workspace_size(dp["B"], dp["Hq"], dp["D"], d["max_pages_per_seq"]),
+                     dtype=torch.uint8, device=dev)
+
+    def step():
+        B_.attn_decode_paged(d["q"], d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"],
+                             scale=dp["scale"], out=out, lse=lse, workspace=ws)
+
+    tokens = int(d["seq_lens"].sum().item())
+    kv_bytes = tokens * dp["Hkv"] * dp["D"] * 2 * 2
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    B_.profile_collect()
+    ms = timed_region(step, args.steps, 0, world)
+    k_ms, n = B_.profile_collect()
+    k_avg = max_over_ranks(k_ms / max(n, 1), world)
+    ach = kv_bytes / (k_avg * 1e-3) / 1e9
+    res = {"workload": DECODE + ("_small_b8" if args.small else ""), "value": world * kv_bytes * args.steps / (ms * 1e-3) / 1e9, "unit": "GB/s",
+           "ms_per_step": ms / args.steps, "kv_tokens": tokens, "kv_bytes_per_step": kv_bytes,
+           "gpu_launches": 2 * args.steps, "l2": "inputs (4.4 GB) larger than L2",
+           "roofline": {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                        "frac": ach / pk["hbm_gbs"], "traffic": traffic_for("decode_kernel", fp),
+                        "kernel": "decode_kernel", "kernel_ms": k_avg, "peak_kind": f"{pk_kind} HBM copy",
+                        "algorithmic": "4096 B per cached token (K+V, 8 heads x 128 x bf16)"}}
+    del d, out, lse, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_mla(args, world, dev, seed, pk, pk_kind, fp):
+    import torch
+    from attention_causal_gqa_b200 import binding as B_
+    from attention_causal_gqa_b200.synthetic import WORKLOADS, workload_inputs
+    mp = dict(WORKLOADS[MLA].params)
+    if args.small:
+        from attention_causal_gqa_b200.synthetic import mla_inputs
+        mp["B"] = 8
+        m = mla_inputs(8, mp["H"], mp["Dc"], mp["Dr"], mp["lmin"], mp["lmax"], mp["std"], seed, dev)
+    else:
+        m = workload_inputs(MLA, seed=seed, device=dev)
+    out = torch.empty_like(m["q_nope"])
+    lse = torch.empty((mp["B"], 1, mp["H"]), dtype=torch.float32, device=dev)
+    ws = torch.empty(B_.mla_workspace_size(mp["B"], mp["H"], mp["Dc"], mp["Dr"], m["T_max"]),
+                     dtype=torch.uint8, device=dev)
+
+    def step():
+        B_.mla_decode(m["q_nope"], m["q_pe"], m["kv_cache"], m["pe_cache"], m["seq_lens"], mp["scale"],
+                      out=out, lse=lse, workspace=ws)
+
+    tokens = int(m["seq_lens"].sum().item())
+    nbytes = tokens * (mp["Dc"] + mp["Dr"]) * 2
+    flops = tokens * mp["H"] * (2.0 * (mp["Dc"] + mp["Dr"]) + 2.0 * mp["Dc"])
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    B_.profile_collect()
+    ms = timed_region(step, args.steps, 0, world)
+    k_ms, n = B_.profile_collect()
+    k_avg = max_over_ranks(k_ms / max(n, 1), world)
+    ach = nbytes / (k_avg * 1e-3) / 1e9
+    res = {"workload": MLA + ("_small_b8" if args.small else ""), "value": world * nbytes * args.steps / (ms * 1e-3) / 1e9, "unit": "GB/s",
+           "ms_per_step": ms / args.steps, "kv_tokens": tokens, "kv_bytes_per_step": nbytes,
+           "tflops": world * flops * args.steps / (ms * 1e-3) / 1e12, "gpu_launches": 2 * args.steps,
+           "l2": "kv/pe caches (1.2 GB) larger than L2",
+           "roofline": {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                        "frac": ach / pk["hbm_gbs"], "traffic": traffic_for("mla_kernel", fp),
+                        "kernel": "mla_kernel", "kernel_ms": k_avg, "peak_kind": f"{pk_kind} HBM copy",
+                        "algorithmic": "1152 B per cached token (kv 512 + pe 64, bf16)",
+                        "tensor_tflops": flops / (k_avg * 1e-3) / 1e12,
+                        "tensor_frac": flops / (k_avg * 1e-3) / 1e12 / pk["bf16_tflops"]}}
+    del m, out, lse, ws
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args):
     import torch
     world, rank, local = dist_setup()
     from attention_causal_gqa_b200 import binding as B_
     from attention_causal_gqa_b200.build import _fingerprint
-    from attention_causal_gqa_b200.synthetic import WORKLOADS, workload_inputs
 
     pk, pk_kind = peaks()
     fp = _fingerprint()[:16]
@@ -259,147 +400,49 @@ def run_ours(args):
     def flush():
         flush_buf.zero_()
 
-    # ------------------------------------------------------------ prefill
-    p = WORKLOADS[PREFILL].params
-    q, k, v = workload_inputs(PREFILL, seed=seed, device=dev)
-    out = torch.empty_like(q)
-    lse = torch.empty((p["B"], p["Hq"], p["S"]), dtype=torch.float32, device=dev)
-    ws = torch.empty(B_.prefill_workspace_size(p["B"], p["Hkv"], p["S"], p["D"]), dtype=torch.uint8, device=dev)
+    def do(w):
+        return args.only is None or args.only == w
 
-    def step_prefill():
-        B_.attn_prefill(q, k, v, causal=True, rope_theta=p["theta"], scale=p["scale"], out=out, lse=lse,
-                        workspace=ws)
-
-    clocks = Clocks(local if world > 1 else int(os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0] or 0))
+    smi_index = local if world > 1 else int((os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0] or "0"))
+    clocks = Clocks(smi_index)
     B_.profile_enable(True)
     B_.profile_collect()
     clocks.start()
-    # warm-up is excluded from the kernel timing hook by collecting after it
-    for _ in range(args.warmup):
-        flush()
-        step_prefill()
-    torch.cuda.synchronize()
-    B_.profile_collect()
-    ms = timed_region(step_prefill, args.steps, 0, world, flush=flush)
-    kern_ms, n_launch = B_.profile_collect()
-    clk = clocks.stop()
-    flops = prefill_flops(p)
-    value = world * flops * args.steps / (ms * 1e-3) / 1e12
-    kern_avg = kern_ms / max(n_launch, 1)
-    kern_avg = max_over_ranks(kern_avg, world)
-    achieved = flops / (kern_avg * 1e-3) / 1e12
-    peak = pk["bf16_tflops"]
-    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-            "traffic": traffic_for("prefill_kernel", fp), "kernel": "prefill_kernel",
-            "peak_kind": f"{pk_kind} dense bf16 (burst)", "kernel_ms": kern_avg,
-            "algorithmic": f"{flops:.4g} flop per launch = B*Hq*4*D*S(S+1)/2"}
-
-    # e2e: host (pinned) buffers, copies inside the timed region
-    qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
-    oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    lh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-
-    def step_e2e():
-        q.copy_(qh, non_blocking=True)
-        k.copy_(kh, non_blocking=True)
-        v.copy_(vh, non_blocking=True)
-        step_prefill()
-        oh.copy_(out, non_blocking=True)
-        lh.copy_(lse, non_blocking=True)
-
-    e2e_steps = max(3, args.steps // 2)
-    ms_e2e = timed_region(step_e2e, e2e_steps, 2, world)
-    e2e_val = world * flops * e2e_steps / (ms_e2e * 1e-3) / 1e12
-    h2d = sum(x.numel() * x.element_size() for x in (qh, kh, vh))
-    d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
-    del qh, kh, vh, oh, lh
-
-    # ------------------------------------------------------------- decode
+    pre = bench_prefill(args, world, dev, seed, flush, pk, pk_kind, fp) if do("prefill") else None
     sub = {}
-    if not args.prefill_only:
-        dp = WORKLOADS[DECODE].params
-        d = workload_inputs(DECODE, seed=seed, device=dev)
-        dout = torch.empty_like(d["q"])
-        dlse = torch.empty((dp["B"], dp["Hq"]), dtype=torch.float32, device=dev)
-        dws = torch.empty(B_.decode_workspace_size(dp["B"], dp["Hq"], dp["D"], d["max_pages_per_seq"]),
-                          dtype=torch.uint8, device=dev)
-
-        def step_decode():
-            B_.attn_decode_paged(d["q"], d["k_pages"], d["v_pages"], d["block_table"], d["seq_lens"],
-                                 scale=dp["scale"], out=dout, lse=dlse, workspace=dws)
-
-        tokens = int(d["seq_lens"].sum().item())
-        kv_bytes = tokens * dp["Hkv"] * dp["D"] * 2 * 2
-        for _ in range(args.warmup):
-            step_decode()
-        torch.cuda.synchronize()
-        B_.profile_collect()
-        dms = timed_region(step_decode, args.steps, 0, world)
-        dk_ms, dn = B_.profile_collect()
-        dk_avg = max_over_ranks(dk_ms / max(dn, 1), world)
-        sub["decode"] = {
-            "workload": DECODE, "value": world * kv_bytes * args.steps / (dms * 1e-3) / 1e9, "unit": "GB/s",
-            "ms_per_step": dms / args.steps, "kv_tokens": tokens, "kv_bytes_per_step": kv_bytes,
-            "gpu_launches": 2 * args.steps,
-            "roofline": {"bound": "hbm", "achieved": kv_bytes / (dk_avg * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
-                         "unit": "GB/s", "frac": kv_bytes / (dk_avg * 1e-3) / 1e9 / pk["hbm_gbs"],
-                         "traffic": traffic_for("decode_kernel", fp), "kernel": "decode_kernel",
-                         "kernel_ms": dk_avg, "peak_kind": f"{pk_kind} HBM copy",
-                         "algorithmic": "4096 B per cached token (K+V, 8 heads x 128 x bf16)"}}
-        del d, dout, dlse, dws
-        torch.cuda.empty_cache()
-
-        # ------------------------------------------------------------ MLA
-        mp = WORKLOADS[MLA].params
-        m = workload_inputs(MLA, seed=seed, device=dev)
-        mout = torch.empty_like(m["q_nope"])
-        mlse = torch.empty((mp["B"], 1, mp["H"]), dtype=torch.float32, device=dev)
-        mws = torch.empty(B_.mla_workspace_size(mp["B"], mp["H"], mp["Dc"], mp["Dr"], m["T_max"]),
-                          dtype=torch.uint8, device=dev)
-
-        def step_mla():
-            B_.mla_decode(m["q_nope"], m["q_pe"], m["kv_cache"], m["pe_cache"], m["seq_lens"], mp["scale"],
-                          out=mout, lse=mlse, workspace=mws)
-
-        mtok = int(m["seq_lens"].sum().item())
-        mbytes = mtok * (mp["Dc"] + mp["Dr"]) * 2
-        mflops = mtok * mp["H"] * (2.0 * (mp["Dc"] + mp["Dr"]) + 2.0 * mp["Dc"])
-        for _ in range(args.warmup):
-            step_mla()
-        torch.cuda.synchronize()
-        B_.profile_collect()
-        mms = timed_region(step_mla, args.steps, 0, world)
-        mk_ms, mn = B_.profile_collect()
-        mk_avg = max_over_ranks(mk_ms / max(mn, 1), world)
-        sub["mla"] = {
-            "workload": MLA, "value": world * mbytes * args.steps / (mms * 1e-3) / 1e9, "unit": "GB/s",
-            "ms_per_step": mms / args.steps, "kv_tokens": mtok, "kv_bytes_per_step": mbytes,
-            "tflops": world * mflops * args.steps / (mms * 1e-3) / 1e12, "gpu_launches": 2 * args.steps,
-            "roofline": {"bound": "hbm", "achieved": mbytes / (mk_avg * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
-                         "unit": "GB/s", "frac": mbytes / (mk_avg * 1e-3) / 1e9 / pk["hbm_gbs"],
-                         "traffic": traffic_for("mla_kernel", fp), "kernel": "mla_kernel", "kernel_ms": mk_avg,
-                         "peak_kind": f"{pk_kind} HBM copy",
-                         "algorithmic": "1152 B per cached token (kv 512 + pe 64, bf16)",
-                         "tensor_frac": mflops / (mk_avg * 1e-3) / 1e12 / pk["bf16_tflops"]}}
-        del m, mout, mlse, mws
+    if do("decode"):
+        sub["decode"] = bench_decode(args, world, dev, seed, pk, pk_kind, fp)
+    if do("mla"):
+        sub["mla"] = bench_mla(args, world, dev, seed, pk, pk_kind, fp)
+    clk = clocks.stop()
     B_.profile_enable(False)
 
-    # -------------------------------------------------------- CPU baseline
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tf, heads, dt = oracle_prefill_sample(q, k, v, p, budget_s=args.cpu_budget)
+    if pre is not None and rank == 0 and world == 1 and not args.no_cpu_baseline:
+        q, k, v = pre["inputs"]
+        tf, heads, dt = oracle_prefill_sample(q, k, v, pre["p"], budget_s=args.cpu_budget)
         cpu = {"value": tf, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": f"{heads} whole heads (all {p['S']} causal rows each) of {PREFILL}, float64, {dt:.1f} s"}
-
-    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": PREFILL, "B": p["B"], "Hq": p["Hq"], "Hkv": p["Hkv"], "S": p["S"], "D": p["D"],
-                       "causal": True, "rope_theta": p["theta"], "l2": "flushed (256 MB write) between steps",
-                       "parallelism": f"replicas x{world}"},
-            "roofline": roof, "cpu_baseline": cpu,
-            "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": 3 * args.steps, "clocks": clk, "source_fingerprint": fp}
+               "sample": f"{heads} whole heads (all {pre['p']['S']} causal rows each) of {PREFILL}, "
+                         f"float64, {dt:.1f} s"}
+    if pre is not None:
+        p = pre["p"]
+        line = {"metric": METRIC, "value": pre["value"], "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": pre["ms"] / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": PREFILL, "B": p["B"], "Hq": p["Hq"], "Hkv": p["Hkv"], "S": p["S"],
+                           "D": p["D"], "causal": True, "rope_theta": p["theta"],
+                           "l2": "flushed (256 MB write) between steps", "parallelism": f"replicas x{world}"},
+                "roofline": pre["roofline"], "cpu_baseline": cpu, "e2e": pre.get("e2e"),
+                "gpu_launches": 3 * args.steps}
+    else:
+        w = sub[args.only]
+        line = {"metric": METRIC, "value": w["value"], "unit": w["unit"], "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": w["ms_per_step"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": w["workload"]}, "roofline": w["roofline"], "cpu_baseline": None,
+                "e2e": None, "gpu_launches": w["gpu_launches"]}
+    line["clocks"] = clk
+    line["source_fingerprint"] = fp
     line.update(sub)
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -416,7 +459,11 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--prefill-only", action="store_true")
+    ap.add_argument("--only", choices=["prefill", "decode", "mla"], default=None,
+                    help="run one workload (for profiling); the JSON line then carries that workload only")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--small", action="store_true",
+                    help="profiling case: decode and MLA with B=8 sequences (inputs still larger than L2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     args = ap.parse_args()
