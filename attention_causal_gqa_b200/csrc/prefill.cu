@@ -17,7 +17,11 @@
 // TMEM holds S_0, S_1 (BN fp32 columns each) and O_0, O_1 (D columns each).
 // Q is rotated (RoPE from the fp32 cos/sin table) by the softmax threads while
 // they stage it into shared memory; K arrives already rotated from the prologue
-// kernel. P goes back to shared memory as the A operand of O += P V.
+// kernel. P (16-bit) is written back into the columns of S_t and feeds O += P V
+// as the A operand straight from TMEM, so shared-memory bandwidth is spent on
+// Q, K and V only. Per tile the tensor pipe runs P_t V_j before Q_t K_{j+1}^T,
+// which both keeps P_t intact until it is consumed and guarantees that O_t is
+// final for step j when S_t(j+1) is reported ready.
 //
 // Operand precision (every shared-memory tile is 16-bit):
 //   kModeBF16   bf16 input, no RoPE: Q K^T and P V in bf16 (exact inputs).
@@ -49,9 +53,8 @@ struct PrefillShape {
   static constexpr int KV_BOX = BN * 128;
   static constexpr int KV_PART = BN * D * 2;
   static constexpr int KV_SLOT = NPART * KV_PART;
-  static constexpr int P_BOX = BM * 128;
-  static constexpr int P_PART = BM * BN * 2;
-  static constexpr int FIXED = 2 * NPART * Q_PART + 2 * NPART * P_PART;
+  static constexpr int P_COLS = BN / 2;      // TMEM columns of one 16-bit P part
+  static constexpr int FIXED = 2 * NPART * Q_PART;
   static constexpr int NST_RAW = (232448 - 1024 - 256 - FIXED) / KV_SLOT;
   static constexpr int NST = NST_RAW > 8 ? 8 : NST_RAW;
   static constexpr int SMEM_BYTES = 1024 /*align slack*/ + FIXED + NST * KV_SLOT + 256 /*barriers*/;
@@ -64,6 +67,7 @@ struct PrefillShape {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(TMEM_NEEDED <= 512, "TMEM budget");
   static_assert(D % 64 == 0 && BN % 64 == 0, "tiles are whole 128-byte swizzle rows");
+  static_assert(NPART * P_COLS <= BN, "P parts fit in the columns of S");
 };
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 domain: rescale O only when the max grows by > 2^8
@@ -141,8 +145,7 @@ __global__ void __launch_bounds__(320, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                           // [2 tiles][NP parts][Q_PART]
-  uint8_t* sP = sQ + 2 * NP * Sh::Q_PART;       // [2 tiles][NP parts][P_PART]
-  uint8_t* sKV = sP + 2 * NP * Sh::P_PART;      // [NST][NP parts][KV_PART]
+  uint8_t* sKV = sQ + 2 * NP * Sh::Q_PART;      // [NST][NP parts][KV_PART]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + Sh::NST * Sh::KV_SLOT);
   uint64_t* kv_full = bars;                     // [NST]
   uint64_t* kv_empty = bars + Sh::NST;          // [NST]
@@ -248,35 +251,39 @@ __global__ void __launch_bounds__(320, 1)
       constexpr int NPROD = Sh::SPLIT ? 3 : 1;
       const int n_kv[2] = {n_kv0, n_kv1};
       bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
+      // Descriptor words: the high word is shared by every operand; the low word
+      // carries the start address (>> 4), advanced by compile-time offsets below.
+      constexpr uint32_t HI = sdesc_hi_sw128(1024);
+      constexpr uint32_t LBO_K = 16;            // unused for K-major swizzled operands
+      const uint32_t q_lo = sdesc_lo(smem_u32(sQ), LBO_K);
+      const uint32_t kv_lo_k = sdesc_lo(smem_u32(sKV), LBO_K);
+      const uint32_t kv_lo_v = sdesc_lo(smem_u32(sKV), Sh::KV_BOX);  // MN-major V: LBO = 64-column block stride
       auto issue_qk = [&](int t, int slot) {
-        const uint32_t a0 = smem_u32(sQ + t * NP * Sh::Q_PART);
-        const uint32_t b0 = smem_u32(sKV + slot * Sh::KV_SLOT);
+        const uint32_t a0 = q_lo + ((t * NP * Sh::Q_PART) >> 4);
+        const uint32_t b0 = kv_lo_k + ((slot * Sh::KV_SLOT) >> 4);
         const uint32_t d = tmem_base + Sh::S_COL0 + t * BN;
 #pragma unroll
         for (int kb = 0; kb < D / 16; ++kb) {
-          const uint32_t koff = (kb >> 2) * 0u + (kb & 3) * 32u;  // 32-byte K step inside a 128-byte row
 #pragma unroll
           for (int x = 0; x < NPROD; ++x) {
             const int pa = x == 2 ? 1 : 0, pb = x == 1 ? 1 : 0;
-            const uint64_t ad = sdesc_sw128(a0 + pa * Sh::Q_PART + (kb >> 2) * Sh::Q_BOX + koff, 16, 1024);
-            const uint64_t bd = sdesc_sw128(b0 + pb * Sh::KV_PART + (kb >> 2) * Sh::KV_BOX + koff, 16, 1024);
-            umma_ss<false>(d, ad, bd, idesc_qk, (kb > 0 || x > 0) ? 1u : 0u);
+            const uint32_t ao = (pa * Sh::Q_PART + (kb >> 2) * Sh::Q_BOX + (kb & 3) * 32) >> 4;
+            const uint32_t bo = (pb * Sh::KV_PART + (kb >> 2) * Sh::KV_BOX + (kb & 3) * 32) >> 4;
+            umma_f16_lohi(d, a0 + ao, HI, b0 + bo, HI, idesc_qk, (kb > 0 || x > 0) ? 1u : 0u);
           }
         }
       };
       auto issue_pv = [&](int t, int slot, bool acc) {
-        const uint32_t a0 = smem_u32(sP + t * NP * Sh::P_PART);
-        const uint32_t b0 = smem_u32(sKV + slot * Sh::KV_SLOT);
+        const uint32_t a0 = tmem_base + Sh::S_COL0 + t * BN;  // P_t lives in the columns of S_t
+        const uint32_t b0 = kv_lo_v + ((slot * Sh::KV_SLOT) >> 4);
         const uint32_t d = tmem_base + Sh::O_COL0 + t * D;
 #pragma unroll
         for (int kb = 0; kb < BN / 16; ++kb) {
 #pragma unroll
           for (int x = 0; x < NPROD; ++x) {
             const int pa = x == 2 ? 1 : 0, pb = x == 1 ? 1 : 0;
-            const uint64_t ad =
-                sdesc_sw128(a0 + pa * Sh::P_PART + (kb >> 2) * Sh::P_BOX + (kb & 3) * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(b0 + pb * Sh::KV_PART + kb * 16 * 128, Sh::KV_BOX, 1024);
-            umma_ss<false>(d, ad, bd, idesc_pv, (acc || kb > 0 || x > 0) ? 1u : 0u);
+            const uint32_t bo = (pb * Sh::KV_PART + kb * 16 * 128) >> 4;
+            umma_f16_ts(d, a0 + pa * Sh::P_COLS + kb * 8, b0 + bo, HI, idesc_pv, (acc || kb > 0 || x > 0) ? 1u : 0u);
           }
         }
       };
@@ -301,6 +308,7 @@ __global__ void __launch_bounds__(320, 1)
             if (j >= n_kv[t]) continue;
             if (!mbar_wait(&p_full[t], j & 1, abort_flag, p.status)) { ok = false; break; }
             tc_fence_after();
+            // P_t V_j first: it reads P_t from the columns that Q_t K_{j+1}^T overwrites.
             issue_pv(t, sV, j > 0);
             umma_commit(&o_done[t]);
             if (j + 1 < n_kv[t]) {
@@ -340,7 +348,7 @@ __global__ void __launch_bounds__(320, 1)
       const TIn* qrow = reinterpret_cast<const TIn*>(p.q) + ((static_cast<size_t>(b) * p.Hq + h) * p.S + grow) * D;
       const float2* cs = p.rope_cs ? p.rope_cs + static_cast<size_t>(grow) * (D / 2) : nullptr;
       bool range_ok = true;
-#pragma unroll 2
+#pragma unroll 4
       for (int c = 0; c < D / 8; ++c) {
         float f[8];
         if (row_valid && n_kv > 0) {
@@ -383,42 +391,45 @@ __global__ void __launch_bounds__(320, 1)
     const float sl2 = p.scale_log2;
     const int limit = p.causal ? min(grow, p.S - 1) : p.S - 1;  // last key this row may see
     bool alive = true;
-    uint8_t* ptile = sP + t * NP * Sh::P_PART;
 
     for (int j = 0; j < n_kv && alive; ++j) {
       bool ok = mbar_wait(&s_full[t], j & 1, abort_flag, p.status);
       if (__any_sync(0xffffffffu, !ok)) { alive = false; break; }
       tc_fence_after();
-      // Pass 1: row max over the tile. The last KEEP 32-column chunks stay in
-      // registers; the others are read again from TMEM in pass 2 (S_t is not
-      // overwritten before this warpgroup arrives on p_full).
+      // The whole S row comes to registers with back-to-back TMEM loads and one wait.
       constexpr int NCH = BN / 32;
-      constexpr int KEEP = NCH > 2 ? 2 : NCH;
       const int thr = limit - j * BN;  // columns > thr are masked
-      float keep[KEEP * 32];
-      float mx = -INFINITY;
+      const bool need_mask = __any_sync(0xffffffffu, thr < BN - 1);  // diagonal or ragged tile
+      uint32_t sr[NCH][32];
 #pragma unroll
-      for (int c = 0; c < NCH; ++c) {
-        uint32_t r[32];
-        tmem_ld32(t_lane + Sh::S_COL0 + t * BN + c * 32, r);
-        tmem_ld_wait();
+      for (int c = 0; c < NCH; ++c) tmem_ld32(t_lane + Sh::S_COL0 + t * BN + c * 32, sr[c]);
+      tmem_ld_wait();
+      if (need_mask) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float x = (c * 32 + e > thr) ? -INFINITY : __uint_as_float(r[e]);
-          mx = fmaxf(mx, x);
-          if (c >= NCH - KEEP) keep[(c - (NCH - KEEP)) * 32 + e] = x;
-        }
+        for (int c = 0; c < NCH; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (c * 32 + e > thr) sr[c][e] = __float_as_uint(-INFINITY);
       }
+      float mxa = -INFINITY, mxb = -INFINITY, mxc = -INFINITY, mxd = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < NCH; ++c)
+#pragma unroll
+        for (int e = 0; e < 32; e += 8) {  // four independent max chains
+          mxa = fmax3f(mxa, __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
+          mxb = fmax3f(mxb, __uint_as_float(sr[c][e + 2]), __uint_as_float(sr[c][e + 3]));
+          mxc = fmax3f(mxc, __uint_as_float(sr[c][e + 4]), __uint_as_float(sr[c][e + 5]));
+          mxd = fmax3f(mxd, __uint_as_float(sr[c][e + 6]), __uint_as_float(sr[c][e + 7]));
+        }
+      const float mx = fmaxf(fmaxf(mxa, mxb), fmaxf(mxc, mxd));
       const float m_tile = mx * sl2;
       const float m_new = fmaxf(m_run, m_tile);
 
-      // PV(j-1) must be complete before P is overwritten and before O is rescaled.
+      // S_t(j) being ready implies P_t V_{j-1} has completed (same in-order tensor
+      // pipe, and the commit covers every earlier MMA), so O_t may be rescaled now.
       float alpha = 1.f;
       bool rescale = false;
       if (j > 0) {
-        ok = mbar_wait(&o_done[t], (j - 1) & 1, abort_flag, p.status);
-        if (__any_sync(0xffffffffu, !ok)) { alive = false; break; }
-        tc_fence_after();
         rescale = __any_sync(0xffffffffu, m_new > m_run + kRescaleThreshold);
         if (rescale) {
           alpha = ex2_approx(m_run - m_new);
@@ -429,43 +440,40 @@ __global__ void __launch_bounds__(320, 1)
         m_run = m_new;
       }
 
-      // Pass 2: P = exp2(s * scale * log2(e) - m), row sum, store swizzled (K-major) for P V.
-      const float neg_m = -m_run;
-      float lsum = 0.f;
+      // P = exp2(s * scale * log2(e) - m) as 16-bit pairs into the columns of S_t, and the row sum.
+      const float2 sl2x2 = make_float2(sl2, sl2);
+      const float2 nmx2 = make_float2(-m_run, -m_run);
+      const uint32_t p_col = t_lane + Sh::S_COL0 + t * BN;
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int c = 0; c < NCH; ++c) {
-        float x[32];
-        if (c < NCH - KEEP) {
-          uint32_t r[32];
-          tmem_ld32(t_lane + Sh::S_COL0 + t * BN + c * 32, r);
-          tmem_ld_wait();
+        uint32_t ph[16];
+        uint32_t pl[Sh::SPLIT ? 16 : 1];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) x[e] = (c * 32 + e > thr) ? -INFINITY : __uint_as_float(r[e]);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) x[e] = keep[(c - (NCH - KEEP)) * 32 + e];
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float f[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float pv = ex2_approx(fmaf(x[i * 8 + e], sl2, neg_m));
-            f[e] = pv;
-            lsum += pv;
-          }
-          const int gc = c * 4 + i;  // 16-byte chunk index within the row
-          const int off = (gc >> 3) * Sh::P_BOX + row * 128 + (((gc & 7) ^ (row & 7)) << 4);
+        for (int e = 0; e < 32; e += 4) {
+          const float2 z0 = ffma2(make_float2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])), sl2x2, nmx2);
+          const float2 z1 = ffma2(make_float2(__uint_as_float(sr[c][e + 2]), __uint_as_float(sr[c][e + 3])), sl2x2, nmx2);
+          const float2 p0 = make_float2(ex2_approx(z0.x), ex2_approx(z0.y));
+          const float2 p1 = make_float2(ex2_approx(z1.x), ex2_approx(z1.y));
+          acc[(e >> 1) & 3] = fadd2(acc[(e >> 1) & 3], p0);
+          acc[((e >> 1) + 1) & 3] = fadd2(acc[((e >> 1) + 1) & 3], p1);
           if constexpr (Sh::SPLIT) {
-            uint4 hi, lo;
-            split8(f, hi, lo);
-            *reinterpret_cast<uint4*>(ptile + off) = hi;
-            *reinterpret_cast<uint4*>(ptile + Sh::P_PART + off) = lo;
+            const float h0 = __bfloat162float(__float2bfloat16_rn(p0.x)), h1 = __bfloat162float(__float2bfloat16_rn(p0.y));
+            const float h2 = __bfloat162float(__float2bfloat16_rn(p1.x)), h3 = __bfloat162float(__float2bfloat16_rn(p1.y));
+            ph[e >> 1] = pack_bf16x2(h0, h1);
+            ph[(e >> 1) + 1] = pack_bf16x2(h2, h3);
+            pl[e >> 1] = pack_bf16x2(p0.x - h0, p0.y - h1);
+            pl[(e >> 1) + 1] = pack_bf16x2(p1.x - h2, p1.y - h3);
           } else {
-            *reinterpret_cast<uint4*>(ptile + off) = pack8<false>(f);
+            ph[e >> 1] = pack_bf16x2(p0.x, p0.y);
+            ph[(e >> 1) + 1] = pack_bf16x2(p1.x, p1.y);
           }
         }
+        tmem_st16(p_col + c * 16, ph);
+        if constexpr (Sh::SPLIT) tmem_st16(p_col + Sh::P_COLS + c * 16, pl);
       }
+      const float2 acc01 = fadd2(acc[0], acc[1]), acc23 = fadd2(acc[2], acc[3]);
+      const float lsum = (acc01.x + acc01.y) + (acc23.x + acc23.y);
       // O *= alpha (warp-uniform decision; exact because P and l use the same m)
       if (rescale) {
 #pragma unroll
@@ -478,10 +486,9 @@ __global__ void __launch_bounds__(320, 1)
           for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
           tmem_st32(ta, r);
         }
-        tmem_st_wait();
       }
+      tmem_st_wait();  // P (and a rescaled O) are in TMEM before the MMA may read them
       l_run += lsum;
-      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&p_full[t]);
     }
