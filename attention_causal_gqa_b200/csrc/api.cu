@@ -81,10 +81,6 @@ int clear_status(void* ws, cudaStream_t st) {
 int decode_splits(int max_pages) {
   return (max_pages + attn::kDecodePagesPerSplit - 1) / attn::kDecodePagesPerSplit;
 }
-int mla_splits(int T_max) {
-  const int tps = attn::kMlaTokensPerTile * attn::kMlaTilesPerSplit;
-  return (T_max + tps - 1) / tps;
-}
 
 // ----------------------------------------------------------- timing hook
 constexpr int kProfSlots = 4096;
@@ -310,12 +306,13 @@ int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, c
   return ok();
 }
 
+// MLA workspace: [status | partial outputs (n_pairs + B) x H x Dc fp32 | partial LSE (n_pairs + B) x H]
 size_t mla_decode_workspace_size(int B, int H, int Dc, int Dr, int T_max) {
   (void)Dr;
-  if (B <= 0 || H <= 0 || Dc <= 0 || T_max <= 0) return kHeader;
-  const size_t ns = mla_splits(T_max);
-  return kHeader + round_up(static_cast<size_t>(B) * ns * H * Dc * sizeof(float), 256) +
-         round_up(static_cast<size_t>(B) * ns * H * sizeof(float), 256);
+  (void)T_max;
+  if (B <= 0 || H <= 0 || Dc <= 0) return kHeader;
+  const size_t slots = static_cast<size_t>(attn::kMlaMaxPairs) + B;
+  return kHeader + round_up(slots * H * Dc * sizeof(float), 256) + round_up(slots * H * sizeof(float), 256);
 }
 
 int mla_decode(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
@@ -330,65 +327,51 @@ int mla_decode(const void* q_nope, const void* q_pe, const void* kv_cache, const
   if (!aligned(q_nope, 16) || !aligned(q_pe, 16) || !aligned(kv_cache, 16) || !aligned(pe_cache, 16) ||
       !aligned(out, 16) || !aligned(seq_lens, 4) || !aligned(lse, 4) || !aligned(workspace, 256))
     return fail(ATTN_ERR_INVALID_ARG, "misaligned pointer");
-  if (T_max > (1 << 26)) return fail(ATTN_ERR_UNSUPPORTED, "T_max too large");
+  if (T_max > (1 << 26) || B > (1 << 20)) return fail(ATTN_ERR_UNSUPPORTED, "problem too large");
   const size_t need = mla_decode_workspace_size(B, H, Dc, Dr, T_max);
   if (workspace_bytes < need)
     return fail(ATTN_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace_bytes, need);
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const int ns = mla_splits(T_max);
+  const size_t slots = static_cast<size_t>(attn::kMlaMaxPairs) + B;
   float* part_o = reinterpret_cast<float*>(ws + kHeader);
-  float* part_lse =
-      reinterpret_cast<float*>(ws + kHeader + round_up(static_cast<size_t>(B) * ns * H * Dc * sizeof(float), 256));
+  float* part_lse = reinterpret_cast<float*>(ws + kHeader + round_up(slots * H * Dc * sizeof(float), 256));
   int rc = clear_status(ws, st);
   if (rc) return rc;
 
-  CUtensorMap tmQn, tmQp, tmKV, tmPE;
-  {
-    const cuuint64_t d[3] = {static_cast<cuuint64_t>(Dc), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
-    const cuuint64_t s[2] = {static_cast<cuuint64_t>(Dc) * 2, static_cast<cuuint64_t>(H) * Dc * 2};
-    const cuuint32_t bx[3] = {64, 128, 1};
-    if ((rc = make_map(&tmQn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, q_nope, d, s, bx, "q_nope"))) return rc;
-  }
-  {
-    const cuuint64_t d[3] = {static_cast<cuuint64_t>(Dr), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
-    const cuuint64_t s[2] = {static_cast<cuuint64_t>(Dr) * 2, static_cast<cuuint64_t>(H) * Dr * 2};
-    const cuuint32_t bx[3] = {64, 128, 1};
-    if ((rc = make_map(&tmQp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, q_pe, d, s, bx, "q_pe"))) return rc;
-  }
+  CUtensorMap tmKV, tmPE;
   {
     const cuuint64_t d[3] = {static_cast<cuuint64_t>(Dc), static_cast<cuuint64_t>(T_max), static_cast<cuuint64_t>(B)};
     const cuuint64_t s[2] = {static_cast<cuuint64_t>(Dc) * 2, static_cast<cuuint64_t>(T_max) * Dc * 2};
-    const cuuint32_t bx[3] = {64, static_cast<cuuint32_t>(attn::kMlaTokensPerTile), 1};
+    const cuuint32_t bx[3] = {64, static_cast<cuuint32_t>(attn::kMlaTile), 1};
     if ((rc = make_map(&tmKV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, kv_cache, d, s, bx, "kv_cache"))) return rc;
   }
   {
     const cuuint64_t d[3] = {static_cast<cuuint64_t>(Dr), static_cast<cuuint64_t>(T_max), static_cast<cuuint64_t>(B)};
     const cuuint64_t s[2] = {static_cast<cuuint64_t>(Dr) * 2, static_cast<cuuint64_t>(T_max) * Dr * 2};
-    const cuuint32_t bx[3] = {64, static_cast<cuuint32_t>(attn::kMlaTokensPerTile), 1};
+    const cuuint32_t bx[3] = {64, static_cast<cuuint32_t>(attn::kMlaTile), 1};
     if ((rc = make_map(&tmPE, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, pe_cache, d, s, bx, "pe_cache"))) return rc;
   }
   attn::MlaParams p{};
+  p.q_nope = q_nope;
+  p.q_pe = q_pe;
   p.seq_lens = seq_lens;
   p.part_o = part_o;
   p.part_lse = part_lse;
-  p.out = out;
-  p.lse = lse;
   p.B = B;
   p.H = H;
   p.Dc = Dc;
   p.Dr = Dr;
   p.T_max = T_max;
-  p.n_splits = ns;
+  p.n_pairs = attn::mla_pairs_for_device();
   p.scale_log2 = scale * 1.4426950408889634f;
   p.status = reinterpret_cast<int*>(ws);
   prof_before(st);
-  cudaError_t e = attn::launch_mla(p, tmQn, tmQp, tmKV, tmPE, st);
+  cudaError_t e = attn::launch_mla(p, tmKV, tmPE, st);
   prof_after(st);
   if (e != cudaSuccess) return cuda_fail(e, "mla launch");
-  e = attn::launch_merge(part_o, part_lse, seq_lens, out, lse, B, H, Dc, ns,
-                         attn::kMlaTokensPerTile * attn::kMlaTilesPerSplit, st);
+  e = attn::launch_mla_merge(part_o, part_lse, seq_lens, out, lse, B, H, T_max, p.n_pairs, st);
   if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   return ok();
 }

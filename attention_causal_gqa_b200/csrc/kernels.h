@@ -54,21 +54,23 @@ cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmK, const C
                           cudaStream_t stream);
 
 // ------------------------------------------------------------------ MLA
-constexpr int kMlaTokensPerTile = 32;
-constexpr int kMlaTilesPerSplit = 16;  // 512 tokens per split
+constexpr int kMlaTile = 32;        // tokens per tile
+constexpr int kMlaMaxPairs = 74;    // two-CTA clusters in the persistent grid (148 SMs)
 
 struct MlaParams {
+  const void* q_nope;       // [B, 1, H, Dc] bf16
+  const void* q_pe;         // [B, 1, H, Dr] bf16
   const int32_t* seq_lens;  // [B]
-  float* part_o;            // [B, n_splits, H, Dc] fp32
-  float* part_lse;          // [B, n_splits, H]
-  void* out;                // [B, H, Dc] bf16
-  float* lse;               // [B, H]
-  int B, H, Dc, Dr, T_max, n_splits;
+  float* part_o;            // [n_pairs + B, H, Dc] fp32 (slot = cluster + sequence)
+  float* part_lse;          // [n_pairs + B, H]
+  int B, H, Dc, Dr, T_max, n_pairs;
   float scale_log2;
   int* status;
 };
-cudaError_t launch_mla(const MlaParams& p, const CUtensorMap& tmQn, const CUtensorMap& tmQp,
-                       const CUtensorMap& tmKV, const CUtensorMap& tmPE, cudaStream_t stream);
+int mla_pairs_for_device();
+cudaError_t launch_mla(const MlaParams& p, const CUtensorMap& tmKV, const CUtensorMap& tmPE, cudaStream_t stream);
+cudaError_t launch_mla_merge(const float* part_o, const float* part_lse, const int32_t* seq_lens, void* out,
+                             float* lse, int B, int H, int T_max, int n_pairs, cudaStream_t stream);
 
 // ------------------------------------------------------------- LSE merge
 // Combines n_valid(b) normalised partials per (b, head) into bf16 out and fp32 lse.

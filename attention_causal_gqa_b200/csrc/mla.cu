@@ -7,15 +7,27 @@
 // [q_nope | q_pe] . [kv_cache | pe_cache]^T ("attention study note", MLA
 // decoupled-RoPE section: the rotary part is concatenated to the content part).
 //
-// Work unit: one split of 512 cached tokens of one sequence and one half of the
-// 512 latent output columns (a CTA pair shares a split; each recomputes S, so
-// the output accumulator of 128 heads x 256 fp32 fits TMEM next to S).
-// Roles (192 threads):
-//   warps 0-3  softmax warpgroup, one thread per head; epilogue
-//   warp  4    TMA producer (Q once, then kv/pe tiles of TN tokens)
-//   warp  5    TMEM allocator and single-thread tcgen05.mma issuer
-// TMEM: S double buffer (2 x TN fp32 columns) and O (256 fp32 columns).
-// Q stays resident in shared memory (9 swizzled 128-byte column blocks).
+// Work split. A cluster of two CTAs (two SMs) shares every token tile and splits
+// the 576 reduction columns: rank 0 owns kv columns 0-255, rank 1 owns kv columns
+// 256-511 plus the 64 rotary columns. Each CTA
+//   * loads only its own columns of each kv/pe tile (no byte is loaded twice),
+//   * computes its partial score block S_r = Q_r . KV_r^T (Q_r kept in TMEM),
+//   * sends S_r to its peer through distributed shared memory and adds the
+//     peer's part (rank-0 part + rank-1 part in both CTAs: identical bits),
+//   * runs the online softmax on the full scores (both CTAs, same m and l),
+//   * accumulates O[:, its 256 columns] += P . KV[:, its 256 columns], with P
+//     written back into the TMEM columns of S and used as the MMA A operand.
+// Scheduling is persistent: the flattened sequence of 32-token tiles of all
+// sequences is cut into one contiguous range per cluster; each maximal piece of
+// a range inside one sequence (a segment) produces one normalised partial result
+// and its LSE, merged per sequence by mla_merge_kernel.
+//
+// Roles per CTA (192 threads): warps 0-3 softmax (one thread per head) and
+// epilogue; warp 4 TMA producer; warp 5 TMEM allocator and MMA issuer.
+// TMEM columns: O [0,256), Q_r [256, 416), S double buffer [416, 480), P double
+// buffer [480, 512). The score exchange is pipelined by one tile: in iteration k a
+// softmax thread sends its partial scores of tile k and then finishes tile k-1,
+// so the distributed-shared-memory latency overlaps a whole iteration.
 #include <cuda_bf16.h>
 
 #include "kernels.h"
@@ -25,81 +37,134 @@ namespace attn {
 
 namespace {
 
-constexpr int kMlaH = 128, kMlaDc = 512, kMlaDr = 64;
-constexpr int kMlaKB = (kMlaDc + kMlaDr) / 64;    // 9 column blocks of 64
-constexpr int kMlaQBox = 128 * 128;                // one 64-column block of Q: 16 KB
-constexpr int kMlaQBytes = kMlaKB * kMlaQBox;      // 147456
-constexpr int kMlaHalf = kMlaDc / 2;               // output columns per CTA
-constexpr int kMlaSplitTokens = kMlaTokensPerTile * kMlaTilesPerSplit;
+constexpr int kH = 128, kDc = 512, kDr = 64;
+constexpr int TN = kMlaTile;              // tokens per tile
+constexpr int KV_BOX = TN * 128;          // one 64-column block of a tile (TN rows of 128 bytes)
+constexpr int NST = 8;                    // kv ring depth
+constexpr int STAGE = 5 * KV_BOX;         // room for the larger (rank-1) share
+constexpr int XBUF = kH * TN * 4;         // one fp32 exchange buffer
+constexpr int O_COL = 0, Q_COL = 256, S_COL = 416, P_COL = 480;  // S: 2 x TN fp32, P: 2 x TN/2 bf16 pairs
+constexpr int TMEM_COLS = 512;
+constexpr int SMEM_BYTES = 1024 + NST * STAGE + 2 * XBUF + 256;
+static_assert(S_COL + 2 * TN <= P_COL && P_COL + TN <= TMEM_COLS, "TMEM budget");
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
-// SWIZZLE_NONE K-major descriptor: 8x16-byte core matrices, LBO along K, SBO along M/N.
-__device__ __forceinline__ uint64_t sdesc_interleave(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
-  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
-  d |= static_cast<uint64_t>(1) << 46;
-  return d;  // layout type 0
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t mapa_peer(uint32_t saddr, uint32_t peer) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(peer));
+  return r;
+}
+// Asynchronous 16-byte store into the peer's shared memory that completes bytes on
+// the peer's mbarrier (transaction count), so no per-store release is needed.
+__device__ __forceinline__ void st_async_v4(uint32_t addr, uint4 v, uint32_t bar_cluster_addr) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
+               "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(bar_cluster_addr)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait for a barrier that the peer CTA arrives on.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                  int* status) {
+  if (mbar_try_wait_acq_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait_acq_cluster(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > ATTN_WAIT_TIMEOUT_NS) {
+      *abort_flag = 1;
+      if (status) atomicOr(status, kDevErrTimeout);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-}  // namespace
+__device__ __forceinline__ int tiles_of(const int32_t* lens, int b, int T_max) {
+  const int L = min(max(__ldg(lens + b), 0), T_max);
+  return (L + TN - 1) / TN;
+}
 
-template <int TN, int NST>
-__global__ void __launch_bounds__(192, 1)
-    mla_kernel(const __grid_constant__ MlaParams p, const __grid_constant__ CUtensorMap tmQn,
-               const __grid_constant__ CUtensorMap tmQp, const __grid_constant__ CUtensorMap tmKV,
-               const __grid_constant__ CUtensorMap tmPE) {
-  constexpr int KV_BOX = TN * 128;             // one 64-column block of a kv/pe tile
-  constexpr int STAGE = kMlaKB * KV_BOX;
-  constexpr int P_BYTES = 128 * TN * 2;
-  constexpr int TMEM_COLS = 512;
-  constexpr int O_COL = 256;
-  static_assert(2 * TN <= O_COL, "S buffers fit below O");
-  static_assert(TN % 32 == 0, "one 32-column TMEM load per tile");
-
-  const int half = blockIdx.x & 1;
-  const int rest = blockIdx.x >> 1;
-  const int split = rest % p.n_splits;
-  const int b = rest / p.n_splits;
-  int L = __ldg(p.seq_lens + b);
-  if (L > p.T_max) {
-    if (threadIdx.x == 0) atomicOr(p.status, kDevErrBadLength);
-    L = p.T_max;
+// Calls fn(b, first_tile, end_tile, global_tile_offset_before) for every segment of
+// cluster `pair` in order. Every role enumerates the same segments.
+template <typename F>
+__device__ __forceinline__ void for_each_segment(const MlaParams& p, int pair, F&& fn) {
+  long long N = 0;
+  for (int b = 0; b < p.B; ++b) N += tiles_of(p.seq_lens, b, p.T_max);
+  const long long lo = N * pair / p.n_pairs, hi = N * (pair + 1) / p.n_pairs;
+  long long s = 0;
+  int done = 0;
+  for (int b = 0; b < p.B && s < hi; ++b) {
+    const int n = tiles_of(p.seq_lens, b, p.T_max);
+    const long long e = s + n;
+    const long long a0 = s > lo ? s : lo, a1 = e < hi ? e : hi;
+    if (a1 > a0) {
+      fn(b, static_cast<int>(a0 - s), static_cast<int>(a1 - s), done);
+      done += static_cast<int>(a1 - a0);
+    }
+    s = e;
   }
-  const int t0 = split * kMlaSplitTokens;
-  if (t0 >= L) return;  // uniform for the whole CTA
-  const int ntok = min(kMlaSplitTokens, L - t0);
-  const int n_tiles = (ntok + TN - 1) / TN;
+}
 
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sKV = sQ + kMlaQBytes;
-  uint8_t* sP = sKV + NST * STAGE;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + P_BYTES);
+template <int R>
+__device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* tmKV, const CUtensorMap* tmPE,
+                                         uint8_t* smem) {
+  constexpr int NKB = R == 0 ? 4 : 5;  // 64-column blocks of the score reduction owned by this CTA
+  constexpr int STAGE_BYTES = NKB * KV_BOX;
+  constexpr uint32_t PEER = 1 - R;
+  uint8_t* sKV = smem;
+  float* xbuf = reinterpret_cast<float*>(smem + NST * STAGE);  // [2][kH][TN], written by the peer
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NST * STAGE + 2 * XBUF);
   uint64_t* kv_full = bars;
-  uint64_t* kv_empty = bars + NST;
-  uint64_t* q_full = bars + 2 * NST;
-  uint64_t* s_full = q_full + 1;   // [2]
-  uint64_t* p_full = s_full + 2;
-  uint64_t* o_done = p_full + 1;
-  uint64_t* mma_done = o_done + 1;
+  uint64_t* kv_empty = kv_full + NST;
+  uint64_t* s_full = kv_empty + NST;  // [2] S(k) computed into S buffer k % 2
+  uint64_t* s_free = s_full + 2;      // [2] S(k) has been read by the softmax
+  uint64_t* p_full = s_free + 2;      // [2] P(k) written into P buffer k % 2
+  uint64_t* o_done = p_full + 2;      // [2] P(k) V(k) completed
+  uint64_t* x_full = o_done + 2;      // [2] the peer's partial scores of tile k landed in xbuf[k % 2]
+  uint64_t* x_empty = x_full + 2;     // [2] the peer has read what this CTA sent for tile k
+  uint64_t* q_ready = x_empty + 2;
+  uint64_t* mma_done = q_ready + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int pair = blockIdx.x >> 1;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NST; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
-    mbar_init(q_full, 1);
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
-    mbar_init(p_full, 128);
-    mbar_init(o_done, 1);
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(&s_full[u], 1);
+      mbar_init(&s_free[u], 128);
+      mbar_init(&p_full[u], 128);
+      mbar_init(&o_done[u], 1);
+      mbar_init(&x_full[u], 1);   // local expect_tx arrive + the peer's st.async bytes
+      mbar_init(&x_empty[u], 1);  // one remote arrive from the peer
+    }
+    mbar_init(q_ready, 128);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -111,208 +176,387 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  cluster_sync_all();  // the peer's barriers exist before any remote arrive
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 4) {
     // --------------------------------------------------------------- producer
     if (lane == 0) {
-      prefetch_tmap(&tmQn);
-      prefetch_tmap(&tmQp);
-      prefetch_tmap(&tmKV);
-      prefetch_tmap(&tmPE);
-      mbar_arrive_expect_tx(q_full, kMlaQBytes);
+      prefetch_tmap(tmKV);
+      if (R == 1) prefetch_tmap(tmPE);
+      int g = 0;
+      bool ok = true;
+      for_each_segment(p, pair, [&](int b, int t0, int t1, int) {
+        for (int t = t0; t < t1 && ok; ++t, ++g) {
+          const int s = g % NST;
+          if (!mbar_wait(&kv_empty[s], ((g / NST) & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
+          uint8_t* dst = sKV + s * STAGE;
+          mbar_arrive_expect_tx(&kv_full[s], STAGE_BYTES);
 #pragma unroll
-      for (int c = 0; c < kMlaDc / 64; ++c) tma_load_3d(sQ + c * kMlaQBox, &tmQn, q_full, c * 64, 0, b);
-      tma_load_3d(sQ + (kMlaDc / 64) * kMlaQBox, &tmQp, q_full, 0, 0, b);
-      for (int j = 0; j < n_tiles; ++j) {
-        const int s = j % NST;
-        if (!mbar_wait(&kv_empty[s], ((j / NST) & 1) ^ 1, abort_flag, p.status)) break;
-        uint8_t* dst = sKV + s * STAGE;
-        mbar_arrive_expect_tx(&kv_full[s], STAGE);
-        const int tok = t0 + j * TN;
-#pragma unroll
-        for (int c = 0; c < kMlaDc / 64; ++c) tma_load_3d(dst + c * KV_BOX, &tmKV, &kv_full[s], c * 64, tok, b);
-        tma_load_3d(dst + (kMlaDc / 64) * KV_BOX, &tmPE, &kv_full[s], 0, tok, b);
-      }
+          for (int c = 0; c < 4; ++c) tma_load_3d(dst + c * KV_BOX, tmKV, &kv_full[s], R * 256 + c * 64, t * TN, b);
+          if (R == 1) tma_load_3d(dst + 4 * KV_BOX, tmPE, &kv_full[s], 0, t * TN, b);
+        }
+      });
     }
   } else if (warp == 5) {
-    // ------------------------------------------------------------- MMA issuer
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_f32acc(1, 128, TN, false, false);
-      constexpr uint32_t idesc_o = idesc_f32acc(1, 128, kMlaHalf, false, true);
-      auto issue_s = [&](int j) {
-        const uint32_t a0 = smem_u32(sQ);
-        const uint32_t b0 = smem_u32(sKV + (j % NST) * STAGE);
-        const uint32_t d = tmem_base + (j & 1) * TN;
+      constexpr uint32_t idesc_o = idesc_f32acc(1, 128, 256, false, true);
+      constexpr uint32_t HI = sdesc_hi_sw128(1024);
+      const uint32_t kv_lo_k = sdesc_lo(smem_u32(sKV), 16);
+      const uint32_t kv_lo_v = sdesc_lo(smem_u32(sKV), KV_BOX);  // MN-major: 64-column blocks KV_BOX apart
+      auto issue_s = [&](int g) {
+        const uint32_t b0 = kv_lo_k + (((g % NST) * STAGE) >> 4);
+        const uint32_t d = tmem_base + S_COL + (g & 1) * TN;
 #pragma unroll
-        for (int kb = 0; kb < kMlaKB * 4; ++kb) {
-          const uint64_t ad = sdesc_sw128(a0 + (kb >> 2) * kMlaQBox + (kb & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(b0 + (kb >> 2) * KV_BOX + (kb & 3) * 32, 16, 1024);
-          umma_ss<false>(d, ad, bd, idesc_s, kb > 0 ? 1u : 0u);
-        }
+        for (int kb = 0; kb < NKB * 4; ++kb)
+          umma_f16_ts(d, tmem_base + Q_COL + kb * 8, b0 + (((kb >> 2) * KV_BOX + (kb & 3) * 32) >> 4), HI, idesc_s,
+                      kb > 0 ? 1u : 0u);
       };
-      auto issue_pv = [&](int j) {
-        const uint32_t a0 = smem_u32(sP);
-        const uint32_t b0 = smem_u32(sKV + (j % NST) * STAGE) + half * 4 * KV_BOX;
-        const uint32_t d = tmem_base + O_COL;
+      auto issue_pv = [&](int g, bool acc) {
+        const uint32_t b0 = kv_lo_v + (((g % NST) * STAGE) >> 4);
+        const uint32_t a0 = tmem_base + P_COL + (g & 1) * (TN / 2);
 #pragma unroll
-        for (int kb = 0; kb < TN / 16; ++kb) {
-          const uint64_t ad = sdesc_interleave(a0 + kb * 2 * 128, 128, TN * 16);
-          const uint64_t bd = sdesc_sw128(b0 + kb * 16 * 128, KV_BOX, 1024);
-          umma_ss<false>(d, ad, bd, idesc_o, (j > 0 || kb > 0) ? 1u : 0u);
-        }
+        for (int kb = 0; kb < TN / 16; ++kb)
+          umma_f16_ts(tmem_base + O_COL, a0 + kb * 8, b0 + ((kb * 16 * 128) >> 4), HI, idesc_o,
+                      (acc || kb > 0) ? 1u : 0u);
       };
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
-      for (int j = 0; ok && j < 2 && j < n_tiles; ++j) {
-        ok = mbar_wait(&kv_full[j % NST], (j / NST) & 1, abort_flag, p.status);
-        if (!ok) break;
+      bool ok = true;
+      int seg = 0;
+      auto s_step = [&](int g) -> bool {  // S(g) once its ring slot is loaded
+        if (!mbar_wait(&kv_full[g % NST], (g / NST) & 1, abort_flag, p.status)) return false;
         tc_fence_after();
-        issue_s(j);
-        umma_commit(&s_full[j & 1]);
-      }
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        if (!mbar_wait(p_full, j & 1, abort_flag, p.status)) break;
+        issue_s(g);
+        umma_commit(&s_full[g & 1]);
+        return true;
+      };
+      auto pv_step = [&](int g, bool acc) -> bool {  // P(g) V(g) once P(g) is in TMEM
+        if (!mbar_wait(&p_full[g & 1], (g >> 1) & 1, abort_flag, p.status)) return false;
         tc_fence_after();
-        issue_pv(j);
-        umma_commit(o_done);
-        umma_commit(&kv_empty[j % NST]);
-        const int jn = j + 2;
-        if (jn < n_tiles) {
-          if (!mbar_wait(&kv_full[jn % NST], (jn / NST) & 1, abort_flag, p.status)) break;
-          tc_fence_after();
-          issue_s(jn);
-          umma_commit(&s_full[jn & 1]);
+        issue_pv(g, acc);
+        umma_commit(&o_done[g & 1]);
+        umma_commit(&kv_empty[g % NST]);
+        return true;
+      };
+      for_each_segment(p, pair, [&](int, int t0, int t1, int g0) {
+        if (!ok) return;
+        const int n = t1 - t0;
+        if (!mbar_wait(q_ready, seg & 1, abort_flag, p.status)) { ok = false; return; }
+        ++seg;
+        tc_fence_after();
+        ok = s_step(g0) && (n < 2 || s_step(g0 + 1));
+        // The softmax, in its iteration k, reads S(k) and then produces P(k-1).
+        for (int i = 0; ok && i < n; ++i) {
+          const int k = g0 + i;
+          if (i + 2 < n) {
+            ok = mbar_wait(&s_free[k & 1], (k >> 1) & 1, abort_flag, p.status) && s_step(k + 2);
+            if (!ok) break;
+          }
+          if (i >= 1) ok = pv_step(k - 1, i > 1);
         }
-      }
+        if (ok) ok = pv_step(g0 + n - 1, n > 1);
+      });
       umma_commit(mma_done);
       mbar_wait(mma_done, 0, abort_flag, p.status);
     }
   } else {
-    // -------------------------------------------------------- softmax warpgroup
-    const int row = warp * 32 + lane;  // head
+    // ------------------------------------------------------ softmax warpgroup
+    const int h = warp * 32 + lane;  // head == TMEM lane
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
     const float sl2 = p.scale_log2;
-    float m_run = -INFINITY, l_run = 0.f;
+    const uint32_t peer_xbuf = mapa_peer(smem_u32(xbuf), PEER);
+    const uint32_t peer_xfull = mapa_peer(smem_u32(x_full), PEER);
+    const uint32_t peer_xempty = mapa_peer(smem_u32(x_empty), PEER);
     bool alive = true;
-    for (int j = 0; j < n_tiles && alive; ++j) {
-      bool ok = mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag, p.status);
-      if (__any_sync(0xffffffffu, !ok)) { alive = false; break; }
-      tc_fence_after();
-      float s[TN];
+    for_each_segment(p, pair, [&](int b, int t0, int t1, int g0) {
+      if (!alive) return;
+      // Q_r row of head h into TMEM (bf16 pairs are already in the operand layout).
+      {
+        const uint32_t* qn = reinterpret_cast<const uint32_t*>(
+            reinterpret_cast<const __nv_bfloat16*>(p.q_nope) + (static_cast<size_t>(b) * kH + h) * kDc + R * 256);
 #pragma unroll
-      for (int c = 0; c < TN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(t_lane + (j & 1) * TN + c * 32, r);
-        tmem_ld_wait();
+        for (int c = 0; c < 4; ++c) {  // 4 x 32 columns = 256 bf16
+          uint32_t r[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[e]);
+          for (int e = 0; e < 32; e += 4) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(qn + c * 32 + e));
+            r[e] = v.x; r[e + 1] = v.y; r[e + 2] = v.z; r[e + 3] = v.w;
+          }
+          tmem_st32(t_lane + Q_COL + c * 32, r);
+        }
+        if (R == 1) {
+          const uint32_t* qp = reinterpret_cast<const uint32_t*>(
+              reinterpret_cast<const __nv_bfloat16*>(p.q_pe) + (static_cast<size_t>(b) * kH + h) * kDr);
+          uint32_t r[32];
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(qp + e));
+            r[e] = v.x; r[e + 1] = v.y; r[e + 2] = v.z; r[e + 3] = v.w;
+          }
+          tmem_st32(t_lane + Q_COL + 128, r);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(q_ready);
       }
-      const int rem = ntok - j * TN;  // valid tokens in this tile
-      if (rem < TN) {
+      const int L = min(max(__ldg(p.seq_lens + b), 0), p.T_max);
+      const int n = t1 - t0;
+      float m_run = -INFINITY, l_run = 0.f;
+      uint32_t prev[TN];  // this CTA's partial scores of tile k-1
 #pragma unroll
-        for (int c = 0; c < TN; ++c)
-          if (c >= rem) s[c] = -INFINITY;
-      }
-      float mx = s[0];
+      for (int c = 0; c < TN; ++c) prev[c] = 0u;
+      for (int i = 0; i <= n; ++i) {
+        const int k = g0 + i;
+        uint32_t cur[TN];
+        if (i < n) {
+          // ---- tile k: read this CTA's partial scores and send them to the peer
+          const int u = k & 1;
+          bool ok = mbar_wait(&s_full[u], (k >> 1) & 1, abort_flag, p.status);
+          if (__any_sync(0xffffffffu, !ok)) { alive = false; return; }
+          tc_fence_after();
+          tmem_ld32(t_lane + S_COL + u * TN, cur);
+          tmem_ld_wait();
+          tc_fence_before();
+          mbar_arrive(&s_free[u]);
+          if (h == 0) mbar_arrive_expect_tx(&x_full[u], XBUF);  // arm for the peer's bytes of tile k
+          ok = mbar_wait_cluster(&x_empty[u], ((k >> 1) & 1) ^ 1, abort_flag, p.status);
+          if (__any_sync(0xffffffffu, !ok)) { alive = false; return; }
+          const uint32_t dst = peer_xbuf + (u * kH + h) * (TN * 4);
 #pragma unroll
-      for (int c = 1; c < TN; ++c) mx = fmaxf(mx, s[c]);
-      const float m_new = fmaxf(m_run, mx * sl2);
-      if (j > 0) {
-        ok = mbar_wait(o_done, (j - 1) & 1, abort_flag, p.status);
-        if (__any_sync(0xffffffffu, !ok)) { alive = false; break; }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, m_new > m_run + 8.0f)) {
-          const float alpha = ex2_approx(m_run - m_new);
-          m_run = m_new;
-          l_run *= alpha;
+          for (int c = 0; c < TN / 4; ++c)  // chunk c of the row is stored at slot (c + h) mod 8
+            st_async_v4(dst + ((c + h) & (TN / 4 - 1)) * 16,
+                        make_uint4(cur[4 * c], cur[4 * c + 1], cur[4 * c + 2], cur[4 * c + 3]), peer_xfull + u * 8);
+        }
+        if (i > 0) {
+          // ---- tile k-1: add the peer's part, online softmax, P into TMEM
+          const int kk = k - 1, uu = kk & 1, ii = i - 1;
+          bool ok = mbar_wait_cluster(&x_full[uu], (kk >> 1) & 1, abort_flag, p.status);
+          if (__any_sync(0xffffffffu, !ok)) { alive = false; return; }
+          float s[TN];
+          {
+            const float* src = xbuf + (uu * kH + h) * TN;
 #pragma unroll
-          for (int c = 0; c < kMlaHalf / 32; ++c) {
-            uint32_t r[32];
-            const uint32_t ta = t_lane + O_COL + c * 32;
-            tmem_ld32(ta, r);
-            tmem_ld_wait();
+            for (int c = 0; c < TN / 4; ++c) {
+              const float4 v = *reinterpret_cast<const float4*>(src + 4 * ((c + h) & (TN / 4 - 1)));
+              const float pv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            tmem_st32(ta, r);
+              for (int e = 0; e < 4; ++e) {
+                const float mv = __uint_as_float(prev[4 * c + e]);
+                s[4 * c + e] = R == 0 ? mv + pv[e] : pv[e] + mv;  // rank-0 part + rank-1 part in both CTAs
+              }
+            }
+          }
+          named_bar_sync(1, 128);  // every row of xbuf[uu] has been read
+          if (h == 0) mbar_arrive_remote(peer_xempty + uu * 8);
+          const int valid = L - (t0 + ii) * TN;  // tokens of this tile inside the sequence
+          if (valid < TN) {
+#pragma unroll
+            for (int c = 0; c < TN; ++c)
+              if (c >= valid) s[c] = -INFINITY;
+          }
+          float mx0 = fmax3f(s[0], s[1], s[2]), mx1 = fmax3f(s[3], s[4], s[5]);
+#pragma unroll
+          for (int c = 6; c + 3 < TN; c += 4) {
+            mx0 = fmax3f(mx0, s[c], s[c + 1]);
+            mx1 = fmax3f(mx1, s[c + 2], s[c + 3]);
+          }
+          mx0 = fmaxf(mx0, s[TN - 2]);
+          mx1 = fmaxf(mx1, s[TN - 1]);
+          const float m_new = fmaxf(m_run, fmaxf(mx0, mx1) * sl2);
+          if (ii > 0) {
+            if (__any_sync(0xffffffffu, m_new > m_run + 8.0f)) {
+              // O must hold P V of every earlier tile before it is scaled
+              ok = mbar_wait(&o_done[(kk - 1) & 1], ((kk - 1) >> 1) & 1, abort_flag, p.status);
+              if (__any_sync(0xffffffffu, !ok)) { alive = false; return; }
+              tc_fence_after();
+              const float alpha = ex2_approx(m_run - m_new);
+              m_run = m_new;
+              l_run *= alpha;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                uint32_t r[32];
+                tmem_ld32(t_lane + O_COL + c * 32, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                tmem_st32(t_lane + O_COL + c * 32, r);
+              }
+            }
+          } else {
+            m_run = m_new;
+          }
+          uint32_t pp[TN / 2];
+          float la = 0.f, lb = 0.f;
+#pragma unroll
+          for (int c = 0; c < TN; c += 2) {
+            const float a = ex2_approx(fmaf(s[c], sl2, -m_run));
+            const float bb = ex2_approx(fmaf(s[c + 1], sl2, -m_run));
+            la += a;
+            lb += bb;
+            pp[c / 2] = pack_bf16x2(a, bb);
+          }
+          l_run += la + lb;
+          if (ii >= 2) {  // P buffer uu last held P(kk-2)
+            ok = mbar_wait(&o_done[uu], ((kk - 2) >> 1) & 1, abort_flag, p.status);
+            if (__any_sync(0xffffffffu, !ok)) { alive = false; return; }
+            tc_fence_after();
+          }
+          tmem_st16(t_lane + P_COL + uu * (TN / 2), pp);
+          if (valid < TN) {
+            // cached rows past the sequence end may hold anything: zero this CTA's
+            // value columns for them so that 0 * garbage cannot reach O
+            uint8_t* st = sKV + (kk % NST) * STAGE;
+            const int nbad = TN - valid;
+            for (int idx = threadIdx.x; idx < 4 * nbad * 8; idx += 128) {
+              const int bx = idx / (nbad * 8), r = valid + (idx / 8) % nbad, ch = idx % 8;
+              *reinterpret_cast<uint4*>(st + bx * KV_BOX + r * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(1, 128);  // every zero row is written before any thread signals P
           }
           tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&p_full[uu]);
         }
-      } else {
-        m_run = m_new;
-      }
-      if (rem < TN) {
-        // cached rows past the sequence end may hold anything: zero this half's
-        // value columns for them so that 0 * garbage cannot reach O
-        uint8_t* st = sKV + (j % NST) * STAGE + half * 4 * KV_BOX;
-        const int nbad = TN - rem;
-        for (int idx = threadIdx.x; idx < 4 * nbad * 8; idx += 128) {
-          const int bx = idx / (nbad * 8), r = rem + (idx / 8) % nbad, ch = idx % 8;
-          *reinterpret_cast<uint4*>(st + bx * KV_BOX + r * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+        if (i < n) {
+#pragma unroll
+          for (int c = 0; c < TN; ++c) prev[c] = cur[c];
         }
       }
-      // P (bf16) in the SWIZZLE_NONE K-major layout: core matrix (row/8, key/8) at
-      // (row/8) * TN*16 + (key/8) * 128, rows 16 bytes apart inside it.
-      const float neg_m = -m_run;
-      float lsum = 0.f;
+      // segment epilogue: O / l for this CTA's 256 columns, and the LSE (rank 0).
+      // P V(g_last - 2) is known complete (waited before P(g_last) was written), so one
+      // wait on the last tile's barrier is exact.
+      const int g_last = g0 + n - 1;
+      bool ok = mbar_wait(&o_done[g_last & 1], (g_last >> 1) & 1, abort_flag, p.status);
+      if (__any_sync(0xffffffffu, !ok)) { alive = false; return; }
+      tc_fence_after();
+      const int slot = pair + b;
+      const float inv_l = 1.f / l_run;
+      float* orow = p.part_o + (static_cast<size_t>(slot) * kH + h) * kDc + R * 256;
 #pragma unroll
-      for (int c = 0; c < TN / 8; ++c) {
-        float f[8];
+      for (int c = 0; c < 8; ++c) {
+        uint32_t r[32];
+        tmem_ld32(t_lane + O_COL + c * 32, r);
+        tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          f[e] = ex2_approx(fmaf(s[c * 8 + e], sl2, neg_m));
-          lsum += f[e];
-        }
-        const uint4 v = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
-                                   pack_bf16x2(f[6], f[7]));
-        *reinterpret_cast<uint4*>(sP + (row >> 3) * (TN * 16) + c * 128 + (row & 7) * 16) = v;
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(orow + c * 32 + e) =
+              make_float4(__uint_as_float(r[e]) * inv_l, __uint_as_float(r[e + 1]) * inv_l,
+                          __uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
       }
-      l_run += lsum;
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(p_full);
-    }
-    if (alive) {
-      bool ok = mbar_wait(o_done, (n_tiles - 1) & 1, abort_flag, p.status);
-      if (!__any_sync(0xffffffffu, !ok)) {
-        tc_fence_after();
-        const float inv_l = 1.f / l_run;
-        float* orow = p.part_o + ((static_cast<size_t>(b) * p.n_splits + split) * kMlaH + row) * kMlaDc + half * kMlaHalf;
-#pragma unroll
-        for (int c = 0; c < kMlaHalf / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(t_lane + O_COL + c * 32, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(orow + c * 32 + e) =
-                make_float4(__uint_as_float(r[e]) * inv_l, __uint_as_float(r[e + 1]) * inv_l,
-                            __uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
-        }
-        if (half == 0)
-          p.part_lse[(static_cast<size_t>(b) * p.n_splits + split) * kMlaH + row] =
-              (m_run + log2f(l_run)) * 0.69314718055994531f;
-      }
-    }
+      if (R == 0) p.part_lse[static_cast<size_t>(slot) * kH + h] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+      tc_fence_before();  // O reads are complete before the next segment's MMAs overwrite O
+    });
   }
 
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // no remote access to this CTA's shared memory is still pending
   if (warp == 5) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
-cudaError_t launch_mla(const MlaParams& p, const CUtensorMap& tmQn, const CUtensorMap& tmQp,
-                       const CUtensorMap& tmKV, const CUtensorMap& tmPE, cudaStream_t stream) {
-  constexpr int TN = kMlaTokensPerTile, NST = 2;
-  constexpr int smem = 1024 + kMlaQBytes + NST * kMlaKB * TN * 128 + 128 * TN * 2 + 128;
-  static_assert(smem <= 232448, "shared memory budget");
-  auto kern = mla_kernel<TN, NST>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+}  // namespace
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+    mla_kernel(const __grid_constant__ MlaParams p, const __grid_constant__ CUtensorMap tmKV,
+               const __grid_constant__ CUtensorMap tmPE) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  if (cluster_ctarank() == 0)
+    mla_body<0>(p, &tmKV, &tmPE, smem);
+  else
+    mla_body<1>(p, &tmKV, &tmPE, smem);
+}
+
+int mla_pairs_for_device() {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int pairs = sms / 2;
+  return pairs < kMlaMaxPairs ? pairs : kMlaMaxPairs;
+}
+
+cudaError_t launch_mla(const MlaParams& p, const CUtensorMap& tmKV, const CUtensorMap& tmPE, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  const int grid = 2 * p.n_splits * p.B;
-  kern<<<grid, 192, smem, stream>>>(p, tmQn, tmQp, tmKV, tmPE);
+  mla_kernel<<<2 * p.n_pairs, 192, SMEM_BYTES, stream>>>(p, tmKV, tmPE);
+  return cudaGetLastError();
+}
+
+// One warp per (b, head): combine the partials of every cluster whose tile range meets
+// sequence b (slot = cluster + b), in cluster order.
+__global__ void mla_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
+                                 const int32_t* __restrict__ seq_lens, __nv_bfloat16* __restrict__ out,
+                                 float* __restrict__ lse, int B, int H, int T_max, int n_pairs) {
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (gw >= B * H) return;
+  const int b = gw / H, h = gw % H;
+  long long N = 0, s_b = 0;
+  for (int i = lane; i < B; i += 32) {
+    const int n = tiles_of(seq_lens, i, T_max);
+    N += n;
+    if (i < b) s_b += n;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    N += __shfl_xor_sync(0xffffffffu, N, o);
+    s_b += __shfl_xor_sync(0xffffffffu, s_b, o);
+  }
+  const long long e_b = s_b + tiles_of(seq_lens, b, T_max);
+  __nv_bfloat16* orow = out + static_cast<size_t>(gw) * kDc;
+  float M = -INFINITY;
+  for (int c = 0; c < n_pairs; ++c) {
+    const long long lo = N * c / n_pairs, hi = N * (c + 1) / n_pairs;
+    if (hi > s_b && lo < e_b && hi > lo) M = fmaxf(M, part_lse[static_cast<size_t>(c + b) * H + h]);
+  }
+  if (!(M > -INFINITY)) {
+    for (int d = lane * 8; d < kDc; d += 256) *reinterpret_cast<uint4*>(orow + d) = make_uint4(0, 0, 0, 0);
+    if (lane == 0) lse[gw] = -INFINITY;
+    return;
+  }
+  float acc[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+  float wsum = 0.f;
+  for (int c = 0; c < n_pairs; ++c) {
+    const long long lo = N * c / n_pairs, hi = N * (c + 1) / n_pairs;
+    if (!(hi > s_b && lo < e_b && hi > lo)) continue;
+    const size_t slot = static_cast<size_t>(c + b);
+    const float w = __expf(part_lse[slot * H + h] - M);
+    wsum += w;
+    const float* po = part_o + (slot * H + h) * kDc;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int d = lane * 8 + i * 256;
+      const float4 v0 = *reinterpret_cast<const float4*>(po + d);
+      const float4 v1 = *reinterpret_cast<const float4*>(po + d + 4);
+      acc[8 * i + 0] += w * v0.x; acc[8 * i + 1] += w * v0.y; acc[8 * i + 2] += w * v0.z; acc[8 * i + 3] += w * v0.w;
+      acc[8 * i + 4] += w * v1.x; acc[8 * i + 5] += w * v1.y; acc[8 * i + 6] += w * v1.z; acc[8 * i + 7] += w * v1.w;
+    }
+  }
+  const float inv = 1.f / wsum;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int d = lane * 8 + i * 256;
+    *reinterpret_cast<uint4*>(orow + d) =
+        make_uint4(pack_bf16x2(acc[8 * i] * inv, acc[8 * i + 1] * inv), pack_bf16x2(acc[8 * i + 2] * inv, acc[8 * i + 3] * inv),
+                   pack_bf16x2(acc[8 * i + 4] * inv, acc[8 * i + 5] * inv), pack_bf16x2(acc[8 * i + 6] * inv, acc[8 * i + 7] * inv));
+  }
+  if (lane == 0) lse[gw] = M + logf(wsum);
+}
+
+cudaError_t launch_mla_merge(const float* part_o, const float* part_lse, const int32_t* seq_lens, void* out,
+                             float* lse, int B, int H, int T_max, int n_pairs, cudaStream_t stream) {
+  const long long warps = static_cast<long long>(B) * H;
+  const int threads = 256;
+  const long long blocks = (warps * 32 + threads - 1) / threads;
+  mla_merge_kernel<<<static_cast<int>(blocks), threads, 0, stream>>>(
+      part_o, part_lse, seq_lens, static_cast<__nv_bfloat16*>(out), lse, B, H, T_max, n_pairs);
   return cudaGetLastError();
 }
 
