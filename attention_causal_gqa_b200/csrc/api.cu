@@ -104,6 +104,8 @@ void prof_after(cudaStream_t st) {
 }  // namespace
 
 namespace attn {
+void set_last_error(const char* msg) { g_last_error = msg; }
+
 __global__ void selftest_wait_kernel(int* status, unsigned long long timeout_ns) {
   __shared__ uint64_t bar;
   if (threadIdx.x == 0) {

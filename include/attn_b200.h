@@ -114,6 +114,31 @@ int mla_decode(const void* q_nope, const void* q_pe, const void* kv_cache, const
                const int32_t* seq_lens, float scale, void* out, float* lse, int B, int H, int Dc, int Dr, int T_max,
                void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * Paged decode for callers that cannot allocate device memory (code running
+ * inside another framework's memory pool with allocation disabled, paths where
+ * cudaMalloc's implicit synchronisation is not allowed, embedders that only pass
+ * buffers they already own). Same arguments, layouts and results as
+ * attn_decode_paged, minus the workspace: the split partials and the status
+ * word live in one file-scope device array of ATTN_DECODE_NOALLOC_MAX_BYTES,
+ * created when the library is loaded and held by every GPU that loads it until
+ * the process exits. The call allocates nothing.
+ *  - Problems whose attn_decode_paged_workspace_size() exceeds the array are
+ *    rejected with ATTN_ERR_WORKSPACE and a message naming both sizes.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call before
+ *    any stream capture.
+ *  - Every call on a device shares the one array and leaves its contents behind;
+ *    calls whose GPU work overlaps (different streams, or host threads) race on it
+ *    and must be serialised by the caller.
+ * There is no counterpart on the method's pages: it exists for these callers only.
+ */
+#define ATTN_DECODE_NOALLOC_MAX_BYTES (32ull << 20)
+int attn_decode_paged_noalloc(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
+                              const int32_t* seq_lens, void* out, float* lse, int B, int Hq, int Hkv, int D,
+                              int page_size, int max_pages_per_seq, int num_pages, float scale, int dtype,
+                              void* stream);
+
 /* Thread-local description of the last error returned on this thread ("" if none). */
 const char* attn_last_error(void);
 
