@@ -132,17 +132,25 @@ def barrier(world):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The slowest rank's value (device times are combined by MAX, never by wall clock)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank runs its own replica of the workload: same shapes, its own seeded values."""
+    return 20261202 + 1000 * rank
 
 
 def timed_region(fn, steps, warmup, world, flush=None):
@@ -394,7 +402,7 @@ def run_ours(args):
     pk, pk_kind = peaks()
     fp = _fingerprint()[:16]
     dev = torch.device("cuda", local if world > 1 else 0)
-    seed = 20261202 + 1000 * rank
+    seed = rank_seed(rank)
     flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
 
     def flush():
