@@ -22,12 +22,15 @@
 // a range inside one sequence (a segment) produces one normalised partial result
 // and its LSE, merged per sequence by mla_merge_kernel.
 //
-// Roles per CTA (192 threads): warps 0-3 softmax (one thread per head) and
-// epilogue; warp 4 TMA producer; warp 5 TMEM allocator and MMA issuer.
+// Roles per CTA (320 threads): warps 0-3 read each partial score tile out of TMEM,
+// keep a copy in shared memory and send one to the peer; warps 4-7 combine the two
+// parts, run the online softmax, write P, and do the Q loads and epilogues (one
+// thread per head in both groups); warp 8 TMA producer; warp 9 TMEM allocator and
+// MMA issuer. The two groups overlap consecutive tiles.
 // TMEM columns: O [0,256), Q_r [256, 416), S double buffer [416, 480), P double
-// buffer [480, 512). The score exchange is pipelined by one tile: in iteration k a
-// softmax thread sends its partial scores of tile k and then finishes tile k-1,
-// so the distributed-shared-memory latency overlaps a whole iteration.
+// buffer [480, 512). Partial scores leave TMEM as soon as they are computed, so
+// the next score tile can start while the exchange and the softmax of this one
+// are still in flight.
 #include <cuda_bf16.h>
 
 #include "kernels.h"
@@ -40,12 +43,13 @@ namespace {
 constexpr int kH = 128, kDc = 512, kDr = 64;
 constexpr int TN = kMlaTile;              // tokens per tile
 constexpr int KV_BOX = TN * 128;          // one 64-column block of a tile (TN rows of 128 bytes)
-constexpr int NST = 8;                    // kv ring depth
+constexpr int NST = 6;                    // kv ring depth
+constexpr int NX = 2;                     // exchange buffers (tiles in flight between the roles)
 constexpr int STAGE = 5 * KV_BOX;         // room for the larger (rank-1) share
 constexpr int XBUF = kH * TN * 4;         // one fp32 exchange buffer
 constexpr int O_COL = 0, Q_COL = 256, S_COL = 416, P_COL = 480;  // S: 2 x TN fp32, P: 2 x TN/2 bf16 pairs
 constexpr int TMEM_COLS = 512;
-constexpr int SMEM_BYTES = 1024 + NST * STAGE + 2 * XBUF + 256;
+constexpr int SMEM_BYTES = 1024 + NST * STAGE + 2 * NX * XBUF + 512;
 static_assert(S_COL + 2 * TN <= P_COL && P_COL + TN <= TMEM_COLS, "TMEM budget");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
@@ -125,24 +129,28 @@ __device__ __forceinline__ void for_each_segment(const MlaParams& p, int pair, F
   }
 }
 
-template <int R>
+// One body for both ranks (a runtime rank keeps the code small enough for the
+// instruction cache; both ranks differ only in loop bounds and column offsets).
 __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* tmKV, const CUtensorMap* tmPE,
-                                         uint8_t* smem) {
-  constexpr int NKB = R == 0 ? 4 : 5;  // 64-column blocks of the score reduction owned by this CTA
-  constexpr int STAGE_BYTES = NKB * KV_BOX;
-  constexpr uint32_t PEER = 1 - R;
+                                         uint8_t* smem, const int R) {
+  const int NKB = R == 0 ? 4 : 5;  // 64-column blocks of the score reduction owned by this CTA
+  const int STAGE_BYTES = NKB * KV_BOX;
+  const uint32_t PEER = 1 - R;
   uint8_t* sKV = smem;
-  float* xbuf = reinterpret_cast<float*>(smem + NST * STAGE);  // [2][kH][TN], written by the peer
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NST * STAGE + 2 * XBUF);
+  float* xbuf = reinterpret_cast<float*>(smem + NST * STAGE);             // [NX][kH][TN] from the peer
+  float* mybuf = reinterpret_cast<float*>(smem + NST * STAGE + NX * XBUF);  // [NX][kH][TN] own partials
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NST * STAGE + 2 * NX * XBUF);
   uint64_t* kv_full = bars;
   uint64_t* kv_empty = kv_full + NST;
-  uint64_t* s_full = kv_empty + NST;  // [2] S(k) computed into S buffer k % 2
-  uint64_t* s_free = s_full + 2;      // [2] S(k) has been read by the softmax
-  uint64_t* p_full = s_free + 2;      // [2] P(k) written into P buffer k % 2
-  uint64_t* o_done = p_full + 2;      // [2] P(k) V(k) completed
-  uint64_t* x_full = o_done + 2;      // [2] the peer's partial scores of tile k landed in xbuf[k % 2]
-  uint64_t* x_empty = x_full + 2;     // [2] the peer has read what this CTA sent for tile k
-  uint64_t* q_ready = x_empty + 2;
+  uint64_t* s_full = kv_empty + NST;   // [2] S(k) computed into S buffer k % 2
+  uint64_t* s_free = s_full + 2;       // [2] S(k) has been read out of TMEM
+  uint64_t* p_full = s_free + 2;       // [2] P(k) written into P buffer k % 2
+  uint64_t* o_done = p_full + 2;       // [2] P(k) V(k) completed
+  uint64_t* x_full = o_done + 2;       // [NX] the peer's partial scores of tile k landed in xbuf[k % NX]
+  uint64_t* x_empty = x_full + NX;     // [NX] the peer has consumed what this CTA sent for tile k
+  uint64_t* my_full = x_empty + NX;    // [NX] own partial scores of tile k are in mybuf[k % NX]
+  uint64_t* my_empty = my_full + NX;   // [NX] the softmax has consumed mybuf[k % NX]
+  uint64_t* q_ready = my_empty + NX;
   uint64_t* mma_done = q_ready + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -161,25 +169,31 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
       mbar_init(&s_free[u], 128);
       mbar_init(&p_full[u], 128);
       mbar_init(&o_done[u], 1);
-      mbar_init(&x_full[u], 1);   // local expect_tx arrive + the peer's st.async bytes
+    }
+    for (int u = 0; u < NX; ++u) {
+      mbar_init(&x_full[u], 1);   // one expect_tx arrive per phase + the peer's st.async bytes
       mbar_init(&x_empty[u], 1);  // one remote arrive from the peer
+      mbar_init(&my_full[u], 128);
+      mbar_init(&my_empty[u], 128);
     }
     mbar_init(q_ready, 128);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
+    // arm the receive buffers for the first NX tiles
+    for (int u = 0; u < NX; ++u) mbar_arrive_expect_tx(&x_full[u], XBUF);
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  cluster_sync_all();  // the peer's barriers exist before any remote arrive
+  cluster_sync_all();  // the peer's barriers exist (and are armed) before any remote access
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // --------------------------------------------------------------- producer
     if (lane == 0) {
       prefetch_tmap(tmKV);
@@ -198,7 +212,7 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
         }
       });
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_f32acc(1, 128, TN, false, false);
@@ -209,10 +223,12 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
       auto issue_s = [&](int g) {
         const uint32_t b0 = kv_lo_k + (((g % NST) * STAGE) >> 4);
         const uint32_t d = tmem_base + S_COL + (g & 1) * TN;
+#pragma unroll 1
+        for (int bx = 0; bx < NKB; ++bx)
 #pragma unroll
-        for (int kb = 0; kb < NKB * 4; ++kb)
-          umma_f16_ts(d, tmem_base + Q_COL + kb * 8, b0 + (((kb >> 2) * KV_BOX + (kb & 3) * 32) >> 4), HI, idesc_s,
-                      kb > 0 ? 1u : 0u);
+          for (int kq = 0; kq < 4; ++kq)
+            umma_f16_ts(d, tmem_base + Q_COL + (bx * 4 + kq) * 8, b0 + ((bx * KV_BOX + kq * 32) >> 4), HI, idesc_s,
+                        (bx > 0 || kq > 0) ? 1u : 0u);
       };
       auto issue_pv = [&](int g, bool acc) {
         const uint32_t b0 = kv_lo_v + (((g % NST) * STAGE) >> 4);
@@ -246,27 +262,65 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
         ++seg;
         tc_fence_after();
         ok = s_step(g0) && (n < 2 || s_step(g0 + 1));
-        // The softmax, in its iteration k, reads S(k) and then produces P(k-1).
+        // S(k+2) goes as soon as S(k) has been read out; P(k) V(k) as soon as P(k) is in TMEM.
         for (int i = 0; ok && i < n; ++i) {
           const int k = g0 + i;
           if (i + 2 < n) {
             ok = mbar_wait(&s_free[k & 1], (k >> 1) & 1, abort_flag, p.status) && s_step(k + 2);
             if (!ok) break;
           }
-          if (i >= 1) ok = pv_step(k - 1, i > 1);
+          ok = pv_step(k, i > 0);
         }
-        if (ok) ok = pv_step(g0 + n - 1, n > 1);
       });
       umma_commit(mma_done);
       mbar_wait(mma_done, 0, abort_flag, p.status);
     }
-  } else {
-    // ------------------------------------------------------ softmax warpgroup
+  } else if (warp < 4) {
+    // ----------------------------------------- exchange warpgroup (WG0): S out of TMEM
     const int h = warp * 32 + lane;  // head == TMEM lane
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
-    const float sl2 = p.scale_log2;
     const uint32_t peer_xbuf = mapa_peer(smem_u32(xbuf), PEER);
     const uint32_t peer_xfull = mapa_peer(smem_u32(x_full), PEER);
+    bool alive = true;
+    for_each_segment(p, pair, [&](int, int t0, int t1, int g0) {
+      for (int i = 0; alive && i < t1 - t0; ++i) {
+        const int k = g0 + i;
+        const int u = k & 1, bx = k % NX;
+        const uint32_t ph = (k / NX) & 1;
+        bool ok = mbar_wait(&s_full[u], (k >> 1) & 1, abort_flag, p.status);
+        if (__any_sync(0xffffffffu, !ok)) { alive = false; return; }
+        tc_fence_after();
+        uint32_t cur[TN];
+        tmem_ld32(t_lane + S_COL + u * TN, cur);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&s_free[u]);
+        // own copy for the softmax warpgroup (chunk c of a row at slot (c + h) mod 8)
+        ok = mbar_wait(&my_empty[bx], ph ^ 1, abort_flag, p.status);
+        if (__any_sync(0xffffffffu, !ok)) { alive = false; return; }
+        float* mine = mybuf + (bx * kH + h) * TN;
+#pragma unroll
+        for (int c = 0; c < TN / 4; ++c)
+          *reinterpret_cast<uint4*>(mine + 4 * ((c + h) & (TN / 4 - 1))) =
+              make_uint4(cur[4 * c], cur[4 * c + 1], cur[4 * c + 2], cur[4 * c + 3]);
+        mbar_arrive(&my_full[bx]);
+        // the peer's copy
+        ok = mbar_wait_cluster(&x_empty[bx], ph ^ 1, abort_flag, p.status);
+        if (__any_sync(0xffffffffu, !ok)) { alive = false; return; }
+        const uint32_t dst = peer_xbuf + (bx * kH + h) * (TN * 4);
+#pragma unroll
+        for (int c = 0; c < TN / 4; ++c)
+          st_async_v4(dst + ((c + h) & (TN / 4 - 1)) * 16,
+                      make_uint4(cur[4 * c], cur[4 * c + 1], cur[4 * c + 2], cur[4 * c + 3]), peer_xfull + bx * 8);
+      }
+    });
+  } else {
+    // ------------------------------------ softmax warpgroup (WG1): scores -> P, epilogue
+    const int wq = warp - 4;
+    const int h = wq * 32 + lane;  // head == TMEM lane
+    const int th = threadIdx.x - 128;
+    const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(wq * 32) << 16);
+    const float sl2 = p.scale_log2;
     const uint32_t peer_xempty = mapa_peer(smem_u32(x_empty), PEER);
     bool alive = true;
     for_each_segment(p, pair, [&](int b, int t0, int t1, int g0) {
@@ -275,7 +329,7 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
       {
         const uint32_t* qn = reinterpret_cast<const uint32_t*>(
             reinterpret_cast<const __nv_bfloat16*>(p.q_nope) + (static_cast<size_t>(b) * kH + h) * kDc + R * 256);
-#pragma unroll
+#pragma unroll 1
         for (int c = 0; c < 4; ++c) {  // 4 x 32 columns = 256 bf16
           uint32_t r[32];
 #pragma unroll
@@ -303,138 +357,120 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
       const int L = min(max(__ldg(p.seq_lens + b), 0), p.T_max);
       const int n = t1 - t0;
       float m_run = -INFINITY, l_run = 0.f;
-      uint32_t prev[TN];  // this CTA's partial scores of tile k-1
-#pragma unroll
-      for (int c = 0; c < TN; ++c) prev[c] = 0u;
-      for (int i = 0; i <= n; ++i) {
+      for (int i = 0; i < n; ++i) {
         const int k = g0 + i;
-        uint32_t cur[TN];
-        if (i < n) {
-          // ---- tile k: read this CTA's partial scores and send them to the peer
-          const int u = k & 1;
-          bool ok = mbar_wait(&s_full[u], (k >> 1) & 1, abort_flag, p.status);
-          if (__any_sync(0xffffffffu, !ok)) { alive = false; return; }
-          tc_fence_after();
-          tmem_ld32(t_lane + S_COL + u * TN, cur);
-          tmem_ld_wait();
-          tc_fence_before();
-          mbar_arrive(&s_free[u]);
-          if (h == 0) mbar_arrive_expect_tx(&x_full[u], XBUF);  // arm for the peer's bytes of tile k
-          ok = mbar_wait_cluster(&x_empty[u], ((k >> 1) & 1) ^ 1, abort_flag, p.status);
-          if (__any_sync(0xffffffffu, !ok)) { alive = false; return; }
-          const uint32_t dst = peer_xbuf + (u * kH + h) * (TN * 4);
+        const int u = k & 1, bx = k % NX;
+        const uint32_t ph = (k / NX) & 1;
+        bool ok = mbar_wait(&my_full[bx], ph, abort_flag, p.status);
+        ok = ok && mbar_wait_cluster(&x_full[bx], ph, abort_flag, p.status);
+        if (__any_sync(0xffffffffu, !ok)) { alive = false; return; }
+        float s[TN];
+        {
+          const float* pe = xbuf + (bx * kH + h) * TN;
+          const float* me = mybuf + (bx * kH + h) * TN;
 #pragma unroll
-          for (int c = 0; c < TN / 4; ++c)  // chunk c of the row is stored at slot (c + h) mod 8
-            st_async_v4(dst + ((c + h) & (TN / 4 - 1)) * 16,
-                        make_uint4(cur[4 * c], cur[4 * c + 1], cur[4 * c + 2], cur[4 * c + 3]), peer_xfull + u * 8);
+          for (int c = 0; c < TN / 4; ++c) {
+            const int slot = (c + h) & (TN / 4 - 1);
+            const float4 v = *reinterpret_cast<const float4*>(pe + 4 * slot);
+            const float4 w = *reinterpret_cast<const float4*>(me + 4 * slot);
+            // rank-0 part + rank-1 part in both CTAs (identical bits)
+            s[4 * c + 0] = R == 0 ? w.x + v.x : v.x + w.x;
+            s[4 * c + 1] = R == 0 ? w.y + v.y : v.y + w.y;
+            s[4 * c + 2] = R == 0 ? w.z + v.z : v.z + w.z;
+            s[4 * c + 3] = R == 0 ? w.w + v.w : v.w + w.w;
+          }
         }
+        mbar_arrive(&my_empty[bx]);
+        named_bar_sync(2, 128);  // every row of xbuf[bx] has been read
+        if (th == 0) {
+          mbar_arrive_remote(peer_xempty + bx * 8);
+          mbar_arrive_expect_tx(&x_full[bx], XBUF);  // re-arm for tile k + NX
+        }
+        const int valid = L - (t0 + i) * TN;  // tokens of this tile inside the sequence
+        if (valid < TN) {
+#pragma unroll
+          for (int c = 0; c < TN; ++c)
+            if (c >= valid) s[c] = -INFINITY;
+        }
+        float mx0 = fmax3f(s[0], s[1], s[2]), mx1 = fmax3f(s[3], s[4], s[5]);
+#pragma unroll
+        for (int c = 6; c + 3 < TN; c += 4) {
+          mx0 = fmax3f(mx0, s[c], s[c + 1]);
+          mx1 = fmax3f(mx1, s[c + 2], s[c + 3]);
+        }
+        mx0 = fmaxf(mx0, s[TN - 2]);
+        mx1 = fmaxf(mx1, s[TN - 1]);
+        const float m_new = fmaxf(m_run, fmaxf(mx0, mx1) * sl2);
         if (i > 0) {
-          // ---- tile k-1: add the peer's part, online softmax, P into TMEM
-          const int kk = k - 1, uu = kk & 1, ii = i - 1;
-          bool ok = mbar_wait_cluster(&x_full[uu], (kk >> 1) & 1, abort_flag, p.status);
-          if (__any_sync(0xffffffffu, !ok)) { alive = false; return; }
-          float s[TN];
-          {
-            const float* src = xbuf + (uu * kH + h) * TN;
-#pragma unroll
-            for (int c = 0; c < TN / 4; ++c) {
-              const float4 v = *reinterpret_cast<const float4*>(src + 4 * ((c + h) & (TN / 4 - 1)));
-              const float pv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float mv = __uint_as_float(prev[4 * c + e]);
-                s[4 * c + e] = R == 0 ? mv + pv[e] : pv[e] + mv;  // rank-0 part + rank-1 part in both CTAs
-              }
-            }
-          }
-          named_bar_sync(1, 128);  // every row of xbuf[uu] has been read
-          if (h == 0) mbar_arrive_remote(peer_xempty + uu * 8);
-          const int valid = L - (t0 + ii) * TN;  // tokens of this tile inside the sequence
-          if (valid < TN) {
-#pragma unroll
-            for (int c = 0; c < TN; ++c)
-              if (c >= valid) s[c] = -INFINITY;
-          }
-          float mx0 = fmax3f(s[0], s[1], s[2]), mx1 = fmax3f(s[3], s[4], s[5]);
-#pragma unroll
-          for (int c = 6; c + 3 < TN; c += 4) {
-            mx0 = fmax3f(mx0, s[c], s[c + 1]);
-            mx1 = fmax3f(mx1, s[c + 2], s[c + 3]);
-          }
-          mx0 = fmaxf(mx0, s[TN - 2]);
-          mx1 = fmaxf(mx1, s[TN - 1]);
-          const float m_new = fmaxf(m_run, fmaxf(mx0, mx1) * sl2);
-          if (ii > 0) {
-            if (__any_sync(0xffffffffu, m_new > m_run + 8.0f)) {
-              // O must hold P V of every earlier tile before it is scaled
-              ok = mbar_wait(&o_done[(kk - 1) & 1], ((kk - 1) >> 1) & 1, abort_flag, p.status);
-              if (__any_sync(0xffffffffu, !ok)) { alive = false; return; }
-              tc_fence_after();
-              const float alpha = ex2_approx(m_run - m_new);
-              m_run = m_new;
-              l_run *= alpha;
-#pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                uint32_t r[32];
-                tmem_ld32(t_lane + O_COL + c * 32, r);
-                tmem_ld_wait();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-                tmem_st32(t_lane + O_COL + c * 32, r);
-              }
-            }
-          } else {
-            m_run = m_new;
-          }
-          uint32_t pp[TN / 2];
-          float la = 0.f, lb = 0.f;
-#pragma unroll
-          for (int c = 0; c < TN; c += 2) {
-            const float a = ex2_approx(fmaf(s[c], sl2, -m_run));
-            const float bb = ex2_approx(fmaf(s[c + 1], sl2, -m_run));
-            la += a;
-            lb += bb;
-            pp[c / 2] = pack_bf16x2(a, bb);
-          }
-          l_run += la + lb;
-          if (ii >= 2) {  // P buffer uu last held P(kk-2)
-            ok = mbar_wait(&o_done[uu], ((kk - 2) >> 1) & 1, abort_flag, p.status);
+          if (__any_sync(0xffffffffu, m_new > m_run + 8.0f)) {
+            // O must hold P V of every earlier tile before it is scaled
+            ok = mbar_wait(&o_done[(k - 1) & 1], ((k - 1) >> 1) & 1, abort_flag, p.status);
             if (__any_sync(0xffffffffu, !ok)) { alive = false; return; }
             tc_fence_after();
-          }
-          tmem_st16(t_lane + P_COL + uu * (TN / 2), pp);
-          if (valid < TN) {
-            // cached rows past the sequence end may hold anything: zero this CTA's
-            // value columns for them so that 0 * garbage cannot reach O
-            uint8_t* st = sKV + (kk % NST) * STAGE;
-            const int nbad = TN - valid;
-            for (int idx = threadIdx.x; idx < 4 * nbad * 8; idx += 128) {
-              const int bx = idx / (nbad * 8), r = valid + (idx / 8) % nbad, ch = idx % 8;
-              *reinterpret_cast<uint4*>(st + bx * KV_BOX + r * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
-            }
-            fence_proxy_async_smem();
-            named_bar_sync(1, 128);  // every zero row is written before any thread signals P
-          }
-          tmem_st_wait();
-          tc_fence_before();
-          mbar_arrive(&p_full[uu]);
-        }
-        if (i < n) {
+            const float alpha = ex2_approx(m_run - m_new);
+            m_run = m_new;
+            l_run *= alpha;
+#pragma unroll 1
+            for (int c = 0; c < 8; ++c) {
+              uint32_t r[32];
+              tmem_ld32(t_lane + O_COL + c * 32, r);
+              tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < TN; ++c) prev[c] = cur[c];
+              for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+              tmem_st32(t_lane + O_COL + c * 32, r);
+            }
+          }
+        } else {
+          m_run = m_new;
         }
+        uint32_t pp[TN / 2];
+        float la = 0.f, lb = 0.f;
+#pragma unroll
+        for (int c = 0; c < TN; c += 2) {
+          const float a = ex2_approx(fmaf(s[c], sl2, -m_run));
+          const float bb = ex2_approx(fmaf(s[c + 1], sl2, -m_run));
+          la += a;
+          lb += bb;
+          pp[c / 2] = pack_bf16x2(a, bb);
+        }
+        l_run += la + lb;
+        if (i >= 2) {  // P buffer u last held P(k-2)
+          ok = mbar_wait(&o_done[u], ((k - 2) >> 1) & 1, abort_flag, p.status);
+          if (__any_sync(0xffffffffu, !ok)) { alive = false; return; }
+          tc_fence_after();
+        }
+        tmem_st16(t_lane + P_COL + u * (TN / 2), pp);
+        if (valid < TN) {
+          // cached rows past the sequence end may hold anything: zero this CTA's
+          // value columns for them so that 0 * garbage cannot reach O
+          uint8_t* st = sKV + (k % NST) * STAGE;
+          const int nbad = TN - valid;
+          for (int idx = th; idx < 4 * nbad * 8; idx += 128) {
+            const int bxx = idx / (nbad * 8), r = valid + (idx / 8) % nbad, ch = idx % 8;
+            *reinterpret_cast<uint4*>(st + bxx * KV_BOX + r * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+          named_bar_sync(2, 128);  // every zero row is written before any thread signals P
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[u]);
       }
       // segment epilogue: O / l for this CTA's 256 columns, and the LSE (rank 0).
       // P V(g_last - 2) is known complete (waited before P(g_last) was written), so one
       // wait on the last tile's barrier is exact.
       const int g_last = g0 + n - 1;
+      if (n < 3 && n >= 2) {  // P V(g_last - 1) may still be pending with only two tiles
+        bool ok1 = mbar_wait(&o_done[(g_last - 1) & 1], ((g_last - 1) >> 1) & 1, abort_flag, p.status);
+        if (__any_sync(0xffffffffu, !ok1)) { alive = false; return; }
+      }
       bool ok = mbar_wait(&o_done[g_last & 1], (g_last >> 1) & 1, abort_flag, p.status);
       if (__any_sync(0xffffffffu, !ok)) { alive = false; return; }
       tc_fence_after();
       const int slot = pair + b;
       const float inv_l = 1.f / l_run;
       float* orow = p.part_o + (static_cast<size_t>(slot) * kH + h) * kDc + R * 256;
-#pragma unroll
+#pragma unroll 1
       for (int c = 0; c < 8; ++c) {
         uint32_t r[32];
         tmem_ld32(t_lane + O_COL + c * 32, r);
@@ -453,7 +489,7 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();  // no remote access to this CTA's shared memory is still pending
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
   }
@@ -461,15 +497,12 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
 
 }  // namespace
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     mla_kernel(const __grid_constant__ MlaParams p, const __grid_constant__ CUtensorMap tmKV,
                const __grid_constant__ CUtensorMap tmPE) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  if (cluster_ctarank() == 0)
-    mla_body<0>(p, &tmKV, &tmPE, smem);
-  else
-    mla_body<1>(p, &tmKV, &tmPE, smem);
+  mla_body(p, &tmKV, &tmPE, smem, static_cast<int>(cluster_ctarank()));
 }
 
 int mla_pairs_for_device() {
@@ -483,7 +516,7 @@ int mla_pairs_for_device() {
 cudaError_t launch_mla(const MlaParams& p, const CUtensorMap& tmKV, const CUtensorMap& tmPE, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  mla_kernel<<<2 * p.n_pairs, 192, SMEM_BYTES, stream>>>(p, tmKV, tmPE);
+  mla_kernel<<<2 * p.n_pairs, 320, SMEM_BYTES, stream>>>(p, tmKV, tmPE);
   return cudaGetLastError();
 }
 
