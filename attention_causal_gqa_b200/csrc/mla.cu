@@ -70,34 +70,10 @@ __device__ __forceinline__ void st_async_v4(uint32_t addr, uint4 v, uint32_t bar
                "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(bar_cluster_addr)
                : "memory");
 }
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait for a barrier that the peer CTA arrives on.
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                                  int* status) {
-  if (mbar_try_wait_acq_cluster(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
-    if (mbar_try_wait_acq_cluster(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > ATTN_WAIT_TIMEOUT_NS) {
-      *abort_flag = 1;
-      if (status) atomicOr(status, kDevErrTimeout);
-      return false;
-    }
-  }
+// Remote arrive without release semantics: used only to say "these bytes were read",
+// where the reads have already returned their values (no write needs publishing).
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t bar_cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
 }
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
@@ -305,7 +281,7 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
               make_uint4(cur[4 * c], cur[4 * c + 1], cur[4 * c + 2], cur[4 * c + 3]);
         mbar_arrive(&my_full[bx]);
         // the peer's copy
-        ok = mbar_wait_cluster(&x_empty[bx], ph ^ 1, abort_flag, p.status);
+        ok = mbar_wait(&x_empty[bx], ph ^ 1, abort_flag, p.status);  // carries no data: plain wait
         if (__any_sync(0xffffffffu, !ok)) { alive = false; return; }
         const uint32_t dst = peer_xbuf + (bx * kH + h) * (TN * 4);
 #pragma unroll
@@ -362,7 +338,9 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
         const int u = k & 1, bx = k % NX;
         const uint32_t ph = (k / NX) & 1;
         bool ok = mbar_wait(&my_full[bx], ph, abort_flag, p.status);
-        ok = ok && mbar_wait_cluster(&x_full[bx], ph, abort_flag, p.status);
+        // the peer's st.async bytes complete on this local barrier, which makes them
+        // visible to a plain wait (same rule as a TMA load)
+        ok = ok && mbar_wait(&x_full[bx], ph, abort_flag, p.status);
         if (__any_sync(0xffffffffu, !ok)) { alive = false; return; }
         float s[TN];
         {
@@ -383,7 +361,7 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
         mbar_arrive(&my_empty[bx]);
         named_bar_sync(2, 128);  // every row of xbuf[bx] has been read
         if (th == 0) {
-          mbar_arrive_remote(peer_xempty + bx * 8);
+          mbar_arrive_remote_relaxed(peer_xempty + bx * 8);
           mbar_arrive_expect_tx(&x_full[bx], XBUF);  // re-arm for tile k + NX
         }
         const int valid = L - (t0 + i) * TN;  // tokens of this tile inside the sequence
