@@ -189,8 +189,8 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
       });
     }
   } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------------ MMA issuer (whole warp)
+    {
       constexpr uint32_t idesc_s = idesc_f32acc(1, 128, TN, false, false);
       constexpr uint32_t idesc_o = idesc_f32acc(1, 128, 256, false, true);
       constexpr uint32_t HI = sdesc_hi_sw128(1024);
@@ -203,7 +203,7 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
         for (int bx = 0; bx < NKB; ++bx)
 #pragma unroll
           for (int kq = 0; kq < 4; ++kq)
-            umma_f16_ts(d, tmem_base + Q_COL + (bx * 4 + kq) * 8, b0 + ((bx * KV_BOX + kq * 32) >> 4), HI, idesc_s,
+            umma_f16_ts_warp(d, tmem_base + Q_COL + (bx * 4 + kq) * 8, b0 + ((bx * KV_BOX + kq * 32) >> 4), HI, idesc_s,
                         (bx > 0 || kq > 0) ? 1u : 0u);
       };
       auto issue_pv = [&](int g, bool acc) {
@@ -211,30 +211,30 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
         const uint32_t a0 = tmem_base + P_COL + (g & 1) * (TN / 2);
 #pragma unroll
         for (int kb = 0; kb < TN / 16; ++kb)
-          umma_f16_ts(tmem_base + O_COL, a0 + kb * 8, b0 + ((kb * 16 * 128) >> 4), HI, idesc_o,
+          umma_f16_ts_warp(tmem_base + O_COL, a0 + kb * 8, b0 + ((kb * 16 * 128) >> 4), HI, idesc_o,
                       (acc || kb > 0) ? 1u : 0u);
       };
       bool ok = true;
       int seg = 0;
       auto s_step = [&](int g) -> bool {  // S(g) once its ring slot is loaded
-        if (!mbar_wait(&kv_full[g % NST], (g / NST) & 1, abort_flag, p.status)) return false;
+        if (!mbar_wait_warp(&kv_full[g % NST], (g / NST) & 1, abort_flag, p.status)) return false;
         tc_fence_after();
         issue_s(g);
-        umma_commit(&s_full[g & 1]);
+        umma_commit_warp(&s_full[g & 1]);
         return true;
       };
       auto pv_step = [&](int g, bool acc) -> bool {  // P(g) V(g) once P(g) is in TMEM
-        if (!mbar_wait(&p_full[g & 1], (g >> 1) & 1, abort_flag, p.status)) return false;
+        if (!mbar_wait_warp(&p_full[g & 1], (g >> 1) & 1, abort_flag, p.status)) return false;
         tc_fence_after();
         issue_pv(g, acc);
-        umma_commit(&o_done[g & 1]);
-        umma_commit(&kv_empty[g % NST]);
+        umma_commit_warp(&o_done[g & 1]);
+        umma_commit_warp(&kv_empty[g % NST]);
         return true;
       };
       for_each_segment(p, pair, [&](int, int t0, int t1, int g0) {
         if (!ok) return;
         const int n = t1 - t0;
-        if (!mbar_wait(q_ready, seg & 1, abort_flag, p.status)) { ok = false; return; }
+        if (!mbar_wait_warp(q_ready, seg & 1, abort_flag, p.status)) { ok = false; return; }
         ++seg;
         tc_fence_after();
         ok = s_step(g0) && (n < 2 || s_step(g0 + 1));
@@ -242,14 +242,14 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
         for (int i = 0; ok && i < n; ++i) {
           const int k = g0 + i;
           if (i + 2 < n) {
-            ok = mbar_wait(&s_free[k & 1], (k >> 1) & 1, abort_flag, p.status) && s_step(k + 2);
+            ok = mbar_wait_warp(&s_free[k & 1], (k >> 1) & 1, abort_flag, p.status) && s_step(k + 2);
             if (!ok) break;
           }
           ok = pv_step(k, i > 0);
         }
       });
-      umma_commit(mma_done);
-      mbar_wait(mma_done, 0, abort_flag, p.status);
+      umma_commit_warp(mma_done);
+      mbar_wait_warp(mma_done, 0, abort_flag, p.status);
     }
   } else if (warp < 4) {
     // ----------------------------------------- exchange warpgroup (WG0): S out of TMEM
