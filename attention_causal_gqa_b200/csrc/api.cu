@@ -197,19 +197,39 @@ int attn_prefill(const void* q, const void* k, const void* v, void* out, float* 
     kbase = kop;
     kdt = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   }
+  // Q operand. Without RoPE, bf16 Q is the operand itself. Otherwise the prologue
+  // writes it into `out`, whose size is exactly that of the operand (rotated fp16 Q
+  // for bf16 input; bf16 hi planes then lo planes for fp32 input). Every Q tile is
+  // loaded and later overwritten by the same CTA, so the reuse is free of races.
+  const long long rows_q = static_cast<long long>(B) * Hq * S;
+  const void* qbase = q;
+  CUtensorMapDataType qdt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  cuuint64_t zq = static_cast<cuuint64_t>(B) * Hq;
+  if (f32) {
+    cudaError_t e = attn::launch_split_f32(static_cast<const float*>(q), out, rope ? cs : nullptr, rows_q, S, D, st);
+    if (e != cudaSuccess) return cuda_fail(e, "Q operand split launch");
+    qbase = out;
+    zq *= 2;
+  } else if (rope) {
+    cudaError_t e = attn::launch_rope_k_f16(q, out, cs, rows_q, S, D, status, st);
+    if (e != cudaSuccess) return cuda_fail(e, "rope Q launch");
+    qbase = out;
+    qdt = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  }
   const int BN = attn::prefill_block_n(D, f32);
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S), zdim};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(S) * D * 2};
   const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(BN), 1};
-  CUtensorMap tmK, tmV;
+  const cuuint64_t qdims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S), zq};
+  const cuuint32_t qbox[3] = {64, 128, 1};
+  CUtensorMap tmQ, tmK, tmV;
+  if ((rc = make_map(&tmQ, qdt, 3, qbase, qdims, strides, qbox, "Q"))) return rc;
   if ((rc = make_map(&tmK, kdt, 3, kbase, dims, strides, box, "K"))) return rc;
   if ((rc = make_map(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, vbase, dims, strides, box, "V"))) return rc;
 
   attn::PrefillParams p{};
-  p.q = q;
   p.out = out;
   p.lse = lse;
-  p.rope_cs = rope ? cs : nullptr;
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
@@ -224,7 +244,7 @@ int attn_prefill(const void* q, const void* k, const void* v, void* out, float* 
                                       : static_cast<long long>(B) * Hq * ((p.n_row_blocks + 1) / 2);
   if (grid > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "grid too large");
   prof_before(st);
-  cudaError_t e = attn::launch_prefill(p, tmK, tmV, D, f32, rope, static_cast<int>(grid), st);
+  cudaError_t e = attn::launch_prefill(p, tmQ, tmK, tmV, D, f32, rope, static_cast<int>(grid), st);
   prof_after(st);
   if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
   return ok();

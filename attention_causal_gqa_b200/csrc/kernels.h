@@ -8,10 +8,8 @@
 namespace attn {
 
 struct PrefillParams {
-  const void* q;          // [B, Hq, S, D] (T)
   void* out;              // [B, Hq, S, D] (T)
   float* lse;             // [B, Hq, S]
-  const float2* rope_cs;  // [S, D/2] (cos, sin) or nullptr when RoPE is off
   int B, Hq, Hkv, S, G;
   int causal;
   float scale_log2;       // scale * log2(e)
@@ -22,7 +20,8 @@ struct PrefillParams {
 
 // RoPE prologue: cos/sin table (angles in fp64), then the key operand.
 cudaError_t launch_rope_table(float2* cs, int S, int D, double theta, cudaStream_t stream);
-// bf16 K [rows, D] -> rotated fp16 K (row r at position r % S); flags values outside fp16 range.
+// bf16 X [rows, D] -> rotated fp16 X (row r at position r % S); flags values outside fp16 range.
+// Used for K and for Q.
 cudaError_t launch_rope_k_f16(const void* k, void* k_f16, const float2* cs, long long rows, int S, int D,
                               int* status, cudaStream_t stream);
 // fp32 X [rows, D] -> bf16 hi parts at out[0, rows) and lo parts at out[rows, 2 rows), rotating
@@ -31,8 +30,9 @@ cudaError_t launch_split_f32(const float* x, void* out, const float2* cs, long l
                              cudaStream_t stream);
 
 int prefill_block_n(int D, bool f32);
-cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV, int D, bool f32,
-                           bool rope, int grid, cudaStream_t stream);
+// tmQ: the Q operand (bf16 Q, rotated fp16 Q, or bf16 hi/lo planes of fp32 Q), 128-row boxes.
+cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                           int D, bool f32, bool rope, int grid, cudaStream_t stream);
 
 // ----------------------------------------------------------- paged decode
 constexpr int kDecodePagesPerSplit = 32;  // pages (of 16 tokens) handled by one split

@@ -12,14 +12,14 @@
 // consecutive row blocks of one head. Roles (320 threads):
 //   warps 0-3  softmax warpgroup of tile 0 (one thread per query row)
 //   warps 4-7  softmax warpgroup of tile 1
-//   warp  8    TMA producer: K/V tiles into a shared-memory ring
-//   warp  9    TMEM allocator and single-thread tcgen05.mma issuer
+//   warp  8    TMA producer: both Q tiles, then K/V tiles into a shared-memory ring
+//   warp  9    TMEM allocator and tcgen05.mma issuer (elected lane of the warp)
 // TMEM holds S_0, S_1 (BN fp32 columns each) and O_0, O_1 (D columns each).
-// Q is rotated (RoPE from the fp32 cos/sin table) by the softmax threads while
-// they stage it into shared memory; K arrives already rotated from the prologue
-// kernel. P (16-bit) is written back into the columns of S_t and feeds O += P V
-// as the A operand straight from TMEM, so shared-memory bandwidth is spent on
-// Q, K and V only. Per tile the tensor pipe runs P_t V_j before Q_t K_{j+1}^T,
+// Q and K arrive by TMA already in operand form: rotated (RoPE, cos/sin table
+// with fp64 angles) and rounded by the prologue kernels, so a CTA starts its
+// first Q K^T as soon as the two tiles land. P (16-bit) is written back into
+// the columns of S_t and feeds O += P V as the A operand straight from TMEM, so
+// shared-memory bandwidth is spent on Q, K and V only. Per tile the tensor pipe runs P_t V_j before Q_t K_{j+1}^T,
 // which both keeps P_t intact until it is consumed and guarantees that O_t is
 // final for step j when S_t(j+1) is reported ready.
 //
@@ -71,54 +71,11 @@ struct PrefillShape {
 };
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 domain: rescale O only when the max grows by > 2^8
-constexpr float kF16Max = 65504.f;
 
-__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
-  const __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-
-// 8 consecutive values -> one 16-byte chunk of 16-bit elements.
-template <bool kF16>
-__device__ __forceinline__ uint4 pack8(const float* f) {
-  if constexpr (kF16)
-    return make_uint4(pack_half2(f[0], f[1]), pack_half2(f[2], f[3]), pack_half2(f[4], f[5]),
-                      pack_half2(f[6], f[7]));
-  else
-    return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
-                      pack_bf16x2(f[6], f[7]));
-}
-
-// hi = bf16(x), lo = bf16(x - hi) for 8 values.
-__device__ __forceinline__ void split8(const float* f, uint4& hi, uint4& lo) {
-  float h[8], l[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    h[e] = __bfloat162float(__float2bfloat16_rn(f[e]));
-    l[e] = f[e] - h[e];
-  }
-  hi = pack8<false>(h);
-  lo = pack8<false>(l);
-}
-
-template <typename TIn>
-__device__ __forceinline__ void load8(const TIn* p, float* f);
-template <>
-__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float* f) {
-  const uint4 raw = __ldg(reinterpret_cast<const uint4*>(p));
-  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
-}
-template <>
-__device__ __forceinline__ void load8<float>(const float* p, float* f) {
-  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
-  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
-  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+// 8 consecutive values -> one 16-byte chunk of bf16 elements.
+__device__ __forceinline__ uint4 pack8_bf16(const float* f) {
+  return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                    pack_bf16x2(f[6], f[7]));
 }
 
 template <typename TIn>
@@ -126,7 +83,7 @@ __device__ __forceinline__ void store32(TIn* dst, const float* f);
 template <>
 __device__ __forceinline__ void store32<__nv_bfloat16>(__nv_bfloat16* dst, const float* f) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) reinterpret_cast<uint4*>(dst)[i] = pack8<false>(f + 8 * i);
+  for (int i = 0; i < 4; ++i) reinterpret_cast<uint4*>(dst)[i] = pack8_bf16(f + 8 * i);
 }
 template <>
 __device__ __forceinline__ void store32<float>(float* dst, const float* f) {
@@ -135,10 +92,13 @@ __device__ __forceinline__ void store32<float>(float* dst, const float* f) {
     reinterpret_cast<float4*>(dst)[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
 }
 
+// Pairs out of every 8 of a softmax row that take the FMA-pipe exp2 (blocks without masking).
+constexpr int kPolyPer8 = 3;
+
 template <int D, int BN, int MODE>
 __global__ void __launch_bounds__(320, 1)
-    prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV) {
+    prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
+                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
   using Sh = PrefillShape<D, BN, MODE>;
   using TIn = typename std::conditional<MODE == kModeSplit, float, __nv_bfloat16>::type;
   constexpr int NP = Sh::NPART;
@@ -201,7 +161,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
-    mbar_init(q_full, 256);
+    mbar_init(q_full, 1);
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
       mbar_init(&p_full[t], 128);
@@ -223,8 +183,20 @@ __global__ void __launch_bounds__(320, 1)
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
+      // Both Q tiles (rows past S arrive as zeros), already in operand form.
+      mbar_arrive_expect_tx(q_full, 2 * NP * Sh::Q_PART);
+      for (int t = 0; t < 2; ++t) {
+        const int zq = b * p.Hq + (t ? h1 : h0), r0 = t ? r0_1 : r0_0;
+#pragma unroll
+        for (int u = 0; u < NP; ++u)
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(sQ + (t * NP + u) * Sh::Q_PART + c * Sh::Q_BOX, &tmQ, q_full, c * 64, r0,
+                        zq + u * p.B * p.Hq);
+      }
       const int zc = b * p.Hkv + kvh;
       const int zlo = p.B * p.Hkv;  // the lo parts follow the hi parts in the split layout
       for (int i = 0; i < 2 * n_max; ++i) {
@@ -243,14 +215,14 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
   } else if (warp == 9) {
-    // -------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // -------------------------------------------------- MMA issuer (whole warp)
+    {
       constexpr uint32_t idesc_qk = idesc_f32acc(Sh::QK_FMT, 128, BN, false, false);
       constexpr uint32_t idesc_pv = idesc_f32acc(1, 128, D, false, true);
       // (A part, B part) products: hi*hi, plus hi*lo and lo*hi for split operands
       constexpr int NPROD = Sh::SPLIT ? 3 : 1;
       const int n_kv[2] = {n_kv0, n_kv1};
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
+      bool ok = mbar_wait_warp(q_full, 0, abort_flag, p.status);
       // Descriptor words: the high word is shared by every operand; the low word
       // carries the start address (>> 4), advanced by compile-time offsets below.
       constexpr uint32_t HI = sdesc_hi_sw128(1024);
@@ -269,7 +241,7 @@ __global__ void __launch_bounds__(320, 1)
             const int pa = x == 2 ? 1 : 0, pb = x == 1 ? 1 : 0;
             const uint32_t ao = (pa * Sh::Q_PART + (kb >> 2) * Sh::Q_BOX + (kb & 3) * 32) >> 4;
             const uint32_t bo = (pb * Sh::KV_PART + (kb >> 2) * Sh::KV_BOX + (kb & 3) * 32) >> 4;
-            umma_f16_lohi(d, a0 + ao, HI, b0 + bo, HI, idesc_qk, (kb > 0 || x > 0) ? 1u : 0u);
+            umma_f16_lohi_warp(d, a0 + ao, HI, b0 + bo, HI, idesc_qk, (kb > 0 || x > 0) ? 1u : 0u);
           }
         }
       };
@@ -283,52 +255,52 @@ __global__ void __launch_bounds__(320, 1)
           for (int x = 0; x < NPROD; ++x) {
             const int pa = x == 2 ? 1 : 0, pb = x == 1 ? 1 : 0;
             const uint32_t bo = (pb * Sh::KV_PART + kb * 16 * 128) >> 4;
-            umma_f16_ts(d, a0 + pa * Sh::P_COLS + kb * 8, b0 + bo, HI, idesc_pv, (acc || kb > 0 || x > 0) ? 1u : 0u);
+            umma_f16_ts_warp(d, a0 + pa * Sh::P_COLS + kb * 8, b0 + bo, HI, idesc_pv, (acc || kb > 0 || x > 0) ? 1u : 0u);
           }
         }
       };
       if (ok && n_max > 0) {
         // K_0 sits in ring slot 0
-        ok = mbar_wait(&kv_full[0], 0, abort_flag, p.status);
+        ok = mbar_wait_warp(&kv_full[0], 0, abort_flag, p.status);
         if (ok) {
           tc_fence_after();
           for (int t = 0; t < 2; ++t)
             if (n_kv[t] > 0) {
               issue_qk(t, 0);
-              umma_commit(&s_full[t]);
+              umma_commit_warp(&s_full[t]);
             }
-          umma_commit(&kv_empty[0]);
+          umma_commit_warp(&kv_empty[0]);
         }
         for (int j = 0; ok && j < n_max; ++j) {
           const int iV = 2 * j + 1, sV = iV % Sh::NST;
           const int iK = 2 * j + 2, sK = iK % Sh::NST;
-          if (!mbar_wait(&kv_full[sV], (iV / Sh::NST) & 1, abort_flag, p.status)) { ok = false; break; }
+          if (!mbar_wait_warp(&kv_full[sV], (iV / Sh::NST) & 1, abort_flag, p.status)) { ok = false; break; }
           bool k_ready = false;
           for (int t = 0; t < 2 && ok; ++t) {
             if (j >= n_kv[t]) continue;
-            if (!mbar_wait(&p_full[t], j & 1, abort_flag, p.status)) { ok = false; break; }
+            if (!mbar_wait_warp(&p_full[t], j & 1, abort_flag, p.status)) { ok = false; break; }
             tc_fence_after();
             // P_t V_j first: it reads P_t from the columns that Q_t K_{j+1}^T overwrites.
             issue_pv(t, sV, j > 0);
-            umma_commit(&o_done[t]);
+            umma_commit_warp(&o_done[t]);
             if (j + 1 < n_kv[t]) {
               if (!k_ready) {
-                if (!mbar_wait(&kv_full[sK], (iK / Sh::NST) & 1, abort_flag, p.status)) { ok = false; break; }
+                if (!mbar_wait_warp(&kv_full[sK], (iK / Sh::NST) & 1, abort_flag, p.status)) { ok = false; break; }
                 tc_fence_after();
                 k_ready = true;
               }
               issue_qk(t, sK);
-              umma_commit(&s_full[t]);
+              umma_commit_warp(&s_full[t]);
             }
           }
           if (!ok) break;
-          umma_commit(&kv_empty[sV]);
-          if (k_ready) umma_commit(&kv_empty[sK]);
+          umma_commit_warp(&kv_empty[sV]);
+          if (k_ready) umma_commit_warp(&kv_empty[sK]);
         }
       }
       // drain: every MMA issued above has completed once this barrier flips
-      umma_commit(mma_done);
-      mbar_wait(mma_done, 0, abort_flag, p.status);
+      umma_commit_warp(mma_done);
+      mbar_wait_warp(mma_done, 0, abort_flag, p.status);
     }
   } else {
     // ------------------------------------------------------- softmax warpgroups
@@ -341,50 +313,6 @@ __global__ void __launch_bounds__(320, 1)
     const int grow = r0 + row;
     const bool row_valid = grow < p.S;
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(wr * 32) << 16);
-
-    // Stage Q (rotated) into the swizzled K-major tile(s).
-    {
-      uint8_t* qtile = sQ + t * NP * Sh::Q_PART;
-      const TIn* qrow = reinterpret_cast<const TIn*>(p.q) + ((static_cast<size_t>(b) * p.Hq + h) * p.S + grow) * D;
-      const float2* cs = p.rope_cs ? p.rope_cs + static_cast<size_t>(grow) * (D / 2) : nullptr;
-      bool range_ok = true;
-#pragma unroll 4
-      for (int c = 0; c < D / 8; ++c) {
-        float f[8];
-        if (row_valid && n_kv > 0) {
-          load8<TIn>(qrow + c * 8, f);
-          if (cs) {
-#pragma unroll
-            for (int e = 0; e < 8; e += 2) {
-              const float2 r = __ldg(cs + (c * 8 + e) / 2);
-              const float x0 = f[e], x1 = f[e + 1];
-              f[e] = x0 * r.x - x1 * r.y;
-              f[e + 1] = x0 * r.y + x1 * r.x;
-            }
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) f[e] = 0.f;
-        }
-        const int box = c >> 3, ch = c & 7;
-        const int off = box * Sh::Q_BOX + row * 128 + ((ch ^ (row & 7)) << 4);
-        if constexpr (MODE == kModeSplit) {
-          uint4 hi, lo;
-          split8(f, hi, lo);
-          *reinterpret_cast<uint4*>(qtile + off) = hi;
-          *reinterpret_cast<uint4*>(qtile + Sh::Q_PART + off) = lo;
-        } else if constexpr (MODE == kModeF16QK) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) range_ok = range_ok && fabsf(f[e]) <= kF16Max;
-          *reinterpret_cast<uint4*>(qtile + off) = pack8<true>(f);
-        } else {
-          *reinterpret_cast<uint4*>(qtile + off) = pack8<false>(f);
-        }
-      }
-      if (!range_ok) atomicOr(p.status, kDevErrRange);
-      fence_proxy_async_smem();
-      mbar_arrive(q_full);
-    }
 
     float m_run = -INFINITY;
     float l_run = 0.f;
@@ -441,37 +369,50 @@ __global__ void __launch_bounds__(320, 1)
       }
 
       // P = exp2(s * scale * log2(e) - m) as 16-bit pairs into the columns of S_t, and the row sum.
+      // In blocks without masked columns, kPolyPer8 of every 8 pairs take the FMA-pipe
+      // exp2 so the MUFU and FMA pipes share the work.
       const float2 sl2x2 = make_float2(sl2, sl2);
       const float2 nmx2 = make_float2(-m_run, -m_run);
       const uint32_t p_col = t_lane + Sh::S_COL0 + t * BN;
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      auto exp_rows = [&](auto poly_tag) {
+        constexpr bool kPoly = decltype(poly_tag)::value;
+        auto ex = [&](float2 z, int q) -> float2 {
+          if (kPoly && (q * kPolyPer8) % 8 < kPolyPer8) return exp2_fma2(z);
+          return make_float2(ex2_approx(z.x), ex2_approx(z.y));
+        };
 #pragma unroll
-      for (int c = 0; c < NCH; ++c) {
-        uint32_t ph[16];
-        uint32_t pl[Sh::SPLIT ? 16 : 1];
+        for (int c = 0; c < NCH; ++c) {
+          uint32_t ph[16];
+          uint32_t pl[Sh::SPLIT ? 16 : 1];
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float2 z0 = ffma2(make_float2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])), sl2x2, nmx2);
-          const float2 z1 = ffma2(make_float2(__uint_as_float(sr[c][e + 2]), __uint_as_float(sr[c][e + 3])), sl2x2, nmx2);
-          const float2 p0 = make_float2(ex2_approx(z0.x), ex2_approx(z0.y));
-          const float2 p1 = make_float2(ex2_approx(z1.x), ex2_approx(z1.y));
-          acc[(e >> 1) & 3] = fadd2(acc[(e >> 1) & 3], p0);
-          acc[((e >> 1) + 1) & 3] = fadd2(acc[((e >> 1) + 1) & 3], p1);
-          if constexpr (Sh::SPLIT) {
-            const float h0 = __bfloat162float(__float2bfloat16_rn(p0.x)), h1 = __bfloat162float(__float2bfloat16_rn(p0.y));
-            const float h2 = __bfloat162float(__float2bfloat16_rn(p1.x)), h3 = __bfloat162float(__float2bfloat16_rn(p1.y));
-            ph[e >> 1] = pack_bf16x2(h0, h1);
-            ph[(e >> 1) + 1] = pack_bf16x2(h2, h3);
-            pl[e >> 1] = pack_bf16x2(p0.x - h0, p0.y - h1);
-            pl[(e >> 1) + 1] = pack_bf16x2(p1.x - h2, p1.y - h3);
-          } else {
-            ph[e >> 1] = pack_bf16x2(p0.x, p0.y);
-            ph[(e >> 1) + 1] = pack_bf16x2(p1.x, p1.y);
+          for (int e = 0; e < 32; e += 4) {
+            const float2 z0 = ffma2(make_float2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])), sl2x2, nmx2);
+            const float2 z1 = ffma2(make_float2(__uint_as_float(sr[c][e + 2]), __uint_as_float(sr[c][e + 3])), sl2x2, nmx2);
+            const float2 p0 = ex(z0, e >> 1);
+            const float2 p1 = ex(z1, (e >> 1) + 1);
+            acc[(e >> 1) & 3] = fadd2(acc[(e >> 1) & 3], p0);
+            acc[((e >> 1) + 1) & 3] = fadd2(acc[((e >> 1) + 1) & 3], p1);
+            if constexpr (Sh::SPLIT) {
+              const float h0 = __bfloat162float(__float2bfloat16_rn(p0.x)), h1 = __bfloat162float(__float2bfloat16_rn(p0.y));
+              const float h2 = __bfloat162float(__float2bfloat16_rn(p1.x)), h3 = __bfloat162float(__float2bfloat16_rn(p1.y));
+              ph[e >> 1] = pack_bf16x2(h0, h1);
+              ph[(e >> 1) + 1] = pack_bf16x2(h2, h3);
+              pl[e >> 1] = pack_bf16x2(p0.x - h0, p0.y - h1);
+              pl[(e >> 1) + 1] = pack_bf16x2(p1.x - h2, p1.y - h3);
+            } else {
+              ph[e >> 1] = pack_bf16x2(p0.x, p0.y);
+              ph[(e >> 1) + 1] = pack_bf16x2(p1.x, p1.y);
+            }
           }
+          tmem_st16(p_col + c * 16, ph);
+          if constexpr (Sh::SPLIT) tmem_st16(p_col + Sh::P_COLS + c * 16, pl);
         }
-        tmem_st16(p_col + c * 16, ph);
-        if constexpr (Sh::SPLIT) tmem_st16(p_col + Sh::P_COLS + c * 16, pl);
-      }
+      };
+      if (Sh::SPLIT || need_mask)
+        exp_rows(std::false_type{});
+      else
+        exp_rows(std::true_type{});
       const float2 acc01 = fadd2(acc[0], acc[1]), acc23 = fadd2(acc[2], acc[3]);
       const float lsum = (acc01.x + acc01.y) + (acc23.x + acc23.y);
       // O *= alpha (warp-uniform decision; exact because P and l use the same m)
@@ -527,13 +468,14 @@ __global__ void __launch_bounds__(320, 1)
 }
 
 template <int D, int BN, int MODE>
-static cudaError_t launch_prefill_t(const PrefillParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
+static cudaError_t launch_prefill_t(const PrefillParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                                    const CUtensorMap& tmV,
                                     int grid, cudaStream_t stream) {
   using Sh = PrefillShape<D, BN, MODE>;
   auto kern = prefill_kernel<D, BN, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sh::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  kern<<<grid, 320, Sh::SMEM_BYTES, stream>>>(p, tmK, tmV);
+  kern<<<grid, 320, Sh::SMEM_BYTES, stream>>>(p, tmQ, tmK, tmV);
   return cudaGetLastError();
 }
 
@@ -542,18 +484,19 @@ int prefill_block_n(int D, bool f32) {
   return f32 ? 64 : 128;
 }
 
-cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV, int D, bool f32,
+cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                           int D, bool f32,
                            bool rope, int grid, cudaStream_t stream) {
   if (f32) {
-    if (D == 64) return launch_prefill_t<64, 64, kModeSplit>(p, tmK, tmV, grid, stream);
+    if (D == 64) return launch_prefill_t<64, 64, kModeSplit>(p, tmQ, tmK, tmV, grid, stream);
     return cudaErrorInvalidValue;
   }
   if (rope) {
-    if (D == 128) return launch_prefill_t<128, 128, kModeF16QK>(p, tmK, tmV, grid, stream);
-    if (D == 64) return launch_prefill_t<64, 128, kModeF16QK>(p, tmK, tmV, grid, stream);
+    if (D == 128) return launch_prefill_t<128, 128, kModeF16QK>(p, tmQ, tmK, tmV, grid, stream);
+    if (D == 64) return launch_prefill_t<64, 128, kModeF16QK>(p, tmQ, tmK, tmV, grid, stream);
   } else {
-    if (D == 128) return launch_prefill_t<128, 128, kModeBF16>(p, tmK, tmV, grid, stream);
-    if (D == 64) return launch_prefill_t<64, 128, kModeBF16>(p, tmK, tmV, grid, stream);
+    if (D == 128) return launch_prefill_t<128, 128, kModeBF16>(p, tmQ, tmK, tmV, grid, stream);
+    if (D == 64) return launch_prefill_t<64, 128, kModeBF16>(p, tmQ, tmK, tmV, grid, stream);
   }
   return cudaErrorInvalidValue;
 }

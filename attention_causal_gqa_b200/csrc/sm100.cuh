@@ -337,6 +337,28 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
   return d;
 }
 
+// 2^z for a pair of arguments on the FMA and integer pipes only, so that part of
+// a softmax row can bypass the MUFU (whose 16 results per clock per SM are the
+// same budget as the tensor core's score rate at head dim 128). Method
+// (Cody-Waite range reduction): n = round(z) via the 1.5 * 2^23 shifter, f = z - n
+// in [-1/2, 1/2], 2^f from a degree-3 polynomial, 2^n added to the exponent field.
+// The coefficients are a minimax fit of 2^f on [-1/2, 1/2] in relative error made
+// for this library by a Remez exchange (maximum relative error 7.5e-5, 25x below
+// the bf16 rounding that P receives). z is clamped below at -126 (result tiny but
+// finite); z must stay below 128.
+__device__ __forceinline__ float2 exp2_fma2(float2 z) {
+  z.x = fmaxf(z.x, -126.f);
+  z.y = fmaxf(z.y, -126.f);
+  const float2 t = fadd2(z, make_float2(12582912.f, 12582912.f));   // low bits of t hold n
+  const float2 n = fadd2(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = ffma2(n, make_float2(-1.f, -1.f), z);
+  float2 q = ffma2(f, make_float2(0.0551716685f, 0.0551716685f), make_float2(0.2426111251f, 0.2426111251f));
+  q = ffma2(q, f, make_float2(0.6932609677f, 0.6932609677f));
+  q = ffma2(q, f, make_float2(0.9999280572f, 0.9999280572f));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

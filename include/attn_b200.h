@@ -51,9 +51,11 @@ enum { ATTN_DEV_TIMEOUT = 1, ATTN_DEV_BAD_PAGE = 2, ATTN_DEV_BAD_LENGTH = 4, ATT
  * h / (Hq/Hkv)); "From 32K to 256K: DeepSeek long-context" (tqpw.cn) section 2.1
  * (RoPE on adjacent pairs, theta_i = rope_theta^(-2i/D)) and 2.5 (cos/sin cache).
  *
- *   q   [B, Hq,  S, D]   dtype (bf16, or fp32 computed as tf32)
+ *   q   [B, Hq,  S, D]   dtype (bf16, or fp32)
  *   k,v [B, Hkv, S, D]   dtype
- *   out [B, Hq,  S, D]   dtype (written)
+ *   out [B, Hq,  S, D]   dtype (written). With RoPE or fp32 input it also holds the
+ *                        prepared Q operand between the prologue and the main kernel
+ *                        (same byte size), so it must not overlap q, k or v.
  *   lse [B, Hq,  S]      fp32  (written)
  * causal: 1 -> key j is visible to query i iff j <= i; 0 -> all keys.
  * rope_theta: > 0 applies RoPE to q and k at positions 0..S-1; <= 0 disables it.
