@@ -93,7 +93,7 @@ __device__ __forceinline__ void store32<float>(float* dst, const float* f) {
 }
 
 // Pairs out of every 8 of a softmax row that take the FMA-pipe exp2 (blocks without masking).
-constexpr int kPolyPer8 = 3;
+constexpr int kPolyPer8 = 2;
 
 template <int D, int BN, int MODE>
 __global__ void __launch_bounds__(320, 1)
