@@ -12,11 +12,12 @@
 // 256-511 plus the 64 rotary columns. Each CTA
 //   * loads only its own columns of each kv/pe tile (no byte is loaded twice),
 //   * computes its partial score block S_r = Q_r . KV_r^T (Q_r kept in TMEM),
-//   * sends S_r to its peer through distributed shared memory and adds the
-//     peer's part (rank-0 part + rank-1 part in both CTAs: identical bits),
+//   * sends S_r to its peer through distributed shared memory (staged, then one
+//     bulk copy per warp) and adds the peer's part (rank-0 part + rank-1 part in
+//     both CTAs: identical bits),
 //   * runs the online softmax on the full scores (both CTAs, same m and l),
 //   * accumulates O[:, its 256 columns] += P . KV[:, its 256 columns], with P
-//     written back into the TMEM columns of S and used as the MMA A operand.
+//     written into TMEM and used as the MMA A operand.
 // Scheduling is persistent: the flattened sequence of 32-token tiles of all
 // sequences is cut into one contiguous range per cluster; each maximal piece of
 // a range inside one sequence (a segment) produces one normalised partial result
@@ -64,16 +65,9 @@ __device__ __forceinline__ uint32_t mapa_peer(uint32_t saddr, uint32_t peer) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(peer));
   return r;
 }
-// Asynchronous 16-byte store into the peer's shared memory that completes bytes on
-// the peer's mbarrier (transaction count), so no per-store release is needed.
-__device__ __forceinline__ void st_async_v4(uint32_t addr, uint4 v, uint32_t bar_cluster_addr) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
-               "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(bar_cluster_addr)
-               : "memory");
-}
-// One bulk copy of a whole staged tile from this CTA's shared memory into the
-// peer's, completing its bytes on the peer's mbarrier (the copy engine moves the
-// 16 KB; far fewer transactions than per-thread remote stores).
+// One bulk copy of a staged block from this CTA's shared memory into the peer's,
+// completing its bytes on the peer's mbarrier (the copy engine moves the block:
+// far fewer transactions than per-thread remote stores).
 __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
                                                   uint32_t bar_cluster) {
   asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -159,7 +153,7 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
       mbar_init(&s_free[u], 128);
       mbar_init(&p_full[u], 128);
       mbar_init(&o_done[u], 1);
-      mbar_init(&x_full[u], 1);   // one expect_tx arrive per phase + the peer's st.async bytes
+      mbar_init(&x_full[u], 1);   // one expect_tx arrive per phase + the bytes of the peer's bulk copies
       mbar_init(&x_empty[u], 1);  // one remote arrive from the peer
       mbar_init(&m_ready[u], 128);
       mbar_init(&l_ready[u], 128);
@@ -330,12 +324,15 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
             *reinterpret_cast<uint4*>(mine + 4 * ((c + h) & (TN / 4 - 1))) =
                 make_uint4(cur[4 * c], cur[4 * c + 1], cur[4 * c + 2], cur[4 * c + 3]);
           fence_proxy_async_smem();
-          named_bar_sync(1 + a, 128);
-          if (th == 0)
-            bulk_copy_to_peer(peer_xbuf + a * XBUF, smem_u32(sbuf + a * kH * TN), XBUF, peer_xfull + a * 8);
+          __syncwarp();
+          // each warp sends its own 32 rows as soon as they are staged
+          const int row0 = (warp & 3) * 32;
+          if (lane == 0)
+            bulk_copy_to_peer(peer_xbuf + a * XBUF + row0 * (TN * 4), smem_u32(sbuf + (a * kH + row0) * TN),
+                              XBUF / 4, peer_xfull + a * 8);
         }
         // add the peer's part: rank-0 part + rank-1 part in both CTAs (identical bits). The
-        // peer's st.async bytes complete on this local barrier, which makes them visible
+        // peer's copied bytes complete on this local barrier, which makes them visible
         // to a plain wait (same rule as a TMA load).
         if (fail(mbar_wait(&x_full[a], ph, abort_flag, p.status))) return;
         float s[TN];
