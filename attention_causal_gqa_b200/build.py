@@ -37,6 +37,20 @@ def _fingerprint() -> str:
     return h.hexdigest()
 
 
+# The file that defines each main kernel; with the shared headers and the arch
+# flags it fixes that kernel's code (profile figures are keyed by this).
+KERNEL_SOURCES = {"prefill_kernel": "prefill.cu", "decode_kernel": "decode.cu", "mla_kernel": "mla.cu"}
+
+
+def kernel_fingerprint(kernel: str) -> str:
+    h = hashlib.sha256()
+    for name in [KERNEL_SOURCES[kernel]] + HEADERS:
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    h.update(" ".join(ARCH).encode())
+    return h.hexdigest()[:16]
+
+
 def build(verbose: bool = False, force: bool = False) -> str:
     stamp = LIB + ".sha256"
     fp = _fingerprint()

@@ -40,6 +40,7 @@ __global__ void merge_kernel(const float* __restrict__ part_o, const float* __re
 #pragma unroll
   for (int i = 0; i < 16; ++i) acc[i] = 0.f;
   float wsum = 0.f;
+#pragma unroll 4
   for (int s = 0; s < ns; ++s) {
     const float w = __expf(pl[static_cast<size_t>(s) * H] - M);
     wsum += w;
@@ -80,6 +81,99 @@ cudaError_t launch_merge(const float* part_o, const float* part_lse, const int32
   merge_kernel<<<static_cast<int>(blocks), threads, 0, stream>>>(part_o, part_lse, seq_lens,
                                                                  static_cast<__nv_bfloat16*>(out), lse, B, H, D,
                                                                  n_splits, tokens_per_split);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ MLA
+__device__ __forceinline__ int mla_tiles_of(const int32_t* lens, int b, int T_max) {
+  const int L = min(max(__ldg(lens + b), 0), T_max);
+  return (L + kMlaTile - 1) / kMlaTile;
+}
+
+// One warp per (b, head). The MLA kernel cuts the N tiles of all sequences into
+// n_pairs contiguous ranges [N c / n_pairs, N (c + 1) / n_pairs), and cluster c
+// writes one partial result per sequence its range meets, at slot c + b. The
+// clusters meeting sequence b (tiles [s_b, e_b)) are those from the one holding
+// tile s_b to the one holding tile e_b - 1: cluster c holds tile x iff
+// floor(N c / P) <= x < floor(N (c + 1) / P), i.e. c = floor(((x + 1) P - 1) / N).
+// They are combined in cluster order (deterministic).
+__global__ void mla_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
+                                 const int32_t* __restrict__ seq_lens, __nv_bfloat16* __restrict__ out,
+                                 float* __restrict__ lse, int B, int H, int T_max, int n_pairs) {
+  constexpr int kDc = 512;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (gw >= B * H) return;
+  const int b = gw / H, h = gw % H;
+  long long N = 0, s_b = 0;
+  for (int i = lane; i < B; i += 32) {
+    const int n = mla_tiles_of(seq_lens, i, T_max);
+    N += n;
+    if (i < b) s_b += n;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    N += __shfl_xor_sync(0xffffffffu, N, o);
+    s_b += __shfl_xor_sync(0xffffffffu, s_b, o);
+  }
+  const long long e_b = s_b + mla_tiles_of(seq_lens, b, T_max);
+  const long long P = n_pairs;
+  int c0 = 0, c1 = -1;  // contributing clusters (none for an empty sequence)
+  if (e_b > s_b) {
+    c0 = static_cast<int>(((s_b + 1) * P - 1) / N);
+    c1 = static_cast<int>((e_b * P - 1) / N);
+  }
+  __nv_bfloat16* orow = out + static_cast<size_t>(gw) * kDc;
+  float M = -INFINITY;
+  for (int c = c0; c <= c1; ++c)
+    if (N * (c + 1) / P > N * c / P) M = fmaxf(M, part_lse[static_cast<size_t>(c + b) * H + h]);
+  if (!(M > -INFINITY)) {
+    for (int d = lane * 8; d < kDc; d += 256) *reinterpret_cast<uint4*>(orow + d) = make_uint4(0, 0, 0, 0);
+    if (lane == 0) lse[gw] = -INFINITY;
+    return;
+  }
+  float acc[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+  float wsum = 0.f;
+#pragma unroll 2
+  for (int c = c0; c <= c1; ++c) {
+    if (!(N * (c + 1) / P > N * c / P)) continue;  // an empty range writes nothing
+    const size_t slot = static_cast<size_t>(c + b);
+    const float w = __expf(part_lse[slot * H + h] - M);
+    wsum += w;
+    const float* po = part_o + (slot * H + h) * kDc;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int d = lane * 8 + i * 256;
+      const float4 v0 = *reinterpret_cast<const float4*>(po + d);
+      const float4 v1 = *reinterpret_cast<const float4*>(po + d + 4);
+      acc[8 * i + 0] += w * v0.x; acc[8 * i + 1] += w * v0.y; acc[8 * i + 2] += w * v0.z; acc[8 * i + 3] += w * v0.w;
+      acc[8 * i + 4] += w * v1.x; acc[8 * i + 5] += w * v1.y; acc[8 * i + 6] += w * v1.z; acc[8 * i + 7] += w * v1.w;
+    }
+  }
+  const float inv = 1.f / wsum;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int d = lane * 8 + i * 256;
+    uint4 u;
+    __nv_bfloat162 t;
+    t = __floats2bfloat162_rn(acc[8 * i] * inv, acc[8 * i + 1] * inv); u.x = *reinterpret_cast<const uint32_t*>(&t);
+    t = __floats2bfloat162_rn(acc[8 * i + 2] * inv, acc[8 * i + 3] * inv); u.y = *reinterpret_cast<const uint32_t*>(&t);
+    t = __floats2bfloat162_rn(acc[8 * i + 4] * inv, acc[8 * i + 5] * inv); u.z = *reinterpret_cast<const uint32_t*>(&t);
+    t = __floats2bfloat162_rn(acc[8 * i + 6] * inv, acc[8 * i + 7] * inv); u.w = *reinterpret_cast<const uint32_t*>(&t);
+    *reinterpret_cast<uint4*>(orow + d) = u;
+  }
+  if (lane == 0) lse[gw] = M + logf(wsum);
+}
+
+cudaError_t launch_mla_merge(const float* part_o, const float* part_lse, const int32_t* seq_lens, void* out,
+                             float* lse, int B, int H, int T_max, int n_pairs, cudaStream_t stream) {
+  const long long warps = static_cast<long long>(B) * H;
+  const int threads = 256;
+  const long long blocks = (warps * 32 + threads - 1) / threads;
+  mla_merge_kernel<<<static_cast<int>(blocks), threads, 0, stream>>>(
+      part_o, part_lse, seq_lens, static_cast<__nv_bfloat16*>(out), lse, B, H, T_max, n_pairs);
   return cudaGetLastError();
 }
 

@@ -21,7 +21,7 @@
 // Scheduling is persistent: the flattened sequence of 32-token tiles of all
 // sequences is cut into one contiguous range per cluster; each maximal piece of
 // a range inside one sequence (a segment) produces one normalised partial result
-// and its LSE, merged per sequence by mla_merge_kernel.
+// and its LSE, merged per sequence by mla_merge_kernel (merge.cu).
 //
 // Roles per CTA (352 threads): warpgroups 0 and 1 take the tiles in turn (tile k
 // goes to warpgroup k % 2, one thread per head): each reads its partial score tile
@@ -496,79 +496,6 @@ cudaError_t launch_mla(const MlaParams& p, const CUtensorMap& tmKV, const CUtens
   cudaError_t e = cudaFuncSetAttribute(mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   mla_kernel<<<2 * p.n_pairs, kMlaThreads, SMEM_BYTES, stream>>>(p, tmKV, tmPE);
-  return cudaGetLastError();
-}
-
-// One warp per (b, head): combine the partials of every cluster whose tile range meets
-// sequence b (slot = cluster + b), in cluster order.
-__global__ void mla_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
-                                 const int32_t* __restrict__ seq_lens, __nv_bfloat16* __restrict__ out,
-                                 float* __restrict__ lse, int B, int H, int T_max, int n_pairs) {
-  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (gw >= B * H) return;
-  const int b = gw / H, h = gw % H;
-  long long N = 0, s_b = 0;
-  for (int i = lane; i < B; i += 32) {
-    const int n = tiles_of(seq_lens, i, T_max);
-    N += n;
-    if (i < b) s_b += n;
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    N += __shfl_xor_sync(0xffffffffu, N, o);
-    s_b += __shfl_xor_sync(0xffffffffu, s_b, o);
-  }
-  const long long e_b = s_b + tiles_of(seq_lens, b, T_max);
-  __nv_bfloat16* orow = out + static_cast<size_t>(gw) * kDc;
-  float M = -INFINITY;
-  for (int c = 0; c < n_pairs; ++c) {
-    const long long lo = N * c / n_pairs, hi = N * (c + 1) / n_pairs;
-    if (hi > s_b && lo < e_b && hi > lo) M = fmaxf(M, part_lse[static_cast<size_t>(c + b) * H + h]);
-  }
-  if (!(M > -INFINITY)) {
-    for (int d = lane * 8; d < kDc; d += 256) *reinterpret_cast<uint4*>(orow + d) = make_uint4(0, 0, 0, 0);
-    if (lane == 0) lse[gw] = -INFINITY;
-    return;
-  }
-  float acc[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-  float wsum = 0.f;
-  for (int c = 0; c < n_pairs; ++c) {
-    const long long lo = N * c / n_pairs, hi = N * (c + 1) / n_pairs;
-    if (!(hi > s_b && lo < e_b && hi > lo)) continue;
-    const size_t slot = static_cast<size_t>(c + b);
-    const float w = __expf(part_lse[slot * H + h] - M);
-    wsum += w;
-    const float* po = part_o + (slot * H + h) * kDc;
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int d = lane * 8 + i * 256;
-      const float4 v0 = *reinterpret_cast<const float4*>(po + d);
-      const float4 v1 = *reinterpret_cast<const float4*>(po + d + 4);
-      acc[8 * i + 0] += w * v0.x; acc[8 * i + 1] += w * v0.y; acc[8 * i + 2] += w * v0.z; acc[8 * i + 3] += w * v0.w;
-      acc[8 * i + 4] += w * v1.x; acc[8 * i + 5] += w * v1.y; acc[8 * i + 6] += w * v1.z; acc[8 * i + 7] += w * v1.w;
-    }
-  }
-  const float inv = 1.f / wsum;
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const int d = lane * 8 + i * 256;
-    *reinterpret_cast<uint4*>(orow + d) =
-        make_uint4(pack_bf16x2(acc[8 * i] * inv, acc[8 * i + 1] * inv), pack_bf16x2(acc[8 * i + 2] * inv, acc[8 * i + 3] * inv),
-                   pack_bf16x2(acc[8 * i + 4] * inv, acc[8 * i + 5] * inv), pack_bf16x2(acc[8 * i + 6] * inv, acc[8 * i + 7] * inv));
-  }
-  if (lane == 0) lse[gw] = M + logf(wsum);
-}
-
-cudaError_t launch_mla_merge(const float* part_o, const float* part_lse, const int32_t* seq_lens, void* out,
-                             float* lse, int B, int H, int T_max, int n_pairs, cudaStream_t stream) {
-  const long long warps = static_cast<long long>(B) * H;
-  const int threads = 256;
-  const long long blocks = (warps * 32 + threads - 1) / threads;
-  mla_merge_kernel<<<static_cast<int>(blocks), threads, 0, stream>>>(
-      part_o, part_lse, seq_lens, static_cast<__nv_bfloat16*>(out), lse, B, H, T_max, n_pairs);
   return cudaGetLastError();
 }
 

@@ -98,8 +98,10 @@ class Clocks:
 
 
 # --------------------------------------------------------------- helpers
-def traffic_for(kernel: str, fingerprint: str):
-    """DRAM bytes per launch from a committed ncu summary, only if taken on this exact source."""
+def traffic_for(kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, only if taken on this kernel's exact source."""
+    from attention_causal_gqa_b200.build import kernel_fingerprint
+    fingerprint = kernel_fingerprint(kernel)
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(path):
         return None
@@ -277,7 +279,7 @@ def bench_prefill(args, world, dev, seed, flush, pk, pk_kind, fp):
     kern_avg = max_over_ranks(kern_ms / max(n_launch, 1), world)
     achieved = flops / (kern_avg * 1e-3) / 1e12
     roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-            "frac": achieved / pk["bf16_tflops"], "traffic": traffic_for("prefill_kernel", fp),
+            "frac": achieved / pk["bf16_tflops"], "traffic": traffic_for("prefill_kernel"),
             "kernel": "prefill_kernel", "kernel_ms": kern_avg, "peak_kind": f"{pk_kind} dense bf16 (burst)",
             "algorithmic": f"{flops:.4g} flop per launch = B*Hq*4*D*S(S+1)/2 (exact causal)"}
     res = {"value": value, "ms": ms, "roofline": roof, "flops": flops, "p": p}
@@ -339,7 +341,7 @@ def bench_decode(args, world, dev, seed, pk, pk_kind, fp):
            "ms_per_step": ms / args.steps, "kv_tokens": tokens, "kv_bytes_per_step": kv_bytes,
            "gpu_launches": 2 * args.steps, "l2": "inputs (4.4 GB) larger than L2",
            "roofline": {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                        "frac": ach / pk["hbm_gbs"], "traffic": traffic_for("decode_kernel", fp),
+                        "frac": ach / pk["hbm_gbs"], "traffic": traffic_for("decode_kernel"),
                         "kernel": "decode_kernel", "kernel_ms": k_avg, "peak_kind": f"{pk_kind} HBM copy",
                         "algorithmic": "4096 B per cached token (K+V, 8 heads x 128 x bf16)"}}
     del d, out, lse, ws
@@ -383,7 +385,7 @@ def bench_mla(args, world, dev, seed, pk, pk_kind, fp):
            "tflops": world * flops * args.steps / (ms * 1e-3) / 1e12, "gpu_launches": 2 * args.steps,
            "l2": "kv/pe caches (1.2 GB) larger than L2",
            "roofline": {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                        "frac": ach / pk["hbm_gbs"], "traffic": traffic_for("mla_kernel", fp),
+                        "frac": ach / pk["hbm_gbs"], "traffic": traffic_for("mla_kernel"),
                         "kernel": "mla_kernel", "kernel_ms": k_avg, "peak_kind": f"{pk_kind} HBM copy",
                         "algorithmic": "1152 B per cached token (kv 512 + pe 64, bf16)",
                         "tensor_tflops": flops / (k_avg * 1e-3) / 1e12,

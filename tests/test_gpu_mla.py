@@ -64,6 +64,27 @@ def test_mla_empty_sequence_and_poison_past_length():
 
 
 @cuda
+def test_mla_empty_sequences_inside_a_cluster_range():
+    """Empty sequences between long ones: the clusters whose tile ranges straddle them
+    write no partial for them, so the merge must not read those slots (the workspace is
+    poisoned with NaN first, so a stray read shows up)."""
+    from attention_causal_gqa_b200 import binding
+    from attention_causal_gqa_b200.synthetic import mla_inputs
+    lens = [2000, 0, 2000, 0, 0, 3000, 0]
+    d = mla_inputs(len(lens), 128, 512, 64, seq_lens=lens, T_max=3072, seed=21, device="cuda")
+    ws = torch.full((binding.mla_workspace_size(len(lens), 128, 512, 64, 3072),), 255, dtype=torch.uint8,
+                    device="cuda")
+    out, lse = binding.mla_decode(d["q_nope"], d["q_pe"], d["kv_cache"], d["pe_cache"], d["seq_lens"], SCALE,
+                                  workspace=ws)
+    torch.cuda.synchronize()
+    ro, rl = _oracle(d)
+    check(out, ro, lse, rl, what="mla empty inside")
+    for b, L in enumerate(lens):
+        if L == 0:
+            assert torch.all(out[b] == 0) and torch.all(torch.isneginf(lse[b]))
+
+
+@cuda
 def test_mla_full_size_sampled():
     from attention_causal_gqa_b200.synthetic import workload_inputs
     d = workload_inputs("mla_decode_b32_h128_dc512_dr64", device="cuda")
