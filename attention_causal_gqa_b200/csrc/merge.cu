@@ -39,24 +39,34 @@ __global__ void merge_kernel(const float* __restrict__ part_o, const float* __re
   float acc[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-  float wsum = 0.f;
-#pragma unroll 4
-  for (int s = 0; s < ns; ++s) {
-    const float w = __expf(pl[static_cast<size_t>(s) * H] - M);
-    wsum += w;
-    const float* po = part_o + ((static_cast<size_t>(b) * n_splits + s) * H + h) * D;
+  // Weights first, one split per lane, then broadcast: the partial loads of the
+  // accumulation loop depend on nothing but their address and can all be in flight.
+  float wpart = 0.f;
+  for (int s0 = 0; s0 < ns; s0 += 32) {
+    const int cnt = min(32, ns - s0);
+    const float w_lane = lane < cnt ? __expf(pl[static_cast<size_t>(s0 + lane) * H] - M) : 0.f;
+    wpart += w_lane;
+    const float* po0 = part_o + ((static_cast<size_t>(b) * n_splits + s0) * H + h) * D;
+#pragma unroll 8
+    for (int i = 0; i < cnt; ++i) {
+      const float w = __shfl_sync(0xffffffffu, w_lane, i);
+      const float* po = po0 + static_cast<size_t>(i) * H * D;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int d = lane * 4 + i * 128;
-      if (d < D) {
-        const float4 v = *reinterpret_cast<const float4*>(po + d);
-        acc[4 * i] += w * v.x;
-        acc[4 * i + 1] += w * v.y;
-        acc[4 * i + 2] += w * v.z;
-        acc[4 * i + 3] += w * v.w;
+      for (int q = 0; q < 4; ++q) {
+        const int d = lane * 4 + q * 128;
+        if (d < D) {
+          const float4 v = *reinterpret_cast<const float4*>(po + d);
+          acc[4 * q] += w * v.x;
+          acc[4 * q + 1] += w * v.y;
+          acc[4 * q + 2] += w * v.z;
+          acc[4 * q + 3] += w * v.w;
+        }
       }
     }
   }
+  float wsum = wpart;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
   const float inv = 1.f / wsum;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {

@@ -6,6 +6,8 @@
 // running phase), then rounded to fp32. Pairs are adjacent elements (2i, 2i+1):
 //   y[2i]   = x[2i] cos - x[2i+1] sin
 //   y[2i+1] = x[2i] sin + x[2i+1] cos
+#include <cmath>
+
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -13,16 +15,19 @@
 
 namespace attn {
 
-__global__ void rope_table_kernel(float2* __restrict__ cs, int S, int D, double theta) {
-  const int half = D / 2;
+// theta^(-2i/D) for every pair i, computed once on the host in fp64.
+struct RopeFreqs {
+  double inv[64];
+};
+
+__global__ void rope_table_kernel(float2* __restrict__ cs, int S, int half, const __grid_constant__ RopeFreqs f) {
   const long long n = static_cast<long long>(S) * half;
   for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < n;
        idx += static_cast<long long>(gridDim.x) * blockDim.x) {
     const int pos = static_cast<int>(idx / half);
-    const int i = static_cast<int>(idx % half);
-    const double inv_freq = pow(theta, -2.0 * i / D);
+    const int i = static_cast<int>(idx - static_cast<long long>(pos) * half);
     double s, c;
-    sincos(static_cast<double>(pos) * inv_freq, &s, &c);
+    sincos(static_cast<double>(pos) * f.inv[i], &s, &c);
     cs[idx] = make_float2(static_cast<float>(c), static_cast<float>(s));
   }
 }
@@ -137,8 +142,12 @@ static int grid_for(long long n, int threads) {
 }
 
 cudaError_t launch_rope_table(float2* cs, int S, int D, double theta, cudaStream_t stream) {
-  const long long n = static_cast<long long>(S) * (D / 2);
-  rope_table_kernel<<<grid_for(n, 256), 256, 0, stream>>>(cs, S, D, theta);
+  const int half = D / 2;
+  if (half < 1 || half > 64) return cudaErrorInvalidValue;
+  RopeFreqs f{};
+  for (int i = 0; i < half; ++i) f.inv[i] = std::pow(theta, -2.0 * i / D);
+  const long long n = static_cast<long long>(S) * half;
+  rope_table_kernel<<<grid_for(n, 256), 256, 0, stream>>>(cs, S, half, f);
   return cudaGetLastError();
 }
 

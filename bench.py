@@ -30,6 +30,7 @@ if ROOT not in sys.path:
 PREFILL = "gqa_prefill_b2_hq32_hkv8_s4096_d128"
 DECODE = "paged_decode_b64_hq32_hkv8_d128"
 MLA = "mla_decode_b32_h128_dc512_dr64"
+PREFILL_LONG = "gqa_prefill_b1_hq32_hkv8_s32768_d128"
 METRIC = "prefill attn TFLOP/s & decode KV-read GB/s, % of B200 roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -253,12 +254,13 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------- our arm
-def bench_prefill(args, world, dev, seed, flush, pk, pk_kind, fp):
+def bench_prefill(args, world, dev, seed, flush, pk, pk_kind, fp, name=None, with_e2e=True):
     import torch
     from attention_causal_gqa_b200 import binding as B_
     from attention_causal_gqa_b200.synthetic import WORKLOADS, workload_inputs
-    p = WORKLOADS[PREFILL].params
-    q, k, v = workload_inputs(PREFILL, seed=seed, device=dev)
+    name = name or PREFILL
+    p = WORKLOADS[name].params
+    q, k, v = workload_inputs(name, seed=seed, device=dev)
     out = torch.empty_like(q)
     lse = torch.empty((p["B"], p["Hq"], p["S"]), dtype=torch.float32, device=dev)
     ws = torch.empty(B_.prefill_workspace_size(p["B"], p["Hkv"], p["S"], p["D"]), dtype=torch.uint8, device=dev)
@@ -283,7 +285,7 @@ def bench_prefill(args, world, dev, seed, flush, pk, pk_kind, fp):
             "kernel": "prefill_kernel", "kernel_ms": kern_avg, "peak_kind": f"{pk_kind} dense bf16 (burst)",
             "algorithmic": f"{flops:.4g} flop per launch = B*Hq*4*D*S(S+1)/2 (exact causal)"}
     res = {"value": value, "ms": ms, "roofline": roof, "flops": flops, "p": p}
-    if not args.no_e2e:
+    if with_e2e and not args.no_e2e:
         # end to end through the public call: pinned host buffers, copies inside the timed region
         qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
         oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
@@ -420,6 +422,14 @@ def run_ours(args):
     clocks.start()
     pre = bench_prefill(args, world, dev, seed, flush, pk, pk_kind, fp) if do("prefill") else None
     sub = {}
+    if do("prefill") and not args.small:
+        # long-context prefill (inputs of 640 MB, larger than L2): call and kernel rates
+        lp = bench_prefill(args, world, dev, seed, flush, pk, pk_kind, fp, name=PREFILL_LONG, with_e2e=False)
+        lp["roofline"]["traffic"] = None  # the committed capture is of the S=4096 workload only
+        sub["prefill_long"] = {"workload": PREFILL_LONG, "value": lp["value"], "unit": "TFLOP/s",
+                               "ms_per_step": lp["ms"] / args.steps, "roofline": lp["roofline"],
+                               "gpu_launches": 4 * args.steps}
+        del lp
     if do("decode"):
         sub["decode"] = bench_decode(args, world, dev, seed, pk, pk_kind, fp)
     if do("mla"):
@@ -443,7 +453,7 @@ def run_ours(args):
                            "D": p["D"], "causal": True, "rope_theta": p["theta"],
                            "l2": "flushed (256 MB write) between steps", "parallelism": f"replicas x{world}"},
                 "roofline": pre["roofline"], "cpu_baseline": cpu, "e2e": pre.get("e2e"),
-                "gpu_launches": 3 * args.steps}
+                "gpu_launches": 4 * args.steps}
     else:
         w = sub[args.only]
         line = {"metric": METRIC, "value": w["value"], "unit": w["unit"], "n_gpus": world, "steps": args.steps,
