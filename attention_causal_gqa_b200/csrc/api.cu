@@ -240,9 +240,14 @@ int attn_prefill(const void* q, const void* k, const void* v, void* out, float* 
   p.pair_heads = (p.G % 2 == 0) ? 1 : 0;
   p.n_row_blocks = (S + 127) / 128;
   p.status = status;
-  const long long grid = p.pair_heads ? static_cast<long long>(B) * (Hq / 2) * p.n_row_blocks
-                                      : static_cast<long long>(B) * Hq * ((p.n_row_blocks + 1) / 2);
-  if (grid > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "grid too large");
+  const long long items = p.pair_heads ? static_cast<long long>(B) * (Hq / 2) * p.n_row_blocks
+                                       : static_cast<long long>(B) * Hq * ((p.n_row_blocks + 1) / 2);
+  if (items > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "too many work items");
+  p.n_items = static_cast<int>(items);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long grid = items < sms ? items : sms;  // one persistent CTA per SM
   prof_before(st);
   cudaError_t e = attn::launch_prefill(p, tmQ, tmK, tmV, D, f32, rope, static_cast<int>(grid), st);
   prof_after(st);

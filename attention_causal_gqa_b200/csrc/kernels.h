@@ -15,6 +15,7 @@ struct PrefillParams {
   float scale_log2;       // scale * log2(e)
   int pair_heads;         // 1: the CTA's two tiles are heads h, h+1; 0: row blocks r, r+1 of one head
   int n_row_blocks;       // ceil(S / 128)
+  int n_items;            // work items (pairs of query tiles); the grid walks them persistently
   int* status;            // device status word
 };
 

@@ -7,9 +7,12 @@
 // rescale of the output accumulator). Query head h reads KV head h / (Hq/Hkv)
 // (same page, GQA worked table).
 //
-// One CTA owns two 128-row query tiles that share one KV head: two heads of
+// A work item is two 128-row query tiles that share one KV head: two heads of
 // the same group over the same rows when the group size is even, otherwise two
-// consecutive row blocks of one head. Roles (320 threads):
+// consecutive row blocks of one head. The grid is persistent (one CTA per SM):
+// each CTA walks its share of the items, heaviest first, and the next item's Q
+// and K/V loads and first Q K^T overlap the current item's last blocks and
+// epilogue. Roles (320 threads):
 //   warps 0-3  softmax warpgroup of tile 0 (one thread per query row)
 //   warps 4-7  softmax warpgroup of tile 1
 //   warp  8    TMA producer: both Q tiles, then K/V tiles into a shared-memory ring
@@ -95,6 +98,51 @@ __device__ __forceinline__ void store32<float>(float* dst, const float* f) {
 // Pairs out of every 8 of a softmax row that take the FMA-pipe exp2 (blocks without masking).
 constexpr int kPolyPer8 = 2;
 
+// A work item: two 128-row query tiles that share one KV head.
+struct PrefillItem {
+  int b, h0, h1, r0_0, r0_1, n_kv0, n_kv1;
+};
+
+// Item w of the list ordered heaviest (last row blocks) first.
+template <int BN>
+__device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int w) {
+  constexpr int BM = 128;
+  PrefillItem it;
+  if (p.pair_heads) {
+    const int units = p.B * (p.Hq / 2);
+    const int rb = p.n_row_blocks - 1 - w / units;
+    const int bh = w % units;
+    it.b = bh / (p.Hq / 2);
+    it.h0 = 2 * (bh % (p.Hq / 2));
+    it.h1 = it.h0 + 1;
+    it.r0_0 = it.r0_1 = rb * BM;
+  } else {
+    const int units = p.B * p.Hq;
+    const int n_rp = (p.n_row_blocks + 1) / 2;
+    const int rp = n_rp - 1 - w / units;
+    const int bh = w % units;
+    it.b = bh / p.Hq;
+    it.h0 = it.h1 = bh % p.Hq;
+    it.r0_0 = 2 * rp * BM;
+    it.r0_1 = it.r0_0 + BM;
+  }
+  auto n_kv_for = [&](int r0) -> int {
+    if (r0 >= p.S) return 0;
+    if (!p.causal) return (p.S + BN - 1) / BN;
+    return (min(p.S, r0 + BM) - 1) / BN + 1;
+  };
+  it.n_kv0 = n_kv_for(it.r0_0);
+  it.n_kv1 = n_kv_for(it.r0_1);
+  return it;
+}
+
+// The persistent grid walks the heaviest-first list in snake order: in round r,
+// CTA c takes item r * G + c (r even) or r * G + G - 1 - c (r odd), so every CTA
+// gets a similar mix of long and short items.
+__device__ __forceinline__ int prefill_item_index(int r, int c, int G) {
+  return r * G + ((r & 1) ? (G - 1 - c) : c);
+}
+
 template <int D, int BN, int MODE>
 __global__ void __launch_bounds__(320, 1)
     prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
@@ -109,51 +157,28 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + Sh::NST * Sh::KV_SLOT);
   uint64_t* kv_full = bars;                     // [NST]
   uint64_t* kv_empty = bars + Sh::NST;          // [NST]
-  uint64_t* q_full = bars + 2 * Sh::NST;        // [1]
-  uint64_t* s_full = q_full + 1;                // [2]
+  uint64_t* q_full = bars + 2 * Sh::NST;        // [1] the item's Q tiles landed
+  uint64_t* q_empty = q_full + 1;               // [1] every Q K^T of the item has completed
+  uint64_t* s_full = q_empty + 1;               // [2]
   uint64_t* p_full = s_full + 2;                // [2]
   uint64_t* o_done = p_full + 2;                // [2]
-  uint64_t* mma_done = o_done + 2;              // [1]
+  uint64_t* o_free = o_done + 2;                // [2] the item's O_t has been read out
+  uint64_t* mma_done = o_free + 2;              // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---------------------------------------------------------------- work item
-  int b, h0, h1, r0_0, r0_1;
-  {
-    const int w = blockIdx.x;
-    if (p.pair_heads) {
-      const int units = p.B * (p.Hq / 2);
-      const int rb = p.n_row_blocks - 1 - w / units;  // heaviest (last) row blocks first
-      const int bh = w % units;
-      b = bh / (p.Hq / 2);
-      h0 = 2 * (bh % (p.Hq / 2));
-      h1 = h0 + 1;
-      r0_0 = r0_1 = rb * Sh::BM;
-    } else {
-      const int units = p.B * p.Hq;
-      const int n_rp = (p.n_row_blocks + 1) / 2;
-      const int rp = n_rp - 1 - w / units;
-      const int bh = w % units;
-      b = bh / p.Hq;
-      h0 = h1 = bh % p.Hq;
-      r0_0 = 2 * rp * Sh::BM;
-      r0_1 = r0_0 + Sh::BM;
+  const int G = gridDim.x;
+  const int n_rounds = (p.n_items + G - 1) / G;
+  // Calls fn(item) for this CTA's items in order; every role walks the same list.
+  auto for_each_item = [&](auto&& fn) {
+    for (int r = 0; r < n_rounds; ++r) {
+      const int w = prefill_item_index(r, blockIdx.x, G);
+      if (w < p.n_items && !fn(prefill_item<BN>(p, w))) return;
     }
-  }
-  const int kvh = h0 / p.G;
-  const int n_kv_all = (p.S + BN - 1) / BN;
-  auto n_kv_for = [&](int r0) -> int {
-    if (r0 >= p.S) return 0;
-    if (!p.causal) return n_kv_all;
-    const int last = min(p.S, r0 + Sh::BM) - 1;
-    return last / BN + 1;
   };
-  const int n_kv0 = n_kv_for(r0_0);
-  const int n_kv1 = n_kv_for(r0_1);
-  const int n_max = max(n_kv0, n_kv1);
 
   // -------------------------------------------------------------------- setup
   if (threadIdx.x == 0) {
@@ -162,10 +187,12 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&kv_empty[i], 1);
     }
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
       mbar_init(&p_full[t], 128);
       mbar_init(&o_done[t], 1);
+      mbar_init(&o_free[t], 128);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -186,33 +213,41 @@ __global__ void __launch_bounds__(320, 1)
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      // Both Q tiles (rows past S arrive as zeros), already in operand form.
-      mbar_arrive_expect_tx(q_full, 2 * NP * Sh::Q_PART);
-      for (int t = 0; t < 2; ++t) {
-        const int zq = b * p.Hq + (t ? h1 : h0), r0 = t ? r0_1 : r0_0;
-#pragma unroll
-        for (int u = 0; u < NP; ++u)
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(sQ + (t * NP + u) * Sh::Q_PART + c * Sh::Q_BOX, &tmQ, q_full, c * 64, r0,
-                        zq + u * p.B * p.Hq);
-      }
-      const int zc = b * p.Hkv + kvh;
       const int zlo = p.B * p.Hkv;  // the lo parts follow the hi parts in the split layout
-      for (int i = 0; i < 2 * n_max; ++i) {
-        const int j = i >> 1;
-        const int s = i % Sh::NST;
-        const uint32_t ph = (i / Sh::NST) & 1;
-        if (!mbar_wait(&kv_empty[s], ph ^ 1, abort_flag, p.status)) break;
-        uint8_t* dst = sKV + s * Sh::KV_SLOT;
-        mbar_arrive_expect_tx(&kv_full[s], Sh::KV_SLOT);
-        const CUtensorMap* map = (i & 1) ? &tmV : &tmK;
+      int kv_i = 0, nq = 0;           // position in the K/V ring sequence; items so far
+      for_each_item([&](const PrefillItem& it) -> bool {
+        // Both Q tiles (rows past S arrive as zeros), already in operand form, once the
+        // previous item's Q K^T products have all completed.
+        if (nq > 0 && !mbar_wait(q_empty, (nq - 1) & 1, abort_flag, p.status)) return false;
+        ++nq;
+        mbar_arrive_expect_tx(q_full, 2 * NP * Sh::Q_PART);
+        for (int t = 0; t < 2; ++t) {
+          const int zq = it.b * p.Hq + (t ? it.h1 : it.h0), r0 = t ? it.r0_1 : it.r0_0;
 #pragma unroll
-        for (int u = 0; u < NP; ++u)
+          for (int u = 0; u < NP; ++u)
 #pragma unroll
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(dst + u * Sh::KV_PART + c * Sh::KV_BOX, map, &kv_full[s], c * 64, j * BN, zc + u * zlo);
-      }
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_3d(sQ + (t * NP + u) * Sh::Q_PART + c * Sh::Q_BOX, &tmQ, q_full, c * 64, r0,
+                          zq + u * p.B * p.Hq);
+        }
+        const int zc = it.b * p.Hkv + it.h0 / p.G;
+        const int n_max = max(it.n_kv0, it.n_kv1);
+        for (int i = 0; i < 2 * n_max; ++i, ++kv_i) {  // K_j at 2j, V_j at 2j + 1
+          const int j = i >> 1;
+          const int s = kv_i % Sh::NST;
+          const uint32_t ph = (kv_i / Sh::NST) & 1;
+          if (!mbar_wait(&kv_empty[s], ph ^ 1, abort_flag, p.status)) return false;
+          uint8_t* dst = sKV + s * Sh::KV_SLOT;
+          mbar_arrive_expect_tx(&kv_full[s], Sh::KV_SLOT);
+          const CUtensorMap* map = (i & 1) ? &tmV : &tmK;
+#pragma unroll
+          for (int u = 0; u < NP; ++u)
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_3d(dst + u * Sh::KV_PART + c * Sh::KV_BOX, map, &kv_full[s], c * 64, j * BN, zc + u * zlo);
+        }
+        return true;
+      });
     }
   } else if (warp == 9) {
     // -------------------------------------------------- MMA issuer (whole warp)
@@ -221,8 +256,7 @@ __global__ void __launch_bounds__(320, 1)
       constexpr uint32_t idesc_pv = idesc_f32acc(1, 128, D, false, true);
       // (A part, B part) products: hi*hi, plus hi*lo and lo*hi for split operands
       constexpr int NPROD = Sh::SPLIT ? 3 : 1;
-      const int n_kv[2] = {n_kv0, n_kv1};
-      bool ok = mbar_wait_warp(q_full, 0, abort_flag, p.status);
+      bool ok = true;
       // Descriptor words: the high word is shared by every operand; the low word
       // carries the start address (>> 4), advanced by compile-time offsets below.
       constexpr uint32_t HI = sdesc_hi_sw128(1024);
@@ -259,33 +293,43 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
       };
-      if (ok && n_max > 0) {
-        // K_0 sits in ring slot 0
-        ok = mbar_wait_warp(&kv_full[0], 0, abort_flag, p.status);
-        if (ok) {
-          tc_fence_after();
-          for (int t = 0; t < 2; ++t)
-            if (n_kv[t] > 0) {
-              issue_qk(t, 0);
-              umma_commit_warp(&s_full[t]);
-            }
-          umma_commit_warp(&kv_empty[0]);
-        }
+      int kv_i = 0, nq = 0;    // position in the K/V ring sequence; items so far
+      int g[2] = {0, 0};       // blocks of tile t processed in earlier items (barrier phases)
+      int ne[2] = {0, 0};      // earlier items with work for tile t (o_free phases)
+      for_each_item([&](const PrefillItem& it) -> bool {
+        const int n_kv[2] = {it.n_kv0, it.n_kv1};
+        const int n_max = max(n_kv[0], n_kv[1]);
+        if (!(ok = mbar_wait_warp(q_full, nq & 1, abort_flag, p.status))) return false;
+        ++nq;
+        auto slot_of = [&](int i) { return (kv_i + i) % Sh::NST; };
+        auto par_of = [&](int i) -> uint32_t { return ((kv_i + i) / Sh::NST) & 1; };
+        // K_0; S_t(0) overwrites the columns that held P_t of the previous item, whose
+        // P V was issued earlier on the same in-order pipe.
+        if (!(ok = mbar_wait_warp(&kv_full[slot_of(0)], par_of(0), abort_flag, p.status))) return false;
+        tc_fence_after();
+        for (int t = 0; t < 2; ++t)
+          if (n_kv[t] > 0) {
+            issue_qk(t, slot_of(0));
+            umma_commit_warp(&s_full[t]);
+          }
+        umma_commit_warp(&kv_empty[slot_of(0)]);
         for (int j = 0; ok && j < n_max; ++j) {
-          const int iV = 2 * j + 1, sV = iV % Sh::NST;
-          const int iK = 2 * j + 2, sK = iK % Sh::NST;
-          if (!mbar_wait_warp(&kv_full[sV], (iV / Sh::NST) & 1, abort_flag, p.status)) { ok = false; break; }
+          const int sV = slot_of(2 * j + 1), sK = slot_of(2 * j + 2);
+          if (!(ok = mbar_wait_warp(&kv_full[sV], par_of(2 * j + 1), abort_flag, p.status))) break;
           bool k_ready = false;
           for (int t = 0; t < 2 && ok; ++t) {
             if (j >= n_kv[t]) continue;
-            if (!mbar_wait_warp(&p_full[t], j & 1, abort_flag, p.status)) { ok = false; break; }
+            if (!(ok = mbar_wait_warp(&p_full[t], (g[t] + j) & 1, abort_flag, p.status))) break;
+            // the item's first P V overwrites O_t: the previous item's result must be out
+            if (j == 0 && ne[t] > 0 && !(ok = mbar_wait_warp(&o_free[t], (ne[t] - 1) & 1, abort_flag, p.status)))
+              break;
             tc_fence_after();
             // P_t V_j first: it reads P_t from the columns that Q_t K_{j+1}^T overwrites.
             issue_pv(t, sV, j > 0);
             umma_commit_warp(&o_done[t]);
             if (j + 1 < n_kv[t]) {
               if (!k_ready) {
-                if (!mbar_wait_warp(&kv_full[sK], (iK / Sh::NST) & 1, abort_flag, p.status)) { ok = false; break; }
+                if (!(ok = mbar_wait_warp(&kv_full[sK], par_of(2 * j + 2), abort_flag, p.status))) break;
                 tc_fence_after();
                 k_ready = true;
               }
@@ -297,7 +341,15 @@ __global__ void __launch_bounds__(320, 1)
           umma_commit_warp(&kv_empty[sV]);
           if (k_ready) umma_commit_warp(&kv_empty[sK]);
         }
-      }
+        if (!ok) return false;
+        umma_commit_warp(q_empty);  // every Q K^T of the item has been issued
+        for (int t = 0; t < 2; ++t) {
+          g[t] += n_kv[t];
+          ne[t] += n_kv[t] > 0;
+        }
+        kv_i += 2 * n_max;
+        return true;
+      });
       // drain: every MMA issued above has completed once this barrier flips
       umma_commit_warp(mma_done);
       mbar_wait_warp(mma_done, 0, abort_flag, p.status);
@@ -307,21 +359,24 @@ __global__ void __launch_bounds__(320, 1)
     const int t = warp >> 2;
     const int wr = warp & 3;
     const int row = wr * 32 + lane;  // TMEM lane == query row within the tile
-    const int h = t ? h1 : h0;
-    const int r0 = t ? r0_1 : r0_0;
-    const int n_kv = t ? n_kv1 : n_kv0;
+    const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(wr * 32) << 16);
+    const float sl2 = p.scale_log2;
+    bool alive = true;
+    int g = 0;  // blocks of this tile processed in earlier items (barrier phases)
+    for_each_item([&](const PrefillItem& it) -> bool {
+    const int h = t ? it.h1 : it.h0;
+    const int r0 = t ? it.r0_1 : it.r0_0;
+    const int n_kv = t ? it.n_kv1 : it.n_kv0;
+    const int b = it.b;
+    if (n_kv == 0) return true;
     const int grow = r0 + row;
     const bool row_valid = grow < p.S;
-    const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(wr * 32) << 16);
-
     float m_run = -INFINITY;
     float l_run = 0.f;
-    const float sl2 = p.scale_log2;
     const int limit = p.causal ? min(grow, p.S - 1) : p.S - 1;  // last key this row may see
-    bool alive = true;
 
     for (int j = 0; j < n_kv && alive; ++j) {
-      bool ok = mbar_wait(&s_full[t], j & 1, abort_flag, p.status);
+      bool ok = mbar_wait(&s_full[t], (g + j) & 1, abort_flag, p.status);
       if (__any_sync(0xffffffffu, !ok)) { alive = false; break; }
       tc_fence_after();
       // The whole S row comes to registers with back-to-back TMEM loads and one wait.
@@ -434,10 +489,11 @@ __global__ void __launch_bounds__(320, 1)
       mbar_arrive(&p_full[t]);
     }
 
-    // Epilogue: O / l and LSE = (m + log2 l) * ln 2.
-    if (alive && n_kv > 0) {
-      bool ok = mbar_wait(&o_done[t], (n_kv - 1) & 1, abort_flag, p.status);
-      if (!__any_sync(0xffffffffu, !ok)) {
+    // Epilogue: O / l and LSE = (m + log2 l) * ln 2; then O_t is free for the next item.
+    if (alive) {
+      bool ok = mbar_wait(&o_done[t], (g + n_kv - 1) & 1, abort_flag, p.status);
+      if (__any_sync(0xffffffffu, !ok)) alive = false;
+      if (alive) {
         tc_fence_after();
         const float inv_l = 1.f / l_run;
         TIn* orow = reinterpret_cast<TIn*>(p.out) + ((static_cast<size_t>(b) * p.Hq + h) * p.S + grow) * D;
@@ -455,8 +511,13 @@ __global__ void __launch_bounds__(320, 1)
         }
         if (row_valid)
           p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.S + grow] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+        tc_fence_before();
+        mbar_arrive(&o_free[t]);
       }
     }
+    g += n_kv;
+    return alive;
+    });
   }
 
   tc_fence_before();
