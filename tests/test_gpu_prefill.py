@@ -39,6 +39,10 @@ def _inputs(B, Hq, Hkv, S, D, dtype="bf16", std=1.0, seed=0):
         (1, 4, 4, 160, 64, "f32", False, 0.0),     # fp32, no RoPE, non-causal, ragged
         (3, 16, 8, 640, 128, "bf16", True, 1e6),   # G=2, theta 1e6, several tiles
         (1, 2, 1, 1000, 128, "bf16", True, 1e4),   # long row pair, many KV tiles
+        (1, 4, 2, 333, 128, "bf16", True, 0.0),    # bf16 without RoPE (Q read straight from q), ragged
+        (2, 8, 8, 200, 64, "bf16", False, 0.0),    # bf16 without RoPE, D=64, non-causal
+        (2, 32, 8, 768, 128, "bf16", True, 1e4),   # 192 work items: CTAs of the persistent grid take two
+        (2, 32, 8, 640, 64, "bf16", False, 0.0),   # 160 work items, no RoPE, D=64, non-causal
     ],
 )
 def test_prefill_matches_oracle_small(B, Hq, Hkv, S, D, dtype, causal, theta):
