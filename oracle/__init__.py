@@ -6,6 +6,7 @@ links it, and it shares no code with the CUDA path.
 """
 from .attention import (  # noqa: F401
     apply_rope,
+    chunk_prefill_ref,
     decode_paged_ref,
     gather_pages,
     lse_merge,
@@ -14,5 +15,6 @@ from .attention import (  # noqa: F401
     online_softmax_merge,
     prefill_ref,
     rope_cache,
+    to_bf16,
     two_pass_softmax_rows,
 )

@@ -285,6 +285,72 @@ def decode_paged_ref(q, k_pages, v_pages, block_table, seq_lens, scale: float | 
     return o, lse
 
 
+# ------------------------------------------- chunked prefill into the paged cache
+def to_bf16(x):
+    """Round values to bfloat16 (round to nearest, ties to even) and return them as
+    float64: the precision a bf16 KV cache stores."""
+    x32 = np.asarray(x, dtype=np.float32)
+    b = x32.view(np.uint32).astype(np.uint64)
+    lsb = (b >> 16) & 1
+    r = ((b + 0x7FFF + lsb) >> 16) << 16
+    return r.astype(np.uint32).view(np.float32).astype(F64)
+
+
+def chunk_prefill_ref(q, k_new, v_new, k_pages, v_pages, block_table, cache_lens, rope_theta: float = 10000.0,
+                      scale: float | None = None, page_size: int = 16, store=to_bf16):
+    """Append a chunk of new tokens to a paged KV cache and attend over the whole cache.
+
+    "From 32K to 256K: DeepSeek long-context", chapter 1 (key architecture path: a
+    streaming KV cache for incremental processing, long sequences cut into chunks, a
+    PagedAttention variant); "attention study note", section "Page Attention" (pages
+    reached through a per-sequence block table).
+
+    q: [B, Hq, S_new, D]; k_new, v_new: [B, Hkv, S_new, D], not rotated. New token i of
+    sequence b sits at position cache_lens[b] + i. k_pages, v_pages: [num_pages,
+    page_size, Hkv, D]; the first cache_lens[b] tokens of sequence b are already there
+    (keys rotated). block_table: [B, max_pages].
+
+    Steps: rotate the new keys at their positions and write them and the new values
+    into their pages with ``store`` (the cache's precision, bf16); rotate the queries at
+    the same positions (float64); query i attends the stored keys t <= cache_lens[b] + i
+    (the causal mask aligned to the end of the cache), two-pass softmax, O = P V.
+    Returns (k_pages', v_pages', o [B, Hq, S_new, D], lse [B, Hq, S_new]).
+    """
+    q = np.asarray(q, dtype=F64)
+    k_new = np.asarray(k_new, dtype=F64)
+    v_new = np.asarray(v_new, dtype=F64)
+    kp = np.array(k_pages, dtype=F64)
+    vp = np.array(v_pages, dtype=F64)
+    B, Hq, S_new, D = q.shape
+    Hkv = k_new.shape[1]
+    G = Hq // Hkv
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(D)
+    use_rope = rope_theta and rope_theta > 0
+    o = np.zeros((B, Hq, S_new, D))
+    lse = np.zeros((B, Hq, S_new))
+    for b in range(B):
+        L = int(cache_lens[b])
+        pos = L + np.arange(S_new)
+        table = np.asarray(block_table[b])
+        for kvh in range(Hkv):
+            kr = apply_rope(k_new[b, kvh], rope_theta, positions=pos) if use_rope else k_new[b, kvh]
+            kp[table[pos // page_size], pos % page_size, kvh] = store(kr)
+            vp[table[pos // page_size], pos % page_size, kvh] = store(v_new[b, kvh])
+        kk = gather_pages(kp, table, L + S_new, page_size)
+        vv = gather_pages(vp, table, L + S_new, page_size)
+        for h in range(Hq):
+            kvh = h // G
+            qr = apply_rope(q[b, h], rope_theta, positions=pos) if use_rope else q[b, h]
+            s = scale * (qr @ kk[:, kvh, :].T)
+            jj = np.arange(L + S_new)[None, :]
+            s = np.where(jj > pos[:, None], -np.inf, s)
+            p, l_ = two_pass_softmax_rows(s)
+            o[b, h] = p @ vv[:, kvh, :]
+            lse[b, h] = l_
+    return kp, vp, o, lse
+
+
 # ------------------------------------------------------------------ MLA decode
 def mla_decode_ref(q_nope, q_pe, kv_cache, pe_cache, seq_lens, scale: float, pairs=None):
     """DeepSeek MLA absorbed decode (einsum vs hand-optimised page, absorbed form).

@@ -395,3 +395,102 @@ def test_mla_ignores_cache_beyond_length():
     pe[:, 6:] = 1e6
     o2, l2 = mla_decode_ref(qn, qp, kv, pe, np.array([6]), 0.5)
     assert np.array_equal(o, o2) and np.array_equal(l, l2)
+
+
+# ------------------------------------------- chunked prefill into the paged cache
+def _paged_setup(rng, B, Hkv, D, cache_lens, S_new, page_size=16, extra=3):
+    """A cache whose pages sit in a random physical order, filled with (rotated, stored)
+    keys for the cached prefix and garbage everywhere else."""
+    from oracle import to_bf16
+    need = [(L + S_new + page_size - 1) // page_size for L in cache_lens]
+    n_pages = sum(need) + extra
+    perm = rng.permutation(n_pages)
+    max_pages = max(need)
+    table = np.zeros((B, max_pages), dtype=np.int64)
+    off = 0
+    for b, n in enumerate(need):
+        table[b, :n] = perm[off:off + n]
+        off += n
+    kp = to_bf16(rng.standard_normal((n_pages, page_size, Hkv, D)))
+    vp = to_bf16(rng.standard_normal((n_pages, page_size, Hkv, D)))
+    return kp, vp, table
+
+
+def test_to_bf16_matches_torch_and_ties_to_even():
+    import torch
+    from oracle import to_bf16
+    x = np.array([1.0, 1.0 + 2.0**-8, 1.0 + 3 * 2.0**-8, -2.5, 1e-30, 3.0e38])
+    r = to_bf16(x)
+    assert r[0] == 1.0 and r[1] == 1.0 and r[2] == 1.0 + 2.0**-6 and r[3] == -2.5
+    y = np.random.default_rng(3).standard_normal(10000) * 7
+    ref = torch.tensor(y, dtype=torch.float32).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(to_bf16(y), ref)
+
+
+def test_chunk_prefill_empty_cache_unrounded_equals_prefill():
+    from oracle import chunk_prefill_ref, prefill_ref
+    rng = np.random.default_rng(40)
+    B, Hq, Hkv, S, D = 2, 4, 2, 37, 16
+    q = rng.standard_normal((B, Hq, S, D))
+    k = rng.standard_normal((B, Hkv, S, D))
+    v = rng.standard_normal((B, Hkv, S, D))
+    kp, vp, table = _paged_setup(rng, B, Hkv, D, [0, 0], S)
+    _, _, o, lse = chunk_prefill_ref(q, k, v, kp, vp, table, [0, 0], rope_theta=1e4, store=lambda x: x)
+    ro, rl = prefill_ref(q, k, v, causal=True, rope_theta=1e4)
+    assert np.allclose(o, ro, atol=1e-12) and np.allclose(lse, rl, atol=1e-12)
+
+
+def test_chunk_prefill_two_chunks_equal_one():
+    from oracle import chunk_prefill_ref
+    rng = np.random.default_rng(41)
+    B, Hq, Hkv, D = 2, 6, 2, 16
+    cache = [5, 40]
+    n1, n2 = 9, 14
+    q = rng.standard_normal((B, Hq, n1 + n2, D))
+    k = rng.standard_normal((B, Hkv, n1 + n2, D))
+    v = rng.standard_normal((B, Hkv, n1 + n2, D))
+    kp, vp, table = _paged_setup(rng, B, Hkv, D, cache, n1 + n2)
+    kp1, vp1, o1, l1 = chunk_prefill_ref(q, k, v, kp, vp, table, cache)
+    kpa, vpa, oa, la = chunk_prefill_ref(q[:, :, :n1], k[:, :, :n1], v[:, :, :n1], kp, vp, table, cache)
+    kpb, vpb, ob, lb = chunk_prefill_ref(q[:, :, n1:], k[:, :, n1:], v[:, :, n1:], kpa, vpa, table,
+                                         [c + n1 for c in cache])
+    assert np.array_equal(kpb, kp1) and np.array_equal(vpb, vp1)
+    assert np.allclose(np.concatenate([oa, ob], axis=2), o1, atol=1e-12)
+    assert np.allclose(np.concatenate([la, lb], axis=2), l1, atol=1e-12)
+
+
+def test_chunk_prefill_appends_rotated_keys_at_their_pages():
+    from oracle import apply_rope, chunk_prefill_ref, gather_pages, to_bf16
+    rng = np.random.default_rng(42)
+    B, Hq, Hkv, D, S_new = 2, 2, 2, 8, 20
+    cache = [3, 17]
+    q = rng.standard_normal((B, Hq, S_new, D))
+    k = rng.standard_normal((B, Hkv, S_new, D))
+    v = rng.standard_normal((B, Hkv, S_new, D))
+    kp, vp, table = _paged_setup(rng, B, Hkv, D, cache, S_new)
+    kp2, vp2, _, _ = chunk_prefill_ref(q, k, v, kp, vp, table, cache, rope_theta=500.0)
+    for b in range(B):
+        L = cache[b]
+        got_k = gather_pages(kp2, table[b], L + S_new, 16)
+        got_v = gather_pages(vp2, table[b], L + S_new, 16)
+        assert np.array_equal(got_k[:L], gather_pages(kp, table[b], L, 16))  # the cached prefix is untouched
+        for kvh in range(Hkv):
+            rot = apply_rope(k[b, kvh], 500.0, positions=L + np.arange(S_new))
+            assert np.array_equal(got_k[L:, kvh], to_bf16(rot))
+            assert np.array_equal(got_v[L:, kvh], to_bf16(v[b, kvh]))
+
+
+def test_chunk_prefill_last_row_equals_decode_over_the_updated_cache():
+    from oracle import apply_rope, chunk_prefill_ref, decode_paged_ref
+    rng = np.random.default_rng(43)
+    B, Hq, Hkv, D, S_new = 3, 8, 2, 16, 7
+    cache = [0, 30, 64]
+    q = rng.standard_normal((B, Hq, S_new, D))
+    k = rng.standard_normal((B, Hkv, S_new, D))
+    v = rng.standard_normal((B, Hkv, S_new, D))
+    kp, vp, table = _paged_setup(rng, B, Hkv, D, cache, S_new)
+    kp2, vp2, o, lse = chunk_prefill_ref(q, k, v, kp, vp, table, cache)
+    q_last = np.stack([apply_rope(q[b, :, -1], 1e4, positions=np.full(Hq, cache[b] + S_new - 1))
+                       for b in range(B)])
+    do, dl = decode_paged_ref(q_last, kp2, vp2, table, [c + S_new for c in cache])
+    assert np.allclose(o[:, :, -1], do, atol=1e-12) and np.allclose(lse[:, :, -1], dl, atol=1e-12)
