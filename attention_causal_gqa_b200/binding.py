@@ -55,6 +55,10 @@ def _load() -> ctypes.CDLL:
     lib.attn_decode_paged_workspace_size.argtypes = [i32] * 5
     lib.attn_decode_paged.restype = i32
     lib.attn_decode_paged.argtypes = [vp] * 7 + [i32] * 7 + [f32, i32, vp, sz, vp]
+    lib.attn_prefill_chunk_workspace_size.restype = sz
+    lib.attn_prefill_chunk_workspace_size.argtypes = [i32] * 5
+    lib.attn_prefill_chunk.restype = i32
+    lib.attn_prefill_chunk.argtypes = [vp] * 9 + [i32] * 9 + [f32, f32, vp, sz, vp]
     lib.mla_decode_workspace_size.restype = sz
     lib.mla_decode_workspace_size.argtypes = [i32] * 5
     lib.mla_decode.restype = i32
@@ -154,6 +158,35 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale=None, ou
     rc = lib.attn_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens), _ptr(out),
                                _ptr(lse), B, Hq, Hkv, D, ps, maxp, P, float(scale or 0.0), ATTN_DTYPE_BF16, _ptr(ws),
                                ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc)
+    return out, lse
+
+
+# -------------------------------------------- chunked prefill into the paged cache
+def prefill_chunk_workspace_size(B, Hkv, S_new, max_cache_len, D) -> int:
+    return int(lib.attn_prefill_chunk_workspace_size(B, Hkv, S_new, max_cache_len, D))
+
+
+def attn_prefill_chunk(q, k, v, k_pages, v_pages, block_table, cache_lens, max_cache_len, rope_theta=10000.0,
+                       scale=None, out=None, lse=None, workspace=None, stream=None):
+    """Append a chunk of new tokens to the paged KV cache and attend over the whole cache.
+    q [B,Hq,S_new,D], k/v [B,Hkv,S_new,D] bf16 (not rotated); k/v_pages [P,16,Hkv,D] bf16, updated in
+    place; block_table [B,maxp] int32; cache_lens [B] int32 (tokens already cached, each <= max_cache_len).
+    Returns (out [B,Hq,S_new,D] bf16, lse [B,Hq,S_new] fp32)."""
+    _need_cuda(q, k, v, k_pages, v_pages, block_table, cache_lens)
+    B, Hq, S_new, D = q.shape
+    Hkv = k.shape[1]
+    P, ps, _, _ = k_pages.shape
+    maxp = block_table.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, S_new), dtype=torch.float32, device=q.device)
+    ws = _workspace(prefill_chunk_workspace_size(B, Hkv, S_new, int(max_cache_len), D), q.device, workspace)
+    rc = lib.attn_prefill_chunk(_ptr(q), _ptr(k), _ptr(v), _ptr(k_pages), _ptr(v_pages), _ptr(block_table),
+                                _ptr(cache_lens), _ptr(out), _ptr(lse), B, Hq, Hkv, S_new, D, ps, maxp, P,
+                                int(max_cache_len), float(rope_theta if rope_theta else 0.0), float(scale or 0.0),
+                                _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
     _check(rc)
     return out, lse
 

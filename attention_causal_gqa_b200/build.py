@@ -14,7 +14,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libattn_b200.so")
-SOURCES = ["api.cu", "rope.cu", "prefill.cu", "decode.cu", "mla.cu", "merge.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "rope.cu", "prefill.cu", "decode.cu", "mla.cu", "merge.cu", "chunk.cu", "noalloc.cu"]
 HEADERS = ["sm100.cuh", "kernels.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

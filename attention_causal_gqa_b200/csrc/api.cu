@@ -255,6 +255,113 @@ int attn_prefill(const void* q, const void* k, const void* v, void* out, float* 
   return ok();
 }
 
+// Chunked-prefill workspace: [status | cos/sin table [Sk_max, D/2] | keys fp16
+// [B*Hkv, Sk_max, D] | values bf16 [B*Hkv, Sk_max, D]], Sk_max = max_cache_len + S_new.
+size_t attn_prefill_chunk_workspace_size(int B, int Hkv, int S_new, int max_cache_len, int D) {
+  if (B <= 0 || Hkv <= 0 || S_new <= 0 || D <= 0 || max_cache_len < 0) return kHeader;
+  const size_t sk = static_cast<size_t>(max_cache_len) + S_new;
+  const size_t table = round_up(sk * (D / 2) * sizeof(float2), 256);
+  const size_t op = round_up(static_cast<size_t>(B) * Hkv * sk * D * 2, 256);
+  return kHeader + table + 2 * op;
+}
+
+int attn_prefill_chunk(const void* q, const void* k, const void* v, void* k_pages, void* v_pages,
+                       const int32_t* block_table, const int32_t* cache_lens, void* out, float* lse, int B, int Hq,
+                       int Hkv, int S_new, int D, int page_size, int max_pages_per_seq, int num_pages,
+                       int max_cache_len, float rope_theta, float scale, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  if (!q || !k || !v || !k_pages || !v_pages || !block_table || !cache_lens || !out || !lse || !workspace)
+    return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || S_new <= 0 || D <= 0 || max_pages_per_seq <= 0 || num_pages <= 0 ||
+      max_cache_len < 0)
+    return fail(ATTN_ERR_INVALID_ARG, "sizes must be positive (B=%d Hq=%d Hkv=%d S_new=%d D=%d pages=%d/%d, max_cache_len=%d)",
+                B, Hq, Hkv, S_new, D, max_pages_per_seq, num_pages, max_cache_len);
+  if (Hq % Hkv != 0) return fail(ATTN_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+  if (D != 64 && D != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d unsupported", D);
+  if (page_size != 16) return fail(ATTN_ERR_UNSUPPORTED, "page size %d unsupported (16)", page_size);
+  if (static_cast<long long>(max_cache_len) + S_new > static_cast<long long>(max_pages_per_seq) * page_size)
+    return fail(ATTN_ERR_INVALID_ARG, "max_cache_len + S_new (%lld) exceeds the block table (%d pages)",
+                static_cast<long long>(max_cache_len) + S_new, max_pages_per_seq);
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16) ||
+      !aligned(out, 16) || !aligned(lse, 4) || !aligned(block_table, 4) || !aligned(cache_lens, 4) ||
+      !aligned(workspace, 256))
+    return fail(ATTN_ERR_INVALID_ARG, "misaligned pointer (tensors 16 B, lse/tables 4 B, workspace 256 B)");
+  const long long rows_q = static_cast<long long>(B) * Hq * S_new;
+  const long long sk = static_cast<long long>(max_cache_len) + S_new;
+  if (rows_q * (D / 8) > 0x7fffffffLL || static_cast<long long>(B) * Hkv * S_new * (D / 8) > 0x7fffffffLL ||
+      sk > (1 << 24))
+    return fail(ATTN_ERR_UNSUPPORTED, "problem too large");
+  const size_t need = attn_prefill_chunk_workspace_size(B, Hkv, S_new, max_cache_len, D);
+  if (workspace_bytes < need) return fail(ATTN_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace_bytes, need);
+  if (!std::isfinite(scale)) return fail(ATTN_ERR_INVALID_ARG, "scale is not finite");
+  if (scale <= 0.f) scale = 1.0f / std::sqrt(static_cast<float>(D));
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* status = reinterpret_cast<int*>(ws);
+  float2* cs = reinterpret_cast<float2*>(ws + kHeader);
+  uint8_t* k_op = ws + kHeader + round_up(static_cast<size_t>(sk) * (D / 2) * sizeof(float2), 256);
+  uint8_t* v_op = k_op + round_up(static_cast<size_t>(B) * Hkv * sk * D * 2, 256);
+  int rc = clear_status(ws, st);
+  if (rc) return rc;
+  const bool rope = rope_theta > 0.f;
+  if (rope) {
+    cudaError_t e = attn::launch_rope_table(cs, static_cast<int>(sk), D, static_cast<double>(rope_theta), st);
+    if (e != cudaSuccess) return cuda_fail(e, "rope table launch");
+  }
+  attn::ChunkGeometry g{cache_lens, block_table, B, Hkv, S_new, D, page_size, max_pages_per_seq, num_pages,
+                        max_cache_len};
+  const float2* rcs = rope ? cs : nullptr;
+  cudaError_t e = attn::launch_kv_append(k, v, k_pages, v_pages, rcs, g, status, st);
+  if (e == cudaSuccess) e = attn::launch_kv_gather(k_pages, v_pages, k_op, v_op, g, static_cast<int>(sk), status, st);
+  // the prepared Q operand goes into `out` (same byte size; each tile is loaded and
+  // later overwritten by the same CTA)
+  if (e == cudaSuccess) e = attn::launch_rope_rows_f16(q, out, rcs, g, Hq, status, st);
+  if (e != cudaSuccess) return cuda_fail(e, "chunk operand launch");
+
+  const int BN = attn::prefill_block_n(D, false);
+  const cuuint64_t qdims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S_new),
+                               static_cast<cuuint64_t>(B) * Hq};
+  const cuuint64_t qstr[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(S_new) * D * 2};
+  const cuuint64_t kdims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(sk), static_cast<cuuint64_t>(B) * Hkv};
+  const cuuint64_t kstr[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(sk) * D * 2};
+  const cuuint32_t qbox[3] = {64, 128, 1};
+  const cuuint32_t kbox[3] = {64, static_cast<cuuint32_t>(BN), 1};
+  CUtensorMap tmQ, tmK, tmV;
+  if ((rc = make_map(&tmQ, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, out, qdims, qstr, qbox, "Q"))) return rc;
+  if ((rc = make_map(&tmK, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, k_op, kdims, kstr, kbox, "K"))) return rc;
+  if ((rc = make_map(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, v_op, kdims, kstr, kbox, "V"))) return rc;
+
+  attn::PrefillParams p{};
+  p.out = out;
+  p.lse = lse;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.S = S_new;
+  p.G = Hq / Hkv;
+  p.causal = 1;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.pair_heads = (p.G % 2 == 0) ? 1 : 0;
+  p.n_row_blocks = (S_new + 127) / 128;
+  p.status = status;
+  p.q_off = cache_lens;
+  p.max_off = max_cache_len;
+  const long long items = p.pair_heads ? static_cast<long long>(B) * (Hq / 2) * p.n_row_blocks
+                                       : static_cast<long long>(B) * Hq * ((p.n_row_blocks + 1) / 2);
+  if (items > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "too many work items");
+  p.n_items = static_cast<int>(items);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long grid = items < sms ? items : sms;
+  prof_before(st);
+  e = attn::launch_prefill(p, tmQ, tmK, tmV, D, false, true, static_cast<int>(grid), st);
+  prof_after(st);
+  if (e != cudaSuccess) return cuda_fail(e, "chunk prefill launch");
+  return ok();
+}
+
 size_t attn_decode_paged_workspace_size(int B, int Hq, int D, int max_pages_per_seq, int page_size) {
   (void)page_size;
   if (B <= 0 || Hq <= 0 || D <= 0 || max_pages_per_seq <= 0) return kHeader;

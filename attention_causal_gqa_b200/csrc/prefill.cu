@@ -101,6 +101,7 @@ constexpr int kPolyPer8 = 2;
 // A work item: two 128-row query tiles that share one KV head.
 struct PrefillItem {
   int b, h0, h1, r0_0, r0_1, n_kv0, n_kv1;
+  int off;  // position of query row 0 among the keys (0 for a plain prefill)
 };
 
 // Item w of the list ordered heaviest (last row blocks) first.
@@ -126,10 +127,16 @@ __device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int 
     it.r0_0 = 2 * rp * BM;
     it.r0_1 = it.r0_0 + BM;
   }
+  it.off = 0;
+  if (p.q_off) {
+    const int o = __ldg(p.q_off + it.b);
+    it.off = o < 0 ? 0 : (o > p.max_off ? p.max_off : o);
+  }
+  // keys 0 .. off + S - 1; with the causal mask query row r sees keys <= off + r
   auto n_kv_for = [&](int r0) -> int {
     if (r0 >= p.S) return 0;
-    if (!p.causal) return (p.S + BN - 1) / BN;
-    return (min(p.S, r0 + BM) - 1) / BN + 1;
+    if (!p.causal) return (it.off + p.S + BN - 1) / BN;
+    return (it.off + min(p.S, r0 + BM) - 1) / BN + 1;
   };
   it.n_kv0 = n_kv_for(it.r0_0);
   it.n_kv1 = n_kv_for(it.r0_1);
@@ -373,7 +380,7 @@ __global__ void __launch_bounds__(320, 1)
     const bool row_valid = grow < p.S;
     float m_run = -INFINITY;
     float l_run = 0.f;
-    const int limit = p.causal ? min(grow, p.S - 1) : p.S - 1;  // last key this row may see
+    const int limit = it.off + (p.causal ? min(grow, p.S - 1) : p.S - 1);  // last key this row may see
 
     for (int j = 0; j < n_kv && alive; ++j) {
       bool ok = mbar_wait(&s_full[t], (g + j) & 1, abort_flag, p.status);

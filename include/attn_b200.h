@@ -99,6 +99,41 @@ int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, c
                       size_t workspace_bytes, void* stream);
 
 /*
+ * Chunked prefill into the paged KV cache: append a chunk of S_new tokens per sequence
+ * and attend the new queries over the whole cache.
+ * Defined by: "From 32K to 256K: DeepSeek long-context" (tqpw.cn) chapter 1 (streaming KV
+ * cache for incremental processing, long sequences cut into chunks, a PagedAttention
+ * variant) and section 2.1 (RoPE); "attention study note", sections "Page Attention"
+ * (block table) and the tiled online-softmax sections (the attention itself).
+ *
+ *   q            [B, Hq,  S_new, D]   bf16, new queries (not rotated)
+ *   k, v         [B, Hkv, S_new, D]   bf16, new keys (not rotated) and values
+ *   k_pages      [num_pages, page_size, Hkv, D] bf16 (keys rotated), updated in place
+ *   v_pages      [num_pages, page_size, Hkv, D] bf16, updated in place
+ *   block_table  [B, max_pages_per_seq] int32; must map every logical page that holds
+ *                a position < cache_lens[b] + S_new
+ *   cache_lens   [B] int32 (device), tokens already cached; new token i of sequence b
+ *                takes position cache_lens[b] + i; 0 <= cache_lens[b] <= max_cache_len
+ *   out          [B, Hq, S_new, D] bf16 (written; also holds the prepared Q operand
+ *                between the prologue and the attention, so it must not overlap q/k/v)
+ *   lse          [B, Hq, S_new] fp32 (written)
+ * The new keys are rotated at their positions (rope_theta > 0; <= 0: no RoPE) and
+ * stored with the values in bf16; query i then attends keys t <= cache_lens[b] + i (the
+ * causal mask aligned to the end of the cache). scale <= 0 selects 1/sqrt(D).
+ * Supported: D in {64, 128}, page_size 16. Q.K^T runs with fp16 operands (bf16 cache
+ * values are exact in fp16; |values| beyond 65504 flag ATTN_DEV_RANGE); P.V in bf16.
+ * Entries outside the page pool or lengths beyond max_cache_len are skipped/clamped and
+ * flagged in the status word (ATTN_DEV_BAD_PAGE, ATTN_DEV_BAD_LENGTH).
+ * workspace: >= attn_prefill_chunk_workspace_size(...) bytes, 256-byte aligned.
+ */
+size_t attn_prefill_chunk_workspace_size(int B, int Hkv, int S_new, int max_cache_len, int D);
+int attn_prefill_chunk(const void* q, const void* k, const void* v, void* k_pages, void* v_pages,
+                       const int32_t* block_table, const int32_t* cache_lens, void* out, float* lse, int B, int Hq,
+                       int Hkv, int S_new, int D, int page_size, int max_pages_per_seq, int num_pages,
+                       int max_cache_len, float rope_theta, float scale, void* workspace, size_t workspace_bytes,
+                       void* stream);
+
+/*
  * DeepSeek MLA absorbed decode (one query token per sequence).
  * Defined by: "DeepSeek-V3 attention: einsum vs hand-optimised" (dksg.cn), absorbed
  * form: scores = (q_nope . kv_cache^T + q_pe . pe_cache^T) * scale,

@@ -42,6 +42,29 @@ def _err(lib):
     return lib.attn_last_error().decode()
 
 
+def test_prefill_chunk_validation_codes(lib):
+    f = lib.attn_prefill_chunk
+    P = ctypes.c_void_p(FAKE)
+    #          q  k  v  kp vp bt cl out lse  B Hq Hkv S_new D  ps maxp np  maxc theta scale ws bytes stream
+    args = [P, P, P, P, P, P, P, P, P, 2, 8, 2, 64, 128, 16, 8, 20, 64, 1e4, 0.0, P, 1 << 30, None]
+
+    def call(**over):
+        a = list(args)
+        for k, v in over.items():
+            a[int(k[1:])] = v
+        return f(*a)
+
+    assert call(_0=None) == 1 and "null" in _err(lib)
+    assert call(_10=6, _11=4) == 1                 # Hq % Hkv
+    assert call(_12=0) == 1                        # S_new = 0
+    assert call(_13=96) == 2                       # D = 96
+    assert call(_14=32) == 2                       # page size 32
+    assert call(_17=65) == 1 and "block table" in _err(lib)   # max_cache_len + S_new > 8 pages * 16
+    need = lib.attn_prefill_chunk_workspace_size(2, 2, 64, 64, 128)
+    assert call(_21=need - 1) == 3
+    assert call(_0=ctypes.c_void_p(FAKE + 8), _21=need) == 1  # misaligned q
+
+
 def test_prefill_validation_codes(lib):
     f = lib.attn_prefill
     P = ctypes.c_void_p(FAKE)
