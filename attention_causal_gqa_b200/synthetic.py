@@ -24,7 +24,7 @@ PAGE_SIZE = 16
 @dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str  # "prefill" | "decode" | "mla"
+    kind: str  # "prefill" | "decode" | "mla" | "chunk"
     params: dict = field(default_factory=dict)
 
 
@@ -42,6 +42,10 @@ WORKLOADS = {
     "paged_decode_b64_hq32_hkv8_d128": Workload(
         "paged_decode_b64_hq32_hkv8_d128", "decode",
         dict(B=64, Hq=32, Hkv=8, D=128, lmin=1024, lmax=32768, std=1.0, scale=1.0 / math.sqrt(128))),
+    "chunk_prefill_b8_hq32_hkv8_d128_n2048_cache4k_28k": Workload(
+        "chunk_prefill_b8_hq32_hkv8_d128_n2048_cache4k_28k", "chunk",
+        dict(B=8, Hq=32, Hkv=8, D=128, S_new=2048, lmin=4096, lmax=28672, std=1.0, theta=1e4,
+             scale=1.0 / math.sqrt(128))),
     "mla_decode_b32_h128_dc512_dr64": Workload(
         "mla_decode_b32_h128_dc512_dr64", "mla",
         dict(B=32, H=128, Dc=512, Dr=64, lmin=4096, lmax=32768, std=1.0, scale=1.0 / math.sqrt(192))),
@@ -134,6 +138,35 @@ def mla_inputs(B, H, Dc, Dr, lmin=4096, lmax=32768, std=1.0, seed=0, device="cpu
                 seq_lens=torch.from_numpy(seq_lens).to(device), T_max=T_max)
 
 
+def chunk_inputs(B, Hq, Hkv, D, S_new, lmin=4096, lmax=28672, std=1.0, seed=0, device="cpu", cache_lens=None,
+                 page_size=PAGE_SIZE):
+    """A chunk of S_new new tokens per sequence and a paged cache that already holds
+    cache_lens[b] tokens (lengths uniform in [lmin, lmax] unless given). Pages for the
+    cached prefix and the chunk are mapped in a seeded random physical order; every
+    slot is filled with random values. q, k, v: [B, H, S_new, D] bf16 (not rotated)."""
+    if cache_lens is None:
+        cache_lens = draw_lengths(B, lmin, lmax, seed)
+    cache_lens = np.asarray(cache_lens, dtype=np.int32)
+    npages = [int(math.ceil((int(L) + S_new) / page_size)) for L in cache_lens]
+    max_pages = max(npages)
+    total = int(sum(npages))
+    rng = np.random.Generator(np.random.PCG64(seed + 7919))
+    perm = rng.permutation(total).astype(np.int32)
+    table = np.full((B, max_pages), -1, dtype=np.int32)
+    off = 0
+    for b, n in enumerate(npages):
+        table[b, :n] = perm[off:off + n]
+        off += n
+    g = _gen(seed, device)
+    q = _randn((B, Hq, S_new, D), std, "bf16", g, device)
+    k = _randn((B, Hkv, S_new, D), std, "bf16", g, device)
+    v = _randn((B, Hkv, S_new, D), std, "bf16", g, device)
+    k_pages = _randn((total, page_size, Hkv, D), std, "bf16", g, device)
+    v_pages = _randn((total, page_size, Hkv, D), std, "bf16", g, device)
+    return dict(q=q, k=k, v=v, k_pages=k_pages, v_pages=v_pages, block_table=torch.from_numpy(table).to(device),
+                cache_lens=torch.from_numpy(cache_lens).to(device), max_cache_len=int(cache_lens.max()))
+
+
 def workload_inputs(name: str, seed: int = 20261202, device="cpu"):
     w = WORKLOADS[name]
     p = w.params
@@ -141,4 +174,6 @@ def workload_inputs(name: str, seed: int = 20261202, device="cpu"):
         return prefill_inputs(p["B"], p["Hq"], p["Hkv"], p["S"], p["D"], p["dtype"], p["std"], seed, device)
     if w.kind == "decode":
         return decode_inputs(p["B"], p["Hq"], p["Hkv"], p["D"], p["lmin"], p["lmax"], p["std"], seed, device)
+    if w.kind == "chunk":
+        return chunk_inputs(p["B"], p["Hq"], p["Hkv"], p["D"], p["S_new"], p["lmin"], p["lmax"], p["std"], seed, device)
     return mla_inputs(p["B"], p["H"], p["Dc"], p["Dr"], p["lmin"], p["lmax"], p["std"], seed, device)

@@ -31,6 +31,7 @@ PREFILL = "gqa_prefill_b2_hq32_hkv8_s4096_d128"
 DECODE = "paged_decode_b64_hq32_hkv8_d128"
 MLA = "mla_decode_b32_h128_dc512_dr64"
 PREFILL_LONG = "gqa_prefill_b1_hq32_hkv8_s32768_d128"
+CHUNK = "chunk_prefill_b8_hq32_hkv8_d128_n2048_cache4k_28k"
 METRIC = "prefill attn TFLOP/s & decode KV-read GB/s, % of B200 roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -309,6 +310,46 @@ def bench_prefill(args, world, dev, seed, flush, pk, pk_kind, fp, name=None, wit
     return res
 
 
+def bench_chunk(args, world, dev, seed, pk, pk_kind):
+    """Chunked prefill into the paged cache: every step appends the same chunk at the same
+    positions (idempotent) and attends over the whole cache."""
+    import numpy as np
+    import torch
+    from attention_causal_gqa_b200 import binding as B_
+    from attention_causal_gqa_b200.synthetic import WORKLOADS, workload_inputs
+    p = WORKLOADS[CHUNK].params
+    d = workload_inputs(CHUNK, seed=seed, device=dev)
+    B, Hq, S, D = p["B"], p["Hq"], p["S_new"], p["D"]
+    out = torch.empty_like(d["q"])
+    lse = torch.empty((B, Hq, S), dtype=torch.float32, device=dev)
+    ws = torch.empty(B_.prefill_chunk_workspace_size(B, p["Hkv"], S, d["max_cache_len"], D), dtype=torch.uint8,
+                     device=dev)
+
+    def step():
+        B_.attn_prefill_chunk(d["q"], d["k"], d["v"], d["k_pages"], d["v_pages"], d["block_table"], d["cache_lens"],
+                              d["max_cache_len"], rope_theta=p["theta"], scale=p["scale"], out=out, lse=lse,
+                              workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    B_.profile_collect()
+    ms = timed_region(step, args.steps, 0, world)
+    kern_ms, n_launch = B_.profile_collect()
+    lens = d["cache_lens"].cpu().numpy().astype(np.float64)
+    # exact causal work: query i of sequence b sees cache_lens[b] + i + 1 keys; QK^T and P V
+    flops = float(np.sum(Hq * 4 * D * (S * lens + S * (S + 1) / 2)))
+    kern_avg = max_over_ranks(kern_ms / max(n_launch, 1), world)
+    achieved = flops / (kern_avg * 1e-3) / 1e12
+    return {"workload": CHUNK, "value": world * flops * args.steps / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "ms_per_step": ms / args.steps, "cached_tokens": int(lens.sum()), "gpu_launches": 5 * args.steps,
+            "l2": "cache (1.2 GB of pages) larger than L2",
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / pk["bf16_tflops"], "traffic": None, "kernel": "prefill_kernel",
+                         "kernel_ms": kern_avg, "peak_kind": f"{pk_kind} dense bf16 (burst)",
+                         "algorithmic": f"{flops:.4g} flop per launch = sum over rows of 4*D*(keys seen)"}}
+
+
 def bench_decode(args, world, dev, seed, pk, pk_kind, fp):
     import torch
     from attention_causal_gqa_b200 import binding as B_
@@ -430,6 +471,8 @@ def run_ours(args):
                                "ms_per_step": lp["ms"] / args.steps, "roofline": lp["roofline"],
                                "gpu_launches": 4 * args.steps}
         del lp
+    if do("prefill") and not args.small:
+        sub["prefill_chunk"] = bench_chunk(args, world, dev, seed, pk, pk_kind)
     if do("decode"):
         sub["decode"] = bench_decode(args, world, dev, seed, pk, pk_kind, fp)
     if do("mla"):
