@@ -7,7 +7,9 @@ links it, and it shares no code with the CUDA path.
 from .attention import (  # noqa: F401
     apply_rope,
     chunk_prefill_ref,
+    decode_paged_fp8_ref,
     decode_paged_ref,
+    e4m3_to_float,
     gather_pages,
     lse_merge,
     mla_decode_ref,

@@ -351,6 +351,31 @@ def chunk_prefill_ref(q, k_new, v_new, k_pages, v_pages, block_table, cache_lens
     return kp, vp, o, lse
 
 
+# ------------------------------------------------------ FP8 (E4M3) paged decode
+def e4m3_to_float(codes):
+    """Value of FP8 E4M3 codes (1 sign bit, 4 exponent bits with bias 7, 3 mantissa
+    bits; exponent 0 encodes subnormals m/8 * 2^-6; 0x7F and 0xFF are NaN, there is no
+    infinity), as float64."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(F64)
+    val = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.power(2.0, e - 7))
+    val = np.where((c & 0x7F) == 0x7F, np.nan, val)
+    return sign * val
+
+
+def decode_paged_fp8_ref(q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale: float | None = None,
+                         page_size: int = 16, pairs=None):
+    """One-token GQA decode over an FP8 (E4M3) paged KV cache with one scale per
+    (page, kv head): the cached key is e4m3(code) * k_scale[page, head] (likewise the
+    value), then exactly ``decode_paged_ref`` on those values.
+    k_codes, v_codes: [num_pages, page_size, Hkv, D] uint8; k_scale, v_scale: [num_pages, Hkv]."""
+    kf = e4m3_to_float(k_codes) * np.asarray(k_scale, dtype=F64)[:, None, :, None]
+    vf = e4m3_to_float(v_codes) * np.asarray(v_scale, dtype=F64)[:, None, :, None]
+    return decode_paged_ref(q, kf, vf, block_table, seq_lens, scale=scale, page_size=page_size, pairs=pairs)
+
+
 # ------------------------------------------------------------------ MLA decode
 def mla_decode_ref(q_nope, q_pe, kv_cache, pe_cache, seq_lens, scale: float, pairs=None):
     """DeepSeek MLA absorbed decode (einsum vs hand-optimised page, absorbed form).

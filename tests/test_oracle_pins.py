@@ -494,3 +494,34 @@ def test_chunk_prefill_last_row_equals_decode_over_the_updated_cache():
                        for b in range(B)])
     do, dl = decode_paged_ref(q_last, kp2, vp2, table, [c + S_new for c in cache])
     assert np.allclose(o[:, :, -1], do, atol=1e-12) and np.allclose(lse[:, :, -1], dl, atol=1e-12)
+
+
+# ------------------------------------------------------ FP8 (E4M3) paged decode
+def test_e4m3_decoding_matches_torch_for_every_code():
+    import torch
+    from oracle import e4m3_to_float
+    codes = np.arange(256, dtype=np.uint8)
+    ours = e4m3_to_float(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(ours), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(ours[ok], ref[ok])
+    assert ours[0x7E] == 448.0 and ours[0x01] == 2.0 ** -9 and ours[0x38] == 1.0  # max, smallest subnormal, one
+
+
+def test_fp8_decode_equals_decode_over_the_dequantised_cache():
+    from oracle import decode_paged_fp8_ref, decode_paged_ref, e4m3_to_float
+    rng = np.random.default_rng(50)
+    B, Hq, Hkv, D, P = 2, 8, 2, 16, 9
+    kc = rng.integers(0, 256, size=(P, 16, Hkv, D), dtype=np.uint8) & 0x77  # no NaN codes
+    vc = rng.integers(0, 256, size=(P, 16, Hkv, D), dtype=np.uint8) & 0x77
+    ks = rng.uniform(0.01, 2.0, size=(P, Hkv))
+    vs = rng.uniform(0.01, 2.0, size=(P, Hkv))
+    table = rng.permutation(P)[:8].reshape(2, 4)
+    lens = [37, 64]
+    q = rng.standard_normal((B, Hq, D))
+    o, l = decode_paged_fp8_ref(q, kc, vc, ks, vs, table, lens)
+    kf = np.stack([[e4m3_to_float(kc[p, :, h]) * ks[p, h] for h in range(Hkv)] for p in range(P)]).transpose(0, 2, 1, 3)
+    vf = np.stack([[e4m3_to_float(vc[p, :, h]) * vs[p, h] for h in range(Hkv)] for p in range(P)]).transpose(0, 2, 1, 3)
+    ro, rl = decode_paged_ref(q, kf, vf, table, lens)
+    assert np.allclose(o, ro, atol=1e-12) and np.allclose(l, rl, atol=1e-12)
