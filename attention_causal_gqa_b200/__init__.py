@@ -5,7 +5,7 @@ The public calls (attn_prefill, attn_prefill_chunk, attn_decode_paged, mla_decod
 ``binding`` and are loaded lazily, so ``synthetic`` can be imported without the
 library; calling any of them without the built library raises.
 """
-__all__ = ["attn_prefill", "attn_prefill_chunk", "attn_decode_paged", "mla_decode", "read_status", "selftest_wait_timeout"]
+__all__ = ["attn_prefill", "attn_prefill_chunk", "attn_decode_paged", "attn_decode_paged_fp8", "mla_decode", "read_status", "selftest_wait_timeout"]
 
 
 def __getattr__(name):

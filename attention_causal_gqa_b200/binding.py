@@ -55,6 +55,8 @@ def _load() -> ctypes.CDLL:
     lib.attn_decode_paged_workspace_size.argtypes = [i32] * 5
     lib.attn_decode_paged.restype = i32
     lib.attn_decode_paged.argtypes = [vp] * 7 + [i32] * 7 + [f32, i32, vp, sz, vp]
+    lib.attn_decode_paged_fp8.restype = i32
+    lib.attn_decode_paged_fp8.argtypes = [vp] * 9 + [i32] * 7 + [f32, vp, sz, vp]
     lib.attn_prefill_chunk_workspace_size.restype = sz
     lib.attn_prefill_chunk_workspace_size.argtypes = [i32] * 5
     lib.attn_prefill_chunk.restype = i32
@@ -158,6 +160,27 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale=None, ou
     rc = lib.attn_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens), _ptr(out),
                                _ptr(lse), B, Hq, Hkv, D, ps, maxp, P, float(scale or 0.0), ATTN_DTYPE_BF16, _ptr(ws),
                                ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc)
+    return out, lse
+
+
+def attn_decode_paged_fp8(q, k_pages, v_pages, k_scale, v_scale, block_table, seq_lens, scale=None, out=None, lse=None,
+                          workspace=None, stream=None):
+    """Paged GQA decode over an FP8 E4M3 cache. q [B,Hq,D] bf16; k/v_pages [P,16,Hkv,D] uint8 codes;
+    k/v_scale [P,Hkv] fp32; block_table [B,maxp] int32; seq_lens [B] int32.
+    Returns (out [B,Hq,D] bf16, lse [B,Hq] fp32)."""
+    _need_cuda(q, k_pages, v_pages, k_scale, v_scale, block_table, seq_lens)
+    B, Hq, D = q.shape
+    P, ps, Hkv, _ = k_pages.shape
+    maxp = block_table.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    ws = _workspace(decode_workspace_size(B, Hq, D, maxp, ps), q.device, workspace)
+    rc = lib.attn_decode_paged_fp8(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(k_scale), _ptr(v_scale),
+                                   _ptr(block_table), _ptr(seq_lens), _ptr(out), _ptr(lse), B, Hq, Hkv, D, ps, maxp,
+                                   P, float(scale or 0.0), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
     _check(rc)
     return out, lse
 

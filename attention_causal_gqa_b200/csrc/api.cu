@@ -440,6 +440,78 @@ int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, c
   return ok();
 }
 
+int attn_decode_paged_fp8(const void* q, const void* k_pages, const void* v_pages, const float* k_scale,
+                          const float* v_scale, const int32_t* block_table, const int32_t* seq_lens, void* out,
+                          float* lse, int B, int Hq, int Hkv, int D, int page_size, int max_pages_per_seq,
+                          int num_pages, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k_pages || !v_pages || !k_scale || !v_scale || !block_table || !seq_lens || !out || !lse || !workspace)
+    return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || max_pages_per_seq <= 0 || num_pages <= 0 || page_size <= 0)
+    return fail(ATTN_ERR_INVALID_ARG, "sizes must be positive");
+  if (Hq % Hkv != 0) return fail(ATTN_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+  if (page_size != 16) return fail(ATTN_ERR_UNSUPPORTED, "page_size %d (only 16)", page_size);
+  if (D != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d (the FP8 cache supports 128)", D);
+  if (Hkv > 8) return fail(ATTN_ERR_UNSUPPORTED, "Hkv %d > 8", Hkv);
+  if (Hq / Hkv > 16) return fail(ATTN_ERR_UNSUPPORTED, "group size %d > 16", Hq / Hkv);
+  if (!aligned(q, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(out, 16) ||
+      !aligned(k_scale, 4) || !aligned(v_scale, 4) || !aligned(block_table, 4) || !aligned(seq_lens, 4) ||
+      !aligned(lse, 4) || !aligned(workspace, 256))
+    return fail(ATTN_ERR_INVALID_ARG, "misaligned pointer");
+  const size_t need = attn_decode_paged_workspace_size(B, Hq, D, max_pages_per_seq, page_size);
+  if (workspace_bytes < need)
+    return fail(ATTN_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace_bytes, need);
+  if (!std::isfinite(scale)) return fail(ATTN_ERR_INVALID_ARG, "scale is not finite");
+  if (scale <= 0.f) scale = 1.0f / std::sqrt(static_cast<float>(D));
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int ns = decode_splits(max_pages_per_seq);
+  float* part_o = reinterpret_cast<float*>(ws + kHeader);
+  float* part_lse =
+      reinterpret_cast<float*>(ws + kHeader + round_up(static_cast<size_t>(B) * ns * Hq * D * sizeof(float), 256));
+  int rc = clear_status(ws, st);
+  if (rc) return rc;
+
+  // 4-D view of a page pool of codes [num_pages][16][Hkv][D]: (d, token, head, page);
+  // its shared-memory image is [head][token][D bytes].
+  const cuuint64_t row = static_cast<cuuint64_t>(Hkv) * D;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), 16, static_cast<cuuint64_t>(Hkv),
+                              static_cast<cuuint64_t>(num_pages)};
+  const cuuint64_t strides[3] = {row, static_cast<cuuint64_t>(D), 16 * row};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(D), 16, static_cast<cuuint32_t>(Hkv), 1};
+  CUtensorMap tmK, tmV;
+  if ((rc = make_map(&tmK, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, k_pages, dims, strides, box, "k_pages"))) return rc;
+  if ((rc = make_map(&tmV, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, v_pages, dims, strides, box, "v_pages"))) return rc;
+
+  attn::DecodeParams p{};
+  p.q = q;
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.part_o = part_o;
+  p.part_lse = part_lse;
+  p.out = out;
+  p.lse = lse;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.D = D;
+  p.G = Hq / Hkv;
+  p.max_pages = max_pages_per_seq;
+  p.num_pages = num_pages;
+  p.n_splits = ns;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.status = reinterpret_cast<int*>(ws);
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  prof_before(st);
+  cudaError_t e = attn::launch_decode(p, tmK, tmV, st);
+  prof_after(st);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  e = attn::launch_merge(part_o, part_lse, seq_lens, out, lse, B, Hq, D, ns, attn::kDecodePagesPerSplit * 16, st);
+  if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  return ok();
+}
+
 // MLA workspace: [status | partial outputs (n_pairs + B) x H x Dc fp32 | partial LSE (n_pairs + B) x H]
 size_t mla_decode_workspace_size(int B, int H, int Dc, int Dr, int T_max) {
   (void)Dr;

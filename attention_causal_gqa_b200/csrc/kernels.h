@@ -68,6 +68,8 @@ struct DecodeParams {
   int max_pages, num_pages, n_splits;
   float scale_log2;
   int* status;
+  const float* k_scale;     // FP8 cache only: [num_pages, Hkv] scales (nullptr: bf16 cache)
+  const float* v_scale;
 };
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
                           cudaStream_t stream);

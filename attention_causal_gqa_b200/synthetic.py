@@ -119,6 +119,28 @@ def decode_inputs(B, Hq, Hkv, D, lmin=1024, lmax=32768, std=1.0, seed=0, device=
                 max_pages_per_seq=max_pages_per_seq, num_pages=num_pages, page_size=page_size)
 
 
+def quantize_e4m3(x, page_axis=0, head_axis=2):
+    """E4M3 codes of x [num_pages, page_size, Hkv, D] with one scale per (page, head) =
+    absmax / 448 (torch's float8_e4m3fn conversion, round to nearest); returns (codes
+    uint8, scales fp32 [num_pages, Hkv])."""
+    xf = x.float()
+    amax = xf.abs().amax(dim=(1, 3)).clamp(min=1e-12)
+    sc = amax / 448.0
+    codes = (xf / sc[:, None, :, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes.contiguous(), sc.contiguous()
+
+
+def decode_inputs_fp8(B, Hq, Hkv, D, lmin=1024, lmax=32768, std=1.0, seed=0, device="cpu", seq_lens=None,
+                      max_pages_per_seq=None, extra_pages=0):
+    """The paged decode inputs of decode_inputs with K and V pages quantised to E4M3
+    (one scale per page and kv head)."""
+    d = decode_inputs(B, Hq, Hkv, D, lmin, lmax, std, seed, device, seq_lens, max_pages_per_seq,
+                      extra_pages=extra_pages)
+    d["k_pages"], d["k_scale"] = quantize_e4m3(d["k_pages"])
+    d["v_pages"], d["v_scale"] = quantize_e4m3(d["v_pages"])
+    return d
+
+
 def mla_inputs(B, H, Dc, Dr, lmin=4096, lmax=32768, std=1.0, seed=0, device="cpu", seq_lens=None,
                T_max=None):
     """Absorbed-MLA decode inputs: q_nope [B,1,H,Dc], q_pe [B,1,H,Dr],

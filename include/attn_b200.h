@@ -99,6 +99,29 @@ int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, c
                       size_t workspace_bytes, void* stream);
 
 /*
+ * Paged GQA decode over an FP8 (E4M3) KV cache with one fp32 scale per (page, kv head).
+ * Defined by the paged decode above, with the cached values read as
+ * e4m3(code) * scale ("7 anti-patterns of DeepSeek attention optimisation" (lpnh.cn),
+ * section 3.3: the FP8 E4M3 format, largest value 448, and scale factors that bring
+ * tensors into its range).
+ *
+ *   q            [B, Hq, D] bf16
+ *   k_pages      [num_pages, page_size, Hkv, D] uint8 E4M3 codes (keys already rotated)
+ *   v_pages      [num_pages, page_size, Hkv, D] uint8 E4M3 codes
+ *   k_scale      [num_pages, Hkv] fp32;  v_scale [num_pages, Hkv] fp32
+ *   block_table, seq_lens, out, lse: as attn_decode_paged.
+ * Supported: D = 128, page_size 16, Hkv <= 8, Hq/Hkv <= 16. NaN codes are out of
+ * contract. Products run in fp16: codes convert exactly, q converts exactly within
+ * +-65504 (else ATTN_DEV_RANGE), P carries the value scale (times 2^8) in fp16, so
+ * 256 * v_scale must stay below about 6.5e4.
+ * workspace: >= attn_decode_paged_workspace_size(B, Hq, D, max_pages_per_seq, page_size).
+ */
+int attn_decode_paged_fp8(const void* q, const void* k_pages, const void* v_pages, const float* k_scale,
+                          const float* v_scale, const int32_t* block_table, const int32_t* seq_lens, void* out,
+                          float* lse, int B, int Hq, int Hkv, int D, int page_size, int max_pages_per_seq,
+                          int num_pages, float scale, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Chunked prefill into the paged KV cache: append a chunk of S_new tokens per sequence
  * and attend the new queries over the whole cache.
  * Defined by: "From 32K to 256K: DeepSeek long-context" (tqpw.cn) chapter 1 (streaming KV

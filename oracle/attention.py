@@ -371,9 +371,24 @@ def decode_paged_fp8_ref(q, k_codes, v_codes, k_scale, v_scale, block_table, seq
     (page, kv head): the cached key is e4m3(code) * k_scale[page, head] (likewise the
     value), then exactly ``decode_paged_ref`` on those values.
     k_codes, v_codes: [num_pages, page_size, Hkv, D] uint8; k_scale, v_scale: [num_pages, Hkv]."""
-    kf = e4m3_to_float(k_codes) * np.asarray(k_scale, dtype=F64)[:, None, :, None]
-    vf = e4m3_to_float(v_codes) * np.asarray(v_scale, dtype=F64)[:, None, :, None]
-    return decode_paged_ref(q, kf, vf, block_table, seq_lens, scale=scale, page_size=page_size, pairs=pairs)
+    # Only the pages of the sequences that are computed are dequantised (same values;
+    # the block table is renumbered onto the compact page list).
+    table = np.asarray(block_table)
+    lens = np.asarray(seq_lens)
+    seqs = range(table.shape[0]) if pairs is None else sorted({b for b, _ in pairs})
+    used = sorted({int(table[b, j]) for b in seqs for j in range((int(lens[b]) + page_size - 1) // page_size)})
+    remap = {pg: i for i, pg in enumerate(used)}
+    table2 = np.zeros_like(table)
+    for b in seqs:
+        for j in range((int(lens[b]) + page_size - 1) // page_size):
+            table2[b, j] = remap[int(table[b, j])]
+    idx = np.asarray(used, dtype=np.int64)
+    kf = e4m3_to_float(np.asarray(k_codes)[idx]) * np.asarray(k_scale, dtype=F64)[idx][:, None, :, None]
+    vf = e4m3_to_float(np.asarray(v_codes)[idx]) * np.asarray(v_scale, dtype=F64)[idx][:, None, :, None]
+    if not used:
+        kf = np.zeros((1,) + np.asarray(k_codes).shape[1:])
+        vf = np.zeros_like(kf)
+    return decode_paged_ref(q, kf, vf, table2, lens, scale=scale, page_size=page_size, pairs=pairs)
 
 
 # ------------------------------------------------------------------ MLA decode
