@@ -10,6 +10,7 @@ __all__ = ["attn_prefill", "attn_prefill_chunk", "attn_decode_paged", "attn_deco
 
 def __getattr__(name):
     if name in __all__ or name in ("prefill_workspace_size", "prefill_chunk_workspace_size", "decode_workspace_size",
+                                   "decode_fp8_workspace_size",
                                    "mla_workspace_size", "AttnError", "lib"):
         from . import binding
         return getattr(binding, name)

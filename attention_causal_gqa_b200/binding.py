@@ -30,7 +30,7 @@ ATTN_DEV_BAD_LENGTH = 4
 EXPORTED = (
     "attn_prefill_workspace_size", "attn_prefill",
     "attn_decode_paged_workspace_size", "attn_decode_paged",
-    "mla_decode_workspace_size", "mla_decode",
+    "attn_decode_paged_fp8_workspace_size", "mla_decode_workspace_size", "mla_decode",
     "attn_last_error", "attn_read_status", "attn_selftest_wait_timeout",
     "attn_profile_enable", "attn_profile_collect",
 )
@@ -61,6 +61,8 @@ def _load() -> ctypes.CDLL:
     lib.attn_prefill_chunk_workspace_size.argtypes = [i32] * 5
     lib.attn_prefill_chunk.restype = i32
     lib.attn_prefill_chunk.argtypes = [vp] * 9 + [i32] * 9 + [f32, f32, vp, sz, vp]
+    lib.attn_decode_paged_fp8_workspace_size.restype = sz
+    lib.attn_decode_paged_fp8_workspace_size.argtypes = [i32] * 5
     lib.mla_decode_workspace_size.restype = sz
     lib.mla_decode_workspace_size.argtypes = [i32] * 5
     lib.mla_decode.restype = i32
@@ -144,6 +146,10 @@ def decode_workspace_size(B, Hq, D, max_pages_per_seq, page_size=16) -> int:
     return int(lib.attn_decode_paged_workspace_size(B, Hq, D, max_pages_per_seq, page_size))
 
 
+def decode_fp8_workspace_size(B, Hq, D, max_pages_per_seq, page_size=16) -> int:
+    return int(lib.attn_decode_paged_fp8_workspace_size(B, Hq, D, max_pages_per_seq, page_size))
+
+
 def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale=None, out=None, lse=None, workspace=None,
                       stream=None):
     """Paged GQA decode. q [B,Hq,D] bf16, k/v_pages [P,16,Hkv,D] bf16, block_table [B,maxp] int32,
@@ -177,7 +183,7 @@ def attn_decode_paged_fp8(q, k_pages, v_pages, k_scale, v_scale, block_table, se
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
-    ws = _workspace(decode_workspace_size(B, Hq, D, maxp, ps), q.device, workspace)
+    ws = _workspace(decode_fp8_workspace_size(B, Hq, D, maxp, ps), q.device, workspace)
     rc = lib.attn_decode_paged_fp8(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(k_scale), _ptr(v_scale),
                                    _ptr(block_table), _ptr(seq_lens), _ptr(out), _ptr(lse), B, Hq, Hkv, D, ps, maxp,
                                    P, float(scale or 0.0), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))

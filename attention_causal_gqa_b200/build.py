@@ -14,7 +14,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libattn_b200.so")
-SOURCES = ["api.cu", "rope.cu", "prefill.cu", "decode.cu", "mla.cu", "merge.cu", "chunk.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "rope.cu", "prefill.cu", "decode.cu", "decode_fp8.cu", "mla.cu", "merge.cu", "chunk.cu", "noalloc.cu"]
 HEADERS = ["sm100.cuh", "kernels.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -39,7 +39,8 @@ def _fingerprint() -> str:
 
 # The file that defines each main kernel; with the shared headers and the arch
 # flags it fixes that kernel's code (profile figures are keyed by this).
-KERNEL_SOURCES = {"prefill_kernel": "prefill.cu", "decode_kernel": "decode.cu", "mla_kernel": "mla.cu"}
+KERNEL_SOURCES = {"prefill_kernel": "prefill.cu", "decode_kernel": "decode.cu", "decode_fp8_kernel": "decode_fp8.cu",
+                  "mla_kernel": "mla.cu"}
 
 
 def kernel_fingerprint(kernel: str) -> str:

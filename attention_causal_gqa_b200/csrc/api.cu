@@ -440,6 +440,14 @@ int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, c
   return ok();
 }
 
+size_t attn_decode_paged_fp8_workspace_size(int B, int Hq, int D, int max_pages_per_seq, int page_size) {
+  (void)page_size;
+  (void)max_pages_per_seq;
+  if (B <= 0 || Hq <= 0 || D <= 0) return kHeader;
+  const size_t slots = static_cast<size_t>(attn::kDecodeFp8MaxRanges) + B;  // range c, sequence b: slot c + b
+  return kHeader + round_up(slots * Hq * D * sizeof(float), 256) + round_up(slots * Hq * sizeof(float), 256);
+}
+
 int attn_decode_paged_fp8(const void* q, const void* k_pages, const void* v_pages, const float* k_scale,
                           const float* v_scale, const int32_t* block_table, const int32_t* seq_lens, void* out,
                           float* lse, int B, int Hq, int Hkv, int D, int page_size, int max_pages_per_seq,
@@ -457,7 +465,7 @@ int attn_decode_paged_fp8(const void* q, const void* k_pages, const void* v_page
       !aligned(k_scale, 4) || !aligned(v_scale, 4) || !aligned(block_table, 4) || !aligned(seq_lens, 4) ||
       !aligned(lse, 4) || !aligned(workspace, 256))
     return fail(ATTN_ERR_INVALID_ARG, "misaligned pointer");
-  const size_t need = attn_decode_paged_workspace_size(B, Hq, D, max_pages_per_seq, page_size);
+  const size_t need = attn_decode_paged_fp8_workspace_size(B, Hq, D, max_pages_per_seq, page_size);
   if (workspace_bytes < need)
     return fail(ATTN_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace_bytes, need);
   if (!std::isfinite(scale)) return fail(ATTN_ERR_INVALID_ARG, "scale is not finite");
@@ -465,10 +473,9 @@ int attn_decode_paged_fp8(const void* q, const void* k_pages, const void* v_page
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const int ns = decode_splits(max_pages_per_seq);
+  const size_t slots = static_cast<size_t>(attn::kDecodeFp8MaxRanges) + B;
   float* part_o = reinterpret_cast<float*>(ws + kHeader);
-  float* part_lse =
-      reinterpret_cast<float*>(ws + kHeader + round_up(static_cast<size_t>(B) * ns * Hq * D * sizeof(float), 256));
+  float* part_lse = reinterpret_cast<float*>(ws + kHeader + round_up(slots * Hq * D * sizeof(float), 256));
   int rc = clear_status(ws, st);
   if (rc) return rc;
 
@@ -498,16 +505,18 @@ int attn_decode_paged_fp8(const void* q, const void* k_pages, const void* v_page
   p.G = Hq / Hkv;
   p.max_pages = max_pages_per_seq;
   p.num_pages = num_pages;
-  p.n_splits = ns;
+  p.n_splits = 0;  // ranges, not fixed splits
   p.scale_log2 = scale * 1.4426950408889634f;
   p.status = reinterpret_cast<int*>(ws);
   p.k_scale = k_scale;
   p.v_scale = v_scale;
   prof_before(st);
-  cudaError_t e = attn::launch_decode(p, tmK, tmV, st);
+  int n_ranges = 0;
+  cudaError_t e = attn::launch_decode_fp8(p, tmK, tmV, &n_ranges, st);
   prof_after(st);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-  e = attn::launch_merge(part_o, part_lse, seq_lens, out, lse, B, Hq, D, ns, attn::kDecodePagesPerSplit * 16, st);
+  e = attn::launch_decode_range_merge(part_o, part_lse, seq_lens, out, lse, B, Hq, max_pages_per_seq * 16, n_ranges,
+                                      st);
   if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   return ok();
 }

@@ -44,40 +44,11 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// Two FP8 E4M3 codes (bytes 0 and 1 of w when sel = 0x1404, bytes 2 and 3 when sel =
-// 0x3424) as an fp16 pair holding exactly value * 2^-8: sign to bit 15, the 4 exponent
-// bits under fp16's bias 15 (instead of E4M3's 7) and the 3 mantissa bits on top of
-// fp16's mantissa; E4M3 subnormals land on fp16 subnormals with the same factor.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_scaled(uint32_t w, uint32_t sel) {
-  const uint32_t u = __byte_perm(w, 0u, sel);  // each byte at bits 8-15 of its half
-  return (u & 0x80008000u) | ((u >> 1) & 0x3F803F80u);
-}
-
-__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w, bool& in_range) {
-  const float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xFFFF0000u);
-  in_range = in_range && fabsf(lo) <= 65504.f && fabsf(hi) <= 65504.f;
-  const __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
 
 
 }  // namespace
 
-// FP8: the pages hold E4M3 codes with one fp32 scale per (page, kv head); the TMA image
-// of a page is [head][token][D bytes]. Each compute warp converts its head's K and V
-// into fp16 (exactly code value * 2^-8) in the same [d/64][token][64] layout as the
-// bf16 path, releases the stage, and runs the products in fp16 (Q converted from
-// bf16, exact in range). The key scale (times 2^8) multiplies the scores in fp32; the
-// value scale (times 2^8) multiplies P before P V, while l sums the unscaled P.
-template <int D, bool FP8>
+template <int D>
 __global__ void __launch_bounds__(kDecThreads, 1)
     decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV) {
@@ -87,13 +58,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   constexpr int PPS = kDecodePagesPerSplit;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int page_bytes = 16 * p.Hkv * D * (FP8 ? 1 : 2);  // one page of K (or V), all heads
+  const int page_bytes = 16 * p.Hkv * D * 2;  // one page of K (or V), all heads
   const int stage_bytes = 2 * page_bytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kDecStages * stage_bytes);
   uint64_t* empty = full + kDecStages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kDecStages);
-  // FP8: each compute warp's converted K and V of the current page, 2 x 16 x D fp16
-  uint8_t* cvt = smem + ((kDecStages * stage_bytes + 256 + 1023) & ~1023);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -145,13 +114,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         if (lane == 0) {
           uint8_t* dst = smem + s * stage_bytes;
           mbar_arrive_expect_tx(&full[s], stage_bytes);
-          if constexpr (FP8) {
-            tma_load_4d(dst, &tmK, &full[s], 0, 0, 0, phys);
-            tma_load_4d(dst + page_bytes, &tmV, &full[s], 0, 0, 0, phys);
-          } else {
-            tma_load_5d(dst, &tmK, &full[s], 0, 0, 0, 0, phys);
-            tma_load_5d(dst + page_bytes, &tmV, &full[s], 0, 0, 0, 0, phys);
-          }
+          tma_load_5d(dst, &tmK, &full[s], 0, 0, 0, 0, phys);
+          tma_load_5d(dst + page_bytes, &tmV, &full[s], 0, 0, 0, 0, phys);
         }
       }
     }
@@ -187,14 +151,6 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         qa[kt][2] = (busy && g < G) ? *reinterpret_cast<const uint32_t*>(qb + g * D + d0 + 8) : 0u;
         qa[kt][3] = (busy && g + 8 < G) ? *reinterpret_cast<const uint32_t*>(qb + (g + 8) * D + d0 + 8) : 0u;
       }
-      if constexpr (FP8) {
-        bool in_range = true;
-#pragma unroll
-        for (int kt = 0; kt < KT; ++kt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) qa[kt][e] = bf16x2_to_f16x2(qa[kt][e], in_range);
-        if (!in_range) atomicOr(p.status, kDevErrRange);
-      }
     }
     float o[NT][4];
 #pragma unroll
@@ -209,48 +165,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       uint8_t* kp = smem + s * stage_bytes;
       uint8_t* vp = kp + page_bytes;
       const int rem = L - pg * 16;  // valid tokens in this page (>= 1)
-      float ks = 1.f, vs = 1.f;     // FP8: 2^8 * the page's scales for this head
-      if constexpr (FP8) {
-        if (busy) {
-          int phys = __ldg(p.block_table + static_cast<size_t>(b) * p.max_pages + pg);
-          if (phys < 0 || phys >= p.num_pages) phys = 0;  // flagged by the producer
-          ks = 256.f * __ldg(p.k_scale + static_cast<size_t>(phys) * p.Hkv + h);
-          vs = 256.f * __ldg(p.v_scale + static_cast<size_t>(phys) * p.Hkv + h);
-          // convert this head's 16 x D codes of K and V; rows past the end become zeros
-          uint8_t* ck = cvt + warp * (2 * 16 * D * 2);
-          uint8_t* cv = ck + 16 * D * 2;
-#pragma unroll
-          for (int i = 0; i < (16 * D / 16) / 32; ++i) {
-            const int idx = lane + 32 * i;           // 16-byte chunk of codes: token t, dims 16j..16j+15
-            const int t = idx / (D / 16), j = idx % (D / 16);
-            const int src = (h * 16 + t) * D + ((j ^ (t & 7)) << 4);
-            const int dim = 16 * j, dh = dim >> 6, ch = (dim & 63) >> 3;
-            const int d0 = (dh * 16 + t) * 128 + ((ch ^ (t & 7)) << 4);
-            const int d1 = (dh * 16 + t) * 128 + (((ch + 1) ^ (t & 7)) << 4);
-            const uint4 kw = *reinterpret_cast<const uint4*>(kp + src);
-            *reinterpret_cast<uint4*>(ck + d0) =
-                make_uint4(e4m3x2_to_f16x2_scaled(kw.x, 0x1404), e4m3x2_to_f16x2_scaled(kw.x, 0x3424),
-                           e4m3x2_to_f16x2_scaled(kw.y, 0x1404), e4m3x2_to_f16x2_scaled(kw.y, 0x3424));
-            *reinterpret_cast<uint4*>(ck + d1) =
-                make_uint4(e4m3x2_to_f16x2_scaled(kw.z, 0x1404), e4m3x2_to_f16x2_scaled(kw.z, 0x3424),
-                           e4m3x2_to_f16x2_scaled(kw.w, 0x1404), e4m3x2_to_f16x2_scaled(kw.w, 0x3424));
-            uint4 vw = *reinterpret_cast<const uint4*>(vp + src);
-            if (t >= rem) vw = make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4*>(cv + d0) =
-                make_uint4(e4m3x2_to_f16x2_scaled(vw.x, 0x1404), e4m3x2_to_f16x2_scaled(vw.x, 0x3424),
-                           e4m3x2_to_f16x2_scaled(vw.y, 0x1404), e4m3x2_to_f16x2_scaled(vw.y, 0x3424));
-            *reinterpret_cast<uint4*>(cv + d1) =
-                make_uint4(e4m3x2_to_f16x2_scaled(vw.z, 0x1404), e4m3x2_to_f16x2_scaled(vw.z, 0x3424),
-                           e4m3x2_to_f16x2_scaled(vw.w, 0x1404), e4m3x2_to_f16x2_scaled(vw.w, 0x3424));
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);  // the codes are consumed: the stage may be refilled
-        kp = cvt + warp * (2 * 16 * D * 2);
-        vp = kp + 16 * D * 2;
-      }
       if (busy) {
-        if (!FP8 && rem < 16) {
+        if (rem < 16) {
           // tokens past the end: zero their V rows so 0 * garbage cannot poison O
           for (int idx = lane; idx < DH * 16 * 8; idx += 32) {
             const int dh = idx / 128, t = (idx / 8) % 16, ch = idx % 8;
@@ -258,8 +174,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           }
           __syncwarp();
         }
-        const uint32_t kbase = smem_u32(kp) + (FP8 ? 0 : h * DH * 16 * 128);
-        const uint32_t vbase = smem_u32(vp) + (FP8 ? 0 : h * DH * 16 * 128);
+        const uint32_t kbase = smem_u32(kp) + h * DH * 16 * 128;
+        const uint32_t vbase = smem_u32(vp) + h * DH * 16 * 128;
         // S = Q K^T over 16 tokens (two n-tiles of 8 tokens)
         float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         const int mi = lane >> 3, r8 = lane & 7;  // ldmatrix: matrix index and row within it
@@ -272,13 +188,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           const uint32_t addr = kbase + (dh * 16 + tok) * 128 + ((ch ^ (tok & 7)) << 4);
           uint32_t b0, b1, b2, b3;
           ldsm_x4(addr, b0, b1, b2, b3);
-          if constexpr (FP8) {
-            mma_f16(sc[0], qa[kt], b0, b1);
-            mma_f16(sc[1], qa[kt], b2, b3);
-          } else {
-            mma_bf16(sc[0], qa[kt], b0, b1);
-            mma_bf16(sc[1], qa[kt], b2, b3);
-          }
+          mma_bf16(sc[0], qa[kt], b0, b1);
+          mma_bf16(sc[1], qa[kt], b2, b3);
         }
         // mask tokens past the end, scale into the log2 domain
         float v[2][4];
@@ -287,7 +198,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int tok = nt * 8 + 2 * c + (e & 1);
-            v[nt][e] = tok < rem ? sc[nt][e] * (sl2 * ks) : -INFINITY;
+            v[nt][e] = tok < rem ? sc[nt][e] * sl2 : -INFINITY;
           }
         float mx0 = fmaxf(fmaxf(v[0][0], v[0][1]), fmaxf(v[1][0], v[1][1]));
         float mx1 = fmaxf(fmaxf(v[0][2], v[0][3]), fmaxf(v[1][2], v[1][3]));
@@ -317,21 +228,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           o[n][3] *= a1;
         }
         uint32_t pa[4];
-        if constexpr (FP8) {
-          auto h2 = [&](float a, float b2) {
-            const __half2 x = __floats2half2_rn(a * vs, b2 * vs);
-            return *reinterpret_cast<const uint32_t*>(&x);
-          };
-          pa[0] = h2(pr[0][0], pr[0][1]);
-          pa[1] = h2(pr[0][2], pr[0][3]);
-          pa[2] = h2(pr[1][0], pr[1][1]);
-          pa[3] = h2(pr[1][2], pr[1][3]);
-        } else {
-          pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
-          pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
-          pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
-          pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
-        }
+        pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
+        pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
+        pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
+        pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
         // O += P V: V is [token][dim]; transposed ldmatrix gives the B fragments
 #pragma unroll
         for (int n2 = 0; n2 < NT / 2; ++n2) {
@@ -342,18 +242,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           const uint32_t addr = vbase + (dh * 16 + tok) * 128 + ((ch ^ (tok & 7)) << 4);
           uint32_t b0, b1, b2, b3;
           ldsm_x4_t(addr, b0, b1, b2, b3);
-          if constexpr (FP8) {
-            mma_f16(o[2 * n2], pa, b0, b1);
-            mma_f16(o[2 * n2 + 1], pa, b2, b3);
-          } else {
-            mma_bf16(o[2 * n2], pa, b0, b1);
-            mma_bf16(o[2 * n2 + 1], pa, b2, b3);
-          }
+          mma_bf16(o[2 * n2], pa, b0, b1);
+          mma_bf16(o[2 * n2 + 1], pa, b2, b3);
         }
-        if (!FP8 && rem < 16) fence_proxy_async_smem();  // generic zero-writes before the next TMA into this slot
+        if (rem < 16) fence_proxy_async_smem();  // generic zero-writes before the next TMA into this slot
       }
       __syncwarp();
-      if (!FP8 && lane == 0) mbar_arrive(&empty[s]);
+      if (lane == 0) mbar_arrive(&empty[s]);
     }
 
     if (busy) {
@@ -379,13 +274,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   }
 }
 
-template <int D, bool FP8>
+template <int D>
 static cudaError_t launch_decode_t(const DecodeParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
                                    cudaStream_t stream) {
-  const int stages = kDecStages * 2 * 16 * p.Hkv * D * (FP8 ? 1 : 2);
-  const int smem = FP8 ? 1024 + ((stages + 256 + 1023) & ~1023) + kDecWarps * 2 * 16 * D * 2
-                       : 1024 + stages + 2 * kDecStages * 8 + 16;
-  auto kern = decode_kernel<D, FP8>;
+  const int smem = 1024 + kDecStages * 2 * 16 * p.Hkv * D * 2 + 2 * kDecStages * 8 + 16;
+  auto kern = decode_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
@@ -399,12 +292,8 @@ static cudaError_t launch_decode_t(const DecodeParams& p, const CUtensorMap& tmK
 
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
                           cudaStream_t stream) {
-  if (p.k_scale) {
-    if (p.D == 128) return launch_decode_t<128, true>(p, tmK, tmV, stream);
-    return cudaErrorInvalidValue;
-  }
-  if (p.D == 128) return launch_decode_t<128, false>(p, tmK, tmV, stream);
-  if (p.D == 64) return launch_decode_t<64, false>(p, tmK, tmV, stream);
+  if (p.D == 128) return launch_decode_t<128>(p, tmK, tmV, stream);
+  if (p.D == 64) return launch_decode_t<64>(p, tmK, tmV, stream);
   return cudaErrorInvalidValue;
 }
 

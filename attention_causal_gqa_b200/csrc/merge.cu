@@ -94,30 +94,34 @@ cudaError_t launch_merge(const float* part_o, const float* part_lse, const int32
   return cudaGetLastError();
 }
 
-// ------------------------------------------------------------------ MLA
-__device__ __forceinline__ int mla_tiles_of(const int32_t* lens, int b, int T_max) {
+// ------------------------------------------------------------ range merge
+template <int UNIT>
+__device__ __forceinline__ int units_of(const int32_t* lens, int b, int T_max) {
   const int L = min(max(__ldg(lens + b), 0), T_max);
-  return (L + kMlaTile - 1) / kMlaTile;
+  return (L + UNIT - 1) / UNIT;
 }
 
-// One warp per (b, head). The MLA kernel cuts the N tiles of all sequences into
-// n_pairs contiguous ranges [N c / n_pairs, N (c + 1) / n_pairs), and cluster c
-// writes one partial result per sequence its range meets, at slot c + b. The
-// clusters meeting sequence b (tiles [s_b, e_b)) are those from the one holding
-// tile s_b to the one holding tile e_b - 1: cluster c holds tile x iff
-// floor(N c / P) <= x < floor(N (c + 1) / P), i.e. c = floor(((x + 1) P - 1) / N).
-// They are combined in cluster order (deterministic).
-__global__ void mla_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
-                                 const int32_t* __restrict__ seq_lens, __nv_bfloat16* __restrict__ out,
-                                 float* __restrict__ lse, int B, int H, int T_max, int n_pairs) {
-  constexpr int kDc = 512;
+// One warp per (b, head). The partial-result kernels that balance work by ranges
+// (the MLA decode with 32-token tiles as units, the FP8 paged decode with 16-token
+// pages) cut the N units of all sequences into n_ranges contiguous ranges
+// [N c / n_ranges, N (c + 1) / n_ranges); range c writes one partial result per
+// sequence it meets, at slot c + b. The ranges meeting sequence b (units [s_b, e_b))
+// are those from the one holding unit s_b to the one holding unit e_b - 1: range c
+// holds unit x iff floor(N c / P) <= x < floor(N (c + 1) / P), i.e.
+// c = floor(((x + 1) P - 1) / N). They are combined in range order (deterministic).
+template <int DIM, int UNIT>
+__global__ void range_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
+                                   const int32_t* __restrict__ seq_lens, __nv_bfloat16* __restrict__ out,
+                                   float* __restrict__ lse, int B, int H, int T_max, int n_ranges) {
+  constexpr int VEC = DIM / 32;  // contiguous columns per lane
+  static_assert(VEC % 4 == 0, "whole float4 columns per lane");
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (gw >= B * H) return;
   const int b = gw / H, h = gw % H;
   long long N = 0, s_b = 0;
   for (int i = lane; i < B; i += 32) {
-    const int n = mla_tiles_of(seq_lens, i, T_max);
+    const int n = units_of<UNIT>(seq_lens, i, T_max);
     N += n;
     if (i < b) s_b += n;
   }
@@ -126,65 +130,79 @@ __global__ void mla_merge_kernel(const float* __restrict__ part_o, const float* 
     N += __shfl_xor_sync(0xffffffffu, N, o);
     s_b += __shfl_xor_sync(0xffffffffu, s_b, o);
   }
-  const long long e_b = s_b + mla_tiles_of(seq_lens, b, T_max);
-  const long long P = n_pairs;
-  int c0 = 0, c1 = -1;  // contributing clusters (none for an empty sequence)
+  const long long e_b = s_b + units_of<UNIT>(seq_lens, b, T_max);
+  const long long P = n_ranges;
+  int c0 = 0, c1 = -1;  // contributing ranges (none for an empty sequence)
   if (e_b > s_b) {
     c0 = static_cast<int>(((s_b + 1) * P - 1) / N);
     c1 = static_cast<int>((e_b * P - 1) / N);
   }
-  __nv_bfloat16* orow = out + static_cast<size_t>(gw) * kDc;
+  __nv_bfloat16* orow = out + static_cast<size_t>(gw) * DIM + lane * VEC;
   float M = -INFINITY;
   for (int c = c0; c <= c1; ++c)
     if (N * (c + 1) / P > N * c / P) M = fmaxf(M, part_lse[static_cast<size_t>(c + b) * H + h]);
+  uint32_t packed[VEC / 2];
   if (!(M > -INFINITY)) {
-    for (int d = lane * 8; d < kDc; d += 256) *reinterpret_cast<uint4*>(orow + d) = make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int i = 0; i < VEC / 2; ++i) packed[i] = 0u;
     if (lane == 0) lse[gw] = -INFINITY;
-    return;
-  }
-  float acc[16];
+  } else {
+    float acc[VEC];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-  float wsum = 0.f;
+    for (int i = 0; i < VEC; ++i) acc[i] = 0.f;
+    float wsum = 0.f;
 #pragma unroll 2
-  for (int c = c0; c <= c1; ++c) {
-    if (!(N * (c + 1) / P > N * c / P)) continue;  // an empty range writes nothing
-    const size_t slot = static_cast<size_t>(c + b);
-    const float w = __expf(part_lse[slot * H + h] - M);
-    wsum += w;
-    const float* po = part_o + (slot * H + h) * kDc;
+    for (int c = c0; c <= c1; ++c) {
+      if (!(N * (c + 1) / P > N * c / P)) continue;  // an empty range writes nothing
+      const size_t slot = static_cast<size_t>(c + b);
+      const float w = __expf(part_lse[slot * H + h] - M);
+      wsum += w;
+      const float* po = part_o + (slot * H + h) * DIM + lane * VEC;
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int d = lane * 8 + i * 256;
-      const float4 v0 = *reinterpret_cast<const float4*>(po + d);
-      const float4 v1 = *reinterpret_cast<const float4*>(po + d + 4);
-      acc[8 * i + 0] += w * v0.x; acc[8 * i + 1] += w * v0.y; acc[8 * i + 2] += w * v0.z; acc[8 * i + 3] += w * v0.w;
-      acc[8 * i + 4] += w * v1.x; acc[8 * i + 5] += w * v1.y; acc[8 * i + 6] += w * v1.z; acc[8 * i + 7] += w * v1.w;
+      for (int q = 0; q < VEC / 4; ++q) {
+        const float4 v = *reinterpret_cast<const float4*>(po + 4 * q);
+        acc[4 * q] += w * v.x;
+        acc[4 * q + 1] += w * v.y;
+        acc[4 * q + 2] += w * v.z;
+        acc[4 * q + 3] += w * v.w;
+      }
     }
-  }
-  const float inv = 1.f / wsum;
+    const float inv = 1.f / wsum;
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const int d = lane * 8 + i * 256;
-    uint4 u;
-    __nv_bfloat162 t;
-    t = __floats2bfloat162_rn(acc[8 * i] * inv, acc[8 * i + 1] * inv); u.x = *reinterpret_cast<const uint32_t*>(&t);
-    t = __floats2bfloat162_rn(acc[8 * i + 2] * inv, acc[8 * i + 3] * inv); u.y = *reinterpret_cast<const uint32_t*>(&t);
-    t = __floats2bfloat162_rn(acc[8 * i + 4] * inv, acc[8 * i + 5] * inv); u.z = *reinterpret_cast<const uint32_t*>(&t);
-    t = __floats2bfloat162_rn(acc[8 * i + 6] * inv, acc[8 * i + 7] * inv); u.w = *reinterpret_cast<const uint32_t*>(&t);
-    *reinterpret_cast<uint4*>(orow + d) = u;
+    for (int i = 0; i < VEC / 2; ++i) {
+      const __nv_bfloat162 t = __floats2bfloat162_rn(acc[2 * i] * inv, acc[2 * i + 1] * inv);
+      packed[i] = *reinterpret_cast<const uint32_t*>(&t);
+    }
+    if (lane == 0) lse[gw] = M + logf(wsum);
   }
-  if (lane == 0) lse[gw] = M + logf(wsum);
+  if constexpr (VEC % 8 == 0) {
+#pragma unroll
+    for (int i = 0; i < VEC / 8; ++i)
+      reinterpret_cast<uint4*>(orow)[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+  } else {
+    reinterpret_cast<uint2*>(orow)[0] = make_uint2(packed[0], packed[1]);
+  }
+}
+
+template <int DIM, int UNIT>
+static cudaError_t launch_range_merge(const float* part_o, const float* part_lse, const int32_t* seq_lens, void* out,
+                                      float* lse, int B, int H, int T_max, int n_ranges, cudaStream_t stream) {
+  const long long warps = static_cast<long long>(B) * H;
+  const int threads = 256;
+  const long long blocks = (warps * 32 + threads - 1) / threads;
+  range_merge_kernel<DIM, UNIT><<<static_cast<int>(blocks), threads, 0, stream>>>(
+      part_o, part_lse, seq_lens, static_cast<__nv_bfloat16*>(out), lse, B, H, T_max, n_ranges);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_mla_merge(const float* part_o, const float* part_lse, const int32_t* seq_lens, void* out,
                              float* lse, int B, int H, int T_max, int n_pairs, cudaStream_t stream) {
-  const long long warps = static_cast<long long>(B) * H;
-  const int threads = 256;
-  const long long blocks = (warps * 32 + threads - 1) / threads;
-  mla_merge_kernel<<<static_cast<int>(blocks), threads, 0, stream>>>(
-      part_o, part_lse, seq_lens, static_cast<__nv_bfloat16*>(out), lse, B, H, T_max, n_pairs);
-  return cudaGetLastError();
+  return launch_range_merge<512, kMlaTile>(part_o, part_lse, seq_lens, out, lse, B, H, T_max, n_pairs, stream);
+}
+
+cudaError_t launch_decode_range_merge(const float* part_o, const float* part_lse, const int32_t* seq_lens, void* out,
+                                      float* lse, int B, int H, int T_max, int n_ranges, cudaStream_t stream) {
+  return launch_range_merge<128, 16>(part_o, part_lse, seq_lens, out, lse, B, H, T_max, n_ranges, stream);
 }
 
 }  // namespace attn

@@ -392,6 +392,49 @@ def bench_decode(args, world, dev, seed, pk, pk_kind, fp):
     return res
 
 
+def bench_decode_fp8(args, world, dev, seed, pk, pk_kind):
+    """The paged decode workload with its K/V pages quantised to E4M3 (one scale per page
+    and kv head): same sequences, half the cache bytes."""
+    import torch
+    from attention_causal_gqa_b200 import binding as B_
+    from attention_causal_gqa_b200.synthetic import WORKLOADS, decode_inputs_fp8
+    dp = dict(WORKLOADS[DECODE].params)
+    B = 8 if args.small else dp["B"]
+    d = decode_inputs_fp8(B, dp["Hq"], dp["Hkv"], dp["D"], dp["lmin"], dp["lmax"], dp["std"], seed, dev)
+    out = torch.empty_like(d["q"])
+    lse = torch.empty((B, dp["Hq"]), dtype=torch.float32, device=dev)
+    ws = torch.empty(B_.decode_fp8_workspace_size(B, dp["Hq"], dp["D"], d["max_pages_per_seq"]), dtype=torch.uint8,
+                     device=dev)
+
+    def step():
+        B_.attn_decode_paged_fp8(d["q"], d["k_pages"], d["v_pages"], d["k_scale"], d["v_scale"], d["block_table"],
+                                 d["seq_lens"], scale=dp["scale"], out=out, lse=lse, workspace=ws)
+
+    tokens = int(d["seq_lens"].sum().item())
+    # codes: Hkv * D bytes each for K and V; scales: 2 * Hkv * 4 bytes per 16-token page
+    kv_bytes = tokens * dp["Hkv"] * dp["D"] * 2 + ((tokens + 15) // 16) * dp["Hkv"] * 8
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    B_.profile_collect()
+    ms = timed_region(step, args.steps, 0, world)
+    k_ms, n = B_.profile_collect()
+    k_avg = max_over_ranks(k_ms / max(n, 1), world)
+    ach = kv_bytes / (k_avg * 1e-3) / 1e9
+    res = {"workload": DECODE + "_fp8_e4m3" + ("_small_b8" if args.small else ""),
+           "value": world * kv_bytes * args.steps / (ms * 1e-3) / 1e9, "unit": "GB/s",
+           "ms_per_step": ms / args.steps, "kv_tokens": tokens, "kv_bytes_per_step": kv_bytes,
+           "gpu_launches": 2 * args.steps, "l2": "inputs (2.2 GB) larger than L2",
+           "roofline": {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                        "frac": ach / pk["hbm_gbs"], "traffic": traffic_for("decode_fp8_kernel"),
+                        "kernel": "decode_fp8_kernel",
+                        "kernel_ms": k_avg, "peak_kind": f"{pk_kind} HBM copy",
+                        "algorithmic": "2048 B of codes per cached token + 64 B of scales per 16-token page"}}
+    del d, out, lse, ws
+    torch.cuda.empty_cache()
+    return res
+
+
 def bench_mla(args, world, dev, seed, pk, pk_kind, fp):
     import torch
     from attention_causal_gqa_b200 import binding as B_
@@ -475,6 +518,7 @@ def run_ours(args):
         sub["prefill_chunk"] = bench_chunk(args, world, dev, seed, pk, pk_kind)
     if do("decode"):
         sub["decode"] = bench_decode(args, world, dev, seed, pk, pk_kind, fp)
+        sub["decode_fp8"] = bench_decode_fp8(args, world, dev, seed, pk, pk_kind)
     if do("mla"):
         sub["mla"] = bench_mla(args, world, dev, seed, pk, pk_kind, fp)
     clk = clocks.stop()

@@ -114,8 +114,13 @@ int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, c
  * contract. Products run in fp16: codes convert exactly, q converts exactly within
  * +-65504 (else ATTN_DEV_RANGE), P carries the value scale (times 2^8) in fp16, so
  * 256 * v_scale must stay below about 6.5e4.
- * workspace: >= attn_decode_paged_workspace_size(B, Hq, D, max_pages_per_seq, page_size).
+ * workspace: >= attn_decode_paged_fp8_workspace_size(B, Hq, D, max_pages_per_seq, page_size)
+ *   (device, 256-byte aligned, caller-owned, scratch): one fp32 partial output and LSE
+ *   per (page range, sequence) pair; the pages of all sequences are cut into one
+ *   contiguous range per CTA of a persistent grid, so every CTA streams the same number
+ *   of pages whatever the length mix.
  */
+size_t attn_decode_paged_fp8_workspace_size(int B, int Hq, int D, int max_pages_per_seq, int page_size);
 int attn_decode_paged_fp8(const void* q, const void* k_pages, const void* v_pages, const float* k_scale,
                           const float* v_scale, const int32_t* block_table, const int32_t* seq_lens, void* out,
                           float* lse, int B, int Hq, int Hkv, int D, int page_size, int max_pages_per_seq,

@@ -31,6 +31,8 @@ def _oracle(d, pairs=None):
     ([5, 300, 2049], 8, 8),      # G = 1
     ([700, 33], 4, 1),           # MQA
     ([257, 4096], 32, 2),        # G = 16
+    ([33, 800, 1601], 48, 8),    # G = 6: a lane's second head column past the group
+    ([100, 1500], 12, 1),        # G = 12: the second 8-head tile half used
 ])
 def test_fp8_decode_matches_oracle(lens, Hq, Hkv):
     from attention_causal_gqa_b200.synthetic import decode_inputs_fp8
