@@ -15,7 +15,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libattn_b200.so")
 SOURCES = ["api.cu", "rope.cu", "prefill.cu", "decode.cu", "decode_fp8.cu", "mla.cu", "merge.cu", "chunk.cu", "noalloc.cu"]
-HEADERS = ["sm100.cuh", "kernels.h"]
+HEADERS = ["sm100.cuh", "kernels.h"]  # shared by every kernel
+PROLOGUE_HEADERS = ["prologue.h"]  # RoPE / KV-cache prologue only (not part of a kernel fingerprint)
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -28,7 +29,7 @@ def nvcc_path() -> str:
 
 def _fingerprint() -> str:
     h = hashlib.sha256()
-    for name in SOURCES + HEADERS:
+    for name in SOURCES + HEADERS + PROLOGUE_HEADERS:
         with open(os.path.join(CSRC, name), "rb") as f:
             h.update(name.encode() + f.read())
     with open(os.path.join(INCLUDE, "attn_b200.h"), "rb") as f:

@@ -9,6 +9,7 @@
 
 #include "../../include/attn_b200.h"
 #include "kernels.h"
+#include "prologue.h"
 #include "sm100.cuh"
 
 namespace {

@@ -19,6 +19,7 @@
 #include <cuda_fp16.h>
 
 #include "kernels.h"
+#include "prologue.h"
 #include "sm100.cuh"
 
 namespace attn {

@@ -1,0 +1,38 @@
+// Launch interfaces of the prologue kernels (RoPE operand preparation, KV-cache append
+// and gather for chunked prefill) between the C-ABI layer and rope.cu / chunk.cu. Kept
+// apart from kernels.h so the attention kernels do not depend on them.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace attn {
+
+// RoPE prologue: cos/sin table (angles in fp64), then the key operand.
+cudaError_t launch_rope_table(float2* cs, int S, int D, double theta, cudaStream_t stream);
+// bf16 X [rows, D] -> rotated fp16 X (row r at position r % S); flags values outside fp16 range.
+// Used for K and for Q.
+cudaError_t launch_rope_k_f16(const void* k, void* k_f16, const float2* cs, long long rows, int S, int D,
+                              int* status, cudaStream_t stream);
+// fp32 X [rows, D] -> bf16 hi parts at out[0, rows) and lo parts at out[rows, 2 rows), rotating
+// first when cs is non-null.
+cudaError_t launch_split_f32(const float* x, void* out, const float2* cs, long long rows, int S, int D,
+                             cudaStream_t stream);
+
+// --------------------------------------------- chunked prefill into the paged cache
+struct ChunkGeometry {
+  const int32_t* cache_lens;   // [B] tokens already cached (new token i sits at cache_lens[b] + i)
+  const int32_t* block_table;  // [B, max_pages]
+  int B, Hkv, S_new, D, page_size, max_pages, num_pages, max_cache_len;
+};
+// rotate the new keys at their positions and write keys and values (bf16) into their pages
+cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* k_pages, void* v_pages, const float2* cs,
+                             const ChunkGeometry& g, int* status, cudaStream_t stream);
+// each sequence's cache into contiguous operands [B*Hkv, Sk_max, D]: keys fp16, values bf16, zeros past it
+cudaError_t launch_kv_gather(const void* k_pages, const void* v_pages, void* k_op, void* v_op, const ChunkGeometry& g,
+                             int Sk_max, int* status, cudaStream_t stream);
+// new queries [B*Hq, S_new, D] rotated at their positions into fp16
+cudaError_t launch_rope_rows_f16(const void* q, void* q_f16, const float2* cs, const ChunkGeometry& g, int Hq,
+                                 int* status, cudaStream_t stream);
+
+}  // namespace attn

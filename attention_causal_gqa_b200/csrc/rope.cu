@@ -12,6 +12,7 @@
 #include <cuda_fp16.h>
 
 #include "kernels.h"
+#include "prologue.h"
 
 namespace attn {
 
