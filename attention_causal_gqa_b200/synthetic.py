@@ -24,11 +24,11 @@ PAGE_SIZE = 16
 @dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str  # "prefill" | "decode" | "mla" | "chunk"
+    kind: str  # "prefill" | "decode" | "mla" | "chunk" | "dsa"
     params: dict = field(default_factory=dict)
 
 
-# The five workloads, named by what they are.
+# The workloads, named by what they are.
 WORKLOADS = {
     "mha_prefill_b1_h4_s256_d64_f32": Workload(
         "mha_prefill_b1_h4_s256_d64_f32", "prefill",
@@ -49,6 +49,12 @@ WORKLOADS = {
     "mla_decode_b32_h128_dc512_dr64": Workload(
         "mla_decode_b32_h128_dc512_dr64", "mla",
         dict(B=32, H=128, Dc=512, Dr=64, lmin=4096, lmax=32768, std=1.0, scale=1.0 / math.sqrt(192))),
+    # the MLA decode workload with a lightning indexer in front: 64 indexer heads of
+    # width 128, the 2048 best-scoring cached tokens attended
+    "dsa_mla_decode_b32_h128_dc512_dr64_hi64_di128_top2048": Workload(
+        "dsa_mla_decode_b32_h128_dc512_dr64_hi64_di128_top2048", "dsa",
+        dict(B=32, H=128, Dc=512, Dr=64, lmin=4096, lmax=32768, std=1.0, scale=1.0 / math.sqrt(192),
+             HI=64, dI=128, top_k=2048)),
 }
 
 _TORCH_DT = {"bf16": torch.bfloat16, "f32": torch.float32}
@@ -160,6 +166,20 @@ def mla_inputs(B, H, Dc, Dr, lmin=4096, lmax=32768, std=1.0, seed=0, device="cpu
                 seq_lens=torch.from_numpy(seq_lens).to(device), T_max=T_max)
 
 
+def dsa_inputs(B, H, Dc, Dr, HI, dI, lmin=4096, lmax=32768, std=1.0, seed=0, device="cpu", seq_lens=None,
+               T_max=None):
+    """The MLA decode inputs of ``mla_inputs`` (same seed, same tensors) plus the lightning
+    indexer's inputs: q_idx [B,HI,dI] bf16 (one query per indexer head), w_idx [B,HI] fp32
+    head weights drawn N(0, 1/HI), k_idx [B,T_max,dI] bf16 (one key per cached token,
+    filled beyond each length too)."""
+    d = mla_inputs(B, H, Dc, Dr, lmin, lmax, std, seed, device, seq_lens, T_max)
+    g = _gen(seed + 104729, device)
+    d["q_idx"] = _randn((B, HI, dI), std, "bf16", g, device)
+    d["w_idx"] = _randn((B, HI), 1.0 / math.sqrt(HI), "f32", g, device)
+    d["k_idx"] = _randn((B, d["T_max"], dI), std, "bf16", g, device)
+    return d
+
+
 def chunk_inputs(B, Hq, Hkv, D, S_new, lmin=4096, lmax=28672, std=1.0, seed=0, device="cpu", cache_lens=None,
                  page_size=PAGE_SIZE):
     """A chunk of S_new new tokens per sequence and a paged cache that already holds
@@ -198,4 +218,7 @@ def workload_inputs(name: str, seed: int = 20261202, device="cpu"):
         return decode_inputs(p["B"], p["Hq"], p["Hkv"], p["D"], p["lmin"], p["lmax"], p["std"], seed, device)
     if w.kind == "chunk":
         return chunk_inputs(p["B"], p["Hq"], p["Hkv"], p["D"], p["S_new"], p["lmin"], p["lmax"], p["std"], seed, device)
+    if w.kind == "dsa":
+        return dsa_inputs(p["B"], p["H"], p["Dc"], p["Dr"], p["HI"], p["dI"], p["lmin"], p["lmax"], p["std"], seed,
+                          device)
     return mla_inputs(p["B"], p["H"], p["Dc"], p["Dr"], p["lmin"], p["lmax"], p["std"], seed, device)

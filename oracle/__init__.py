@@ -9,6 +9,9 @@ from .attention import (  # noqa: F401
     chunk_prefill_ref,
     decode_paged_fp8_ref,
     decode_paged_ref,
+    dsa_index_scores_ref,
+    dsa_mla_decode_ref,
+    dsa_topk_ref,
     e4m3_to_float,
     gather_pages,
     lse_merge,

@@ -27,6 +27,11 @@ definition allows:
 * "DeepSeek-V3 attention: einsum vs hand-optimised" (dksg.cn), absorbed MLA
   scores: scores = (q_nope . kv_cache^T + q_pe . pe_cache^T) * scale, and
   out = softmax(scores) . kv_cache.
+* "attention study note", section "Lighting Indexer": index score of a token =
+  sum over indexer heads j of w_j * ReLU(q_j . k_s); only the most relevant tokens
+  are attended (DeepSeek sparse attention).
+* "7 anti-patterns of DeepSeek attention optimisation" (lpnh.cn), section 3.3: the
+  FP8 E4M3 format (largest value 448) with scale factors.
 
 Readings taken where the pages are silent or garbled (all also listed in the
 design notes): RoPE positions start at 0 for Q and K; the score scale multiplies
@@ -451,3 +456,64 @@ def mla_naive_ref(x_q, c_kv, k_pe, w_uk, w_uv, q_pe, scale: float):
         outs.append((p @ V)[0])
         lses.append(l_[0])
     return np.stack(outs), np.array(lses)
+
+
+# ---------------------------------------------------------------------------
+# DeepSeek sparse attention: lightning indexer, top-k selection, MLA over the
+# selected tokens ("attention study note", section "Lighting Indexer").
+# ---------------------------------------------------------------------------
+def dsa_index_scores_ref(q_idx, w_idx, k_idx, seq_lens):
+    """Lightning-indexer scores for one decode query per sequence.
+
+    The page forms indexer queries q_j (one per indexer head j) and one indexer key
+    k_s per token, and sums w_j * ReLU(q_j . k_s) over the heads into the token's
+    index score:  I[b, s] = sum_j w[b, j] * max(q[b, j] . k[b, s], 0)  for s < seq_lens[b],
+    and -inf for the slots past the sequence (never selected).
+    q_idx [B, H_I, d_I], w_idx [B, H_I], k_idx [B, T, d_I]. Returns [B, T] float64."""
+    q = np.asarray(q_idx, dtype=F64)
+    w = np.asarray(w_idx, dtype=F64)
+    B, T = k_idx.shape[0], k_idx.shape[1]
+    out = np.full((B, T), -np.inf)
+    for b in range(B):
+        L = min(max(int(seq_lens[b]), 0), T)
+        if L == 0:
+            continue
+        k = np.asarray(k_idx[b, :L], dtype=F64)
+        dots = q[b] @ k.T  # [H_I, L]
+        out[b, :L] = w[b] @ np.maximum(dots, 0.0)
+    return out
+
+
+def dsa_topk_ref(scores, seq_lens, top_k: int):
+    """The tokens kept for attention: the min(top_k, L) cached tokens with the largest
+    index scores. Ties are broken toward the smaller token index (a reading: the page
+    does not say), so the set is unique. Returned per sequence in ascending token order."""
+    res = []
+    for b in range(scores.shape[0]):
+        L = min(max(int(seq_lens[b]), 0), scores.shape[1])
+        n = min(int(top_k), L)
+        if n <= 0:
+            res.append(np.zeros(0, dtype=np.int64))
+            continue
+        s = np.asarray(scores[b, :L], dtype=F64)
+        order = np.lexsort((np.arange(L), -s))  # score descending, then index ascending
+        res.append(np.sort(order[:n]))
+    return res
+
+
+def dsa_mla_decode_ref(q_nope, q_pe, kv_cache, pe_cache, indices, scale: float, pairs=None):
+    """MLA absorbed decode restricted to the selected tokens: exactly ``mla_decode_ref``
+    over the rows kv_cache[b, indices[b]] and pe_cache[b, indices[b]] (attention is
+    invariant to the order of its keys, so the ascending order changes nothing)."""
+    B = q_nope.shape[0]
+    n = [len(ix) for ix in indices]
+    t = max([1] + n)
+    kv = np.zeros((B, t, kv_cache.shape[2]))
+    pe = np.zeros((B, t, pe_cache.shape[2]))
+    seqs = range(B) if pairs is None else sorted({b for b, _ in pairs})
+    for b in seqs:
+        ix = np.asarray(indices[b], dtype=np.int64)
+        if len(ix):
+            kv[b, :len(ix)] = np.asarray(kv_cache[b][ix], dtype=F64)
+            pe[b, :len(ix)] = np.asarray(pe_cache[b][ix], dtype=F64)
+    return mla_decode_ref(q_nope, q_pe, kv, pe, n, scale, pairs=pairs)

@@ -525,3 +525,82 @@ def test_fp8_decode_equals_decode_over_the_dequantised_cache():
     vf = np.stack([[e4m3_to_float(vc[p, :, h]) * vs[p, h] for h in range(Hkv)] for p in range(P)]).transpose(0, 2, 1, 3)
     ro, rl = decode_paged_ref(q, kf, vf, table, lens)
     assert np.allclose(o, ro, atol=1e-12) and np.allclose(l, rl, atol=1e-12)
+
+
+# ------------------------------------------- DSA: lightning indexer + top-k MLA
+def test_indexer_hand_worked_example():
+    """Attention study note, "Lighting Indexer": score = sum_j w_j * ReLU(q_j . k_s).
+    Two heads q1 = (1, 0), q2 = (0, 1), weights (0.5, 2); keys (2, -3), (-1, 1), (1, 1):
+    token 0: 0.5*2 + 2*ReLU(-3) = 1; token 1: 0.5*ReLU(-1) + 2*1 = 2; token 2: 0.5 + 2 = 2.5."""
+    from oracle import dsa_index_scores_ref, dsa_topk_ref
+    q = np.array([[[1.0, 0.0], [0.0, 1.0]]])
+    w = np.array([[0.5, 2.0]])
+    k = np.array([[[2.0, -3.0], [-1.0, 1.0], [1.0, 1.0], [9.0, 9.0]]])
+    s = dsa_index_scores_ref(q, w, k, [3])
+    assert s[0, :3].tolist() == [1.0, 2.0, 2.5] and s[0, 3] == -np.inf  # slot past the length never counts
+    assert dsa_topk_ref(s, [3], 2)[0].tolist() == [1, 2]
+
+
+def test_indexer_matches_scalar_brute_force():
+    from oracle import dsa_index_scores_ref
+    rng = np.random.default_rng(60)
+    B, HI, d, T = 2, 3, 4, 6
+    q, w, k = rng.standard_normal((B, HI, d)), rng.standard_normal((B, HI)), rng.standard_normal((B, T, d))
+    lens = [6, 4]
+    s = dsa_index_scores_ref(q, w, k, lens)
+    for b in range(B):
+        for t in range(T):
+            if t >= lens[b]:
+                assert s[b, t] == -np.inf
+                continue
+            acc = 0.0
+            for j in range(HI):
+                dot = sum(float(q[b, j, i]) * float(k[b, t, i]) for i in range(d))
+                acc += float(w[b, j]) * (dot if dot > 0 else 0.0)
+            assert abs(s[b, t] - acc) < 1e-12
+
+
+def test_topk_ties_prefer_the_smaller_index_and_short_sequences_keep_everything():
+    from oracle import dsa_topk_ref
+    s = np.array([[3.0, 1.0, 3.0, 2.0, 3.0, -np.inf], [0.5, 0.5, 0.5, 0.5, 0.5, 0.5]])
+    got = dsa_topk_ref(s, [5, 6], 2)
+    assert got[0].tolist() == [0, 2] and got[1].tolist() == [0, 1]
+    assert dsa_topk_ref(s, [5, 6], 4)[0].tolist() == [0, 2, 3, 4]
+    assert dsa_topk_ref(s, [5, 0], 99)[0].tolist() == [0, 1, 2, 3, 4] and len(dsa_topk_ref(s, [5, 0], 99)[1]) == 0
+    # brute force over every subset on a small random row: the chosen set has the largest sum
+    rng = np.random.default_rng(61)
+    row = rng.standard_normal(7)
+    import itertools
+    best = max(itertools.combinations(range(7), 3), key=lambda c: sum(row[i] for i in c))
+    assert dsa_topk_ref(row[None, :], [7], 3)[0].tolist() == sorted(best)
+
+
+def test_dsa_with_every_token_selected_is_dense_mla():
+    from oracle import dsa_index_scores_ref, dsa_mla_decode_ref, dsa_topk_ref, mla_decode_ref
+    rng = np.random.default_rng(62)
+    B, H, Dc, Dr, T = 2, 3, 8, 4, 20
+    qn, qp = rng.standard_normal((B, 1, H, Dc)), rng.standard_normal((B, 1, H, Dr))
+    kv, pe = rng.standard_normal((B, T, Dc)), rng.standard_normal((B, T, Dr))
+    lens = [20, 13]
+    s = dsa_index_scores_ref(rng.standard_normal((B, 2, 5)), rng.standard_normal((B, 2)),
+                             rng.standard_normal((B, T, 5)), lens)
+    o, l = dsa_mla_decode_ref(qn, qp, kv, pe, dsa_topk_ref(s, lens, 64), 0.3)
+    ro, rl = mla_decode_ref(qn, qp, kv, pe, lens, 0.3)
+    assert np.allclose(o, ro, atol=1e-12) and np.allclose(l, rl, atol=1e-12)
+
+
+def test_dsa_equals_dense_softmax_with_unselected_tokens_masked():
+    """Attending only the selected tokens = the dense score row with -inf on the others."""
+    from oracle import dsa_mla_decode_ref, two_pass_softmax_rows
+    rng = np.random.default_rng(63)
+    B, H, Dc, Dr, T = 1, 2, 8, 4, 30
+    qn, qp = rng.standard_normal((B, 1, H, Dc)), rng.standard_normal((B, 1, H, Dr))
+    kv, pe = rng.standard_normal((B, T, Dc)), rng.standard_normal((B, T, Dr))
+    sel = np.array([2, 3, 11, 17, 29])
+    o, l = dsa_mla_decode_ref(qn, qp, kv, pe, [sel], 0.25)
+    for h in range(H):
+        sc = (kv[0] @ qn[0, 0, h] + pe[0] @ qp[0, 0, h]) * 0.25
+        masked = np.full(T, -np.inf)
+        masked[sel] = sc[sel]
+        p, lse = two_pass_softmax_rows(masked[None, :])
+        assert np.allclose(o[0, 0, h], (p @ kv[0])[0], atol=1e-12) and abs(l[0, 0, h] - lse[0]) < 1e-12
