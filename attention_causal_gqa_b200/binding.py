@@ -26,11 +26,14 @@ ATTN_DTYPE_BF16 = 1
 ATTN_DEV_TIMEOUT = 1
 ATTN_DEV_BAD_PAGE = 2
 ATTN_DEV_BAD_LENGTH = 4
+ATTN_DEV_RANGE = 8
+ATTN_DEV_BAD_INDEX = 16
 
 EXPORTED = (
     "attn_prefill_workspace_size", "attn_prefill",
     "attn_decode_paged_workspace_size", "attn_decode_paged",
     "attn_decode_paged_fp8_workspace_size", "mla_decode_workspace_size", "mla_decode",
+    "dsa_index_topk_workspace_size", "dsa_index_topk", "dsa_mla_decode_workspace_size", "dsa_mla_decode",
     "attn_last_error", "attn_read_status", "attn_selftest_wait_timeout",
     "attn_profile_enable", "attn_profile_collect",
 )
@@ -67,6 +70,14 @@ def _load() -> ctypes.CDLL:
     lib.mla_decode_workspace_size.argtypes = [i32] * 5
     lib.mla_decode.restype = i32
     lib.mla_decode.argtypes = [vp] * 5 + [f32, vp, vp] + [i32] * 5 + [vp, sz, vp]
+    lib.dsa_index_topk_workspace_size.restype = sz
+    lib.dsa_index_topk_workspace_size.argtypes = [i32] * 5
+    lib.dsa_index_topk.restype = i32
+    lib.dsa_index_topk.argtypes = [vp] * 6 + [i32] * 5 + [vp, sz, vp]
+    lib.dsa_mla_decode_workspace_size.restype = sz
+    lib.dsa_mla_decode_workspace_size.argtypes = [i32] * 5
+    lib.dsa_mla_decode.restype = i32
+    lib.dsa_mla_decode.argtypes = [vp] * 6 + [i32, f32, vp, vp] + [i32] * 5 + [vp, sz, vp]
     lib.attn_last_error.restype = ctypes.c_char_p
     lib.attn_last_error.argtypes = []
     lib.attn_read_status.restype = i32
@@ -243,6 +254,51 @@ def mla_decode(q_nope, q_pe, kv_cache, pe_cache, seq_lens, scale, out=None, lse=
     rc = lib.mla_decode(_ptr(q_nope), _ptr(q_pe), _ptr(kv_cache), _ptr(pe_cache), _ptr(seq_lens), float(scale),
                         _ptr(out), _ptr(lse), B, H, Dc, Dr, T, _ptr(ws), ws.numel() * ws.element_size(),
                         _stream(stream))
+    _check(rc)
+    return out, lse
+
+
+# ------------------------------------------------- DeepSeek sparse attention
+def dsa_index_topk(q_idx, w_idx, k_idx, seq_lens, top_k, scores=None, topk_idx=None, workspace=None, stream=None):
+    """Lightning-indexer scores and top-k selection. q_idx [B,H_I,d_I] bf16, w_idx [B,H_I] fp32,
+    k_idx [B,T,d_I] bf16, seq_lens [B] int32. Returns (scores [B,T] fp32, topk_idx [B,top_k] int32)."""
+    _need_cuda(q_idx, w_idx, k_idx, seq_lens)
+    B, HI, dI = q_idx.shape
+    T = k_idx.shape[1]
+    if scores is None:
+        scores = torch.empty((B, T), dtype=torch.float32, device=q_idx.device)
+    if topk_idx is None:
+        topk_idx = torch.empty((B, int(top_k)), dtype=torch.int32, device=q_idx.device)
+    ws = _workspace(lib.dsa_index_topk_workspace_size(B, HI, dI, T, int(top_k)), q_idx.device, workspace)
+    rc = lib.dsa_index_topk(_ptr(q_idx), _ptr(w_idx), _ptr(k_idx), _ptr(seq_lens), _ptr(scores), _ptr(topk_idx), B, HI,
+                            dI, T, int(top_k), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc)
+    return scores, topk_idx
+
+
+def dsa_mla_workspace_size(B, H, Dc, Dr, top_k) -> int:
+    return int(lib.dsa_mla_decode_workspace_size(B, H, Dc, Dr, top_k))
+
+
+def dsa_mla_decode(q_nope, q_pe, kv_cache, pe_cache, seq_lens, topk_idx, scale, out=None, lse=None, workspace=None,
+                   stream=None):
+    """MLA absorbed decode over the selected tokens topk_idx [B, top_k] int32 (from dsa_index_topk).
+    Other tensors as mla_decode. Returns (out [B,1,H,Dc] bf16, lse [B,1,H] fp32)."""
+    _need_cuda(q_nope, q_pe, kv_cache, pe_cache, seq_lens, topk_idx)
+    B, _, H, Dc = q_nope.shape
+    Dr = q_pe.shape[-1]
+    T = kv_cache.shape[1]
+    top_k = topk_idx.shape[1]
+    if not scale or scale <= 0:
+        raise ValueError("dsa_mla_decode needs an explicit positive scale")
+    if out is None:
+        out = torch.empty_like(q_nope)
+    if lse is None:
+        lse = torch.empty((B, 1, H), dtype=torch.float32, device=q_nope.device)
+    ws = _workspace(dsa_mla_workspace_size(B, H, Dc, Dr, top_k), q_nope.device, workspace)
+    rc = lib.dsa_mla_decode(_ptr(q_nope), _ptr(q_pe), _ptr(kv_cache), _ptr(pe_cache), _ptr(seq_lens), _ptr(topk_idx),
+                            top_k, float(scale), _ptr(out), _ptr(lse), B, H, Dc, Dr, T, _ptr(ws),
+                            ws.numel() * ws.element_size(), _stream(stream))
     _check(rc)
     return out, lse
 

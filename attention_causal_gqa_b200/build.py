@@ -14,9 +14,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libattn_b200.so")
-SOURCES = ["api.cu", "rope.cu", "prefill.cu", "decode.cu", "decode_fp8.cu", "mla.cu", "merge.cu", "chunk.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "rope.cu", "prefill.cu", "decode.cu", "decode_fp8.cu", "mla.cu", "merge.cu", "chunk.cu", "dsa.cu", "noalloc.cu"]
 HEADERS = ["sm100.cuh", "kernels.h"]  # shared by every kernel
-PROLOGUE_HEADERS = ["prologue.h"]  # RoPE / KV-cache prologue only (not part of a kernel fingerprint)
+PROLOGUE_HEADERS = ["prologue.h", "dsa.h"]  # included by their own kernels only (not in every fingerprint)
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -41,12 +41,13 @@ def _fingerprint() -> str:
 # The file that defines each main kernel; with the shared headers and the arch
 # flags it fixes that kernel's code (profile figures are keyed by this).
 KERNEL_SOURCES = {"prefill_kernel": "prefill.cu", "decode_kernel": "decode.cu", "decode_fp8_kernel": "decode_fp8.cu",
-                  "mla_kernel": "mla.cu"}
+                  "mla_kernel": "mla.cu", "dsa_index_kernel": ("dsa.cu", "dsa.h")}
 
 
 def kernel_fingerprint(kernel: str) -> str:
     h = hashlib.sha256()
-    for name in [KERNEL_SOURCES[kernel]] + HEADERS:
+    srcs = KERNEL_SOURCES[kernel]
+    for name in ([srcs] if isinstance(srcs, str) else list(srcs)) + HEADERS:
         with open(os.path.join(CSRC, name), "rb") as f:
             h.update(name.encode() + f.read())
     h.update(" ".join(ARCH).encode())

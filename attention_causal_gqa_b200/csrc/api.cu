@@ -8,6 +8,7 @@
 #include <string>
 
 #include "../../include/attn_b200.h"
+#include "dsa.h"
 #include "kernels.h"
 #include "prologue.h"
 #include "sm100.cuh"
@@ -531,30 +532,15 @@ size_t mla_decode_workspace_size(int B, int H, int Dc, int Dr, int T_max) {
   return kHeader + round_up(slots * H * Dc * sizeof(float), 256) + round_up(slots * H * sizeof(float), 256);
 }
 
-int mla_decode(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
-               const int32_t* seq_lens, float scale, void* out, float* lse, int B, int H, int Dc, int Dr, int T_max,
-               void* workspace, size_t workspace_bytes, void* stream) {
-  if (!q_nope || !q_pe || !kv_cache || !pe_cache || !seq_lens || !out || !lse || !workspace)
-    return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
-  if (B <= 0 || H <= 0 || Dc <= 0 || Dr <= 0 || T_max <= 0) return fail(ATTN_ERR_INVALID_ARG, "sizes must be positive");
-  if (H != 128 || Dc != 512 || Dr != 64)
-    return fail(ATTN_ERR_UNSUPPORTED, "MLA decode supports H=128, Dc=512, Dr=64 (got %d, %d, %d)", H, Dc, Dr);
-  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(ATTN_ERR_INVALID_ARG, "scale must be positive");
-  if (!aligned(q_nope, 16) || !aligned(q_pe, 16) || !aligned(kv_cache, 16) || !aligned(pe_cache, 16) ||
-      !aligned(out, 16) || !aligned(seq_lens, 4) || !aligned(lse, 4) || !aligned(workspace, 256))
-    return fail(ATTN_ERR_INVALID_ARG, "misaligned pointer");
-  if (T_max > (1 << 26) || B > (1 << 20)) return fail(ATTN_ERR_UNSUPPORTED, "problem too large");
-  const size_t need = mla_decode_workspace_size(B, H, Dc, Dr, T_max);
-  if (workspace_bytes < need)
-    return fail(ATTN_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace_bytes, need);
-
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
+// The MLA decode launches after validation: partials at `parts` (the workspace past its
+// header), device flags into `status`.
+static int mla_run(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
+                   const int32_t* seq_lens, float scale, void* out, float* lse, int B, int H, int Dc, int Dr,
+                   int T_max, uint8_t* parts, int* status, cudaStream_t st) {
   const size_t slots = static_cast<size_t>(attn::kMlaMaxPairs) + B;
-  float* part_o = reinterpret_cast<float*>(ws + kHeader);
-  float* part_lse = reinterpret_cast<float*>(ws + kHeader + round_up(slots * H * Dc * sizeof(float), 256));
-  int rc = clear_status(ws, st);
-  if (rc) return rc;
+  float* part_o = reinterpret_cast<float*>(parts);
+  float* part_lse = reinterpret_cast<float*>(parts + round_up(slots * H * Dc * sizeof(float), 256));
+  int rc = ATTN_OK;
 
   CUtensorMap tmKV, tmPE;
   {
@@ -582,7 +568,7 @@ int mla_decode(const void* q_nope, const void* q_pe, const void* kv_cache, const
   p.T_max = T_max;
   p.n_pairs = attn::mla_pairs_for_device();
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.status = reinterpret_cast<int*>(ws);
+  p.status = status;
   prof_before(st);
   cudaError_t e = attn::launch_mla(p, tmKV, tmPE, st);
   prof_after(st);
@@ -590,6 +576,120 @@ int mla_decode(const void* q_nope, const void* q_pe, const void* kv_cache, const
   e = attn::launch_mla_merge(part_o, part_lse, seq_lens, out, lse, B, H, T_max, p.n_pairs, st);
   if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   return ok();
+}
+
+int mla_decode(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
+               const int32_t* seq_lens, float scale, void* out, float* lse, int B, int H, int Dc, int Dr, int T_max,
+               void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q_nope || !q_pe || !kv_cache || !pe_cache || !seq_lens || !out || !lse || !workspace)
+    return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
+  if (B <= 0 || H <= 0 || Dc <= 0 || Dr <= 0 || T_max <= 0) return fail(ATTN_ERR_INVALID_ARG, "sizes must be positive");
+  if (H != 128 || Dc != 512 || Dr != 64)
+    return fail(ATTN_ERR_UNSUPPORTED, "MLA decode supports H=128, Dc=512, Dr=64 (got %d, %d, %d)", H, Dc, Dr);
+  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(ATTN_ERR_INVALID_ARG, "scale must be positive");
+  if (!aligned(q_nope, 16) || !aligned(q_pe, 16) || !aligned(kv_cache, 16) || !aligned(pe_cache, 16) ||
+      !aligned(out, 16) || !aligned(seq_lens, 4) || !aligned(lse, 4) || !aligned(workspace, 256))
+    return fail(ATTN_ERR_INVALID_ARG, "misaligned pointer");
+  if (T_max > (1 << 26) || B > (1 << 20)) return fail(ATTN_ERR_UNSUPPORTED, "problem too large");
+  const size_t need = mla_decode_workspace_size(B, H, Dc, Dr, T_max);
+  if (workspace_bytes < need)
+    return fail(ATTN_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace_bytes, need);
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int rc = clear_status(ws, st);
+  if (rc) return rc;
+  return mla_run(q_nope, q_pe, kv_cache, pe_cache, seq_lens, scale, out, lse, B, H, Dc, Dr, T_max, ws + kHeader,
+                 reinterpret_cast<int*>(ws), st);
+}
+
+// ------------------------------------------------ DeepSeek sparse attention
+size_t dsa_index_topk_workspace_size(int B, int H_I, int d_I, int T_max, int top_k) {
+  (void)B;
+  (void)H_I;
+  (void)d_I;
+  (void)T_max;
+  (void)top_k;
+  return kHeader;  // the status word only
+}
+
+int dsa_index_topk(const void* q_idx, const float* w_idx, const void* k_idx, const int32_t* seq_lens, float* scores,
+                   int32_t* topk_idx, int B, int H_I, int d_I, int T_max, int top_k, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  if (!q_idx || !w_idx || !k_idx || !seq_lens || !scores || !topk_idx || !workspace)
+    return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
+  if (B <= 0 || H_I <= 0 || d_I <= 0 || T_max <= 0 || top_k <= 0)
+    return fail(ATTN_ERR_INVALID_ARG, "sizes must be positive");
+  if (d_I != attn::kDsaIndexDim) return fail(ATTN_ERR_UNSUPPORTED, "indexer width %d (supported: 128)", d_I);
+  if (H_I % 16 != 0 || H_I > attn::kDsaMaxIndexHeads)
+    return fail(ATTN_ERR_UNSUPPORTED, "indexer heads %d (supported: multiples of 16 up to 64)", H_I);
+  if (T_max > (1 << 26) || B > 65535 || top_k > (1 << 26)) return fail(ATTN_ERR_UNSUPPORTED, "problem too large");
+  if (!aligned(q_idx, 16) || !aligned(k_idx, 16) || !aligned(w_idx, 4) || !aligned(seq_lens, 4) ||
+      !aligned(scores, 4) || !aligned(topk_idx, 4) || !aligned(workspace, 256))
+    return fail(ATTN_ERR_INVALID_ARG, "misaligned pointer");
+  const size_t need = dsa_index_topk_workspace_size(B, H_I, d_I, T_max, top_k);
+  if (workspace_bytes < need)
+    return fail(ATTN_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace_bytes, need);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int rc = clear_status(workspace, st);
+  if (rc) return rc;
+  attn::DsaIndexParams p{};
+  p.q = q_idx;
+  p.w = w_idx;
+  p.k = k_idx;
+  p.seq_lens = seq_lens;
+  p.scores = scores;
+  p.B = B;
+  p.HI = H_I;
+  p.T_max = T_max;
+  prof_before(st);
+  cudaError_t e = attn::launch_dsa_index(p, st);
+  prof_after(st);
+  if (e != cudaSuccess) return cuda_fail(e, "indexer launch");
+  e = attn::launch_dsa_topk(scores, seq_lens, topk_idx, B, T_max, top_k, st);
+  if (e != cudaSuccess) return cuda_fail(e, "top-k launch");
+  return ok();
+}
+
+// workspace: [status | MLA partials | kv_sel B x top_k x Dc | pe_sel B x top_k x Dr | n_sel B]
+size_t dsa_mla_decode_workspace_size(int B, int H, int Dc, int Dr, int top_k) {
+  if (B <= 0 || H <= 0 || Dc <= 0 || Dr <= 0 || top_k <= 0) return kHeader;
+  const size_t mla = mla_decode_workspace_size(B, H, Dc, Dr, top_k);
+  const size_t rows = static_cast<size_t>(B) * top_k;
+  return mla + round_up(rows * Dc * 2, 256) + round_up(rows * Dr * 2, 256) + round_up(static_cast<size_t>(B) * 4, 256);
+}
+
+int dsa_mla_decode(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
+                   const int32_t* seq_lens, const int32_t* topk_idx, int top_k, float scale, void* out, float* lse,
+                   int B, int H, int Dc, int Dr, int T_max, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q_nope || !q_pe || !kv_cache || !pe_cache || !seq_lens || !topk_idx || !out || !lse || !workspace)
+    return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
+  if (B <= 0 || H <= 0 || Dc <= 0 || Dr <= 0 || T_max <= 0 || top_k <= 0)
+    return fail(ATTN_ERR_INVALID_ARG, "sizes must be positive");
+  if (H != 128 || Dc != 512 || Dr != 64)
+    return fail(ATTN_ERR_UNSUPPORTED, "MLA decode supports H=128, Dc=512, Dr=64 (got %d, %d, %d)", H, Dc, Dr);
+  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(ATTN_ERR_INVALID_ARG, "scale must be positive");
+  if (!aligned(q_nope, 16) || !aligned(q_pe, 16) || !aligned(kv_cache, 16) || !aligned(pe_cache, 16) ||
+      !aligned(out, 16) || !aligned(seq_lens, 4) || !aligned(topk_idx, 4) || !aligned(lse, 4) ||
+      !aligned(workspace, 256))
+    return fail(ATTN_ERR_INVALID_ARG, "misaligned pointer");
+  if (T_max > (1 << 26) || B > (1 << 20) || top_k > (1 << 26)) return fail(ATTN_ERR_UNSUPPORTED, "problem too large");
+  const size_t need = dsa_mla_decode_workspace_size(B, H, Dc, Dr, top_k);
+  if (workspace_bytes < need)
+    return fail(ATTN_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace_bytes, need);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t rows = static_cast<size_t>(B) * top_k;
+  uint8_t* kv_sel = ws + mla_decode_workspace_size(B, H, Dc, Dr, top_k);
+  uint8_t* pe_sel = kv_sel + round_up(rows * Dc * 2, 256);
+  int32_t* n_sel = reinterpret_cast<int32_t*>(pe_sel + round_up(rows * Dr * 2, 256));
+  int* status = reinterpret_cast<int*>(ws);
+  int rc = clear_status(ws, st);
+  if (rc) return rc;
+  cudaError_t e = attn::launch_dsa_gather(kv_cache, pe_cache, topk_idx, seq_lens, kv_sel, pe_sel, n_sel, B, T_max,
+                                          top_k, Dc, Dr, status, st);
+  if (e != cudaSuccess) return cuda_fail(e, "gather launch");
+  return mla_run(q_nope, q_pe, kv_sel, pe_sel, n_sel, scale, out, lse, B, H, Dc, Dr, top_k, ws + kHeader, status, st);
 }
 
 int attn_read_status(const void* workspace, int* flags, void* stream) {

@@ -30,6 +30,7 @@ if ROOT not in sys.path:
 PREFILL = "gqa_prefill_b2_hq32_hkv8_s4096_d128"
 DECODE = "paged_decode_b64_hq32_hkv8_d128"
 MLA = "mla_decode_b32_h128_dc512_dr64"
+DSA = "dsa_mla_decode_b32_h128_dc512_dr64_hi64_di128_top2048"
 PREFILL_LONG = "gqa_prefill_b1_hq32_hkv8_s32768_d128"
 CHUNK = "chunk_prefill_b8_hq32_hkv8_d128_n2048_cache4k_28k"
 METRIC = "prefill attn TFLOP/s & decode KV-read GB/s, % of B200 roofline"
@@ -481,6 +482,69 @@ def bench_mla(args, world, dev, seed, pk, pk_kind, fp):
     return res
 
 
+def bench_dsa(args, world, dev, seed, pk, pk_kind, dense_ms=None):
+    """DeepSeek sparse attention on the MLA workload: lightning indexer + top-k over every
+    cached token, then the MLA decode over the 2048 selected tokens per sequence."""
+    import torch
+    from attention_causal_gqa_b200 import binding as B_
+    from attention_causal_gqa_b200.synthetic import WORKLOADS, dsa_inputs, workload_inputs
+    p = dict(WORKLOADS[DSA].params)
+    if args.small:
+        p["B"] = 8
+        d = dsa_inputs(8, p["H"], p["Dc"], p["Dr"], p["HI"], p["dI"], p["lmin"], p["lmax"], p["std"], seed, dev)
+    else:
+        d = workload_inputs(DSA, seed=seed, device=dev)
+    B, T, K = p["B"], d["T_max"], p["top_k"]
+    scores = torch.empty((B, T), dtype=torch.float32, device=dev)
+    idx = torch.empty((B, K), dtype=torch.int32, device=dev)
+    out = torch.empty_like(d["q_nope"])
+    lse = torch.empty((B, 1, p["H"]), dtype=torch.float32, device=dev)
+    ws1 = torch.empty(256, dtype=torch.uint8, device=dev)
+    ws2 = torch.empty(B_.dsa_mla_workspace_size(B, p["H"], p["Dc"], p["Dr"], K), dtype=torch.uint8, device=dev)
+
+    def index():
+        B_.dsa_index_topk(d["q_idx"], d["w_idx"], d["k_idx"], d["seq_lens"], K, scores=scores, topk_idx=idx,
+                          workspace=ws1)
+
+    def attend():
+        B_.dsa_mla_decode(d["q_nope"], d["q_pe"], d["kv_cache"], d["pe_cache"], d["seq_lens"], idx, p["scale"],
+                          out=out, lse=lse, workspace=ws2)
+
+    def step():
+        index()
+        attend()
+
+    tokens = int(d["seq_lens"].sum().item())
+    selected = int(d["seq_lens"].clamp(max=K).sum().item())
+    idx_bytes = tokens * (p["dI"] * 2 + 4)  # indexer keys read + scores written
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    B_.profile_collect()
+    ms = timed_region(step, args.steps, 0, world)
+    B_.profile_collect()  # (the step's two brackets; kernel times are taken one call at a time below)
+    ms_index = timed_region(index, args.steps, 0, world)
+    k_ms, n = B_.profile_collect()
+    k_idx = max_over_ranks(k_ms / max(n, 1), world)
+    ms_attend = timed_region(attend, args.steps, 0, world)
+    m_ms, mn = B_.profile_collect()
+    k_mla = max_over_ranks(m_ms / max(mn, 1), world)
+    ach = idx_bytes / (k_idx * 1e-3) / 1e9
+    res = {"workload": DSA + ("_small_b8" if args.small else ""), "value": world * tokens * args.steps / (ms * 1e-3),
+           "unit": "cached tokens/s", "ms_per_step": ms / args.steps, "kv_tokens": tokens,
+           "selected_tokens": selected, "index_call_ms": ms_index / args.steps,
+           "sparse_mla_call_ms": ms_attend / args.steps, "mla_kernel_ms": k_mla,
+           "dense_mla_ms_per_step": dense_ms, "gpu_launches": 5 * args.steps,
+           "l2": "indexer keys (268 MB) and caches larger than L2",
+           "roofline": {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                        "frac": ach / pk["hbm_gbs"], "traffic": traffic_for("dsa_index_kernel"),
+                        "kernel": "dsa_index_kernel", "kernel_ms": k_idx, "peak_kind": f"{pk_kind} HBM copy",
+                        "algorithmic": "260 B per cached token (128 bf16 indexer key + fp32 score)"}}
+    del d, scores, idx, out, lse, ws1, ws2
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args):
     import torch
     world, rank, local = dist_setup()
@@ -521,6 +585,9 @@ def run_ours(args):
         sub["decode_fp8"] = bench_decode_fp8(args, world, dev, seed, pk, pk_kind)
     if do("mla"):
         sub["mla"] = bench_mla(args, world, dev, seed, pk, pk_kind, fp)
+    if do("mla") or do("dsa"):
+        dense = sub["mla"]["ms_per_step"] if "mla" in sub else None
+        sub["dsa"] = bench_dsa(args, world, dev, seed, pk, pk_kind, dense_ms=dense)
     clk = clocks.stop()
     B_.profile_enable(False)
 
@@ -566,7 +633,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--only", choices=["prefill", "decode", "mla"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "mla", "dsa"], default=None,
                     help="run one workload (for profiling); the JSON line then carries that workload only")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--small", action="store_true",

@@ -41,7 +41,7 @@ enum {
 enum { ATTN_DTYPE_F32 = 0, ATTN_DTYPE_BF16 = 1 };
 
 /* Device status flags (attn_read_status). */
-enum { ATTN_DEV_TIMEOUT = 1, ATTN_DEV_BAD_PAGE = 2, ATTN_DEV_BAD_LENGTH = 4, ATTN_DEV_RANGE = 8 };
+enum { ATTN_DEV_TIMEOUT = 1, ATTN_DEV_BAD_PAGE = 2, ATTN_DEV_BAD_LENGTH = 4, ATTN_DEV_RANGE = 8, ATTN_DEV_BAD_INDEX = 16 };
 
 /*
  * Causal GQA/MQA/MHA prefill with RoPE.
@@ -178,6 +178,45 @@ size_t mla_decode_workspace_size(int B, int H, int Dc, int Dr, int T_max);
 int mla_decode(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
                const int32_t* seq_lens, float scale, void* out, float* lse, int B, int H, int Dc, int Dr, int T_max,
                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * DeepSeek sparse attention, step 1: lightning-indexer scores and the top-k selection.
+ * Defined by: "attention study note" (makinaruto), section "Lighting Indexer": indexer
+ * queries q_j (one per indexer head j), one indexer key k_s per cached token, and the
+ * index score sum_j w_j * ReLU(q_j . k_s); only the most relevant tokens are attended.
+ *
+ *   q_idx    [B, H_I, d_I] bf16   indexer queries of each sequence's decode token
+ *   w_idx    [B, H_I] fp32        indexer head weights
+ *   k_idx    [B, T_max, d_I] bf16 indexer keys of the cached tokens
+ *   seq_lens [B] int32            cached tokens per sequence (clamped to [0, T_max])
+ *   scores   [B, T_max] fp32      out: I[b, s] for s < seq_lens[b], -inf past it
+ *   topk_idx [B, top_k] int32     out: the min(top_k, seq_lens[b]) tokens with the largest
+ *                                 scores (ties: smaller token index first), in ascending
+ *                                 token order, then -1
+ * Scores are fp32 (bf16 products accumulated in fp32, then ReLU, weights and the head sum
+ * in fp32); the selection is exact with respect to those scores. Supported: d_I = 128,
+ * H_I a multiple of 16 up to 64. All device pointers, caller-owned; 16-byte aligned q_idx
+ * and k_idx. workspace: >= dsa_index_topk_workspace_size() bytes (status word).
+ */
+size_t dsa_index_topk_workspace_size(int B, int H_I, int d_I, int T_max, int top_k);
+int dsa_index_topk(const void* q_idx, const float* w_idx, const void* k_idx, const int32_t* seq_lens, float* scores,
+                   int32_t* topk_idx, int B, int H_I, int d_I, int T_max, int top_k, void* workspace,
+                   size_t workspace_bytes, void* stream);
+
+/*
+ * DeepSeek sparse attention, step 2: the MLA absorbed decode (mla_decode) over the
+ * selected tokens only: scores, softmax and output use the rows kv_cache[b, t] and
+ * pe_cache[b, t] for t = topk_idx[b, i], i < min(seq_lens[b], top_k) (as written by
+ * dsa_index_topk; any distinct indices in [0, seq_lens[b]) are accepted, an index outside
+ * it flags ATTN_DEV_BAD_INDEX and reads row 0). Same tensors, layouts and limits as
+ * mla_decode. The selected rows are gathered into the workspace, then attended by the
+ * MLA kernel. workspace: >= dsa_mla_decode_workspace_size(B, H, Dc, Dr, top_k) bytes,
+ * 256-byte aligned, caller-owned scratch (status word first).
+ */
+size_t dsa_mla_decode_workspace_size(int B, int H, int Dc, int Dr, int top_k);
+int dsa_mla_decode(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
+                   const int32_t* seq_lens, const int32_t* topk_idx, int top_k, float scale, void* out, float* lse,
+                   int B, int H, int Dc, int Dr, int T_max, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Paged decode for callers that cannot allocate device memory (code running
