@@ -30,7 +30,7 @@ ATTN_DEV_RANGE = 8
 ATTN_DEV_BAD_INDEX = 16
 
 EXPORTED = (
-    "attn_prefill_workspace_size", "attn_prefill",
+    "attn_prefill_workspace_size", "attn_prefill", "attn_prefill_ex",
     "attn_decode_paged_workspace_size", "attn_decode_paged",
     "attn_decode_paged_fp8_workspace_size", "mla_decode_workspace_size", "mla_decode",
     "dsa_index_topk_workspace_size", "dsa_index_topk", "dsa_mla_decode_workspace_size", "dsa_mla_decode",
@@ -52,6 +52,8 @@ def _load() -> ctypes.CDLL:
     vp, i32, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.attn_prefill_workspace_size.restype = sz
     lib.attn_prefill_workspace_size.argtypes = [i32] * 5
+    lib.attn_prefill_ex.restype = i32
+    lib.attn_prefill_ex.argtypes = [vp] * 5 + [i32] * 6 + [f32, f32, i32, f32, i32, vp, sz, vp]
     lib.attn_prefill.restype = i32
     lib.attn_prefill.argtypes = [vp] * 5 + [i32] * 6 + [f32, f32, i32, vp, sz, vp]
     lib.attn_decode_paged_workspace_size.restype = sz
@@ -131,10 +133,26 @@ def prefill_workspace_size(B, Hkv, S, D, dtype=torch.bfloat16) -> int:
     return int(lib.attn_prefill_workspace_size(B, Hkv, S, D, dt))
 
 
+ROPE_LAYOUTS = {"interleaved": 0, "half": 1}  # ATTN_ROPE_INTERLEAVED, ATTN_ROPE_HALF_SPLIT
+
+
+def ntk_aware_theta(theta: float, scale: float, head_dim: int) -> float:
+    """NTK-aware RoPE base for a context stretched by `scale` (the long-context page names the
+    method; the rule is the published one): theta * scale^(D / (D - 2)), which divides the
+    lowest rotary frequency by `scale` and leaves the highest unchanged."""
+    return float(theta) * float(scale) ** (head_dim / (head_dim - 2.0))
+
+
+def length_scaled_theta(theta: float, length: int, base_length: int, alpha: float) -> float:
+    """The long-context page's length-aware base (section 2.4): theta * (L / L0)^alpha."""
+    return float(theta) * (float(length) / float(base_length)) ** float(alpha)
+
+
 def attn_prefill(q, k, v, causal=True, rope_theta=10000.0, scale=None, out=None, lse=None, workspace=None,
-                 stream=None):
+                 stream=None, rope_freq_scale=1.0, rope_layout="interleaved"):
     """Causal GQA prefill with RoPE. q [B,Hq,S,D], k/v [B,Hkv,S,D] (bf16 or fp32).
-    Returns (out [B,Hq,S,D] same dtype, lse [B,Hq,S] fp32)."""
+    rope_freq_scale multiplies every rotary frequency; rope_layout "interleaved" pairs
+    (2i, 2i+1), "half" pairs (i, i + D/2). Returns (out [B,Hq,S,D] same dtype, lse [B,Hq,S] fp32)."""
     _need_cuda(q, k, v)
     B, Hq, S, D = q.shape
     Hkv = k.shape[1]
@@ -145,9 +163,17 @@ def attn_prefill(q, k, v, causal=True, rope_theta=10000.0, scale=None, out=None,
         lse = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
     ws_bytes = prefill_workspace_size(B, Hkv, S, D, q.dtype)
     ws = _workspace(ws_bytes, q.device, workspace)
-    rc = lib.attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, S, D, int(bool(causal)),
-                          float(rope_theta if rope_theta else 0.0), float(scale or 0.0), dt, _ptr(ws),
-                          ws.numel() * ws.element_size(), _stream(stream))
+    if rope_layout not in ROPE_LAYOUTS:
+        raise ValueError(f"rope_layout must be one of {sorted(ROPE_LAYOUTS)}")
+    if float(rope_freq_scale) == 1.0 and rope_layout == "interleaved":
+        rc = lib.attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, S, D, int(bool(causal)),
+                              float(rope_theta if rope_theta else 0.0), float(scale or 0.0), dt, _ptr(ws),
+                              ws.numel() * ws.element_size(), _stream(stream))
+    else:
+        rc = lib.attn_prefill_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, S, D,
+                                 int(bool(causal)), float(rope_theta if rope_theta else 0.0), float(rope_freq_scale),
+                                 ROPE_LAYOUTS[rope_layout], float(scale or 0.0), dt, _ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream))
     _check(rc)
     return out, lse
 

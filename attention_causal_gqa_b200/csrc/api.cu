@@ -144,14 +144,19 @@ size_t attn_prefill_workspace_size(int B, int Hkv, int S, int D, int dtype) {
   return kHeader + table + round_up(n * 2, 256);
 }
 
-int attn_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv, int S,
-                 int D, int causal, float rope_theta, float scale, int dtype, void* workspace,
-                 size_t workspace_bytes, void* stream) {
+int attn_prefill_ex(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv, int S,
+                    int D, int causal, float rope_theta, float rope_freq_scale, int rope_layout, float scale, int dtype,
+                    void* workspace, size_t workspace_bytes, void* stream) {
   if (!q || !k || !v || !out || !lse || !workspace) return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || S <= 0 || D <= 0)
     return fail(ATTN_ERR_INVALID_ARG, "sizes must be positive (B=%d Hq=%d Hkv=%d S=%d D=%d)", B, Hq, Hkv, S, D);
   if (Hq % Hkv != 0) return fail(ATTN_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
   if (dtype != ATTN_DTYPE_BF16 && dtype != ATTN_DTYPE_F32) return fail(ATTN_ERR_UNSUPPORTED, "dtype %d", dtype);
+  if (rope_layout != ATTN_ROPE_INTERLEAVED && rope_layout != ATTN_ROPE_HALF_SPLIT)
+    return fail(ATTN_ERR_INVALID_ARG, "rope_layout %d", rope_layout);
+  if (!(rope_freq_scale > 0.f) || !std::isfinite(rope_freq_scale))
+    return fail(ATTN_ERR_INVALID_ARG, "rope_freq_scale must be positive and finite");
+  const bool half_split = rope_layout == ATTN_ROPE_HALF_SPLIT;
   const bool f32 = dtype == ATTN_DTYPE_F32;
   if (!(f32 ? D == 64 : (D == 64 || D == 128)))
     return fail(ATTN_ERR_UNSUPPORTED, "head dim %d unsupported for %s", D, f32 ? "fp32" : "bf16");
@@ -178,7 +183,8 @@ int attn_prefill(const void* q, const void* k, const void* v, void* out, float* 
 
   const bool rope = rope_theta > 0.f;
   if (rope) {
-    cudaError_t e = attn::launch_rope_table(cs, S, D, static_cast<double>(rope_theta), st);
+    cudaError_t e = attn::launch_rope_table(cs, S, D, static_cast<double>(rope_theta),
+                                            static_cast<double>(rope_freq_scale), st);
     if (e != cudaSuccess) return cuda_fail(e, "rope table launch");
   }
   const long long rows = static_cast<long long>(B) * Hkv * S;
@@ -187,14 +193,15 @@ int attn_prefill(const void* q, const void* k, const void* v, void* out, float* 
   CUtensorMapDataType kdt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   cuuint64_t zdim = static_cast<cuuint64_t>(B) * Hkv;
   if (f32) {
-    cudaError_t e = attn::launch_split_f32(static_cast<const float*>(k), kop, rope ? cs : nullptr, rows, S, D, st);
-    if (e == cudaSuccess) e = attn::launch_split_f32(static_cast<const float*>(v), vop, nullptr, rows, S, D, st);
+    cudaError_t e =
+        attn::launch_split_f32(static_cast<const float*>(k), kop, rope ? cs : nullptr, rows, S, D, half_split, st);
+    if (e == cudaSuccess) e = attn::launch_split_f32(static_cast<const float*>(v), vop, nullptr, rows, S, D, false, st);
     if (e != cudaSuccess) return cuda_fail(e, "operand split launch");
     kbase = kop;
     vbase = vop;
     zdim *= 2;
   } else if (rope) {
-    cudaError_t e = attn::launch_rope_k_f16(k, kop, cs, rows, S, D, status, st);
+    cudaError_t e = attn::launch_rope_k_f16(k, kop, cs, rows, S, D, half_split, status, st);
     if (e != cudaSuccess) return cuda_fail(e, "rope K launch");
     kbase = kop;
     kdt = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -208,12 +215,13 @@ int attn_prefill(const void* q, const void* k, const void* v, void* out, float* 
   CUtensorMapDataType qdt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   cuuint64_t zq = static_cast<cuuint64_t>(B) * Hq;
   if (f32) {
-    cudaError_t e = attn::launch_split_f32(static_cast<const float*>(q), out, rope ? cs : nullptr, rows_q, S, D, st);
+    cudaError_t e =
+        attn::launch_split_f32(static_cast<const float*>(q), out, rope ? cs : nullptr, rows_q, S, D, half_split, st);
     if (e != cudaSuccess) return cuda_fail(e, "Q operand split launch");
     qbase = out;
     zq *= 2;
   } else if (rope) {
-    cudaError_t e = attn::launch_rope_k_f16(q, out, cs, rows_q, S, D, status, st);
+    cudaError_t e = attn::launch_rope_k_f16(q, out, cs, rows_q, S, D, half_split, status, st);
     if (e != cudaSuccess) return cuda_fail(e, "rope Q launch");
     qbase = out;
     qdt = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -255,6 +263,13 @@ int attn_prefill(const void* q, const void* k, const void* v, void* out, float* 
   prof_after(st);
   if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
   return ok();
+}
+
+int attn_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv, int S,
+                 int D, int causal, float rope_theta, float scale, int dtype, void* workspace, size_t workspace_bytes,
+                 void* stream) {
+  return attn_prefill_ex(q, k, v, out, lse, B, Hq, Hkv, S, D, causal, rope_theta, 1.0f, ATTN_ROPE_INTERLEAVED, scale,
+                         dtype, workspace, workspace_bytes, stream);
 }
 
 // Chunked-prefill workspace: [status | cos/sin table [Sk_max, D/2] | keys fp16
@@ -308,7 +323,7 @@ int attn_prefill_chunk(const void* q, const void* k, const void* v, void* k_page
   if (rc) return rc;
   const bool rope = rope_theta > 0.f;
   if (rope) {
-    cudaError_t e = attn::launch_rope_table(cs, static_cast<int>(sk), D, static_cast<double>(rope_theta), st);
+    cudaError_t e = attn::launch_rope_table(cs, static_cast<int>(sk), D, static_cast<double>(rope_theta), 1.0, st);
     if (e != cudaSuccess) return cuda_fail(e, "rope table launch");
   }
   attn::ChunkGeometry g{cache_lens, block_table, B, Hkv, S_new, D, page_size, max_pages_per_seq, num_pages,

@@ -8,16 +8,17 @@
 
 namespace attn {
 
-// RoPE prologue: cos/sin table (angles in fp64), then the key operand.
-cudaError_t launch_rope_table(float2* cs, int S, int D, double theta, cudaStream_t stream);
+// RoPE prologue: cos/sin table of pos * freq_scale * theta^(-2i/D) (angles in fp64), then
+// the operands. half_split: element d pairs with d + D/2 instead of 2i with 2i + 1.
+cudaError_t launch_rope_table(float2* cs, int S, int D, double theta, double freq_scale, cudaStream_t stream);
 // bf16 X [rows, D] -> rotated fp16 X (row r at position r % S); flags values outside fp16 range.
 // Used for K and for Q.
 cudaError_t launch_rope_k_f16(const void* k, void* k_f16, const float2* cs, long long rows, int S, int D,
-                              int* status, cudaStream_t stream);
+                              bool half_split, int* status, cudaStream_t stream);
 // fp32 X [rows, D] -> bf16 hi parts at out[0, rows) and lo parts at out[rows, 2 rows), rotating
 // first when cs is non-null.
 cudaError_t launch_split_f32(const float* x, void* out, const float2* cs, long long rows, int S, int D,
-                             cudaStream_t stream);
+                             bool half_split, cudaStream_t stream);
 
 // --------------------------------------------- chunked prefill into the paged cache
 struct ChunkGeometry {

@@ -1,11 +1,14 @@
 // RoPE prologue ("From 32K to 256K: DeepSeek long-context", section 2.1 for the
 // rotation, section 2.5 for the cos/sin cache [max_len, head_dim/2, 2]).
 //
-// The table stores cos and sin of pos * theta^(-2i/D) for every integer position
-// and pair; each angle is formed in fp64 straight from the integer position (no
-// running phase), then rounded to fp32. Pairs are adjacent elements (2i, 2i+1):
+// The table stores cos and sin of pos * f * theta^(-2i/D) for every integer position
+// and pair (f: a frequency scale, 1 for plain RoPE; section 2.2 scales the frequencies
+// by a factor, section 2.4 rescales the base theta, which callers pass as theta); each
+// angle is formed in fp64 straight from the integer position (no running phase), then
+// rounded to fp32. Pairs are adjacent elements (2i, 2i+1) by default:
 //   y[2i]   = x[2i] cos - x[2i+1] sin
 //   y[2i+1] = x[2i] sin + x[2i+1] cos
+// and (i, i + D/2) in the half-split layout (the concatenated-halves form of section 2.4).
 #include <cmath>
 
 #include <cuda_bf16.h>
@@ -86,39 +89,120 @@ __global__ void __launch_bounds__(256) rope_f16_kernel(const uint4* __restrict__
   if (!in_range) atomicOr(status, 8);
 }
 
-// fp32 X [heads, S, D] -> hi = bf16(x) in out[0, heads), lo = bf16(x - hi) in
-// out[heads, 2 heads), rotating first when cs is non-null.
+// The cos/sin of pairs 8c .. 8c+7 (half-split layout: chunk c of the first half).
 template <int CPR>
+__device__ __forceinline__ void load_cs8(const float2* __restrict__ cs, int pos, int c, float2 (&a)[8]) {
+  const float4* t = reinterpret_cast<const float4*>(cs + static_cast<size_t>(pos) * (CPR * 4) + c * 8);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float4 u = __ldg(t + k);
+    a[2 * k] = make_float2(u.x, u.y);
+    a[2 * k + 1] = make_float2(u.z, u.w);
+  }
+}
+
+// Half-split layout of rope_f16_kernel: the thread of chunk c < CPR/2 rotates it together
+// with its partner chunk c + CPR/2 (element d pairs with d + D/2); the others have no work.
+template <int CPR>
+__global__ void __launch_bounds__(256) rope_f16_half_kernel(const uint4* __restrict__ x, uint4* __restrict__ y,
+                                                            const float2* __restrict__ cs, int heads, int S,
+                                                            int* __restrict__ status) {
+  int pos, c;
+  if (!chunk_position<CPR>(S, pos, c) || c >= CPR / 2) return;
+  float2 a[8];
+  load_cs8<CPR>(cs, pos, c, a);
+  bool in_range = true;
+  for (int hd = blockIdx.y; hd < heads; hd += gridDim.y) {
+    const size_t idx = (static_cast<size_t>(hd) * S + pos) * CPR + c;
+    const uint4 rl = x[idx], rh = x[idx + CPR / 2];
+    const uint32_t wl[4] = {rl.x, rl.y, rl.z, rl.w}, wh[4] = {rh.x, rh.y, rh.z, rh.w};
+    uint32_t ol[4], oh[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float lo[2] = {__uint_as_float(wl[e] << 16), __uint_as_float(wl[e] & 0xFFFF0000u)};
+      float hi[2] = {__uint_as_float(wh[e] << 16), __uint_as_float(wh[e] & 0xFFFF0000u)};
+      float yl[2], yh[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const float2 cz = a[2 * e + k];
+        yl[k] = lo[k] * cz.x - hi[k] * cz.y;
+        yh[k] = lo[k] * cz.y + hi[k] * cz.x;
+        in_range = in_range && fabsf(yl[k]) <= 65504.f && fabsf(yh[k]) <= 65504.f;
+      }
+      const __half2 vl = __floats2half2_rn(yl[0], yl[1]), vh = __floats2half2_rn(yh[0], yh[1]);
+      ol[e] = *reinterpret_cast<const uint32_t*>(&vl);
+      oh[e] = *reinterpret_cast<const uint32_t*>(&vh);
+    }
+    y[idx] = make_uint4(ol[0], ol[1], ol[2], ol[3]);
+    y[idx + CPR / 2] = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+  }
+  if (!in_range) atomicOr(status, 8);
+}
+
+// fp32 X [heads, S, D] -> hi = bf16(x) in out[0, heads), lo = bf16(x - hi) in
+// out[heads, 2 heads), rotating first when cs is non-null. HALF: half-split pairs (the
+// thread of chunk c < CPR/2 handles chunks c and c + CPR/2).
+template <int CPR, bool HALF>
 __global__ void __launch_bounds__(256) split_f32_kernel(const float4* __restrict__ x, uint4* __restrict__ out,
                                                         const float2* __restrict__ cs, int heads, int S) {
   int pos, c;
   if (!chunk_position<CPR>(S, pos, c)) return;
-  float2 a[4];
-  if (cs) load_cs4<CPR>(cs, pos, c, a);
+  if (HALF && c >= CPR / 2) return;
+  constexpr int NC = HALF ? 2 : 1;  // chunks per thread
+  float2 a[8];
+  if (cs) {
+    if constexpr (HALF) {
+      load_cs8<CPR>(cs, pos, c, a);
+    } else {
+      float2 a4[4];
+      load_cs4<CPR>(cs, pos, c, a4);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) a[e] = a4[e];
+    }
+  }
   const size_t n = static_cast<size_t>(heads) * S * CPR;
   for (int hd = blockIdx.y; hd < heads; hd += gridDim.y) {
     const size_t idx = (static_cast<size_t>(hd) * S + pos) * CPR + c;
-    const float4 u = x[2 * idx], v = x[2 * idx + 1];
-    float f[8] = {u.x, u.y, u.z, u.w, v.x, v.y, v.z, v.w};
-    if (cs) {
+    float f[NC][8];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float x0 = f[2 * e], x1 = f[2 * e + 1];
-        f[2 * e] = x0 * a[e].x - x1 * a[e].y;
-        f[2 * e + 1] = x0 * a[e].y + x1 * a[e].x;
+    for (int q = 0; q < NC; ++q) {
+      const size_t ix = idx + q * (CPR / 2);
+      const float4 u = x[2 * ix], v = x[2 * ix + 1];
+      f[q][0] = u.x; f[q][1] = u.y; f[q][2] = u.z; f[q][3] = u.w;
+      f[q][4] = v.x; f[q][5] = v.y; f[q][6] = v.z; f[q][7] = v.w;
+    }
+    if (cs) {
+      if constexpr (HALF) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float x0 = f[0][e], x1 = f[NC - 1][e];
+          f[0][e] = x0 * a[e].x - x1 * a[e].y;
+          f[NC - 1][e] = x0 * a[e].y + x1 * a[e].x;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float x0 = f[0][2 * e], x1 = f[0][2 * e + 1];
+          f[0][2 * e] = x0 * a[e].x - x1 * a[e].y;
+          f[0][2 * e + 1] = x0 * a[e].y + x1 * a[e].x;
+        }
       }
     }
-    uint32_t hw[4], lw[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
-      const float2 hf = __bfloat1622float2(h);
-      const __nv_bfloat162 l = __floats2bfloat162_rn(f[2 * e] - hf.x, f[2 * e + 1] - hf.y);
-      hw[e] = *reinterpret_cast<const uint32_t*>(&h);
-      lw[e] = *reinterpret_cast<const uint32_t*>(&l);
+    for (int q = 0; q < NC; ++q) {
+      uint32_t hw[4], lw[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(f[q][2 * e], f[q][2 * e + 1]);
+        const float2 hf = __bfloat1622float2(h);
+        const __nv_bfloat162 l = __floats2bfloat162_rn(f[q][2 * e] - hf.x, f[q][2 * e + 1] - hf.y);
+        hw[e] = *reinterpret_cast<const uint32_t*>(&h);
+        lw[e] = *reinterpret_cast<const uint32_t*>(&l);
+      }
+      const size_t ix = idx + q * (CPR / 2);
+      out[ix] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      out[ix + n] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
-    out[idx] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-    out[idx + n] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
   }
 }
 
@@ -142,38 +226,44 @@ static int grid_for(long long n, int threads) {
   return static_cast<int>(g);
 }
 
-cudaError_t launch_rope_table(float2* cs, int S, int D, double theta, cudaStream_t stream) {
+cudaError_t launch_rope_table(float2* cs, int S, int D, double theta, double freq_scale, cudaStream_t stream) {
   const int half = D / 2;
   if (half < 1 || half > 64) return cudaErrorInvalidValue;
   RopeFreqs f{};
-  for (int i = 0; i < half; ++i) f.inv[i] = std::pow(theta, -2.0 * i / D);
+  for (int i = 0; i < half; ++i) f.inv[i] = freq_scale * std::pow(theta, -2.0 * i / D);
   const long long n = static_cast<long long>(S) * half;
   rope_table_kernel<<<grid_for(n, 256), 256, 0, stream>>>(cs, S, half, f);
   return cudaGetLastError();
 }
 
 cudaError_t launch_rope_k_f16(const void* k, void* k_f16, const float2* cs, long long rows, int S, int D,
-                              int* status, cudaStream_t stream) {
+                              bool half_split, int* status, cudaStream_t stream) {
   const long long heads = rows / S;
   if (heads * S != rows || heads > 0x7fffffffLL) return cudaErrorInvalidValue;
   const dim3 grid = operand_grid(static_cast<int>(heads), S, D / 8);
   const uint4* x = static_cast<const uint4*>(k);
   uint4* y = static_cast<uint4*>(k_f16);
-  if (D == 128) rope_f16_kernel<16><<<grid, 256, 0, stream>>>(x, y, cs, static_cast<int>(heads), S, status);
-  else if (D == 64) rope_f16_kernel<8><<<grid, 256, 0, stream>>>(x, y, cs, static_cast<int>(heads), S, status);
+  const int h = static_cast<int>(heads);
+  if (D == 128 && half_split) rope_f16_half_kernel<16><<<grid, 256, 0, stream>>>(x, y, cs, h, S, status);
+  else if (D == 128) rope_f16_kernel<16><<<grid, 256, 0, stream>>>(x, y, cs, h, S, status);
+  else if (D == 64 && half_split) rope_f16_half_kernel<8><<<grid, 256, 0, stream>>>(x, y, cs, h, S, status);
+  else if (D == 64) rope_f16_kernel<8><<<grid, 256, 0, stream>>>(x, y, cs, h, S, status);
   else return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
 
 cudaError_t launch_split_f32(const float* x, void* out, const float2* cs, long long rows, int S, int D,
-                             cudaStream_t stream) {
+                             bool half_split, cudaStream_t stream) {
   const long long heads = rows / S;
   if (heads * S != rows || heads > 0x7fffffffLL) return cudaErrorInvalidValue;
   const dim3 grid = operand_grid(static_cast<int>(heads), S, D / 8);
   const float4* xx = reinterpret_cast<const float4*>(x);
   uint4* o = static_cast<uint4*>(out);
-  if (D == 64) split_f32_kernel<8><<<grid, 256, 0, stream>>>(xx, o, cs, static_cast<int>(heads), S);
-  else if (D == 128) split_f32_kernel<16><<<grid, 256, 0, stream>>>(xx, o, cs, static_cast<int>(heads), S);
+  const int h = static_cast<int>(heads);
+  if (D == 64 && half_split) split_f32_kernel<8, true><<<grid, 256, 0, stream>>>(xx, o, cs, h, S);
+  else if (D == 64) split_f32_kernel<8, false><<<grid, 256, 0, stream>>>(xx, o, cs, h, S);
+  else if (D == 128 && half_split) split_f32_kernel<16, true><<<grid, 256, 0, stream>>>(xx, o, cs, h, S);
+  else if (D == 128) split_f32_kernel<16, false><<<grid, 256, 0, stream>>>(xx, o, cs, h, S);
   else return cudaErrorInvalidValue;
   return cudaGetLastError();
 }

@@ -40,6 +40,9 @@ enum {
 
 enum { ATTN_DTYPE_F32 = 0, ATTN_DTYPE_BF16 = 1 };
 
+/* RoPE pair layouts (attn_prefill_ex). */
+enum { ATTN_ROPE_INTERLEAVED = 0, ATTN_ROPE_HALF_SPLIT = 1 };
+
 /* Device status flags (attn_read_status). */
 enum { ATTN_DEV_TIMEOUT = 1, ATTN_DEV_BAD_PAGE = 2, ATTN_DEV_BAD_LENGTH = 4, ATTN_DEV_RANGE = 8, ATTN_DEV_BAD_INDEX = 16 };
 
@@ -73,6 +76,23 @@ size_t attn_prefill_workspace_size(int B, int Hkv, int S, int D, int dtype);
 int attn_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv, int S,
                  int D, int causal, float rope_theta, float scale, int dtype, void* workspace,
                  size_t workspace_bytes, void* stream);
+
+/*
+ * attn_prefill with the RoPE scaling variants of "From 32K to 256K: DeepSeek
+ * long-context" (tqpw.cn): section 2.2 scales the rotary frequencies by a factor and
+ * section 2.4 rescales the base (theta' = theta * (L / L0)^alpha; NTK-aware scaling is
+ * likewise a rescaled base), and section 2.4's embedding concatenates the two halves.
+ *   rope_theta       the (possibly rescaled) base; <= 0 disables RoPE as in attn_prefill
+ *   rope_freq_scale  f > 0: the angle of pair i at position p is p * f * rope_theta^(-2i/D)
+ *                    (1 = plain RoPE; 1/s interpolates positions by s)
+ *   rope_layout      ATTN_ROPE_INTERLEAVED: pairs (2i, 2i+1) (attn_prefill's layout);
+ *                    ATTN_ROPE_HALF_SPLIT: pairs (i, i + D/2), i < D/2
+ * Everything else as attn_prefill, which equals attn_prefill_ex(..., rope_freq_scale = 1,
+ * ATTN_ROPE_INTERLEAVED, ...). Invalid layout or non-positive scale: ATTN_ERR_INVALID_ARG.
+ */
+int attn_prefill_ex(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv, int S,
+                    int D, int causal, float rope_theta, float rope_freq_scale, int rope_layout, float scale, int dtype,
+                    void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Paged split-KV GQA decode: one query token per sequence attends to all

@@ -50,43 +50,57 @@ _ROW_BLOCK = 1024  # rows of the score matrix materialised at once (memory only)
 
 
 # --------------------------------------------------------------------------- RoPE
-def rope_cache(seq_len: int, head_dim: int, theta: float) -> np.ndarray:
+def rope_cache(seq_len: int, head_dim: int, theta: float, freq_scale: float = 1.0) -> np.ndarray:
     """cos/sin cache [seq_len, head_dim/2, 2] in float64.
 
     Long-context page, section 2.5 (cache layout) and section 2.1 (theta_i =
     theta^(-2i/d)). Each angle is pos * theta_i computed directly from the
-    integer position, never by accumulation.
+    integer position, never by accumulation. freq_scale multiplies every theta_i
+    (section 2.2's frequency scaling; 1 = plain RoPE).
     """
     if head_dim % 2:
         raise ValueError("RoPE needs an even head dimension")
     i = np.arange(head_dim // 2, dtype=F64)
-    inv_freq = np.power(F64(theta), -2.0 * i / head_dim)
+    inv_freq = F64(freq_scale) * np.power(F64(theta), -2.0 * i / head_dim)
     pos = np.arange(seq_len, dtype=F64)
     ang = pos[:, None] * inv_freq[None, :]
     return np.stack([np.cos(ang), np.sin(ang)], axis=-1)
 
 
-def apply_rope(x: np.ndarray, theta: float, positions: np.ndarray | None = None) -> np.ndarray:
-    """Rotate adjacent pairs (x[2i], x[2i+1]) of the last axis by pos * theta_i.
+def _pair_slices(d: int, layout: str):
+    """The two members of each rotated pair: adjacent (2i, 2i+1) ("interleaved", the
+    long-context page's section 2.1) or the two halves (i, i + d/2) ("half", the
+    concatenated-halves form of its section 2.4)."""
+    if layout == "interleaved":
+        return slice(0, None, 2), slice(1, None, 2)
+    if layout == "half":
+        return slice(0, d // 2), slice(d // 2, d)
+    raise ValueError(f"unknown RoPE layout {layout!r}")
 
-    Long-context page, section 2.1: [x0 cos - x1 sin, x0 sin + x1 cos].
-    ``x`` is [..., S, D]; positions default to 0..S-1.
+
+def apply_rope(x: np.ndarray, theta: float, positions: np.ndarray | None = None, freq_scale: float = 1.0,
+               layout: str = "interleaved") -> np.ndarray:
+    """Rotate the pairs of the last axis by pos * freq_scale * theta_i.
+
+    Long-context page, section 2.1: [x0 cos - x1 sin, x0 sin + x1 cos] on the pair
+    (x0, x1). ``x`` is [..., S, D]; positions default to 0..S-1.
     """
     x = np.asarray(x, dtype=F64)
     s, d = x.shape[-2], x.shape[-1]
     if positions is None:
-        cs = rope_cache(s, d, theta)
+        cs = rope_cache(s, d, theta, freq_scale)
     else:
         i = np.arange(d // 2, dtype=F64)
-        inv_freq = np.power(F64(theta), -2.0 * i / d)
+        inv_freq = F64(freq_scale) * np.power(F64(theta), -2.0 * i / d)
         ang = np.asarray(positions, dtype=F64)[:, None] * inv_freq[None, :]
         cs = np.stack([np.cos(ang), np.sin(ang)], axis=-1)
     cos, sin = cs[..., 0], cs[..., 1]
-    x0 = x[..., 0::2]
-    x1 = x[..., 1::2]
+    a, b = _pair_slices(d, layout)
+    x0 = x[..., a]
+    x1 = x[..., b]
     out = np.empty_like(x)
-    out[..., 0::2] = x0 * cos - x1 * sin
-    out[..., 1::2] = x0 * sin + x1 * cos
+    out[..., a] = x0 * cos - x1 * sin
+    out[..., b] = x0 * sin + x1 * cos
     return out
 
 
@@ -155,11 +169,12 @@ def lse_merge(partial_o, partial_lse):
 
 # -------------------------------------------------------------------- prefill
 def prefill_ref(q, k, v, causal: bool = True, rope_theta: float = 10000.0, scale: float | None = None,
-                rows=None):
+                rows=None, rope_freq_scale: float = 1.0, rope_layout: str = "interleaved"):
     """Exact (causal) GQA/MQA/MHA attention with RoPE on Q and K.
 
     q: [B, Hq, S, D]; k, v: [B, Hkv, S, D] (any float dtype, upcast to float64).
-    rope_theta <= 0 disables RoPE. scale defaults to 1/sqrt(D).
+    rope_theta <= 0 disables RoPE; rope_freq_scale and rope_layout as ``apply_rope``.
+    scale defaults to 1/sqrt(D).
     rows: optional iterable of (b, h, i) triples; when given, only those output rows
     are computed and returned as (o [n, D], lse [n]). Otherwise returns full
     (o [B, Hq, S, D], lse [B, Hq, S]).
@@ -179,13 +194,14 @@ def prefill_ref(q, k, v, causal: bool = True, rope_theta: float = 10000.0, scale
     if scale is None or scale <= 0:
         scale = 1.0 / math.sqrt(D)
     if rope_theta and rope_theta > 0:
-        cs = rope_cache(S, D, rope_theta)
+        cs = rope_cache(S, D, rope_theta, rope_freq_scale)
+        pa, pb = _pair_slices(D, rope_layout)
 
         def rot(x):
             out = np.empty_like(x)
             c, s_ = cs[..., 0], cs[..., 1]
-            out[..., 0::2] = x[..., 0::2] * c - x[..., 1::2] * s_
-            out[..., 1::2] = x[..., 0::2] * s_ + x[..., 1::2] * c
+            out[..., pa] = x[..., pa] * c - x[..., pb] * s_
+            out[..., pb] = x[..., pa] * s_ + x[..., pb] * c
             return out
     else:
         def rot(x):
@@ -202,7 +218,8 @@ def prefill_ref(q, k, v, causal: bool = True, rope_theta: float = 10000.0, scale
                 cache_k[(b, kvh)] = rot(k[b, kvh])
             kr = cache_k[(b, kvh)]
             qi = q[b, h, i][None, :]
-            qi_r = rot_one(qi, i, D, rope_theta) if (rope_theta and rope_theta > 0) else qi
+            qi_r = (rot_one(qi, i, D, rope_theta, rope_freq_scale, rope_layout) if (rope_theta and rope_theta > 0)
+                    else qi)
             hi = i + 1 if causal else S
             s = scale * (qi_r @ kr[:hi].T)
             p, l_ = two_pass_softmax_rows(s)
@@ -231,9 +248,9 @@ def prefill_ref(q, k, v, causal: bool = True, rope_theta: float = 10000.0, scale
     return o, lse
 
 
-def rot_one(x, pos: int, D: int, theta: float):
+def rot_one(x, pos: int, D: int, theta: float, freq_scale: float = 1.0, layout: str = "interleaved"):
     """RoPE of row vector(s) x [n, D] at a single position ``pos``."""
-    return apply_rope(x, theta, positions=np.full(x.shape[0], pos))
+    return apply_rope(x, theta, positions=np.full(x.shape[0], pos), freq_scale=freq_scale, layout=layout)
 
 
 # --------------------------------------------------------------- paged decode

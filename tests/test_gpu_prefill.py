@@ -104,3 +104,24 @@ def test_prefill_rejects_bad_arguments():
     with pytest.raises(AttnError) as e:
         attn_prefill(q, k, v)
     assert e.value.code == 2
+
+
+@cuda
+@pytest.mark.parametrize(
+    "B,Hq,Hkv,S,D,dtype,causal,theta,fscale,layout",
+    [
+        (1, 8, 2, 300, 128, "bf16", True, 1e4, 0.25, "interleaved"),   # positions interpolated by 4
+        (1, 8, 2, 300, 128, "bf16", True, 1e4, 1.0, "half"),           # half-split pairs
+        (2, 4, 4, 257, 64, "bf16", False, 500.0, 0.5, "half"),          # D = 64, non-causal
+        (1, 4, 4, 200, 64, "f32", True, 1e4, 1.0, "half"),             # fp32 operands (hi/lo split)
+        (1, 4, 2, 640, 128, "bf16", True, 8.1e4, 2.0, "half"),         # an NTK-style base, frequencies stretched
+    ],
+)
+def test_prefill_rope_variants(B, Hq, Hkv, S, D, dtype, causal, theta, fscale, layout):
+    from attention_causal_gqa_b200 import attn_prefill
+    q, k, v = _inputs(B, Hq, Hkv, S, D, dtype, seed=B * 7 + S)
+    out, lse = attn_prefill(q, k, v, causal=causal, rope_theta=theta, rope_freq_scale=fscale, rope_layout=layout)
+    torch.cuda.synchronize()
+    ro, rl = prefill_ref(to_np(q), to_np(k), to_np(v), causal=causal, rope_theta=theta, rope_freq_scale=fscale,
+                         rope_layout=layout)
+    check(out, ro, lse, rl, what=f"prefill rope {fscale} {layout} {dtype} D={D}")

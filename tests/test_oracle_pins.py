@@ -604,3 +604,68 @@ def test_dsa_equals_dense_softmax_with_unselected_tokens_masked():
         masked[sel] = sc[sel]
         p, lse = two_pass_softmax_rows(masked[None, :])
         assert np.allclose(o[0, 0, h], (p @ kv[0])[0], atol=1e-12) and abs(l[0, 0, h] - lse[0]) < 1e-12
+
+
+# ------------------------------------------------------ RoPE scaling variants
+def _interleave_halves(x):
+    """(x[i], x[i + D/2]) -> positions (2i, 2i + 1)."""
+    d = x.shape[-1]
+    out = np.empty_like(x)
+    out[..., 0::2] = x[..., :d // 2]
+    out[..., 1::2] = x[..., d // 2:]
+    return out
+
+
+def test_half_split_rope_is_interleaved_rope_on_permuted_dims():
+    from oracle import apply_rope
+    rng = np.random.default_rng(70)
+    x = rng.standard_normal((5, 16))
+    half = apply_rope(x, 500.0, layout="half")
+    inter = apply_rope(_interleave_halves(x), 500.0)
+    assert np.allclose(_interleave_halves(half), inter, atol=1e-13)
+    # and it is not the same function (a plausible mix-up)
+    assert not np.allclose(half, apply_rope(x, 500.0), atol=1e-3)
+
+
+def test_half_split_rope_closed_form_d4():
+    """D = 4, half layout: pairs (0, 2) with theta_0 = 1 and (1, 3) with theta_1 = theta^-1/2."""
+    from oracle import apply_rope
+    x = np.array([[1.0, 2.0, 3.0, 4.0]])
+    p, th = 3, 16.0
+    y = apply_rope(x, th, positions=np.array([p]), layout="half")[0]
+    a0, a1 = p * 1.0, p * th ** -0.5
+    want = [1 * math.cos(a0) - 3 * math.sin(a0), 2 * math.cos(a1) - 4 * math.sin(a1),
+            1 * math.sin(a0) + 3 * math.cos(a0), 2 * math.sin(a1) + 4 * math.cos(a1)]
+    assert np.allclose(y, want, atol=1e-14)
+
+
+def test_frequency_scale_equals_scaled_positions():
+    from oracle import apply_rope
+    rng = np.random.default_rng(71)
+    x = rng.standard_normal((6, 32))
+    pos = np.arange(6) * 7
+    a = apply_rope(x, 1e4, positions=4 * pos, freq_scale=0.25)
+    b = apply_rope(x, 1e4, positions=pos)
+    assert np.array_equal(a, b)  # 4p * (theta_i / 4) = p * theta_i exactly in binary
+
+
+def test_prefill_half_split_equals_interleaved_on_permuted_q_k():
+    from oracle import prefill_ref
+    rng = np.random.default_rng(72)
+    q, k, v = rng.standard_normal((1, 4, 40, 16)), rng.standard_normal((1, 2, 40, 16)), rng.standard_normal((1, 2, 40, 16))
+    o1, l1 = prefill_ref(q, k, v, rope_theta=100.0, rope_layout="half", rope_freq_scale=0.5)
+    o2, l2 = prefill_ref(_interleave_halves(q), _interleave_halves(k), v, rope_theta=100.0, rope_freq_scale=0.5)
+    assert np.allclose(o1, o2, atol=1e-12) and np.allclose(l1, l2, atol=1e-12)
+
+
+def test_ntk_aware_and_length_scaled_bases():
+    """NTK-aware: the lowest frequency is divided by the stretch, the highest stays 1.
+    Length-aware base of the long-context page (section 2.4): theta at L = L0."""
+    from attention_causal_gqa_b200.binding import length_scaled_theta, ntk_aware_theta
+    D, s, th = 128, 8.0, 1e4
+    t2 = ntk_aware_theta(th, s, D)
+    lowest = lambda t: t ** (-2.0 * (D // 2 - 1) / D)  # noqa: E731
+    assert abs(lowest(t2) - lowest(th) / s) < 1e-12 * lowest(th)
+    assert ntk_aware_theta(th, 1.0, D) == th
+    assert length_scaled_theta(th, 4096, 4096, 0.2) == th
+    assert length_scaled_theta(th, 8192, 4096, 1.0) == 2 * th
