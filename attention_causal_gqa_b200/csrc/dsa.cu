@@ -14,9 +14,10 @@
 //   memory. HBM-bound on the keys (256 B per token, 64 flop per byte).
 // * dsa_topk_kernel: one CTA per sequence. Radix selection on order-preserving 32-bit
 //   keys (four 8-bit digit passes with shared-memory histograms, over the keys staged in
-//   shared memory once) finds the k-th largest score; a final pass keeps every score
-//   above it and, of the scores equal to it, the ones with the smallest token indices,
-//   writing the selection in ascending token order (block-wide ballot prefix sums).
+//   shared memory once; warp w owns a contiguous segment of them) finds the k-th largest
+//   score; a final pass keeps every score above it and, of the scores equal to it, the ones
+//   with the smallest token indices, writing the selection in ascending token order (warp
+//   ballots within a segment, one warp's scan across segments: two block barriers).
 // * dsa_gather_kernel: one warp per two selected tokens copies their latent rows (Dc) and
 //   rotary rows (Dr), all loads in flight first, into contiguous [B, top_k, .] buffers that
 //   the MLA decode reads as caches.
@@ -184,7 +185,6 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const float* __r
   __shared__ unsigned whist[kTopkThreads / 32][256];  // one histogram per warp, summed into hist
   __shared__ unsigned hist[256];
   __shared__ unsigned wcnt[2][kTopkThreads / 32];
-  __shared__ unsigned tile_tot[2];
   __shared__ uint32_t sh_prefix;
   __shared__ unsigned sh_need;
   const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -207,6 +207,9 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const float* __r
     if constexpr (SMEM) return skeys[i];
     else return order_key(s[i]);
   };
+  // warp w owns the contiguous keys [seg0, seg1)
+  const int seg = (L + kTopkThreads / 32 - 1) / (kTopkThreads / 32);
+  const int seg0 = min(L, warp * seg), seg1 = min(L, seg0 + seg);
   // radix selection of the top_k-th largest key, most significant digit first:
   // `need` counts how many keys still to take from the band that matches `prefix`
   uint32_t prefix = 0u, mask = 0u;
@@ -217,7 +220,7 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const float* __r
     // the digits are few and repeated (the top digit is sign and exponent): each thread
     // counts a run of equal digits in a register and adds it with one atomic when it ends
     unsigned cur = 256u, cnt = 0u;
-    for (int i = tid; i < L; i += kTopkThreads) {
+    for (int i = seg0 + lane; i < seg1; i += 32) {
       const uint32_t key = key_at(i);
       if ((key & mask) != prefix) continue;
       const unsigned dg = (key >> shift) & 0xFFu;
@@ -274,42 +277,57 @@ __global__ void __launch_bounds__(kTopkThreads) dsa_topk_kernel(const float* __r
   // first `need` keys equal to it in token order; write positions by ballot prefix sums
   const uint32_t tau = prefix;
   const unsigned lt = (1u << lane) - 1u;
-  unsigned eq_base = 0u, out_base = 0u;
-  // exclusive prefix of the per-warp counts c[0..31] in place, the total into *tot (warp 0)
-  auto warp_scan = [&](unsigned* c, unsigned* tot) {
-    const unsigned v = c[lane];
-    unsigned incl = v;
+  // (a) per warp: how many of its keys are above tau and equal to it
+  unsigned n_gt = 0u, n_eq = 0u;
+  for (int i0 = seg0; i0 < seg1; i0 += 32) {
+    const int i = i0 + lane;
+    uint32_t key = 0u;
+    if (i < seg1) key = key_at(i);
+    n_gt += __popc(__ballot_sync(0xffffffffu, i < seg1 && key > tau));
+    n_eq += __popc(__ballot_sync(0xffffffffu, i < seg1 && key == tau));
+  }
+  if (lane == 0) {
+    wcnt[0][warp] = n_eq;
+    wcnt[1][warp] = n_gt;
+  }
+  __syncthreads();
+  // (b) one warp: equal keys before each warp, then each warp's share and output offset
+  if (warp == 0) {
+    const unsigned eq = wcnt[0][lane], gtc = wcnt[1][lane];
+    unsigned incl = eq;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += t;
     }
-    c[lane] = incl - v;
-    if (lane == 31) *tot = incl;
-  };
-  for (int base = 0; base < L; base += kTopkThreads) {
-    const int i = base + tid;
-    bool gt = false, eq = false;
-    if (i < L) {
-      const uint32_t key = key_at(i);
-      gt = key > tau;
-      eq = key == tau;
+    const unsigned eq_pre = incl - eq;
+    const unsigned take = eq_pre >= need ? 0u : min(eq, need - eq_pre);
+    const unsigned mine = gtc + take;
+    unsigned oin = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned t = __shfl_up_sync(0xffffffffu, oin, o);
+      if (lane >= o) oin += t;
     }
+    wcnt[0][lane] = eq_pre;
+    wcnt[1][lane] = oin - mine;
+  }
+  __syncthreads();
+  // (c) per warp, in token order: keys above tau, and equal ones while their rank < need
+  const unsigned eq_pre = wcnt[0][warp];
+  unsigned eq_seen = 0u, out_off = wcnt[1][warp];
+  for (int i0 = seg0; i0 < seg1; i0 += 32) {
+    const int i = i0 + lane;
+    uint32_t key = 0u;
+    if (i < seg1) key = key_at(i);
+    const bool gt = i < seg1 && key > tau, eq = i < seg1 && key == tau;
     const unsigned be = __ballot_sync(0xffffffffu, eq);
-    if (lane == 0) wcnt[0][warp] = __popc(be);
-    __syncthreads();
-    if (warp == 0) warp_scan(wcnt[0], &tile_tot[0]);
-    __syncthreads();
-    const bool sel = gt || (eq && eq_base + wcnt[0][warp] + __popc(be & lt) < need);
+    const bool sel = gt || (eq && eq_pre + eq_seen + __popc(be & lt) < need);
     const unsigned bs = __ballot_sync(0xffffffffu, sel);
-    if (lane == 0) wcnt[1][warp] = __popc(bs);
-    __syncthreads();
-    if (warp == 0) warp_scan(wcnt[1], &tile_tot[1]);
-    __syncthreads();
-    const unsigned pos = out_base + wcnt[1][warp] + __popc(bs & lt);
+    const unsigned pos = out_off + __popc(bs & lt);
     if (sel && pos < static_cast<unsigned>(top_k)) out[pos] = i;
-    eq_base += tile_tot[0];
-    out_base += tile_tot[1];
+    eq_seen += __popc(be);
+    out_off += __popc(bs);
   }
 }
 
