@@ -119,3 +119,62 @@ def test_workspace_sizes_grow_with_problem(lib):
     assert lib.mla_decode_workspace_size(32, 128, 512, 64, 32768) > lib.mla_decode_workspace_size(1, 128, 512, 64, 512)
     assert lib.attn_selftest_wait_timeout(ctypes.c_void_p(FAKE), 100, 10 ** 6, None) == 3
     assert lib.attn_selftest_wait_timeout(ctypes.c_void_p(FAKE), 256, 10, None) == 1
+
+
+def test_prefill_ex_validation_codes(lib):
+    f = lib.attn_prefill_ex
+    P = ctypes.c_void_p(FAKE)
+    need = lib.attn_prefill_workspace_size(1, 2, 256, 128, 1)
+
+    def call(layout=0, fscale=1.0, ws=need, D=128, dt=1):
+        return f(P, P, P, P, P, 1, 8, 2, 256, D, 1, 1e4, fscale, layout, 0.0, dt, P, ws, None)
+    assert call(layout=2) == 1
+    assert call(fscale=0.0) == 1
+    assert call(fscale=-1.0) == 1
+    assert call(fscale=float("inf")) == 1
+    assert call(dt=0) == 2
+    assert call(ws=need - 1) == 3
+    assert call(layout=1, ws=need - 1) == 3  # the half-split layout itself is accepted
+
+
+def test_decode_fp8_validation_codes(lib):
+    f = lib.attn_decode_paged_fp8
+    P = ctypes.c_void_p(FAKE)
+    need = lib.attn_decode_paged_fp8_workspace_size(2, 32, 128, 64, 16)
+
+    def call(D=128, Hkv=8, Hq=32, ps=16, ws=need, ks=P):
+        return f(P, P, P, ks, P, P, P, P, P, 2, Hq, Hkv, D, ps, 64, 100, 0.0, P, ws, None)
+    assert call(D=64) == 2
+    assert call(Hkv=16, Hq=32) == 2
+    assert call(ps=32) == 2
+    assert call(Hq=30) == 1
+    assert call(ws=need - 1) == 3
+    assert call(ks=None) == 1
+    # one partial per (page range, sequence): independent of the longest sequence
+    assert need == lib.attn_decode_paged_fp8_workspace_size(2, 32, 128, 4096, 16)
+
+
+def test_dsa_validation_codes(lib):
+    P = ctypes.c_void_p(FAKE)
+    f = lib.dsa_index_topk
+    wsi = lib.dsa_index_topk_workspace_size(2, 64, 128, 4096, 2048)
+
+    def idx(HI=64, dI=128, k=2048, ws=wsi, w=P):
+        return f(P, w, P, P, P, P, 2, HI, dI, 4096, k, P, ws, None)
+    assert idx(dI=64) == 2
+    assert idx(HI=24) == 2
+    assert idx(HI=128) == 2
+    assert idx(k=0) == 1
+    assert idx(w=None) == 1
+    assert idx(ws=wsi - 1) == 3
+    g = lib.dsa_mla_decode
+    need = lib.dsa_mla_decode_workspace_size(2, 128, 512, 64, 2048)
+    assert need > lib.mla_decode_workspace_size(2, 128, 512, 64, 2048)  # plus the gathered rows
+
+    def mla(H=128, k=2048, scale=0.07, ws=need, ix=P):
+        return g(P, P, P, P, P, ix, k, scale, P, P, 2, H, 512, 64, 4096, P, ws, None)
+    assert mla(H=64) == 2
+    assert mla(k=0) == 1
+    assert mla(scale=0.0) == 1
+    assert mla(ix=None) == 1
+    assert mla(ws=need - 1) == 3
