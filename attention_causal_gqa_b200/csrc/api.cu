@@ -648,6 +648,22 @@ int dsa_index_topk(const void* q_idx, const float* w_idx, const void* k_idx, con
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int rc = clear_status(workspace, st);
   if (rc) return rc;
+  // q as (d, head, b) and k as (d, token, b), 64-column boxes with 128-byte swizzle; the Q box
+  // is 64 heads high (rows past H_I read as zeros)
+  CUtensorMap tmQ, tmK;
+  {
+    const cuuint64_t d[3] = {static_cast<cuuint64_t>(d_I), static_cast<cuuint64_t>(H_I), static_cast<cuuint64_t>(B)};
+    const cuuint64_t s[2] = {static_cast<cuuint64_t>(d_I) * 2, static_cast<cuuint64_t>(H_I) * d_I * 2};
+    const cuuint32_t bx[3] = {64, 64, 1};
+    if ((rc = make_map(&tmQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, q_idx, d, s, bx, "q_idx"))) return rc;
+  }
+  {
+    const cuuint64_t d[3] = {static_cast<cuuint64_t>(d_I), static_cast<cuuint64_t>(T_max),
+                             static_cast<cuuint64_t>(B)};
+    const cuuint64_t s[2] = {static_cast<cuuint64_t>(d_I) * 2, static_cast<cuuint64_t>(T_max) * d_I * 2};
+    const cuuint32_t bx[3] = {64, 128, 1};
+    if ((rc = make_map(&tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, k_idx, d, s, bx, "k_idx"))) return rc;
+  }
   attn::DsaIndexParams p{};
   p.q = q_idx;
   p.w = w_idx;
@@ -657,8 +673,9 @@ int dsa_index_topk(const void* q_idx, const float* w_idx, const void* k_idx, con
   p.B = B;
   p.HI = H_I;
   p.T_max = T_max;
+  p.status = static_cast<int*>(workspace);
   prof_before(st);
-  cudaError_t e = attn::launch_dsa_index(p, st);
+  cudaError_t e = attn::launch_dsa_index(p, tmQ, tmK, st);
   prof_after(st);
   if (e != cudaSuccess) return cuda_fail(e, "indexer launch");
   e = attn::launch_dsa_topk(scores, seq_lens, topk_idx, B, T_max, top_k, st);

@@ -24,31 +24,16 @@
 #include <cuda_bf16.h>
 
 #include "dsa.h"
+#include "kernels.h"
+#include "sm100.cuh"
 
 namespace attn {
 
 namespace {
 
-constexpr int kIdxTokens = 64;   // tokens per indexer block (one key tile in shared memory)
-constexpr int kIdxBlocks = 4;    // blocks per indexer CTA: Q loaded once, the next tile copied during the current
-constexpr int kIdxThreads = 128;  // four warps: 16 indexer heads each
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkSmemKeys = 48 * 1024;  // sequences up to this many tokens keep their keys in shared memory
 constexpr int kGatherRows = 2;            // selected rows per gather warp
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
 
 // Order-preserving map of a float onto an unsigned key (larger float, larger key).
 __device__ __forceinline__ uint32_t order_key(float x) {
@@ -56,123 +41,131 @@ __device__ __forceinline__ uint32_t order_key(float x) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// 16-byte asynchronous copy global -> shared; src_bytes = 0 writes zeros without reading.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
+constexpr int kTcTok = 128;    // tokens per tile: the M of the score MMA
+constexpr int kTcTiles = 16;   // tiles per CTA
+constexpr int kTcThreads = 128;
+constexpr int kTcQBox = 64 * 128;          // bytes of one 64-column block of Q (64 head rows)
+constexpr int kTcKBox = kTcTok * 128;      // bytes of one 64-column block of a key tile
+constexpr int kTcQBytes = 2 * kTcQBox;     // Q: 64 heads x 128 dims
+constexpr int kTcKBytes = 2 * kTcKBox;     // key tile: 128 tokens x 128 dims
+constexpr int kTcSmem = 1024 + kTcQBytes + 2 * kTcKBytes + 1024;
 
-__global__ void __launch_bounds__(kIdxThreads) dsa_index_kernel(const DsaIndexParams p) {
-  constexpr int D = kDsaIndexDim;
-  constexpr int TILE = kIdxTokens * D * 2;  // bytes of one key tile
-  // two key tiles [token][16 chunks of 16 B], chunk ^ (token & 7), copied while the other is used
-  __shared__ __align__(128) uint8_t kblk[2][TILE];
-  __shared__ float red[kIdxThreads / 32][kIdxTokens];
-  const int b = blockIdx.y, c0 = blockIdx.x * (kIdxTokens * kIdxBlocks);
+// Scores on the 5th-generation tensor cores: S^T = K Q^T with the tile's 128 tokens as M,
+// the (up to) 64 indexer heads as N and d = 128 as K, accumulated in TMEM (two 64-column
+// accumulators, so tile j + 1's MMAs run while tile j is read back). Q (64 x 128) and each
+// key tile (128 x 128) arrive by TMA with 128-byte swizzle; one warp issues the MMAs. In the
+// epilogue each thread owns one token (its TMEM lane): ReLU, head weights and the sum over
+// heads in a fixed order from two tcgen05.ld of 32 columns.
+__global__ void __launch_bounds__(kTcThreads, 1)
+    dsa_index_kernel(const DsaIndexParams p, const __grid_constant__ CUtensorMap tmQ,
+                     const __grid_constant__ CUtensorMap tmK) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = smem + kTcQBytes;  // two stages
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kTcQBytes + 2 * kTcKBytes);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;    // [2]
+  uint64_t* mma_done = bars + 3;  // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* s_w = reinterpret_cast<float*>(tmem_slot + 2);  // 64 head weights (0 past HI)
+
+  const int b = blockIdx.y, c0 = blockIdx.x * (kTcTok * kTcTiles);
   const int L = min(max(__ldg(p.seq_lens + b), 0), p.T_max);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5;
   float* srow = p.scores + static_cast<size_t>(b) * p.T_max;
-  const int c1 = min(c0 + kIdxTokens * kIdxBlocks, p.T_max);
+  const int c1 = min(c0 + kTcTok * kTcTiles, p.T_max);
   if (c0 >= L) {  // the whole range lies past the sequence
-    for (int t = c0 + tid; t < c1; t += kIdxThreads) srow[t] = -INFINITY;
+    for (int t = c0 + tid; t < c1; t += kTcThreads) srow[t] = -INFINITY;
     return;
   }
-  const int nblk = (min(c1, L) - c0 + kIdxTokens - 1) / kIdxTokens;  // tiles holding tokens of the sequence
-  const uint8_t* kbase = static_cast<const uint8_t*>(p.k) + static_cast<size_t>(b) * p.T_max * (D * 2);
-  const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(&kblk[0][0]));
-  auto copy_tile = [&](int j) {  // key rows c0 + 64 j ..; rows past the sequence become zeros
-    const int t0 = c0 + j * kIdxTokens;
-#pragma unroll
-    for (int i = tid; i < kIdxTokens * 16; i += kIdxThreads) {
-      const int r = i >> 4, ch = i & 15;
-      const bool in = t0 + r < L;
-      const uint8_t* src = kbase + static_cast<size_t>(in ? t0 + r : 0) * (D * 2) + ch * 16;
-      cp_async16(sbase + (j & 1) * TILE + r * (D * 2) + ((ch ^ (r & 7)) << 4), src, in ? 16 : 0);
+  const int ntiles = (min(c1, L) - c0 + kTcTok - 1) / kTcTok;
+  if (tid == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&mma_done[s], 1);
     }
-    cp_async_commit();
-  };
-  copy_tile(0);
-  // this warp's 16 heads: A fragments of Q (rows = heads) and the two head weights of the lane
-  const int g = lane >> 2, c = lane & 3;
-  const int h0 = 16 * warp;
-  const bool active = h0 < p.HI;
-  uint32_t qa[D / 16][4];
-  float w0 = 0.f, w1 = 0.f;
-  if (active) {
-    const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(p.q) + (static_cast<size_t>(b) * p.HI + h0) * D;
-#pragma unroll
-    for (int kt = 0; kt < D / 16; ++kt) {
-      const int d0 = kt * 16 + 2 * c;
-      qa[kt][0] = *reinterpret_cast<const uint32_t*>(qb + g * D + d0);
-      qa[kt][1] = *reinterpret_cast<const uint32_t*>(qb + (g + 8) * D + d0);
-      qa[kt][2] = *reinterpret_cast<const uint32_t*>(qb + g * D + d0 + 8);
-      qa[kt][3] = *reinterpret_cast<const uint32_t*>(qb + (g + 8) * D + d0 + 8);
-    }
-    w0 = __ldg(p.w + static_cast<size_t>(b) * p.HI + h0 + g);
-    w1 = __ldg(p.w + static_cast<size_t>(b) * p.HI + h0 + g + 8);
+    *abort_flag = 0;
+    fence_mbar_init();
   }
-  const int mi = lane >> 3, r8 = lane & 7;  // ldmatrix: matrix index and row within it
-  for (int j = 0; j < nblk; ++j) {
-    if (j + 1 < nblk) {
-      copy_tile(j + 1);
-      cp_async_wait<1>();  // tile j has landed (tile j + 1 may still be in flight)
-    } else {
-      cp_async_wait<0>();
+  if (tid < 64) s_w[tid] = tid < p.HI ? __ldg(p.w + static_cast<size_t>(b) * p.HI + tid) : 0.f;
+  if (warp == 0) tmem_alloc(tmem_slot, 128);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto load_tile = [&](int j) {  // key rows c0 + 128 j .. into stage j & 1
+    uint8_t* dst = sK + (j & 1) * kTcKBytes;
+    mbar_arrive_expect_tx(&k_full[j & 1], kTcKBytes);
+    tma_load_3d(dst, &tmK, &k_full[j & 1], 0, c0 + j * kTcTok, b);
+    tma_load_3d(dst + kTcKBox, &tmK, &k_full[j & 1], 64, c0 + j * kTcTok, b);
+  };
+  if (tid == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    mbar_arrive_expect_tx(q_full, kTcQBytes);
+    tma_load_3d(sQ, &tmQ, q_full, 0, 0, b);
+    tma_load_3d(sQ + kTcQBox, &tmQ, q_full, 64, 0, b);
+    load_tile(0);
+    if (ntiles > 1) load_tile(1);
+  }
+  constexpr uint32_t idesc = idesc_f32acc(1, kTcTok, 64, false, false);  // bf16 x bf16 -> f32, K-major both
+  constexpr uint32_t HI = sdesc_hi_sw128(1024);
+  const uint32_t q_lo = sdesc_lo(smem_u32(sQ), 16);
+  const uint32_t k_lo = sdesc_lo(smem_u32(sK), 16);
+  bool ok = true;
+  auto issue = [&](int j) {  // warp 0: the 8 k-steps of tile j into accumulator j & 1
+    ok = ok && mbar_wait_warp(&k_full[j & 1], (j >> 1) & 1, abort_flag, p.status);
+    if (j == 0) ok = ok && mbar_wait_warp(q_full, 0, abort_flag, p.status);
+    if (!ok) return;
+    tc_fence_after();
+    const uint32_t a0 = k_lo + (((j & 1) * kTcKBytes) >> 4);
+    const uint32_t d = tmem + (j & 1) * 64;
+#pragma unroll
+    for (int kb = 0; kb < 8; ++kb) {
+      const uint32_t ao = ((kb >> 2) * kTcKBox + (kb & 3) * 32) >> 4;
+      const uint32_t bo = ((kb >> 2) * kTcQBox + (kb & 3) * 32) >> 4;
+      umma_f16_lohi_warp(d, a0 + ao, HI, q_lo + bo, HI, idesc, kb > 0 ? 1u : 0u);
     }
-    __syncthreads();  // tile j visible to every warp; red free again
-    if (active) {
-      const uint32_t base = sbase + (j & 1) * TILE;
+    umma_commit_warp(&mma_done[j & 1]);
+  };
+  if (warp == 0) issue(0);
+  for (int j = 0; j < ntiles; ++j) {
+    if (warp == 0 && j + 1 < ntiles) issue(j + 1);
+    ok = ok && mbar_wait(&mma_done[j & 1], (j >> 1) & 1, abort_flag, p.status);
+    if (__syncthreads_or(!ok)) break;
+    tc_fence_after();
+    // stage j & 1 is free once its MMAs are done: bring in tile j + 2
+    if (tid == 0 && j + 2 < ntiles) load_tile(j + 2);
+    // epilogue: this thread's token is row 32 warp + lane of the accumulator
+    float score = 0.f;
+    {
+      uint32_t v[32];
+      const uint32_t base = tmem + (static_cast<uint32_t>(32 * warp) << 16) + (j & 1) * 64;
 #pragma unroll
-      for (int np = 0; np < kIdxTokens / 16; ++np) {  // 16 tokens: two n-tiles of 8
-        float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int half = 0; half < 2; ++half) {
+        tmem_ld32(base + 32 * half, v);
+        tmem_ld_wait();
 #pragma unroll
-        for (int kt = 0; kt < D / 16; ++kt) {
-          // matrices: (tokens 0-7, dims lo), (tokens 0-7, dims hi), (tokens 8-15, lo), (8-15, hi)
-          const int tok = 16 * np + (mi >> 1) * 8 + r8;
-          const int ch = 2 * kt + (mi & 1);
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(base + tok * (D * 2) + ((ch ^ (tok & 7)) << 4), b0, b1, b2, b3);
-          mma_bf16_16816(acc0, qa[kt], b0, b1);
-          mma_bf16_16816(acc1, qa[kt], b2, b3);
-        }
-        // ReLU, head weights, sum over this lane's two heads, then over the 8 row groups.
-        // The rounding steps are spelled out (no free contraction into fused multiply-adds)
-        // so every token takes the same ones: equal keys give bit-equal scores.
-        float v[4];
-        v[0] = __fmaf_rn(w1, fmaxf(acc0[2], 0.f), __fmul_rn(w0, fmaxf(acc0[0], 0.f)));  // token 16np + 2c
-        v[1] = __fmaf_rn(w1, fmaxf(acc0[3], 0.f), __fmul_rn(w0, fmaxf(acc0[1], 0.f)));  // token 16np + 2c + 1
-        v[2] = __fmaf_rn(w1, fmaxf(acc1[2], 0.f), __fmul_rn(w0, fmaxf(acc1[0], 0.f)));  // token 16np + 8 + 2c
-        v[3] = __fmaf_rn(w1, fmaxf(acc1[3], 0.f), __fmul_rn(w0, fmaxf(acc1[1], 0.f)));
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-#pragma unroll
-          for (int sh = 4; sh < 32; sh <<= 1) v[e] = __fadd_rn(v[e], __shfl_xor_sync(0xffffffffu, v[e], sh));
-        }
-        if (g == 0) {
-          red[warp][16 * np + 2 * c] = v[0];
-          red[warp][16 * np + 2 * c + 1] = v[1];
-          red[warp][16 * np + 8 + 2 * c] = v[2];
-          red[warp][16 * np + 8 + 2 * c + 1] = v[3];
-        }
+        for (int h = 0; h < 32; ++h) score = __fmaf_rn(s_w[32 * half + h], fmaxf(__uint_as_float(v[h]), 0.f), score);
       }
-    } else {
-      for (int i = lane; i < kIdxTokens; i += 32) red[warp][i] = 0.f;
     }
-    __syncthreads();  // red complete; tile j no longer read (the copy into it is issued next round)
-    const int t = c0 + j * kIdxTokens + tid;
-    if (tid < kIdxTokens && t < p.T_max) {
-      float sum = 0.f;
-#pragma unroll
-      for (int w = 0; w < kIdxThreads / 32; ++w) sum = __fadd_rn(sum, red[w][tid]);
-      srow[t] = t < L ? sum : -INFINITY;
-    }
+    const int t = c0 + j * kTcTok + tid;
+    if (t < p.T_max) srow[t] = t < L ? score : -INFINITY;
+    tc_fence_before();
+    __syncthreads();  // accumulator j & 1 read by every warp before tile j + 2's MMAs reuse it
   }
   // slots of this CTA's range past the sequence's last tile
-  for (int t = c0 + nblk * kIdxTokens + tid; t < c1; t += kIdxThreads) srow[t] = -INFINITY;
+  for (int t = c0 + ntiles * kTcTok + tid; t < c1; t += kTcThreads) srow[t] = -INFINITY;
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
 }
 
 // SMEM: the sequence's keys are converted once into shared memory (T_max <= kTopkSmemKeys)
@@ -381,10 +374,13 @@ __global__ void __launch_bounds__(256, 4) dsa_gather_kernel(const __nv_bfloat16*
 
 }  // namespace
 
-cudaError_t launch_dsa_index(const DsaIndexParams& p, cudaStream_t stream) {
-  if (p.HI < 16 || p.HI > kDsaMaxIndexHeads || p.HI % 16 != 0) return cudaErrorInvalidValue;
-  const dim3 grid((p.T_max + kIdxTokens * kIdxBlocks - 1) / (kIdxTokens * kIdxBlocks), p.B);
-  dsa_index_kernel<<<grid, kIdxThreads, 0, stream>>>(p);
+cudaError_t launch_dsa_index(const DsaIndexParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                             cudaStream_t stream) {
+  if (p.HI < 1 || p.HI > kDsaMaxIndexHeads) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(dsa_index_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((p.T_max + kTcTok * kTcTiles - 1) / (kTcTok * kTcTiles), p.B);
+  dsa_index_kernel<<<grid, kTcThreads, kTcSmem, stream>>>(p, tmQ, tmK);
   return cudaGetLastError();
 }
 

@@ -4,6 +4,7 @@
 #pragma once
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace attn {
@@ -19,8 +20,12 @@ struct DsaIndexParams {
   const int32_t* seq_lens;  // [B]
   float* scores;            // [B, T_max] out: index scores, -inf past each length
   int B, HI, T_max;
+  int* status;              // device status word (bounded waits)
 };
-cudaError_t launch_dsa_index(const DsaIndexParams& p, cudaStream_t stream);
+// tmQ: 3-D bf16 map of q (d, head, b), box 64 x 64 x 1; tmK: 3-D bf16 map of k (d, token, b),
+// box 64 x 128 x 1; both with 128-byte swizzle
+cudaError_t launch_dsa_index(const DsaIndexParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                             cudaStream_t stream);
 
 // idx [B, top_k]: the min(top_k, L) best tokens in ascending order, -1 after them
 cudaError_t launch_dsa_topk(const float* scores, const int32_t* seq_lens, int32_t* idx, int B, int T_max, int top_k,
