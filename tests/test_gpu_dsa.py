@@ -173,3 +173,15 @@ def test_dsa_full_size_sampled():
     ro, rl = _oracle_out(d, idx, pairs, compact=True)
     ix = torch.tensor(pairs, device="cuda")
     check(out[ix[:, 0], 0, ix[:, 1]], ro, lse[ix[:, 0], 0, ix[:, 1]], rl, what="dsa full")
+
+
+@cuda
+def test_selection_past_the_shared_memory_staging_limit():
+    """Sequences longer than the top-k kernel stages in shared memory (48K tokens) take the
+    path that re-reads the scores on every pass."""
+    from attention_causal_gqa_b200.synthetic import dsa_inputs
+    lens = [50000, 7000]
+    d = dsa_inputs(2, 128, 512, 64, 64, 128, seq_lens=lens, T_max=50000, seed=99, device="cuda")
+    scores, idx = _index(d, 2048)
+    _check_scores(d, scores, rows=[0])
+    _check_selection(scores, idx, lens, 2048)
