@@ -282,13 +282,17 @@ size_t attn_prefill_chunk_workspace_size(int B, int Hkv, int S_new, int max_cach
   return kHeader + table + 2 * op;
 }
 
-int attn_prefill_chunk(const void* q, const void* k, const void* v, void* k_pages, void* v_pages,
-                       const int32_t* block_table, const int32_t* cache_lens, void* out, float* lse, int B, int Hq,
-                       int Hkv, int S_new, int D, int page_size, int max_pages_per_seq, int num_pages,
-                       int max_cache_len, float rope_theta, float scale, void* workspace, size_t workspace_bytes,
-                       void* stream) {
+int attn_prefill_chunk_ex(const void* q, const void* k, const void* v, void* k_pages, void* v_pages,
+                          const int32_t* block_table, const int32_t* cache_lens, void* out, float* lse, int B, int Hq,
+                          int Hkv, int S_new, int D, int page_size, int max_pages_per_seq, int num_pages,
+                          int max_cache_len, float rope_theta, float rope_freq_scale, int rope_layout, float scale,
+                          void* workspace, size_t workspace_bytes, void* stream) {
   if (!q || !k || !v || !k_pages || !v_pages || !block_table || !cache_lens || !out || !lse || !workspace)
     return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
+  if (rope_layout != ATTN_ROPE_INTERLEAVED && rope_layout != ATTN_ROPE_HALF_SPLIT)
+    return fail(ATTN_ERR_INVALID_ARG, "rope_layout %d", rope_layout);
+  if (!(rope_freq_scale > 0.f) || !std::isfinite(rope_freq_scale))
+    return fail(ATTN_ERR_INVALID_ARG, "rope_freq_scale must be positive and finite");
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || S_new <= 0 || D <= 0 || max_pages_per_seq <= 0 || num_pages <= 0 ||
       max_cache_len < 0)
     return fail(ATTN_ERR_INVALID_ARG, "sizes must be positive (B=%d Hq=%d Hkv=%d S_new=%d D=%d pages=%d/%d, max_cache_len=%d)",
@@ -323,11 +327,12 @@ int attn_prefill_chunk(const void* q, const void* k, const void* v, void* k_page
   if (rc) return rc;
   const bool rope = rope_theta > 0.f;
   if (rope) {
-    cudaError_t e = attn::launch_rope_table(cs, static_cast<int>(sk), D, static_cast<double>(rope_theta), 1.0, st);
+    cudaError_t e = attn::launch_rope_table(cs, static_cast<int>(sk), D, static_cast<double>(rope_theta),
+                                            static_cast<double>(rope_freq_scale), st);
     if (e != cudaSuccess) return cuda_fail(e, "rope table launch");
   }
   attn::ChunkGeometry g{cache_lens, block_table, B, Hkv, S_new, D, page_size, max_pages_per_seq, num_pages,
-                        max_cache_len};
+                        max_cache_len, rope_layout == ATTN_ROPE_HALF_SPLIT ? 1 : 0};
   const float2* rcs = rope ? cs : nullptr;
   cudaError_t e = attn::launch_kv_append(k, v, k_pages, v_pages, rcs, g, status, st);
   if (e == cudaSuccess) e = attn::launch_kv_gather(k_pages, v_pages, k_op, v_op, g, static_cast<int>(sk), status, st);
@@ -377,6 +382,16 @@ int attn_prefill_chunk(const void* q, const void* k, const void* v, void* k_page
   prof_after(st);
   if (e != cudaSuccess) return cuda_fail(e, "chunk prefill launch");
   return ok();
+}
+
+int attn_prefill_chunk(const void* q, const void* k, const void* v, void* k_pages, void* v_pages,
+                       const int32_t* block_table, const int32_t* cache_lens, void* out, float* lse, int B, int Hq,
+                       int Hkv, int S_new, int D, int page_size, int max_pages_per_seq, int num_pages,
+                       int max_cache_len, float rope_theta, float scale, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  return attn_prefill_chunk_ex(q, k, v, k_pages, v_pages, block_table, cache_lens, out, lse, B, Hq, Hkv, S_new, D,
+                               page_size, max_pages_per_seq, num_pages, max_cache_len, rope_theta, 1.0f,
+                               ATTN_ROPE_INTERLEAVED, scale, workspace, workspace_bytes, stream);
 }
 
 size_t attn_decode_paged_workspace_size(int B, int Hq, int D, int max_pages_per_seq, int page_size) {

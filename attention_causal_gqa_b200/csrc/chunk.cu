@@ -36,6 +36,21 @@ __device__ __forceinline__ int clamp_len(const int32_t* lens, int b, int max_len
 }
 
 // Rotate the 8 values of chunk c of a row at position pos (cs == nullptr: no rotation).
+// Half-split layout: chunk c < D/16 (elements 8c .. 8c+7) pairs element by element with
+// chunk c + D/16; pair 8c + e turns by the table's angle 8c + e.
+__device__ __forceinline__ void rotate16_half(const uint4 lo_raw, const uint4 hi_raw, const float2* __restrict__ cs,
+                                              int pos, int c, int D, float (&lo)[8], float (&hi)[8]) {
+  const uint32_t wl[4] = {lo_raw.x, lo_raw.y, lo_raw.z, lo_raw.w}, wh[4] = {hi_raw.x, hi_raw.y, hi_raw.z, hi_raw.w};
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float x0 = __uint_as_float((e & 1) ? (wl[e >> 1] & 0xFFFF0000u) : (wl[e >> 1] << 16));
+    const float x1 = __uint_as_float((e & 1) ? (wh[e >> 1] & 0xFFFF0000u) : (wh[e >> 1] << 16));
+    const float2 a = __ldg(cs + static_cast<size_t>(pos) * (D / 2) + c * 8 + e);
+    lo[e] = x0 * a.x - x1 * a.y;
+    hi[e] = x0 * a.y + x1 * a.x;
+  }
+}
+
 __device__ __forceinline__ void rotate8(const uint4 raw, const float2* __restrict__ cs, int pos, int c, int D,
                                         float (&f)[8]) {
   const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
@@ -104,6 +119,16 @@ __global__ void kv_append_kernel(const uint4* __restrict__ k_new, const uint4* _
     const int page = page_of(g.block_table, b, pos / g.page_size, g.max_pages, g.num_pages, status);
     if (page < 0) continue;
     const size_t dst = ((static_cast<size_t>(page) * g.page_size + pos % g.page_size) * g.Hkv + kvh) * cpr + c;
+    if (g.half_split && cs) {  // the thread of chunk c < cpr/2 writes chunks c and c + cpr/2
+      if (c >= cpr / 2) continue;
+      float lo[8], hi[8];
+      rotate16_half(k_new[idx], k_new[idx + cpr / 2], cs, pos, c, g.D, lo, hi);
+      k_pages[dst] = pack8_bf16_rn(lo);
+      k_pages[dst + cpr / 2] = pack8_bf16_rn(hi);
+      v_pages[dst] = v_new[idx];
+      v_pages[dst + cpr / 2] = v_new[idx + cpr / 2];
+      continue;
+    }
     float f[8];
     rotate8(k_new[idx], cs, pos, c, g.D, f);
     k_pages[dst] = pack8_bf16_rn(f);
@@ -152,6 +177,14 @@ __global__ void rope_rows_f16_kernel(const uint4* __restrict__ x, uint4* __restr
     const int c = idx % cpr, r = idx / cpr;
     const int i = r % g.S_new, b = r / (g.S_new * Hq);
     const int pos = clamp_len(g.cache_lens, b, g.max_cache_len, status) + i;
+    if (g.half_split && cs) {  // the thread of chunk c < cpr/2 writes chunks c and c + cpr/2
+      if (c >= cpr / 2) continue;
+      float lo[8], hi[8];
+      rotate16_half(x[idx], x[idx + cpr / 2], cs, pos, c, g.D, lo, hi);
+      y[idx] = pack8_f16_checked(lo, in_range);
+      y[idx + cpr / 2] = pack8_f16_checked(hi, in_range);
+      continue;
+    }
     float f[8];
     rotate8(x[idx], cs, pos, c, g.D, f);
     y[idx] = pack8_f16_checked(f, in_range);

@@ -25,6 +25,7 @@ struct ChunkGeometry {
   const int32_t* cache_lens;   // [B] tokens already cached (new token i sits at cache_lens[b] + i)
   const int32_t* block_table;  // [B, max_pages]
   int B, Hkv, S_new, D, page_size, max_pages, num_pages, max_cache_len;
+  int half_split;              // RoPE pairs (i, i + D/2) instead of (2i, 2i + 1)
 };
 // rotate the new keys at their positions and write keys and values (bf16) into their pages
 cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* k_pages, void* v_pages, const float2* cs,

@@ -182,6 +182,18 @@ int attn_prefill_chunk(const void* q, const void* k, const void* v, void* k_page
                        void* stream);
 
 /*
+ * attn_prefill_chunk with the RoPE variants of attn_prefill_ex (rope_freq_scale multiplies
+ * every rotary frequency; rope_layout ATTN_ROPE_INTERLEAVED or ATTN_ROPE_HALF_SPLIT): the new
+ * keys are stored rotated in that form, and the cached keys must have been rotated the same
+ * way. attn_prefill_chunk equals this call with 1 and ATTN_ROPE_INTERLEAVED.
+ */
+int attn_prefill_chunk_ex(const void* q, const void* k, const void* v, void* k_pages, void* v_pages,
+                          const int32_t* block_table, const int32_t* cache_lens, void* out, float* lse, int B, int Hq,
+                          int Hkv, int S_new, int D, int page_size, int max_pages_per_seq, int num_pages,
+                          int max_cache_len, float rope_theta, float rope_freq_scale, int rope_layout, float scale,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * DeepSeek MLA absorbed decode (one query token per sequence).
  * Defined by: "DeepSeek-V3 attention: einsum vs hand-optimised" (dksg.cn), absorbed
  * form: scores = (q_nope . kv_cache^T + q_pe . pe_cache^T) * scale,

@@ -319,7 +319,8 @@ def to_bf16(x):
 
 
 def chunk_prefill_ref(q, k_new, v_new, k_pages, v_pages, block_table, cache_lens, rope_theta: float = 10000.0,
-                      scale: float | None = None, page_size: int = 16, store=to_bf16):
+                      scale: float | None = None, page_size: int = 16, store=to_bf16, rope_freq_scale: float = 1.0,
+                      rope_layout: str = "interleaved"):
     """Append a chunk of new tokens to a paged KV cache and attend over the whole cache.
 
     "From 32K to 256K: DeepSeek long-context", chapter 1 (key architecture path: a
@@ -336,6 +337,8 @@ def chunk_prefill_ref(q, k_new, v_new, k_pages, v_pages, block_table, cache_lens
     into their pages with ``store`` (the cache's precision, bf16); rotate the queries at
     the same positions (float64); query i attends the stored keys t <= cache_lens[b] + i
     (the causal mask aligned to the end of the cache), two-pass softmax, O = P V.
+    rope_freq_scale and rope_layout as ``apply_rope`` (the cached keys are taken as
+    rotated the same way).
     Returns (k_pages', v_pages', o [B, Hq, S_new, D], lse [B, Hq, S_new]).
     """
     q = np.asarray(q, dtype=F64)
@@ -356,14 +359,16 @@ def chunk_prefill_ref(q, k_new, v_new, k_pages, v_pages, block_table, cache_lens
         pos = L + np.arange(S_new)
         table = np.asarray(block_table[b])
         for kvh in range(Hkv):
-            kr = apply_rope(k_new[b, kvh], rope_theta, positions=pos) if use_rope else k_new[b, kvh]
+            kr = (apply_rope(k_new[b, kvh], rope_theta, positions=pos, freq_scale=rope_freq_scale, layout=rope_layout)
+                  if use_rope else k_new[b, kvh])
             kp[table[pos // page_size], pos % page_size, kvh] = store(kr)
             vp[table[pos // page_size], pos % page_size, kvh] = store(v_new[b, kvh])
         kk = gather_pages(kp, table, L + S_new, page_size)
         vv = gather_pages(vp, table, L + S_new, page_size)
         for h in range(Hq):
             kvh = h // G
-            qr = apply_rope(q[b, h], rope_theta, positions=pos) if use_rope else q[b, h]
+            qr = (apply_rope(q[b, h], rope_theta, positions=pos, freq_scale=rope_freq_scale, layout=rope_layout)
+                  if use_rope else q[b, h])
             s = scale * (qr @ kk[:, kvh, :].T)
             jj = np.arange(L + S_new)[None, :]
             s = np.where(jj > pos[:, None], -np.inf, s)

@@ -95,3 +95,28 @@ def test_chunk_bad_page_is_flagged_not_faulted():
     d["table"][0, 2] = 10 ** 6  # the page of positions 32..47 lies outside the pool
     out, lse, dev, ws = _run(d, 1e4)
     assert binding.read_status(ws) & 2
+
+
+@cuda
+@pytest.mark.parametrize("B,Hq,Hkv,D,cache_lens,S_new,fscale,layout", [
+    (2, 8, 2, 128, [0, 300], 77, 1.0, "half"),          # half-split pairs
+    (2, 4, 4, 64, [33, 200], 129, 0.25, "half"),        # D = 64, frequencies scaled
+    (1, 8, 2, 128, [500], 64, 0.5, "interleaved"),      # interpolated positions
+])
+def test_chunk_prefill_rope_variants(B, Hq, Hkv, D, cache_lens, S_new, fscale, layout):
+    from attention_causal_gqa_b200 import binding
+    d = _setup(B, Hq, Hkv, D, cache_lens, S_new, seed=S_new * 11 + D)
+    dev = {k: v.cuda() for k, v in d.items()}
+    mcl = max(cache_lens)
+    ws = torch.empty(binding.prefill_chunk_workspace_size(B, Hkv, S_new, mcl, D), dtype=torch.uint8, device="cuda")
+    out, lse = binding.attn_prefill_chunk(dev["q"], dev["k"], dev["v"], dev["k_pages"], dev["v_pages"], dev["table"],
+                                          dev["cache_lens"], mcl, rope_theta=1e4, workspace=ws,
+                                          rope_freq_scale=fscale, rope_layout=layout)
+    torch.cuda.synchronize()
+    kp, vp, ro, rl = chunk_prefill_ref(to_np(d["q"]), to_np(d["k"]), to_np(d["v"]), to_np(d["k_pages"]),
+                                       to_np(d["v_pages"]), d["table"].numpy(), cache_lens, rope_theta=1e4,
+                                       rope_freq_scale=fscale, rope_layout=layout)
+    check(out, ro, lse, rl, what=f"chunk rope {fscale} {layout} D={D}")
+    assert binding.read_status(ws) == 0
+    assert np.array_equal(to_np(dev["v_pages"]), vp)
+    assert _within_one_bf16_step(to_np(dev["k_pages"]), kp)

@@ -669,3 +669,21 @@ def test_ntk_aware_and_length_scaled_bases():
     assert ntk_aware_theta(th, 1.0, D) == th
     assert length_scaled_theta(th, 4096, 4096, 0.2) == th
     assert length_scaled_theta(th, 8192, 4096, 1.0) == 2 * th
+
+
+def test_chunk_prefill_half_split_equals_interleaved_on_permuted_dims():
+    """The layouts differ by a fixed permutation of d: outputs agree, stored keys are permuted."""
+    from oracle import chunk_prefill_ref
+    rng = np.random.default_rng(73)
+    B, Hq, Hkv, D, S_new = 2, 4, 2, 16, 5
+    cache = [0, 21]
+    q = rng.standard_normal((B, Hq, S_new, D))
+    k = rng.standard_normal((B, Hkv, S_new, D))
+    v = rng.standard_normal((B, Hkv, S_new, D))
+    kp, vp, table = _paged_setup(rng, B, Hkv, D, cache, S_new)
+    kh, vh, oh, lh = chunk_prefill_ref(q, k, v, kp, vp, table, cache, rope_theta=50.0, rope_freq_scale=0.5,
+                                       rope_layout="half", store=lambda x: x)
+    ki, vi, oi, li = chunk_prefill_ref(_interleave_halves(q), _interleave_halves(k), v, _interleave_halves(kp), vp,
+                                       table, cache, rope_theta=50.0, rope_freq_scale=0.5, store=lambda x: x)
+    assert np.allclose(oh, oi, atol=1e-12) and np.allclose(lh, li, atol=1e-12)
+    assert np.allclose(_interleave_halves(kh), ki, atol=1e-12)
