@@ -178,3 +178,16 @@ def test_dsa_validation_codes(lib):
     assert mla(scale=0.0) == 1
     assert mla(ix=None) == 1
     assert mla(ws=need - 1) == 3
+
+
+def test_prefill_chunk_ex_validation_codes(lib):
+    f = lib.attn_prefill_chunk_ex
+    P = ctypes.c_void_p(FAKE)
+    need = lib.attn_prefill_chunk_workspace_size(2, 2, 64, 64, 128)
+
+    def call(layout=0, fscale=1.0, ws=need):
+        return f(P, P, P, P, P, P, P, P, P, 2, 8, 2, 64, 128, 16, 8, 20, 64, 1e4, fscale, layout, 0.0, P, ws, None)
+    assert call(layout=5) == 1
+    assert call(fscale=0.0) == 1
+    assert call(ws=need - 1) == 3
+    assert call(layout=1, ws=need - 1) == 3  # the half-split layout itself is accepted
