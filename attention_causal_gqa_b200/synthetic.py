@@ -136,6 +136,28 @@ def quantize_e4m3(x, page_axis=0, head_axis=2):
     return codes.contiguous(), sc.contiguous()
 
 
+def quantize_e4m3_rows(x, block=128):
+    """E4M3 codes of x [..., D] with one scale per row and `block`-wide column block =
+    absmax / 448 (round to nearest); returns (codes uint8 [..., D], scales fp32 [..., D/block])."""
+    xf = x.float()
+    shp = xf.shape
+    blk = xf.reshape(*shp[:-1], shp[-1] // block, block)
+    sc = (blk.abs().amax(dim=-1) / 448.0).clamp(min=1e-12)
+    codes = (blk / sc[..., None]).to(torch.float8_e4m3fn).view(torch.uint8).reshape(shp)
+    return codes.contiguous(), sc.contiguous()
+
+
+def dsa_inputs_fp8(B, H, Dc, Dr, HI, dI, lmin=4096, lmax=32768, std=1.0, seed=0, device="cpu", seq_lens=None,
+                   T_max=None):
+    """The DSA inputs of ``dsa_inputs`` with the latent cache quantised to E4M3 (one scale
+    per token and 128-wide latent block): kv_codes [B,T,Dc] uint8, kv_scale [B,T,Dc/128] fp32;
+    the rotary cache stays bf16."""
+    d = dsa_inputs(B, H, Dc, Dr, HI, dI, lmin, lmax, std, seed, device, seq_lens, T_max)
+    d["kv_codes"], d["kv_scale"] = quantize_e4m3_rows(d["kv_cache"])
+    del d["kv_cache"]
+    return d
+
+
 def decode_inputs_fp8(B, Hq, Hkv, D, lmin=1024, lmax=32768, std=1.0, seed=0, device="cpu", seq_lens=None,
                       max_pages_per_seq=None, extra_pages=0):
     """The paged decode inputs of decode_inputs with K and V pages quantised to E4M3

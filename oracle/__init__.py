@@ -10,6 +10,7 @@ from .attention import (  # noqa: F401
     decode_paged_fp8_ref,
     decode_paged_ref,
     dsa_index_scores_ref,
+    dsa_mla_decode_fp8_ref,
     dsa_mla_decode_ref,
     dsa_topk_ref,
     e4m3_to_float,

@@ -539,3 +539,26 @@ def dsa_mla_decode_ref(q_nope, q_pe, kv_cache, pe_cache, indices, scale: float, 
             kv[b, :len(ix)] = np.asarray(kv_cache[b][ix], dtype=F64)
             pe[b, :len(ix)] = np.asarray(pe_cache[b][ix], dtype=F64)
     return mla_decode_ref(q_nope, q_pe, kv, pe, n, scale, pairs=pairs)
+
+
+def dsa_mla_decode_fp8_ref(q_nope, q_pe, kv_codes, kv_scale, pe_cache, indices, scale: float, pairs=None,
+                           block: int = 128):
+    """Sparse MLA decode over an FP8 (E4M3) latent cache: the latent row of token t is
+    e4m3(kv_codes[b, t, c]) * kv_scale[b, t, c // block] ("7 anti-patterns of DeepSeek
+    attention optimisation", section 3.3: E4M3 with scale factors; one scale per token and
+    128-wide latent block is a reading), the rotary cache stays bf16; then exactly
+    ``dsa_mla_decode_ref`` over those values. Only the selected rows are dequantised."""
+    B, Dc = kv_codes.shape[0], kv_codes.shape[2]
+    n = [len(ix) for ix in indices]
+    t = max([1] + n)
+    kv = np.zeros((B, t, Dc))
+    pe = np.zeros((B, t, pe_cache.shape[2]))
+    seqs = range(B) if pairs is None else sorted({b for b, _ in pairs})
+    for b in seqs:
+        ix = np.asarray(indices[b], dtype=np.int64)
+        if len(ix):
+            codes = np.asarray(kv_codes[b][ix])
+            sc = np.asarray(kv_scale[b][ix], dtype=F64)
+            kv[b, :len(ix)] = e4m3_to_float(codes) * np.repeat(sc, block, axis=1)[:, :Dc]
+            pe[b, :len(ix)] = np.asarray(pe_cache[b][ix], dtype=F64)
+    return dsa_mla_decode_ref(q_nope, q_pe, kv, pe, [np.arange(m) for m in n], scale, pairs=pairs)

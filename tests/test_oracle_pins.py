@@ -687,3 +687,23 @@ def test_chunk_prefill_half_split_equals_interleaved_on_permuted_dims():
                                        table, cache, rope_theta=50.0, rope_freq_scale=0.5, store=lambda x: x)
     assert np.allclose(oh, oi, atol=1e-12) and np.allclose(lh, li, atol=1e-12)
     assert np.allclose(_interleave_halves(kh), ki, atol=1e-12)
+
+
+def test_dsa_fp8_latent_equals_dsa_over_the_dequantised_cache():
+    from oracle import dsa_mla_decode_fp8_ref, dsa_mla_decode_ref, e4m3_to_float
+    rng = np.random.default_rng(74)
+    B, H, Dc, Dr, T = 2, 3, 256, 8, 12
+    codes = rng.integers(0, 256, size=(B, T, Dc), dtype=np.uint8) & 0xF7  # no NaN codes
+    sc = rng.uniform(0.01, 3.0, size=(B, T, Dc // 128))
+    pe = rng.standard_normal((B, T, Dr))
+    qn, qp = rng.standard_normal((B, 1, H, Dc)), rng.standard_normal((B, 1, H, Dr))
+    sel = [np.array([1, 4, 5, 11]), np.array([0, 2])]
+    o, l = dsa_mla_decode_fp8_ref(qn, qp, codes, sc, pe, sel, 0.2)
+    kv = e4m3_to_float(codes) * np.repeat(sc, 128, axis=2)
+    ro, rl = dsa_mla_decode_ref(qn, qp, kv, pe, sel, 0.2)
+    assert np.allclose(o, ro, atol=1e-12) and np.allclose(l, rl, atol=1e-12)
+    # block b of the latent uses scale b: scaling one block's scale changes only that block's values
+    sc2 = sc.copy()
+    sc2[:, :, 1] *= 2.0
+    o2, _ = dsa_mla_decode_fp8_ref(qn, qp, codes, sc2, pe, sel, 0.2)
+    assert not np.allclose(o2, o)
