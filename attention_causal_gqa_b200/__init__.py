@@ -6,7 +6,7 @@ The public calls (attn_prefill, attn_prefill_chunk, attn_decode_paged, mla_decod
 library; calling any of them without the built library raises.
 """
 __all__ = ["attn_prefill", "attn_prefill_chunk", "attn_decode_paged", "attn_decode_paged_fp8", "mla_decode", "dsa_index_topk",
-           "dsa_mla_decode", "read_status", "selftest_wait_timeout"]
+           "dsa_mla_decode", "dsa_mla_decode_fp8", "read_status", "selftest_wait_timeout"]
 
 
 def __getattr__(name):

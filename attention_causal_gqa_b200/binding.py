@@ -34,6 +34,7 @@ EXPORTED = (
     "attn_decode_paged_workspace_size", "attn_decode_paged",
     "attn_decode_paged_fp8_workspace_size", "mla_decode_workspace_size", "mla_decode",
     "dsa_index_topk_workspace_size", "dsa_index_topk", "dsa_mla_decode_workspace_size", "dsa_mla_decode",
+    "dsa_mla_decode_fp8",
     "attn_last_error", "attn_read_status", "attn_selftest_wait_timeout",
     "attn_profile_enable", "attn_profile_collect",
 )
@@ -82,6 +83,8 @@ def _load() -> ctypes.CDLL:
     lib.dsa_mla_decode_workspace_size.argtypes = [i32] * 5
     lib.dsa_mla_decode.restype = i32
     lib.dsa_mla_decode.argtypes = [vp] * 6 + [i32, f32, vp, vp] + [i32] * 5 + [vp, sz, vp]
+    lib.dsa_mla_decode_fp8.restype = i32
+    lib.dsa_mla_decode_fp8.argtypes = [vp] * 7 + [i32, f32, vp, vp] + [i32] * 5 + [vp, sz, vp]
     lib.attn_last_error.restype = ctypes.c_char_p
     lib.attn_last_error.argtypes = []
     lib.attn_read_status.restype = i32
@@ -337,6 +340,29 @@ def dsa_mla_decode(q_nope, q_pe, kv_cache, pe_cache, seq_lens, topk_idx, scale, 
     rc = lib.dsa_mla_decode(_ptr(q_nope), _ptr(q_pe), _ptr(kv_cache), _ptr(pe_cache), _ptr(seq_lens), _ptr(topk_idx),
                             top_k, float(scale), _ptr(out), _ptr(lse), B, H, Dc, Dr, T, _ptr(ws),
                             ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc)
+    return out, lse
+
+
+def dsa_mla_decode_fp8(q_nope, q_pe, kv_codes, kv_scale, pe_cache, seq_lens, topk_idx, scale, out=None, lse=None,
+                       workspace=None, stream=None):
+    """dsa_mla_decode over an E4M3 latent cache: kv_codes [B,T,512] uint8, kv_scale [B,T,4] fp32
+    (one scale per token and 128-wide block), pe_cache [B,T,64] bf16. Returns (out, lse) as mla_decode."""
+    _need_cuda(q_nope, q_pe, kv_codes, kv_scale, pe_cache, seq_lens, topk_idx)
+    B, _, H, Dc = q_nope.shape
+    Dr = q_pe.shape[-1]
+    T = kv_codes.shape[1]
+    top_k = topk_idx.shape[1]
+    if not scale or scale <= 0:
+        raise ValueError("dsa_mla_decode_fp8 needs an explicit positive scale")
+    if out is None:
+        out = torch.empty_like(q_nope)
+    if lse is None:
+        lse = torch.empty((B, 1, H), dtype=torch.float32, device=q_nope.device)
+    ws = _workspace(dsa_mla_workspace_size(B, H, Dc, Dr, top_k), q_nope.device, workspace)
+    rc = lib.dsa_mla_decode_fp8(_ptr(q_nope), _ptr(q_pe), _ptr(kv_codes), _ptr(kv_scale), _ptr(pe_cache),
+                                _ptr(seq_lens), _ptr(topk_idx), top_k, float(scale), _ptr(out), _ptr(lse), B, H, Dc,
+                                Dr, T, _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
     _check(rc)
     return out, lse
 

@@ -14,9 +14,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libattn_b200.so")
-SOURCES = ["api.cu", "rope.cu", "prefill.cu", "decode.cu", "decode_fp8.cu", "mla.cu", "merge.cu", "chunk.cu", "dsa.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "rope.cu", "prefill.cu", "decode.cu", "decode_fp8.cu", "mla.cu", "merge.cu", "chunk.cu", "dsa.cu", "dsa_fp8.cu", "noalloc.cu"]
 HEADERS = ["sm100.cuh", "kernels.h"]  # shared by every kernel
-PROLOGUE_HEADERS = ["prologue.h", "dsa.h"]  # included by their own kernels only (not in every fingerprint)
+PROLOGUE_HEADERS = ["prologue.h", "dsa.h", "dsa_fp8.h"]  # included by their own kernels only (not in every fingerprint)
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

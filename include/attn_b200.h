@@ -251,6 +251,21 @@ int dsa_mla_decode(const void* q_nope, const void* q_pe, const void* kv_cache, c
                    int B, int H, int Dc, int Dr, int T_max, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * dsa_mla_decode over an FP8 (E4M3) latent cache: the latent row of token t is
+ * e4m3(kv_codes[b, t, c]) * kv_scale[b, t, c / 128] ("7 anti-patterns of DeepSeek attention
+ * optimisation", section 3.3: E4M3, largest value 448, with scale factors); the rotary cache
+ * pe_cache stays bf16. kv_codes [B, T_max, 512] uint8, kv_scale [B, T_max, 4] fp32; the
+ * other arguments, the workspace (dsa_mla_decode_workspace_size) and the limits as
+ * dsa_mla_decode. The selected rows are dequantised into bf16 (the MLA kernel's operand
+ * type, so each latent value is rounded to bf16) and attended by the MLA decode kernel.
+ * NaN codes are out of contract.
+ */
+int dsa_mla_decode_fp8(const void* q_nope, const void* q_pe, const void* kv_codes, const float* kv_scale,
+                       const void* pe_cache, const int32_t* seq_lens, const int32_t* topk_idx, int top_k, float scale,
+                       void* out, float* lse, int B, int H, int Dc, int Dr, int T_max, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/*
  * Paged decode for callers that cannot allocate device memory (code running
  * inside another framework's memory pool with allocation disabled, paths where
  * cudaMalloc's implicit synchronisation is not allowed, embedders that only pass

@@ -185,3 +185,41 @@ def test_selection_past_the_shared_memory_staging_limit():
     scores, idx = _index(d, 2048)
     _check_scores(d, scores, rows=[0])
     _check_selection(scores, idx, lens, 2048)
+
+
+# ------------------------------------------------ FP8 (E4M3) latent cache, sparse MLA
+def _oracle_fp8(d, idx, pairs=None):
+    from oracle import dsa_mla_decode_fp8_ref
+    sl = d["seq_lens"].cpu().numpy()
+    ix = [idx[b, :min(int(sl[b]), idx.shape[1])].cpu().numpy().astype(np.int64) for b in range(len(sl))]
+    return dsa_mla_decode_fp8_ref(to_np(d["q_nope"]), to_np(d["q_pe"]), d["kv_codes"].cpu().numpy(),
+                                  d["kv_scale"].cpu().numpy(), to_np(d["pe_cache"]), ix, SCALE, pairs=pairs)
+
+
+@cuda
+@pytest.mark.parametrize("lens,T,top_k", [([40, 900, 2000], 2048, 256), ([33, 0, 1025], 1088, 2048)])
+def test_sparse_mla_fp8_latent_matches_oracle(lens, T, top_k):
+    from attention_causal_gqa_b200 import dsa_mla_decode_fp8
+    from attention_causal_gqa_b200.synthetic import dsa_inputs_fp8
+    d = dsa_inputs_fp8(len(lens), 128, 512, 64, 64, 128, seq_lens=lens, T_max=T, seed=T + 3 * top_k, device="cuda")
+    _, idx = _index(d, top_k)
+    out, lse = dsa_mla_decode_fp8(d["q_nope"], d["q_pe"], d["kv_codes"], d["kv_scale"], d["pe_cache"],
+                                  d["seq_lens"], idx, SCALE)
+    torch.cuda.synchronize()
+    ro, rl = _oracle_fp8(d, idx)
+    check(out, ro, lse, rl, what=f"dsa fp8 {lens}")
+
+
+@cuda
+def test_sparse_mla_fp8_bad_index_is_flagged():
+    from attention_causal_gqa_b200 import binding
+    from attention_causal_gqa_b200.synthetic import dsa_inputs_fp8
+    lens = [300, 200]
+    d = dsa_inputs_fp8(2, 128, 512, 64, 16, 128, seq_lens=lens, T_max=320, seed=8, device="cuda")
+    _, idx = _index(d, 64)
+    idx[0, 3] = -5
+    ws = torch.empty(binding.dsa_mla_workspace_size(2, 128, 512, 64, 64), dtype=torch.uint8, device="cuda")
+    out, _ = binding.dsa_mla_decode_fp8(d["q_nope"], d["q_pe"], d["kv_codes"], d["kv_scale"], d["pe_cache"],
+                                        d["seq_lens"], idx, SCALE, workspace=ws)
+    assert binding.read_status(ws) & binding.ATTN_DEV_BAD_INDEX
+    assert torch.isfinite(out.float()).all()
