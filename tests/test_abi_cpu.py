@@ -191,3 +191,16 @@ def test_prefill_chunk_ex_validation_codes(lib):
     assert call(fscale=0.0) == 1
     assert call(ws=need - 1) == 3
     assert call(layout=1, ws=need - 1) == 3  # the half-split layout itself is accepted
+
+
+def test_dsa_fp8_validation_codes(lib):
+    P = ctypes.c_void_p(FAKE)
+    g = lib.dsa_mla_decode_fp8
+    need = lib.dsa_mla_decode_workspace_size(2, 128, 512, 64, 2048)
+
+    def call(Dc=512, k=2048, sc=P, ws=need):
+        return g(P, P, P, sc, P, P, P, k, 0.07, P, P, 2, 128, Dc, 64, 4096, P, ws, None)
+    assert call(Dc=256) == 2
+    assert call(k=0) == 1
+    assert call(sc=None) == 1
+    assert call(ws=need - 1) == 3
