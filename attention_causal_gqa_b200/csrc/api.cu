@@ -721,7 +721,8 @@ int dsa_mla_decode(const void* q_nope, const void* q_pe, const void* kv_cache, c
       !aligned(out, 16) || !aligned(seq_lens, 4) || !aligned(topk_idx, 4) || !aligned(lse, 4) ||
       !aligned(workspace, 256))
     return fail(ATTN_ERR_INVALID_ARG, "misaligned pointer");
-  if (T_max > (1 << 26) || B > (1 << 20) || top_k > (1 << 26)) return fail(ATTN_ERR_UNSUPPORTED, "problem too large");
+  if (T_max > (1 << 26) || B > (1 << 20) || top_k > (1 << 26) || static_cast<long long>(B) * top_k > (1LL << 30))
+    return fail(ATTN_ERR_UNSUPPORTED, "problem too large");
   const size_t need = dsa_mla_decode_workspace_size(B, H, Dc, Dr, top_k);
   if (workspace_bytes < need)
     return fail(ATTN_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace_bytes, need);
@@ -755,7 +756,8 @@ int dsa_mla_decode_fp8(const void* q_nope, const void* q_pe, const void* kv_code
       !aligned(pe_cache, 16) || !aligned(out, 16) || !aligned(seq_lens, 4) || !aligned(topk_idx, 4) ||
       !aligned(lse, 4) || !aligned(workspace, 256))
     return fail(ATTN_ERR_INVALID_ARG, "misaligned pointer");
-  if (T_max > (1 << 26) || B > (1 << 20) || top_k > (1 << 26)) return fail(ATTN_ERR_UNSUPPORTED, "problem too large");
+  if (T_max > (1 << 26) || B > (1 << 20) || top_k > (1 << 26) || static_cast<long long>(B) * top_k > (1LL << 30))
+    return fail(ATTN_ERR_UNSUPPORTED, "problem too large");
   const size_t need = dsa_mla_decode_workspace_size(B, H, Dc, Dr, top_k);
   if (workspace_bytes < need)
     return fail(ATTN_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace_bytes, need);

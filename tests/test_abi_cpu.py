@@ -204,3 +204,10 @@ def test_dsa_fp8_validation_codes(lib):
     assert call(k=0) == 1
     assert call(sc=None) == 1
     assert call(ws=need - 1) == 3
+
+
+def test_dsa_gather_grid_limit(lib):
+    """B * top_k selected rows beyond 2^30 would not fit the gather's grid: rejected up front."""
+    P = ctypes.c_void_p(FAKE)
+    g = lib.dsa_mla_decode
+    assert g(P, P, P, P, P, P, 1 << 21, 0.07, P, P, 1024, 128, 512, 64, 1 << 22, P, 1 << 62, None) == 2
