@@ -529,11 +529,25 @@ def bench_dsa(args, world, dev, seed, pk, pk_kind, dense_ms=None):
     ms_attend = timed_region(attend, args.steps, 0, world)
     m_ms, mn = B_.profile_collect()
     k_mla = max_over_ranks(m_ms / max(mn, 1), world)
+    # the same selection attended over an E4M3 latent cache (one scale per token and 128-wide block)
+    from attention_causal_gqa_b200.synthetic import quantize_e4m3_rows
+    kv_codes, kv_scale = quantize_e4m3_rows(d["kv_cache"])
+
+    def attend_fp8():
+        B_.dsa_mla_decode_fp8(d["q_nope"], d["q_pe"], kv_codes, kv_scale, d["pe_cache"], d["seq_lens"], idx,
+                              p["scale"], out=out, lse=lse, workspace=ws2)
+
+    for _ in range(args.warmup):
+        attend_fp8()
+    ms_attend_fp8 = timed_region(attend_fp8, args.steps, 0, world)
+    B_.profile_collect()
+    del kv_codes, kv_scale
     ach = idx_bytes / (k_idx * 1e-3) / 1e9
     res = {"workload": DSA + ("_small_b8" if args.small else ""), "value": world * tokens * args.steps / (ms * 1e-3),
            "unit": "cached tokens/s", "ms_per_step": ms / args.steps, "kv_tokens": tokens,
            "selected_tokens": selected, "index_call_ms": ms_index / args.steps,
            "sparse_mla_call_ms": ms_attend / args.steps, "mla_kernel_ms": k_mla,
+           "sparse_mla_fp8_latent_call_ms": ms_attend_fp8 / args.steps,
            "dense_mla_ms_per_step": dense_ms, "gpu_launches": 5 * args.steps,
            "l2": "indexer keys (268 MB) and caches larger than L2",
            "roofline": {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
