@@ -64,12 +64,13 @@ EncodeTiledFn encode_fn() {
 
 // Tiled tensor map with 128-byte swizzle; dims/strides innermost first, strides in bytes for dims 1..rank-1.
 int make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const cuuint64_t* dims,
-             const cuuint64_t* strides, const cuuint32_t* box, const char* what) {
+             const cuuint64_t* strides, const cuuint32_t* box, const char* what,
+             CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = fn(m, dt, static_cast<cuuint32_t>(rank), const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(ATTN_ERR_CUDA, "tensor map encode failed for %s (CUresult %d)", what, (int)r);
   return ATTN_OK;
@@ -583,8 +584,11 @@ static int mla_run(const void* q_nope, const void* q_pe, const void* kv_cache, c
   {
     const cuuint64_t d[3] = {static_cast<cuuint64_t>(Dr), static_cast<cuuint64_t>(T_max), static_cast<cuuint64_t>(B)};
     const cuuint64_t s[2] = {static_cast<cuuint64_t>(Dr) * 2, static_cast<cuuint64_t>(T_max) * Dr * 2};
-    const cuuint32_t bx[3] = {64, static_cast<cuuint32_t>(attn::kMlaTile), 1};
-    if ((rc = make_map(&tmPE, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, pe_cache, d, s, bx, "pe_cache"))) return rc;
+    // each CTA of a cluster loads its 32 of the 64 rotary columns: 64-byte rows, 64-byte swizzle
+    const cuuint32_t bx[3] = {32, static_cast<cuuint32_t>(attn::kMlaTile), 1};
+    if ((rc = make_map(&tmPE, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, pe_cache, d, s, bx, "pe_cache",
+                       CU_TENSOR_MAP_SWIZZLE_64B)))
+      return rc;
   }
   attn::MlaParams p{};
   p.q_nope = q_nope;

@@ -58,7 +58,7 @@ cudaError_t launch_decode_range_merge(const float* part_o, const float* part_lse
                                       float* lse, int B, int H, int T_max, int n_ranges, cudaStream_t stream);
 
 // ------------------------------------------------------------------ MLA
-constexpr int kMlaTile = 32;        // tokens per tile
+constexpr int kMlaTile = 64;        // tokens per tile
 constexpr int kMlaMaxPairs = 74;    // two-CTA clusters in the persistent grid (148 SMs)
 
 struct MlaParams {

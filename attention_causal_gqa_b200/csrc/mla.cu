@@ -7,32 +7,41 @@
 // [q_nope | q_pe] . [kv_cache | pe_cache]^T ("attention study note", MLA
 // decoupled-RoPE section: the rotary part is concatenated to the content part).
 //
-// Work split. A cluster of two CTAs (two SMs) shares every token tile and splits
-// the 576 reduction columns: rank 0 owns kv columns 0-255, rank 1 owns kv columns
-// 256-511 plus the 64 rotary columns. Each CTA
-//   * loads only its own columns of each kv/pe tile (no byte is loaded twice),
-//   * computes its partial score block S_r = Q_r . KV_r^T (Q_r kept in TMEM),
-//   * sends S_r to its peer through distributed shared memory (staged, then one
-//     bulk copy per warp) and adds the peer's part (rank-0 part + rank-1 part in
-//     both CTAs: identical bits),
-//   * runs the online softmax on the full scores (both CTAs, same m and l),
-//   * accumulates O[:, its 256 columns] += P . KV[:, its 256 columns], with P
-//     written into TMEM and used as the MMA A operand.
-// Scheduling is persistent: the flattened sequence of 32-token tiles of all
+// Work split. O (128 heads x 512 fp32) fills a whole SM's tensor memory, so a
+// cluster of two CTAs shares every 64-token tile: rank r owns kv columns
+// [256 r, 256 r + 256) and rotary columns [32 r, 32 r + 32) -- 288 of the 576
+// reduction columns each, 18 MMAs per tile on both SMs. Each CTA
+//   * loads only its own columns of each tile (no byte is loaded twice),
+//   * computes its partial score block S_r = Q_r . K_r^T (M = 128 heads, N = 64
+//     tokens, Q_r kept in tensor memory as the A operand),
+//   * sends S_r to its peer through distributed shared memory and adds the peer's
+//     part (rank-0 part + rank-1 part in both CTAs: identical bits, hence the same
+//     running max and sum on both sides),
+//   * accumulates O[:, its 256 kv columns] += P . V with P in tensor memory.
+// The exchange runs on its own warps: four sender warps read each partial score
+// tile out of TMEM as soon as it is computed, stage it and copy it to the peer,
+// while the softmax warps work on the previous tile.
+// Scheduling is persistent: the flattened sequence of 64-token tiles of all
 // sequences is cut into one contiguous range per cluster; each maximal piece of
 // a range inside one sequence (a segment) produces one normalised partial result
-// and its LSE, merged per sequence by mla_merge_kernel (merge.cu).
+// and its LSE, merged per sequence by the range merge (merge.cu).
 //
-// Roles per CTA (352 threads): warpgroups 0 and 1 take the tiles in turn (tile k
-// goes to warpgroup k % 2, one thread per head): each reads its partial score tile
-// out of TMEM, sends it to the peer, adds the peer's part, and runs the online
-// softmax on it, writing P. Only the running max (early in a tile) and the running
-// sum (late in a tile) pass from one warpgroup to the other, through shared memory,
-// so two tiles are in flight at once. The owner of a segment's first tile loads
-// Q_r into TMEM; the owner of its last tile writes the partial result. Warp 8 is
-// the TMA producer, warp 9 allocates TMEM and issues Q K^T, warp 10 issues P V.
-// TMEM columns: O [0,256), Q_r [256, 416), S double buffer [416, 480) (tile k in
-// buffer k % 2), P double buffer [480, 512).
+// Roles per CTA (480 threads). A warp reaches only its TMEM lane quarter
+// q = warp % 4, i.e. heads [32 q, 32 q + 32), one thread per head.
+//   * Softmax warps 0-7: warpgroup w (warps 4w .. 4w + 3) handles tokens
+//     [32 w, 32 w + 32) of every tile. Warps q and q + 4 share the heads and
+//     combine their half-tile maxima through shared memory; each keeps the running
+//     sum of its own tokens. They add the staged own part and the peer's part,
+//     run the online softmax and write P into TMEM.
+//   * Sender warps 11-14 (quarter warp % 4): read the 64 partial scores of their
+//     heads out of TMEM (freeing the S buffer for the next tile), stage them in
+//     shared memory and send them to the same sender's receive block on the peer
+//     with one bulk copy that completes on the peer's barrier.
+//   * Warp 8 is the TMA producer, warp 9 allocates TMEM and issues Q K^T, warp 10
+//     issues P V.
+// Every wait is bounded; no named barrier is used, so a role that gives up
+// cannot strand the others.
+// TMEM columns: O [0, 256), Q_r [256, 400), S [416, 480), P [480, 512).
 #include <cuda_bf16.h>
 
 #include "kernels.h"
@@ -44,15 +53,21 @@ namespace {
 
 constexpr int kH = 128, kDc = 512, kDr = 64;
 constexpr int TN = kMlaTile;              // tokens per tile
-constexpr int KV_BOX = TN * 128;          // one 64-column block of a tile (TN rows of 128 bytes)
-constexpr int NST = 7;                    // kv ring depth
-constexpr int STAGE = 5 * KV_BOX;         // room for the larger (rank-1) share
-constexpr int XBUF = kH * TN * 4;         // one fp32 exchange buffer (one per tile parity)
-constexpr int O_COL = 0, Q_COL = 256, S_COL = 416, P_COL = 480;  // S: 2 x TN fp32, P: 2 x TN/2 bf16 pairs
+constexpr int HALF = TN / 2;              // tokens per softmax warpgroup
+constexpr int KV_BOX = TN * 128;          // one 64-column kv block of a tile (TN rows of 128 bytes)
+constexpr int PE_BOX = TN * 64;           // this CTA's 32 rotary columns (TN rows of 64 bytes)
+constexpr int STAGE = 4 * KV_BOX + PE_BOX;
+constexpr int NST = 4;                    // ring depth
+constexpr int XCHUNK = 32 * TN * 4;       // one quarter's block of partial scores: 32 heads x 64 tokens fp32
+constexpr int XBUF = 4 * XCHUNK;
+constexpr int O_COL = 0, Q_COL = 256, S_COL = 416, P_COL = 480;
 constexpr int TMEM_COLS = 512;
-constexpr int kMlaThreads = 352;
-constexpr int SMEM_BYTES = 1024 + NST * STAGE + 4 * XBUF + 4 * kH * 4 + 512;
-static_assert(S_COL + 2 * TN <= P_COL && P_COL + TN <= TMEM_COLS, "TMEM budget");
+constexpr int kMlaThreads = 480;
+constexpr int kNumBars = 2 * NST + 4 + 12 + 8 + 3;
+constexpr int SMEM_BYTES = 1024 + NST * STAGE + 2 * XBUF + 2 * (2 * 2 * kH * 4) + kNumBars * 8 + 16;
+static_assert(TN == 64, "the exchange and P layout assume 64-token tiles");
+static_assert(Q_COL + 144 <= S_COL && S_COL + TN <= P_COL && P_COL + TN / 2 <= TMEM_COLS, "TMEM budget");
+static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -66,8 +81,7 @@ __device__ __forceinline__ uint32_t mapa_peer(uint32_t saddr, uint32_t peer) {
   return r;
 }
 // One bulk copy of a staged block from this CTA's shared memory into the peer's,
-// completing its bytes on the peer's mbarrier (the copy engine moves the block:
-// far fewer transactions than per-thread remote stores).
+// completing its bytes on the peer's mbarrier.
 __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
                                                   uint32_t bar_cluster) {
   asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -76,7 +90,7 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t
                : "memory");
 }
 // Remote arrive without release semantics: used only to say "these bytes were read",
-// where the reads have already returned their values (no write needs publishing).
+// after the values read have been used (no write needs publishing).
 __device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t bar_cluster_addr) {
   asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
 }
@@ -110,31 +124,41 @@ __device__ __forceinline__ void for_each_segment(const MlaParams& p, int pair, F
   }
 }
 
-// One body for both ranks (a runtime rank keeps the code small enough for the
-// instruction cache; both ranks differ only in loop bounds and column offsets).
+// 32 consecutive bf16 pairs (128 bytes) of a row into registers.
+__device__ __forceinline__ void load_row32(const uint32_t* src, uint32_t (&r)[32]) {
+#pragma unroll
+  for (int e = 0; e < 32; e += 4) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + e));
+    r[e] = v.x;
+    r[e + 1] = v.y;
+    r[e + 2] = v.z;
+    r[e + 3] = v.w;
+  }
+}
+
 __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* tmKV, const CUtensorMap* tmPE,
                                          uint8_t* smem, const int R) {
-  const int NKB = R == 0 ? 4 : 5;  // 64-column blocks of the score reduction owned by this CTA
-  const int STAGE_BYTES = NKB * KV_BOX;
   const uint32_t PEER = 1 - R;
   uint8_t* sKV = smem;
-  float* xbuf = reinterpret_cast<float*>(smem + NST * STAGE);               // [2][kH][TN] from the peer
-  float* sbuf = xbuf + 2 * kH * TN;                                         // [2][kH][TN] own, staged for the copy
-  float* m_sh = reinterpret_cast<float*>(smem + NST * STAGE + 4 * XBUF);    // [2][kH] running max after tile k
-  float* l_sh = m_sh + 2 * kH;                                              // [2][kH] running sum after tile k
-  uint64_t* bars = reinterpret_cast<uint64_t*>(l_sh + 2 * kH);
+  // partial-score blocks [4 quarters][2 token halves][32 heads][32 tokens]: from the peer / own, staged
+  float* xrecv = reinterpret_cast<float*>(smem + NST * STAGE);
+  float* xsend = xrecv + XBUF / 4;
+  float* mx_sh = xsend + XBUF / 4;                                // [2 parity][2 wg][kH] half-tile maxima
+  float* l_sh = mx_sh + 2 * 2 * kH;                               // [2 parity][2 wg][kH] half sums at a segment end
+  uint64_t* bars = reinterpret_cast<uint64_t*>(l_sh + 2 * 2 * kH);
   uint64_t* kv_full = bars;
   uint64_t* kv_empty = kv_full + NST;
-  uint64_t* s_full = kv_empty + NST;   // [2] S(k) computed into S buffer k % 2
-  uint64_t* s_free = s_full + 2;       // [2] S(k) has been read out of TMEM
-  uint64_t* p_full = s_free + 2;       // [2] P(k) written into P buffer k % 2
-  uint64_t* o_done = p_full + 2;       // [2] P(k) V(k) completed
-  uint64_t* x_full = o_done + 2;       // [2] the peer's partial scores of tile k landed in xbuf[k % 2]
-  uint64_t* x_empty = x_full + 2;      // [2] the peer has consumed what this CTA sent for tile k
-  uint64_t* m_ready = x_empty + 2;     // [2] running max after tile k is in m_sh[k % 2]
-  uint64_t* l_ready = m_ready + 2;     // [2] running sum after tile k is in l_sh[k % 2]
-  uint64_t* q_ready = l_ready + 2;     // Q_r of the segment is in TMEM
-  uint64_t* o_free = q_ready + 1;      // the segment's partial result has been read out of O
+  uint64_t* s_full = kv_empty + NST;  // S(k) computed
+  uint64_t* s_free = s_full + 1;      // the sender warps have read S(k) out of TMEM
+  uint64_t* p_full = s_free + 1;      // P(k) written (and any O rescale done)
+  uint64_t* o_done = p_full + 1;      // P(k) V(k) completed
+  uint64_t* x_full = o_done + 1;      // [4] the peer's block for quarter q landed in xrecv
+  uint64_t* x_empty = x_full + 4;     // [4] the peer's softmax warps of quarter q consumed what was sent
+  uint64_t* own_free = x_empty + 4;   // [4] this CTA's softmax warps of quarter q consumed the staged block
+  uint64_t* mx_bar = own_free + 4;    // [4] warps q and q + 4 published their half maxima
+  uint64_t* l_bar = mx_bar + 4;       // [4] warps q and q + 4 published their half sums
+  uint64_t* q_ready = l_bar + 4;      // Q_r of the segment is in TMEM
+  uint64_t* o_free = q_ready + 1;     // the segment's partial result has been read out of O
   uint64_t* mma_done = o_free + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -148,23 +172,24 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
-    for (int u = 0; u < 2; ++u) {
-      mbar_init(&s_full[u], 1);
-      mbar_init(&s_free[u], 128);
-      mbar_init(&p_full[u], 128);
-      mbar_init(&o_done[u], 1);
-      mbar_init(&x_full[u], 1);   // one expect_tx arrive per phase + the bytes of the peer's bulk copies
-      mbar_init(&x_empty[u], 1);  // one remote arrive from the peer
-      mbar_init(&m_ready[u], 128);
-      mbar_init(&l_ready[u], 128);
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 128);
+    mbar_init(p_full, 256);
+    mbar_init(o_done, 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&x_full[i], 1);    // the sender's expect_tx arrive + the bytes of the peer's bulk copy
+      mbar_init(&x_empty[i], 2);   // remote arrives from the peer's two softmax warps of quarter i
+      mbar_init(&own_free[i], 2);  // this CTA's two softmax warps of quarter i
     }
-    mbar_init(q_ready, 128);
-    mbar_init(o_free, 128);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&mx_bar[i], 64);
+      mbar_init(&l_bar[i], 64);
+    }
+    mbar_init(q_ready, 256);
+    mbar_init(o_free, 256);
     mbar_init(mma_done, 2);
     *abort_flag = 0;
     fence_mbar_init();
-    // arm the receive buffers for the first two tiles
-    for (int u = 0; u < 2; ++u) mbar_arrive_expect_tx(&x_full[u], XBUF);
   }
   if (warp == 9) {
     tmem_alloc(tmem_slot, TMEM_COLS);
@@ -180,7 +205,7 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
     // --------------------------------------------------------------- producer
     if (lane == 0) {
       prefetch_tmap(tmKV);
-      if (R == 1) prefetch_tmap(tmPE);
+      prefetch_tmap(tmPE);
       int g = 0;
       bool ok = true;
       for_each_segment(p, pair, [&](int b, int t0, int t1, int) {
@@ -188,19 +213,20 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
           const int s = g % NST;
           if (!mbar_wait(&kv_empty[s], ((g / NST) & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
           uint8_t* dst = sKV + s * STAGE;
-          mbar_arrive_expect_tx(&kv_full[s], STAGE_BYTES);
+          mbar_arrive_expect_tx(&kv_full[s], STAGE);
 #pragma unroll
           for (int c = 0; c < 4; ++c) tma_load_3d(dst + c * KV_BOX, tmKV, &kv_full[s], R * 256 + c * 64, t * TN, b);
-          if (R == 1) tma_load_3d(dst + 4 * KV_BOX, tmPE, &kv_full[s], 0, t * TN, b);
+          tma_load_3d(dst + 4 * KV_BOX, tmPE, &kv_full[s], R * 32, t * TN, b);
         }
       });
     }
-  } else if (warp >= 9) {
+  } else if (warp == 9 || warp == 10) {
     // ------------------------------ MMA issuers (whole warps): 9 = scores, 10 = P V
-    constexpr uint32_t HI = sdesc_hi_sw128(1024);
+    constexpr uint32_t HI128 = sdesc_hi_sw128(1024);
     bool ok = true;
     int seg = 0;
     if (warp == 9) {
+      constexpr uint32_t HI64 = sdesc_hi_sw64(512);
       constexpr uint32_t idesc_s = idesc_f32acc(1, 128, TN, false, false);
       const uint32_t kv_lo_k = sdesc_lo(smem_u32(sKV), 16);
       for_each_segment(p, pair, [&](int, int t0, int t1, int g0) {
@@ -210,18 +236,23 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
         tc_fence_after();
         for (int i = 0; ok && i < t1 - t0; ++i) {
           const int k = g0 + i;
-          if (k >= 2 && !(ok = mbar_wait_warp(&s_free[k & 1], ((k - 2) >> 1) & 1, abort_flag, p.status))) break;
+          // single S buffer: S(k - 1) must have been read out by the sender warps
+          if (k >= 1 && !(ok = mbar_wait_warp(s_free, (k - 1) & 1, abort_flag, p.status))) break;
           if (!(ok = mbar_wait_warp(&kv_full[k % NST], (k / NST) & 1, abort_flag, p.status))) break;
           tc_fence_after();
           const uint32_t b0 = kv_lo_k + (((k % NST) * STAGE) >> 4);
-          const uint32_t d = tmem_base + S_COL + (k & 1) * TN;
+          const uint32_t d = tmem_base + S_COL;
 #pragma unroll 1
-          for (int bx = 0; bx < NKB; ++bx)
+          for (int bx = 0; bx < 4; ++bx)
 #pragma unroll
             for (int kq = 0; kq < 4; ++kq)
-              umma_f16_ts_warp(d, tmem_base + Q_COL + (bx * 4 + kq) * 8, b0 + ((bx * KV_BOX + kq * 32) >> 4), HI,
+              umma_f16_ts_warp(d, tmem_base + Q_COL + (bx * 4 + kq) * 8, b0 + ((bx * KV_BOX + kq * 32) >> 4), HI128,
                                idesc_s, (bx > 0 || kq > 0) ? 1u : 0u);
-          umma_commit_warp(&s_full[k & 1]);
+#pragma unroll
+          for (int kq = 0; kq < 2; ++kq)  // the 32 rotary columns: 64-byte rows, 64-byte swizzle
+            umma_f16_ts_warp(d, tmem_base + Q_COL + 128 + kq * 8, b0 + ((4 * KV_BOX + kq * 32) >> 4), HI64, idesc_s,
+                             1u);
+          umma_commit_warp(s_full);
         }
       });
     } else {
@@ -231,240 +262,246 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
         if (!ok) return;
         for (int i = 0; ok && i < t1 - t0; ++i) {
           const int k = g0 + i;
-          if (!(ok = mbar_wait_warp(&p_full[k & 1], (k >> 1) & 1, abort_flag, p.status))) break;
+          if (!(ok = mbar_wait_warp(p_full, k & 1, abort_flag, p.status))) break;
           // the first P V of a segment overwrites O: the previous segment's result must be out
           if (i == 0 && seg > 0 && !(ok = mbar_wait_warp(o_free, (seg - 1) & 1, abort_flag, p.status))) break;
           tc_fence_after();
           const uint32_t b0 = kv_lo_v + (((k % NST) * STAGE) >> 4);
-          const uint32_t a0 = tmem_base + P_COL + (k & 1) * (TN / 2);
+          const uint32_t a0 = tmem_base + P_COL;
 #pragma unroll
           for (int kb = 0; kb < TN / 16; ++kb)
-            umma_f16_ts_warp(tmem_base + O_COL, a0 + kb * 8, b0 + ((kb * 16 * 128) >> 4), HI, idesc_o,
+            umma_f16_ts_warp(tmem_base + O_COL, a0 + kb * 8, b0 + ((kb * 16 * 128) >> 4), HI128, idesc_o,
                              (i > 0 || kb > 0) ? 1u : 0u);
-          umma_commit_warp(&o_done[k & 1]);
-          umma_commit_warp(&kv_empty[k % NST]);  // S(k) is complete too: P(k) was computed from it
+          umma_commit_warp(o_done);
+          umma_commit_warp(&kv_empty[k % NST]);  // S(k) was complete before P(k) existed
         }
         ++seg;
       });
     }
     umma_commit_warp(mma_done);
     mbar_wait_warp(mma_done, 0, abort_flag, p.status);
+  } else if (warp >= 11) {
+    // ------------------------------------------ sender warps: quarter q = warp % 4
+    const int q = warp & 3;
+    const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    float* stage = xsend + (q * 2 * 32 + lane) * HALF;  // this lane's row of token half 0 (half 1: 32 rows on)
+    const uint32_t peer_recv = mapa_peer(smem_u32(xrecv + q * 2 * 32 * HALF), PEER);
+    const uint32_t peer_full = mapa_peer(smem_u32(&x_full[q]), PEER);
+    const uint32_t send_src = smem_u32(xsend + q * 2 * 32 * HALF);
+    bool ok = true;
+    for_each_segment(p, pair, [&](int, int t0, int t1, int g0) {
+      for (int i = 0; ok && i < t1 - t0; ++i) {
+        const int k = g0 + i;
+        // S(k) out of TMEM; the buffer may then take S(k + 1)
+        if (!(ok = mbar_wait_warp(s_full, k & 1, abort_flag, p.status))) break;
+        tc_fence_after();
+        uint32_t r0[32], r1[32];
+        tmem_ld32(t_lane + S_COL, r0);
+        tmem_ld32(t_lane + S_COL + HALF, r1);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(s_free);
+        // the staged block of tile k - 1 has been read here, and the peer has consumed
+        // what it received of tile k - 1 (its copy had landed, so the staging block was read)
+        if (!(ok = mbar_wait_warp(&own_free[q], (k & 1) ^ 1, abort_flag, p.status))) break;
+        if (!(ok = mbar_wait_warp(&x_empty[q], (k & 1) ^ 1, abort_flag, p.status))) break;
+        if (lane == 0) mbar_arrive_expect_tx(&x_full[q], XCHUNK);  // receive tile k from the peer
+#pragma unroll
+        for (int c = 0; c < HALF / 4; ++c) {
+          const int cc = 4 * ((c + lane) & (HALF / 4 - 1));
+          *reinterpret_cast<uint4*>(stage + cc) = make_uint4(r0[4 * c], r0[4 * c + 1], r0[4 * c + 2], r0[4 * c + 3]);
+          *reinterpret_cast<uint4*>(stage + 32 * HALF + cc) =
+              make_uint4(r1[4 * c], r1[4 * c + 1], r1[4 * c + 2], r1[4 * c + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) bulk_copy_to_peer(peer_recv, send_src, XCHUNK, peer_full);
+      }
+    });
   } else {
-    // ----------------------------- softmax warpgroups: tile k is handled by warpgroup k % 2
-    const int a = warp >> 2;
-    const int h = (warp & 3) * 32 + lane;  // head == TMEM lane
-    const int th = threadIdx.x - 128 * a;
-    const uint32_t t_lane = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    // ------------------------------------------------- softmax warpgroups
+    const int w = warp >> 2;               // token half
+    const int q = warp & 3;                // lane quarter
+    const int h = q * 32 + lane;           // head == TMEM lane
+    const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     const float sl2 = p.scale_log2;
-    const uint32_t peer_xbuf = mapa_peer(smem_u32(xbuf), PEER);
-    const uint32_t peer_xfull = mapa_peer(smem_u32(x_full), PEER);
-    const uint32_t peer_xempty = mapa_peer(smem_u32(x_empty), PEER);
-    float* my_x = xbuf + (a * kH + h) * TN;
+    const int row = ((q * 2 + w) * 32 + lane) * HALF;
+    const float* my_recv = xrecv + row;
+    const float* my_own = xsend + row;
+    const uint32_t peer_empty = mapa_peer(smem_u32(&x_empty[q]), PEER);
     bool alive = true;
     auto fail = [&](bool ok) -> bool {
       if (__any_sync(0xffffffffu, !ok)) alive = false;
       return !alive;
     };
+    int seg = 0;
     for_each_segment(p, pair, [&](int b, int t0, int t1, int g0) {
       if (!alive) return;
       const int n = t1 - t0;
-      // Q_r row of head h into TMEM (bf16 pairs are already in the operand layout), by
-      // the owner of the segment's first tile, once the last score tile of the previous
-      // segment has been read (then every earlier Q K^T has completed).
-      if ((g0 & 1) == a) {
-        if (g0 > 0 && fail(mbar_wait(&m_ready[a ^ 1], ((g0 - 1) >> 1) & 1, abort_flag, p.status))) return;
+      // Q_r of sequence b into TMEM (bf16 pairs are already in the operand layout). Every
+      // S MMA of the previous segment has completed: its last score tile was staged.
+      {
         const uint32_t* qn = reinterpret_cast<const uint32_t*>(
-            reinterpret_cast<const __nv_bfloat16*>(p.q_nope) + (static_cast<size_t>(b) * kH + h) * kDc + R * 256);
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {  // 4 x 32 columns = 256 bf16
-          uint32_t r[32];
-#pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(qn + c * 32 + e));
-            r[e] = v.x; r[e + 1] = v.y; r[e + 2] = v.z; r[e + 3] = v.w;
-          }
-          tmem_st32(t_lane + Q_COL + c * 32, r);
-        }
-        if (R == 1) {
+            reinterpret_cast<const __nv_bfloat16*>(p.q_nope) + (static_cast<size_t>(b) * kH + h) * kDc + R * 256 +
+            w * 128);
+        uint32_t r[32];
+        load_row32(qn, r);
+        tmem_st32(t_lane + Q_COL + w * 64, r);
+        load_row32(qn + 32, r);
+        tmem_st32(t_lane + Q_COL + w * 64 + 32, r);
+        if (w == 1) {
           const uint32_t* qp = reinterpret_cast<const uint32_t*>(
-              reinterpret_cast<const __nv_bfloat16*>(p.q_pe) + (static_cast<size_t>(b) * kH + h) * kDr);
-          uint32_t r[32];
+              reinterpret_cast<const __nv_bfloat16*>(p.q_pe) + (static_cast<size_t>(b) * kH + h) * kDr + R * 32);
+          uint32_t r16[16];
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
+          for (int e = 0; e < 16; e += 4) {
             const uint4 v = __ldg(reinterpret_cast<const uint4*>(qp + e));
-            r[e] = v.x; r[e + 1] = v.y; r[e + 2] = v.z; r[e + 3] = v.w;
+            r16[e] = v.x;
+            r16[e + 1] = v.y;
+            r16[e + 2] = v.z;
+            r16[e + 3] = v.w;
           }
-          tmem_st32(t_lane + Q_COL + 128, r);
+          tmem_st16(t_lane + Q_COL + 128, r16);
         }
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(q_ready);
       }
       const int L = min(max(__ldg(p.seq_lens + b), 0), p.T_max);
-      float m_k = -INFINITY, l_k = 0.f;
-      for (int i = (g0 & 1) == a ? 0 : 1; i < n; i += 2) {
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int i = 0; i < n; ++i) {
         const int k = g0 + i;
-        const uint32_t ph = (k >> 1) & 1;
-        // partial scores of tile k out of TMEM; the buffer is free for S(k + 2) at once
-        if (fail(mbar_wait(&s_full[a], ph, abort_flag, p.status))) return;
-        tc_fence_after();
-        uint32_t cur[TN];
-        tmem_ld32(t_lane + S_COL + a * TN, cur);
-        tmem_ld_wait();
-        tc_fence_before();
-        mbar_arrive(&s_free[a]);
-        // send them to the peer (chunk c of a row at slot (c + h) mod 8): stage the tile,
-        // then one thread copies all of it. The staging buffer and the peer's receive
-        // buffer are both free once the peer has consumed tile k - 2 (its copy had landed).
-        if (fail(mbar_wait(&x_empty[a], ph ^ 1, abort_flag, p.status))) return;  // carries no data: plain wait
-        {
-          float* mine = sbuf + (a * kH + h) * TN;
+        // own staged part + the peer's part of tile k: rank-0 part + rank-1 part in both CTAs
+        if (fail(mbar_wait(&x_full[q], k & 1, abort_flag, p.status))) return;
+        float s[HALF];
 #pragma unroll
-          for (int c = 0; c < TN / 4; ++c)
-            *reinterpret_cast<uint4*>(mine + 4 * ((c + h) & (TN / 4 - 1))) =
-                make_uint4(cur[4 * c], cur[4 * c + 1], cur[4 * c + 2], cur[4 * c + 3]);
-          fence_proxy_async_smem();
-          __syncwarp();
-          // each warp sends its own 32 rows as soon as they are staged
-          const int row0 = (warp & 3) * 32;
-          if (lane == 0)
-            bulk_copy_to_peer(peer_xbuf + a * XBUF + row0 * (TN * 4), smem_u32(sbuf + (a * kH + row0) * TN),
-                              XBUF / 4, peer_xfull + a * 8);
+        for (int c = 0; c < HALF / 4; ++c) {
+          const int cc = 4 * ((c + lane) & (HALF / 4 - 1));
+          const float4 v = *reinterpret_cast<const float4*>(my_recv + cc);
+          const float4 o = *reinterpret_cast<const float4*>(my_own + cc);
+          s[4 * c + 0] = R == 0 ? o.x + v.x : v.x + o.x;
+          s[4 * c + 1] = R == 0 ? o.y + v.y : v.y + o.y;
+          s[4 * c + 2] = R == 0 ? o.z + v.z : v.z + o.z;
+          s[4 * c + 3] = R == 0 ? o.w + v.w : v.w + o.w;
         }
-        // add the peer's part: rank-0 part + rank-1 part in both CTAs (identical bits). The
-        // peer's copied bytes complete on this local barrier, which makes them visible
-        // to a plain wait (same rule as a TMA load).
-        if (fail(mbar_wait(&x_full[a], ph, abort_flag, p.status))) return;
-        float s[TN];
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&own_free[q]);
+          mbar_arrive_remote_relaxed(peer_empty);
+        }
+        const int valid = L - (t0 + i) * TN - w * HALF;  // tokens of this half inside the sequence
+        if (valid < HALF) {
 #pragma unroll
-        for (int c = 0; c < TN / 4; ++c) {
-          const float4 v = *reinterpret_cast<const float4*>(my_x + 4 * ((c + h) & (TN / 4 - 1)));
-          const float w0 = __uint_as_float(cur[4 * c]), w1 = __uint_as_float(cur[4 * c + 1]);
-          const float w2 = __uint_as_float(cur[4 * c + 2]), w3 = __uint_as_float(cur[4 * c + 3]);
-          s[4 * c + 0] = R == 0 ? w0 + v.x : v.x + w0;
-          s[4 * c + 1] = R == 0 ? w1 + v.y : v.y + w1;
-          s[4 * c + 2] = R == 0 ? w2 + v.z : v.z + w2;
-          s[4 * c + 3] = R == 0 ? w3 + v.w : v.w + w3;
-        }
-        named_bar_sync(1 + a, 128);  // every row of xbuf[a] has been read
-        if (th == 0) {
-          mbar_arrive_remote_relaxed(peer_xempty + a * 8);
-          mbar_arrive_expect_tx(&x_full[a], XBUF);  // re-arm for tile k + 2
-        }
-        const int valid = L - (t0 + i) * TN;  // tokens of this tile inside the sequence
-        if (valid < TN) {
-#pragma unroll
-          for (int c = 0; c < TN; ++c)
+          for (int c = 0; c < HALF; ++c)
             if (c >= valid) s[c] = -INFINITY;
         }
         float mx0 = fmax3f(s[0], s[1], s[2]), mx1 = fmax3f(s[3], s[4], s[5]);
 #pragma unroll
-        for (int c = 6; c + 3 < TN; c += 4) {
+        for (int c = 6; c + 3 < HALF; c += 4) {
           mx0 = fmax3f(mx0, s[c], s[c + 1]);
           mx1 = fmax3f(mx1, s[c + 2], s[c + 3]);
         }
-        mx0 = fmaxf(mx0, s[TN - 2]);
-        mx1 = fmaxf(mx1, s[TN - 1]);
-        const float m_tile = fmaxf(mx0, mx1) * sl2;
-        // running max after tile k - 1 (from the other warpgroup; ignored at a segment start)
-        float m_prev = -INFINITY;
-        if (k > 0) {
-          if (fail(mbar_wait(&m_ready[a ^ 1], ((k - 1) >> 1) & 1, abort_flag, p.status))) return;
-          if (i > 0) m_prev = m_sh[(a ^ 1) * kH + h];
-        }
+        mx0 = fmaxf(mx0, s[HALF - 2]);
+        mx1 = fmaxf(mx1, s[HALF - 1]);
+        // the other half's maximum (warp q + 4 or q - 4 holds the same heads)
+        float* mslot = mx_sh + (k & 1) * 2 * kH;
+        mslot[w * kH + h] = fmaxf(mx0, mx1);
+        mbar_arrive(&mx_bar[q]);
+        if (fail(mbar_wait(&mx_bar[q], k & 1, abort_flag, p.status))) return;
+        const float m_tile = fmaxf(mslot[h], mslot[kH + h]) * sl2;
         bool rescale = false;
+        float alpha = 1.f;
         if (i == 0) {
-          m_k = m_tile;
-        } else {
-          rescale = __any_sync(0xffffffffu, m_tile > m_prev + 8.0f);
-          m_k = rescale ? fmaxf(m_prev, m_tile) : m_prev;
+          m_run = m_tile;
+        } else if (__any_sync(0xffffffffu, m_tile > m_run + 8.0f)) {
+          rescale = true;
+          const float m_new = fmaxf(m_run, m_tile);
+          alpha = ex2_approx(m_run - m_new);
+          m_run = m_new;
         }
-        m_sh[a * kH + h] = m_k;
-        mbar_arrive(&m_ready[a]);
-        const float alpha = rescale ? ex2_approx(m_prev - m_k) : 1.f;
-        if (rescale) {
-          // O must hold P V of tile k - 1 before it is scaled
-          if (fail(mbar_wait(&o_done[a ^ 1], ((k - 1) >> 1) & 1, abort_flag, p.status))) return;
+        // P = 2^(s * scale * log2 e - m); in a half without masked tokens 1 of every 4
+        // pairs takes the FMA-pipe exp2, which relieves the MUFU (shared by two warps)
+        uint32_t pp[HALF / 2];
+        float2 lsum = make_float2(0.f, 0.f);
+        const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-m_run, -m_run);
+        const bool soft = valid >= HALF;
+#pragma unroll
+        for (int c = 0; c < HALF; c += 2) {
+          const float2 z = ffma2(make_float2(s[c], s[c + 1]), sc2, nm2);
+          float2 e;
+          if (soft && (c & 6) == 6) {
+            e = exp2_fma2(z);
+          } else {
+            e.x = ex2_approx(z.x);
+            e.y = ex2_approx(z.y);
+          }
+          lsum = fadd2(lsum, e);
+          pp[c / 2] = pack_bf16x2(e.x, e.y);
+        }
+        // one P buffer: P(k - 1) V(k - 1) must be complete before P(k) replaces it
+        // (and before O is rescaled)
+        if (k >= 1) {
+          if (fail(mbar_wait(o_done, (k - 1) & 1, abort_flag, p.status))) return;
           tc_fence_after();
+        }
+        if (rescale) {
 #pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
+          for (int c = 0; c < 4; ++c) {
             uint32_t r[32];
-            tmem_ld32(t_lane + O_COL + c * 32, r);
+            tmem_ld32(t_lane + O_COL + w * 128 + c * 32, r);
             tmem_ld_wait();
 #pragma unroll
             for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            tmem_st32(t_lane + O_COL + c * 32, r);
+            tmem_st32(t_lane + O_COL + w * 128 + c * 32, r);
           }
         }
-        uint32_t pp[TN / 2];
-        float la = 0.f, lb = 0.f;
-#pragma unroll
-        for (int c = 0; c < TN; c += 2) {
-          const float e0 = ex2_approx(fmaf(s[c], sl2, -m_k));
-          const float e1 = ex2_approx(fmaf(s[c + 1], sl2, -m_k));
-          la += e0;
-          lb += e1;
-          pp[c / 2] = pack_bf16x2(e0, e1);
-        }
-        // P buffer a last held P(k - 2): its P V must be complete before it is overwritten
-        if (k >= 2) {
-          if (fail(mbar_wait(&o_done[a], ((k - 2) >> 1) & 1, abort_flag, p.status))) return;
-          tc_fence_after();
-        }
-        tmem_st16(t_lane + P_COL + a * (TN / 2), pp);
-        if (valid < TN) {
-          // cached rows past the sequence end may hold anything: zero this CTA's
-          // value columns for them so that 0 * garbage cannot reach O
+        tmem_st16(t_lane + P_COL + w * (HALF / 2), pp);
+        if (valid < HALF) {
+          // cached rows past the sequence end may hold anything: zero this CTA's value
+          // columns for them so that 0 * garbage cannot reach O
           uint8_t* st = sKV + (k % NST) * STAGE;
-          const int nbad = TN - valid;
-          for (int idx = th; idx < 4 * nbad * 8; idx += 128) {
-            const int bxx = idx / (nbad * 8), r = valid + (idx / 8) % nbad, ch = idx % 8;
+          const int r0 = w * HALF + max(valid, 0), nbad = (w + 1) * HALF - r0;
+          for (int idx = q * 32 + lane; idx < 4 * nbad * 8; idx += 128) {
+            const int bxx = idx / (nbad * 8), r = r0 + (idx / 8) % nbad, ch = idx % 8;
             *reinterpret_cast<uint4*>(st + bxx * KV_BOX + r * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
           }
           fence_proxy_async_smem();
-          named_bar_sync(1 + a, 128);  // every zero row is written before any thread signals P
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&p_full[a]);
-        // running sum after tile k (from the other warpgroup's sum after tile k - 1)
-        float l_prev = 0.f;
-        if (k > 0) {
-          if (fail(mbar_wait(&l_ready[a ^ 1], ((k - 1) >> 1) & 1, abort_flag, p.status))) return;
-          if (i > 0) l_prev = l_sh[(a ^ 1) * kH + h];
-        }
-        l_k = l_prev * alpha + (la + lb);
-        l_sh[a * kH + h] = l_k;
-        mbar_arrive(&l_ready[a]);
+        mbar_arrive(p_full);
+        l_run = l_run * alpha + (lsum.x + lsum.y);
       }
-      // segment epilogue by the owner of the last tile: O / l for this CTA's 256
-      // columns, and the LSE (rank 0). P V of the segment's earlier tiles completed
-      // before P V of its last one.
+      // segment epilogue: O / l for this CTA's 256 columns (128 per warpgroup) and the
+      // LSE (rank 0). P V of the segment's last tile completes after all earlier ones.
       const int k_last = g0 + n - 1;
-      if ((k_last & 1) == a) {
-        if (fail(mbar_wait(&o_done[a], (k_last >> 1) & 1, abort_flag, p.status))) return;
-        tc_fence_after();
-        const int slot = pair + b;
-        const float inv_l = 1.f / l_k;
-        float* orow = p.part_o + (static_cast<size_t>(slot) * kH + h) * kDc + R * 256;
+      if (fail(mbar_wait(o_done, k_last & 1, abort_flag, p.status))) return;
+      tc_fence_after();
+      float* lslot = l_sh + (seg & 1) * 2 * kH;
+      lslot[w * kH + h] = l_run;
+      mbar_arrive(&l_bar[q]);
+      if (fail(mbar_wait(&l_bar[q], seg & 1, abort_flag, p.status))) return;
+      const float l_tot = lslot[h] + lslot[kH + h];
+      const int slot = pair + b;
+      const float inv_l = 1.f / l_tot;
+      float* orow = p.part_o + (static_cast<size_t>(slot) * kH + h) * kDc + R * 256 + w * 128;
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          uint32_t r[32];
-          tmem_ld32(t_lane + O_COL + c * 32, r);
-          tmem_ld_wait();
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(t_lane + O_COL + w * 128 + c * 32, r);
+        tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(orow + c * 32 + e) =
-                make_float4(__uint_as_float(r[e]) * inv_l, __uint_as_float(r[e + 1]) * inv_l,
-                            __uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
-        }
-        if (R == 0) p.part_lse[static_cast<size_t>(slot) * kH + h] = (m_k + log2f(l_k)) * 0.69314718055994531f;
-        tc_fence_before();  // O reads are complete before the next segment's P V overwrites O
-        mbar_arrive(o_free);
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(orow + c * 32 + e) =
+              make_float4(__uint_as_float(r[e]) * inv_l, __uint_as_float(r[e + 1]) * inv_l,
+                          __uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
       }
+      if (R == 0 && w == 0) p.part_lse[static_cast<size_t>(slot) * kH + h] = (m_run + log2f(l_tot)) * 0.69314718055994531f;
+      tc_fence_before();  // O reads are complete before the next segment's P V overwrites O
+      mbar_arrive(o_free);
+      ++seg;
     });
   }
-
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();  // no remote access to this CTA's shared memory is still pending

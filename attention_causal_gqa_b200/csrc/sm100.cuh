@@ -195,6 +195,10 @@ __host__ __device__ constexpr uint32_t sdesc_lo(uint32_t saddr, uint32_t lbo_byt
 __host__ __device__ constexpr uint32_t sdesc_hi_sw128(uint32_t sbo_bytes) {
   return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
 }
+// Same with 64-byte swizzle (layout type 4): K-major rows of 64 bytes, 8-row groups SBO apart.
+__host__ __device__ constexpr uint32_t sdesc_hi_sw64(uint32_t sbo_bytes) {
+  return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (4u << 29);
+}
 
 // Instruction descriptor for kind::f16 / kind::tf32 with an f32 accumulator.
 //   bits 4-5 D format (1 = f32); bits 7-9 A format; bits 10-12 B format

@@ -40,7 +40,10 @@ def _oracle(d, pairs=None, scale=SCALE):
 
 @cuda
 @pytest.mark.parametrize("lens,T_max", [([1, 31, 32, 33], 64), ([600, 1500, 513, 511, 512], 1536),
-                                        ([2048, 100], 2048)])
+                                        ([2048, 100], 2048),
+                                        # 64-token tile edges, half tiles, and a cache length that
+                                        # is not a multiple of the tile (last box read past T_max)
+                                        ([1, 63, 64, 65, 96, 97, 127, 129, 160], 160)])
 def test_mla_matches_oracle_small(lens, T_max):
     from attention_causal_gqa_b200.synthetic import mla_inputs
     d = mla_inputs(len(lens), 128, 512, 64, seq_lens=lens, T_max=T_max, seed=T_max + len(lens), device="cuda")
