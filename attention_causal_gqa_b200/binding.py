@@ -35,7 +35,8 @@ EXPORTED = (
     "attn_decode_paged_fp8_workspace_size", "mla_decode_workspace_size", "mla_decode",
     "dsa_index_topk_workspace_size", "dsa_index_topk", "dsa_mla_decode_workspace_size", "dsa_mla_decode",
     "dsa_mla_decode_fp8",
-    "attn_last_error", "attn_read_status", "attn_selftest_wait_timeout",
+    "attn_last_error", "attn_read_status", "attn_selftest_wait_timeout", "attn_selftest_exp2",
+    "attn_rope_ntk_theta", "attn_rope_length_scaled_theta", "attn_decode_paged_noalloc_status", "attn_lse_merge",
     "attn_profile_enable", "attn_profile_collect",
 )
 
@@ -89,6 +90,14 @@ def _load() -> ctypes.CDLL:
     lib.attn_last_error.argtypes = []
     lib.attn_read_status.restype = i32
     lib.attn_read_status.argtypes = [vp, ctypes.POINTER(i32), vp]
+    lib.attn_lse_merge.restype = i32
+    lib.attn_lse_merge.argtypes = [vp, vp, i32, ctypes.c_longlong, i32, vp, vp, vp]
+    lib.attn_rope_ntk_theta.restype = ctypes.c_double
+    lib.attn_rope_ntk_theta.argtypes = [ctypes.c_double, ctypes.c_double, i32]
+    lib.attn_rope_length_scaled_theta.restype = ctypes.c_double
+    lib.attn_rope_length_scaled_theta.argtypes = [ctypes.c_double, i32, i32, ctypes.c_double]
+    lib.attn_selftest_exp2.restype = i32
+    lib.attn_selftest_exp2.argtypes = [vp, vp, i32, vp]
     lib.attn_selftest_wait_timeout.restype = i32
     lib.attn_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_ulonglong, vp]
     lib.attn_profile_enable.restype = i32
@@ -124,6 +133,18 @@ def _need_cuda(*ts):
             raise ValueError("attn_b200 takes contiguous tensors")
 
 
+def _flags_or_raise(ws, stream, what: str) -> None:
+    """Waits for the stream and raises AttnError when the call's device status word has
+    flags (ATTN_DEV_*): an out-of-range operand, a bad page, a bad length or a timeout
+    means the outputs are not valid."""
+    flags = read_status(ws, stream)
+    if flags:
+        names = [n for bit, n in ((ATTN_DEV_TIMEOUT, "timeout"), (ATTN_DEV_BAD_PAGE, "bad page"),
+                                  (ATTN_DEV_BAD_LENGTH, "bad length"), (ATTN_DEV_RANGE, "fp16 operand range"),
+                                  (ATTN_DEV_BAD_INDEX, "bad index")) if flags & bit]
+        raise AttnError(ATTN_ERR_DEVICE, f"{what}: device status flags {flags:#x} ({', '.join(names)})")
+
+
 def _workspace(nbytes: int, device, workspace):
     if workspace is not None:
         if workspace.numel() * workspace.element_size() < nbytes:
@@ -139,25 +160,38 @@ def prefill_workspace_size(B, Hkv, S, D, dtype=torch.bfloat16) -> int:
 
 
 ROPE_LAYOUTS = {"interleaved": 0, "half": 1}  # ATTN_ROPE_INTERLEAVED, ATTN_ROPE_HALF_SPLIT
+ATTN_ROPE_BF16_OPERANDS = 4
 
 
 def ntk_aware_theta(theta: float, scale: float, head_dim: int) -> float:
-    """NTK-aware RoPE base for a context stretched by `scale` (the long-context page names the
-    method; the rule is the published one): theta * scale^(D / (D - 2)), which divides the
-    lowest rotary frequency by `scale` and leaves the highest unchanged."""
-    return float(theta) * float(scale) ** (head_dim / (head_dim - 2.0))
+    """NTK-aware RoPE base for a context stretched by `scale` (computed by the library:
+    attn_rope_ntk_theta)."""
+    r = float(lib.attn_rope_ntk_theta(float(theta), float(scale), int(head_dim)))
+    if not r > 0.0:
+        raise AttnError(ATTN_ERR_INVALID_ARG, lib.attn_last_error().decode())
+    return r
 
 
 def length_scaled_theta(theta: float, length: int, base_length: int, alpha: float) -> float:
-    """The long-context page's length-aware base (section 2.4): theta * (L / L0)^alpha."""
-    return float(theta) * (float(length) / float(base_length)) ** float(alpha)
+    """Length-aware RoPE base theta * (L / L0)^alpha (computed by the library:
+    attn_rope_length_scaled_theta)."""
+    r = float(lib.attn_rope_length_scaled_theta(float(theta), int(length), int(base_length), float(alpha)))
+    if not r > 0.0:
+        raise AttnError(ATTN_ERR_INVALID_ARG, lib.attn_last_error().decode())
+    return r
 
 
 def attn_prefill(q, k, v, causal=True, rope_theta=10000.0, scale=None, out=None, lse=None, workspace=None,
-                 stream=None, rope_freq_scale=1.0, rope_layout="interleaved"):
+                 stream=None, rope_freq_scale=1.0, rope_layout="interleaved", check=False, bf16_operands=False):
     """Causal GQA prefill with RoPE. q [B,Hq,S,D], k/v [B,Hkv,S,D] (bf16 or fp32).
     rope_freq_scale multiplies every rotary frequency; rope_layout "interleaved" pairs
-    (2i, 2i+1), "half" pairs (i, i + D/2). Returns (out [B,Hq,S,D] same dtype, lse [B,Hq,S] fp32)."""
+    (2i, 2i+1), "half" pairs (i, i + D/2). Returns (out [B,Hq,S,D] same dtype, lse [B,Hq,S] fp32).
+
+    With RoPE on bf16 input the rotated q and k are fp16 tensor-core operands; a rotated
+    value beyond 65504 sets ATTN_DEV_RANGE and makes the result invalid. check=True waits
+    for the call, and when that flag is set re-runs it with bf16 operands
+    (ATTN_ROPE_BF16_OPERANDS, valid for any bf16 input at 8x the operand rounding) before
+    raising on any flag left; bf16_operands=True asks for that form directly."""
     _need_cuda(q, k, v)
     B, Hq, S, D = q.shape
     Hkv = k.shape[1]
@@ -170,16 +204,26 @@ def attn_prefill(q, k, v, causal=True, rope_theta=10000.0, scale=None, out=None,
     ws = _workspace(ws_bytes, q.device, workspace)
     if rope_layout not in ROPE_LAYOUTS:
         raise ValueError(f"rope_layout must be one of {sorted(ROPE_LAYOUTS)}")
-    if float(rope_freq_scale) == 1.0 and rope_layout == "interleaved":
-        rc = lib.attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, S, D, int(bool(causal)),
-                              float(rope_theta if rope_theta else 0.0), float(scale or 0.0), dt, _ptr(ws),
-                              ws.numel() * ws.element_size(), _stream(stream))
-    else:
-        rc = lib.attn_prefill_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, S, D,
-                                 int(bool(causal)), float(rope_theta if rope_theta else 0.0), float(rope_freq_scale),
-                                 ROPE_LAYOUTS[rope_layout], float(scale or 0.0), dt, _ptr(ws),
-                                 ws.numel() * ws.element_size(), _stream(stream))
-    _check(rc)
+
+    def run(bf16_ops):
+        if float(rope_freq_scale) == 1.0 and rope_layout == "interleaved" and not bf16_ops:
+            rc = lib.attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, S, D,
+                                  int(bool(causal)), float(rope_theta if rope_theta else 0.0), float(scale or 0.0), dt,
+                                  _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+        else:
+            layout = ROPE_LAYOUTS[rope_layout] | (ATTN_ROPE_BF16_OPERANDS if bf16_ops else 0)
+            rc = lib.attn_prefill_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, S, D,
+                                     int(bool(causal)), float(rope_theta if rope_theta else 0.0),
+                                     float(rope_freq_scale), layout, float(scale or 0.0), dt, _ptr(ws),
+                                     ws.numel() * ws.element_size(), _stream(stream))
+        _check(rc)
+
+    run(bf16_operands)
+    if check:
+        rope_bf16 = dt == ATTN_DTYPE_BF16 and bool(rope_theta) and rope_theta > 0
+        if rope_bf16 and not bf16_operands and read_status(ws, stream) & ATTN_DEV_RANGE:
+            run(True)
+        _flags_or_raise(ws, stream, "attn_prefill")
     return out, lse
 
 
@@ -193,7 +237,7 @@ def decode_fp8_workspace_size(B, Hq, D, max_pages_per_seq, page_size=16) -> int:
 
 
 def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale=None, out=None, lse=None, workspace=None,
-                      stream=None):
+                      stream=None, check=False):
     """Paged GQA decode. q [B,Hq,D] bf16, k/v_pages [P,16,Hkv,D] bf16, block_table [B,maxp] int32,
     seq_lens [B] int32. Returns (out [B,Hq,D] bf16, lse [B,Hq] fp32)."""
     _need_cuda(q, k_pages, v_pages, block_table, seq_lens)
@@ -209,11 +253,13 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale=None, ou
                                _ptr(lse), B, Hq, Hkv, D, ps, maxp, P, float(scale or 0.0), ATTN_DTYPE_BF16, _ptr(ws),
                                ws.numel() * ws.element_size(), _stream(stream))
     _check(rc)
+    if check:  # waits; raises on a bad page, a length beyond the table or a timeout
+        _flags_or_raise(ws, stream, "attn_decode_paged")
     return out, lse
 
 
 def attn_decode_paged_fp8(q, k_pages, v_pages, k_scale, v_scale, block_table, seq_lens, scale=None, out=None, lse=None,
-                          workspace=None, stream=None):
+                          workspace=None, stream=None, check=False):
     """Paged GQA decode over an FP8 E4M3 cache. q [B,Hq,D] bf16; k/v_pages [P,16,Hkv,D] uint8 codes;
     k/v_scale [P,Hkv] fp32; block_table [B,maxp] int32; seq_lens [B] int32.
     Returns (out [B,Hq,D] bf16, lse [B,Hq] fp32)."""
@@ -230,6 +276,8 @@ def attn_decode_paged_fp8(q, k_pages, v_pages, k_scale, v_scale, block_table, se
                                    _ptr(block_table), _ptr(seq_lens), _ptr(out), _ptr(lse), B, Hq, Hkv, D, ps, maxp,
                                    P, float(scale or 0.0), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
     _check(rc)
+    if check:  # waits; raises when q left the fp16 range (ATTN_DEV_RANGE) or on any other flag
+        _flags_or_raise(ws, stream, "attn_decode_paged_fp8")
     return out, lse
 
 
@@ -240,7 +288,7 @@ def prefill_chunk_workspace_size(B, Hkv, S_new, max_cache_len, D) -> int:
 
 def attn_prefill_chunk(q, k, v, k_pages, v_pages, block_table, cache_lens, max_cache_len, rope_theta=10000.0,
                        scale=None, out=None, lse=None, workspace=None, stream=None, rope_freq_scale=1.0,
-                       rope_layout="interleaved"):
+                       rope_layout="interleaved", check=False):
     """Append a chunk of new tokens to the paged KV cache and attend over the whole cache.
     q [B,Hq,S_new,D], k/v [B,Hkv,S_new,D] bf16 (not rotated); k/v_pages [P,16,Hkv,D] bf16, updated in
     place; block_table [B,maxp] int32; cache_lens [B] int32 (tokens already cached, each <= max_cache_len).
@@ -269,6 +317,8 @@ def attn_prefill_chunk(q, k, v, k_pages, v_pages, block_table, cache_lens, max_c
                                        float(rope_freq_scale), ROPE_LAYOUTS[rope_layout], float(scale or 0.0),
                                        _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
     _check(rc)
+    if check:  # waits; raises when a rotated query or a cached key left the fp16 range, or on any other flag
+        _flags_or_raise(ws, stream, "attn_prefill_chunk")
     return out, lse
 
 
@@ -278,7 +328,7 @@ def mla_workspace_size(B, H, Dc, Dr, T_max) -> int:
 
 
 def mla_decode(q_nope, q_pe, kv_cache, pe_cache, seq_lens, scale, out=None, lse=None, workspace=None,
-               stream=None):
+               stream=None, check=False):
     """MLA absorbed decode. q_nope [B,1,H,Dc], q_pe [B,1,H,Dr], kv_cache [B,T,Dc], pe_cache [B,T,Dr] (bf16),
     seq_lens [B] int32. Returns (out [B,1,H,Dc] bf16, lse [B,1,H] fp32)."""
     _need_cuda(q_nope, q_pe, kv_cache, pe_cache, seq_lens)
@@ -296,6 +346,25 @@ def mla_decode(q_nope, q_pe, kv_cache, pe_cache, seq_lens, scale, out=None, lse=
                         _ptr(out), _ptr(lse), B, H, Dc, Dr, T, _ptr(ws), ws.numel() * ws.element_size(),
                         _stream(stream))
     _check(rc)
+    if check:  # waits; raises on a timeout flag
+        _flags_or_raise(ws, stream, "mla_decode")
+    return out, lse
+
+
+def lse_merge(o_parts, lse_parts, out=None, lse=None, stream=None):
+    """Combines partial results over disjoint key sets (e.g. gathered from the ranks of a
+    sequence-parallel decode). o_parts [n, ..., D] bf16, lse_parts [n, ...] fp32 (same
+    leading shape). Returns (out [..., D] bf16, lse [...] fp32)."""
+    _need_cuda(o_parts, lse_parts)
+    n, D = o_parts.shape[0], o_parts.shape[-1]
+    if tuple(lse_parts.shape) != tuple(o_parts.shape[:-1]) or o_parts.dtype != torch.bfloat16:
+        raise ValueError("o_parts [n, ..., D] bf16 and lse_parts [n, ...] fp32 with matching shapes")
+    rows = lse_parts[0].numel()
+    if out is None:
+        out = torch.empty(o_parts.shape[1:], dtype=torch.bfloat16, device=o_parts.device)
+    if lse is None:
+        lse = torch.empty(lse_parts.shape[1:], dtype=torch.float32, device=o_parts.device)
+    _check(lib.attn_lse_merge(_ptr(o_parts), _ptr(lse_parts), n, rows, D, _ptr(out), _ptr(lse), _stream(stream)))
     return out, lse
 
 
@@ -374,6 +443,14 @@ def read_status(workspace, stream=None) -> int:
     if rc not in (ATTN_OK, ATTN_ERR_DEVICE):
         _check(rc)
     return flags.value
+
+
+def selftest_exp2(z: torch.Tensor, stream=None) -> torch.Tensor:
+    """2^z as the prefill softmax's FMA-pipe exponential computes it (z: CUDA fp32)."""
+    assert z.is_cuda and z.dtype == torch.float32 and z.is_contiguous()
+    y = torch.empty_like(z)
+    _check(lib.attn_selftest_exp2(_ptr(z), _ptr(y), z.numel(), _stream(stream)))
+    return y
 
 
 def selftest_wait_timeout(timeout_ns: int, workspace=None, stream=None) -> int:

@@ -129,6 +129,16 @@ __global__ void selftest_wait_kernel(int* status, unsigned long long timeout_ns)
   }
   __syncthreads();
 }
+// Evaluates the FMA-pipe exp2 of the softmax (exp2_fma2, sm100.cuh) on a caller buffer,
+// two arguments per thread as the kernels use it.
+__global__ void selftest_exp2_kernel(const float* __restrict__ z, float* __restrict__ y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float2 in = make_float2(z[i], i + 1 < n ? z[i + 1] : 0.f);
+  const float2 r = exp2_fma2(in);
+  y[i] = r.x;
+  if (i + 1 < n) y[i + 1] = r.y;
+}
 }  // namespace attn
 
 extern "C" {
@@ -154,6 +164,8 @@ int attn_prefill_ex(const void* q, const void* k, const void* v, void* out, floa
     return fail(ATTN_ERR_INVALID_ARG, "sizes must be positive (B=%d Hq=%d Hkv=%d S=%d D=%d)", B, Hq, Hkv, S, D);
   if (Hq % Hkv != 0) return fail(ATTN_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
   if (dtype != ATTN_DTYPE_BF16 && dtype != ATTN_DTYPE_F32) return fail(ATTN_ERR_UNSUPPORTED, "dtype %d", dtype);
+  const bool bf16_ops = (rope_layout & ATTN_ROPE_BF16_OPERANDS) != 0;
+  rope_layout &= ~ATTN_ROPE_BF16_OPERANDS;
   if (rope_layout != ATTN_ROPE_INTERLEAVED && rope_layout != ATTN_ROPE_HALF_SPLIT)
     return fail(ATTN_ERR_INVALID_ARG, "rope_layout %d", rope_layout);
   if (!(rope_freq_scale > 0.f) || !std::isfinite(rope_freq_scale))
@@ -203,10 +215,10 @@ int attn_prefill_ex(const void* q, const void* k, const void* v, void* out, floa
     vbase = vop;
     zdim *= 2;
   } else if (rope) {
-    cudaError_t e = attn::launch_rope_k_f16(k, kop, cs, rows, S, D, half_split, status, st);
+    cudaError_t e = attn::launch_rope_k_f16(k, kop, cs, rows, S, D, half_split, status, st, bf16_ops);
     if (e != cudaSuccess) return cuda_fail(e, "rope K launch");
     kbase = kop;
-    kdt = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    kdt = bf16_ops ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   }
   // Q operand. Without RoPE, bf16 Q is the operand itself. Otherwise the prologue
   // writes it into `out`, whose size is exactly that of the operand (rotated fp16 Q
@@ -223,10 +235,10 @@ int attn_prefill_ex(const void* q, const void* k, const void* v, void* out, floa
     qbase = out;
     zq *= 2;
   } else if (rope) {
-    cudaError_t e = attn::launch_rope_k_f16(q, out, cs, rows_q, S, D, half_split, status, st);
+    cudaError_t e = attn::launch_rope_k_f16(q, out, cs, rows_q, S, D, half_split, status, st, bf16_ops);
     if (e != cudaSuccess) return cuda_fail(e, "rope Q launch");
     qbase = out;
-    qdt = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    qdt = bf16_ops ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   }
   const int BN = attn::prefill_block_n(D, f32);
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S), zdim};
@@ -261,7 +273,8 @@ int attn_prefill_ex(const void* q, const void* k, const void* v, void* out, floa
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long grid = items < sms ? items : sms;  // one persistent CTA per SM
   prof_before(st);
-  cudaError_t e = attn::launch_prefill(p, tmQ, tmK, tmV, D, f32, rope, static_cast<int>(grid), st);
+  // rotated operands in fp16 select the f16 Q.K^T form of the kernel; bf16 ones the plain form
+  cudaError_t e = attn::launch_prefill(p, tmQ, tmK, tmV, D, f32, rope && !bf16_ops, static_cast<int>(grid), st);
   prof_after(st);
   if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
   return ok();
@@ -790,6 +803,62 @@ int attn_read_status(const void* workspace, int* flags, void* stream) {
   if (e != cudaSuccess) return cuda_fail(e, "status copy");
   *flags = v;
   if (v) return fail(ATTN_ERR_DEVICE, "device status flags 0x%x", v);
+  return ok();
+}
+
+int attn_lse_merge(const void* o_parts, const float* lse_parts, int n_parts, long long rows, int D, void* out,
+                   float* lse, void* stream) {
+  if (!o_parts || !lse_parts || !out || !lse) return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
+  if (n_parts < 1 || n_parts > (1 << 16) || rows < 1 || rows > (1LL << 36))
+    return fail(ATTN_ERR_INVALID_ARG, "n_parts (%d) or rows (%lld) out of range", n_parts, rows);
+  if (D != 64 && D != 128 && D != 256 && D != 512)
+    return fail(ATTN_ERR_UNSUPPORTED, "head dim %d (64, 128, 256 or 512)", D);
+  if (!aligned(o_parts, 4) || !aligned(out, 4) || !aligned(lse_parts, 4) || !aligned(lse, 4))
+    return fail(ATTN_ERR_INVALID_ARG, "misaligned pointer (4 bytes)");
+  cudaError_t e =
+      attn::launch_parts_merge(o_parts, lse_parts, n_parts, rows, D, out, lse, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  return ok();
+}
+
+double attn_rope_ntk_theta(double theta, double scale, int head_dim) {
+  if (!(theta > 0.0) || !std::isfinite(theta) || !(scale >= 1.0) || !std::isfinite(scale) || head_dim < 4 ||
+      head_dim % 2 != 0) {
+    fail(ATTN_ERR_INVALID_ARG, "attn_rope_ntk_theta: theta > 0, scale >= 1 and an even head_dim >= 4 are required");
+    return 0.0;
+  }
+  // the lowest rotary frequency theta^(-(D-2)/D) divided by `scale`, the highest (pair 0) unchanged
+  const double r = theta * std::pow(scale, static_cast<double>(head_dim) / (head_dim - 2.0));
+  if (!std::isfinite(r)) {
+    fail(ATTN_ERR_INVALID_ARG, "attn_rope_ntk_theta: result overflows");
+    return 0.0;
+  }
+  ok();
+  return r;
+}
+
+double attn_rope_length_scaled_theta(double theta, int length, int base_length, double alpha) {
+  if (!(theta > 0.0) || !std::isfinite(theta) || length <= 0 || base_length <= 0 || !std::isfinite(alpha)) {
+    fail(ATTN_ERR_INVALID_ARG,
+         "attn_rope_length_scaled_theta: theta > 0, positive lengths and a finite alpha are required");
+    return 0.0;
+  }
+  const double r = theta * std::pow(static_cast<double>(length) / base_length, alpha);
+  if (!(r > 0.0) || !std::isfinite(r)) {
+    fail(ATTN_ERR_INVALID_ARG, "attn_rope_length_scaled_theta: result out of range");
+    return 0.0;
+  }
+  ok();
+  return r;
+}
+
+int attn_selftest_exp2(const float* z, float* y, int n, void* stream) {
+  if (!z || !y) return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
+  if (n <= 0 || n > (1 << 30)) return fail(ATTN_ERR_INVALID_ARG, "n must be within 1 .. 2^30");
+  const int pairs = (n + 1) / 2;
+  attn::selftest_exp2_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(z, y, n);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "selftest launch");
   return ok();
 }
 

@@ -82,4 +82,9 @@ cudaError_t launch_mla_merge(const float* part_o, const float* part_lse, const i
 cudaError_t launch_merge(const float* part_o, const float* part_lse, const int32_t* seq_lens, void* out, float* lse,
                          int B, int H, int D, int n_splits, int tokens_per_split, cudaStream_t stream);
 
+// Merges n_parts bf16 partial outputs [n_parts, rows, D] with fp32 LSEs [n_parts, rows]
+// over disjoint key sets into out [rows, D] bf16 and lse [rows] (D in {64, 128, 256, 512}).
+cudaError_t launch_parts_merge(const void* o_parts, const float* lse_parts, int n_parts, long long rows, int D,
+                               void* out, float* lse, cudaStream_t stream);
+
 }  // namespace attn

@@ -94,6 +94,70 @@ cudaError_t launch_merge(const float* part_o, const float* part_lse, const int32
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------ parts merge
+// Partial results of the same query rows over disjoint key sets, one per part (the
+// slices of every sequence's cache that different GPUs hold): bf16 outputs
+// [n_parts, rows, D] and fp32 LSEs [n_parts, rows], combined in part order. One warp
+// per row; lane l owns the column pairs 2l + 64 i.
+template <int D>
+__global__ void parts_merge_kernel(const __nv_bfloat16* __restrict__ o_parts, const float* __restrict__ lse_parts,
+                                   int n_parts, long long rows, __nv_bfloat16* __restrict__ out,
+                                   float* __restrict__ lse) {
+  constexpr int NP = D / 64;  // column pairs per lane
+  const long long r = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  float M = -INFINITY;
+  for (int s = lane; s < n_parts; s += 32) M = fmaxf(M, lse_parts[static_cast<size_t>(s) * rows + r]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  __nv_bfloat162* orow = reinterpret_cast<__nv_bfloat162*>(out + r * D);
+  if (!(M > -INFINITY)) {  // every part empty: no key at all
+#pragma unroll
+    for (int i = 0; i < NP; ++i) orow[lane + 32 * i] = __floats2bfloat162_rn(0.f, 0.f);
+    if (lane == 0) lse[r] = -INFINITY;
+    return;
+  }
+  float2 acc[NP];
+#pragma unroll
+  for (int i = 0; i < NP; ++i) acc[i] = make_float2(0.f, 0.f);
+  float wsum = 0.f;
+  for (int s = 0; s < n_parts; ++s) {
+    const float ls = lse_parts[static_cast<size_t>(s) * rows + r];
+    if (!(ls > -INFINITY)) continue;  // an empty part carries no weight (its output is not read)
+    const float w = __expf(ls - M);
+    wsum += w;
+    const __nv_bfloat162* po = reinterpret_cast<const __nv_bfloat162*>(o_parts + (static_cast<size_t>(s) * rows + r) * D);
+#pragma unroll
+    for (int i = 0; i < NP; ++i) {
+      const float2 v = __bfloat1622float2(po[lane + 32 * i]);
+      acc[i].x += w * v.x;
+      acc[i].y += w * v.y;
+    }
+  }
+  const float inv = 1.f / wsum;
+#pragma unroll
+  for (int i = 0; i < NP; ++i) orow[lane + 32 * i] = __floats2bfloat162_rn(acc[i].x * inv, acc[i].y * inv);
+  if (lane == 0) lse[r] = M + logf(wsum);
+}
+
+cudaError_t launch_parts_merge(const void* o_parts, const float* lse_parts, int n_parts, long long rows, int D,
+                               void* out, float* lse, cudaStream_t stream) {
+  const int threads = 256;
+  const long long blocks = (rows * 32 + threads - 1) / threads;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const auto* op = static_cast<const __nv_bfloat16*>(o_parts);
+  auto* o = static_cast<__nv_bfloat16*>(out);
+  switch (D) {
+    case 64: parts_merge_kernel<64><<<static_cast<int>(blocks), threads, 0, stream>>>(op, lse_parts, n_parts, rows, o, lse); break;
+    case 128: parts_merge_kernel<128><<<static_cast<int>(blocks), threads, 0, stream>>>(op, lse_parts, n_parts, rows, o, lse); break;
+    case 256: parts_merge_kernel<256><<<static_cast<int>(blocks), threads, 0, stream>>>(op, lse_parts, n_parts, rows, o, lse); break;
+    case 512: parts_merge_kernel<512><<<static_cast<int>(blocks), threads, 0, stream>>>(op, lse_parts, n_parts, rows, o, lse); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------ range merge
 template <int UNIT>
 __device__ __forceinline__ int units_of(const int32_t* lens, int b, int T_max) {

@@ -5,8 +5,9 @@
 // allocation disabled, real-time paths where cudaMalloc's implicit device-wide
 // synchronisation is not allowed, or embedders that only hand over buffers they
 // own. For them the split partials and the status word live in one file-scope
-// device array of fixed size, created when the library is loaded and kept by
-// every GPU that loads it until the process exits.
+// device array of fixed size, kept by every GPU that loads the library until the
+// process exits. With CUDA's lazy module loading the array is reserved when this
+// file's device code is first loaded on a device, i.e. by the first call here.
 #include <cstdio>
 #include <mutex>
 #include <string>
@@ -31,6 +32,34 @@ namespace attn {
 void set_last_error(const char* msg);  // api.cu
 }
 
+namespace {
+
+// Device address of the array on the current device, looked up once per device with
+// that device current (the array's name is only a host-side handle).
+int scratch_for_current_device(void** out, const char* who) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    char buf[160];
+    snprintf(buf, sizeof(buf), "%s: no usable current device", who);
+    attn::set_last_error(buf);
+    return ATTN_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_scratch_ptr[dev]) {
+    if (cudaGetSymbolAddress(&g_scratch_ptr[dev], g_decode_scratch) != cudaSuccess) {
+      g_scratch_ptr[dev] = nullptr;
+      char buf[160];
+      snprintf(buf, sizeof(buf), "%s: cudaGetSymbolAddress failed", who);
+      attn::set_last_error(buf);
+      return ATTN_ERR_CUDA;
+    }
+  }
+  *out = g_scratch_ptr[dev];
+  return ATTN_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 int attn_decode_paged_noalloc(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
@@ -47,30 +76,25 @@ int attn_decode_paged_noalloc(const void* q, const void* k_pages, const void* v_
     attn::set_last_error(buf);
     return ATTN_ERR_WORKSPACE;
   }
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-    attn::set_last_error("attn_decode_paged_noalloc: no usable current device");
-    return ATTN_ERR_CUDA;
-  }
   void* ptr = nullptr;
-  {
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_ptr[dev]) {
-      // The array's name is only a host-side handle: its device address comes from
-      // the runtime, once per device, with that device current.
-      if (cudaGetSymbolAddress(&g_scratch_ptr[dev], g_decode_scratch) != cudaSuccess) {
-        g_scratch_ptr[dev] = nullptr;
-        attn::set_last_error("attn_decode_paged_noalloc: cudaGetSymbolAddress failed");
-        return ATTN_ERR_CUDA;
-      }
-    }
-    ptr = g_scratch_ptr[dev];
-  }
+  const int rc = scratch_for_current_device(&ptr, "attn_decode_paged_noalloc");
+  if (rc != ATTN_OK) return rc;
   // The existing entry point clears the status word at the start of the scratch;
   // the split partials are fully written before they are read, so nothing else
   // needs to start at zero.
   return attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, out, lse, B, Hq, Hkv, D, page_size,
                            max_pages_per_seq, num_pages, scale, dtype, ptr, kScratchBytes, stream);
+}
+
+int attn_decode_paged_noalloc_status(int* flags, void* stream) {
+  if (!flags) {
+    attn::set_last_error("attn_decode_paged_noalloc_status: null pointer argument");
+    return ATTN_ERR_INVALID_ARG;
+  }
+  void* ptr = nullptr;
+  const int rc = scratch_for_current_device(&ptr, "attn_decode_paged_noalloc_status");
+  if (rc != ATTN_OK) return rc;
+  return attn_read_status(ptr, flags, stream);
 }
 
 }  // extern "C"

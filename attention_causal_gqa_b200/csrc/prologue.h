@@ -14,7 +14,8 @@ cudaError_t launch_rope_table(float2* cs, int S, int D, double theta, double fre
 // bf16 X [rows, D] -> rotated fp16 X (row r at position r % S); flags values outside fp16 range.
 // Used for K and for Q.
 cudaError_t launch_rope_k_f16(const void* k, void* k_f16, const float2* cs, long long rows, int S, int D,
-                              bool half_split, int* status, cudaStream_t stream);
+                              bool half_split, int* status, cudaStream_t stream,
+                              bool bf16_out = false);
 // fp32 X [rows, D] -> bf16 hi parts at out[0, rows) and lo parts at out[rows, 2 rows), rotating
 // first when cs is non-null.
 cudaError_t launch_split_f32(const float* x, void* out, const float2* cs, long long rows, int S, int D,

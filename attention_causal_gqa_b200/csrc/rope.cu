@@ -59,9 +59,22 @@ __device__ __forceinline__ void load_cs4(const float2* __restrict__ cs, int pos,
   a[3] = make_float2(t1.z, t1.w);
 }
 
-// bf16 X [heads, S, D] -> rotated fp16 X (used for K and for Q). Values beyond
-// the fp16 range set the range flag of the status word.
-template <int CPR>
+// Two 16-bit values of a rotated operand: fp16 (flags values beyond its range) or bf16.
+template <bool BF16>
+__device__ __forceinline__ uint32_t pack_operand(float a, float b, bool& in_range) {
+  if (BF16) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&v);
+  }
+  in_range = in_range && fabsf(a) <= 65504.f && fabsf(b) <= 65504.f;
+  const __half2 v = __floats2half2_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// bf16 X [heads, S, D] -> rotated fp16 X (used for K and for Q), or rotated bf16 X for
+// inputs beyond the fp16 range (BF16). fp16 values beyond its range set the range flag
+// of the status word.
+template <int CPR, bool BF16>
 __global__ void __launch_bounds__(256) rope_f16_kernel(const uint4* __restrict__ x, uint4* __restrict__ y,
                                                        const float2* __restrict__ cs, int heads, int S,
                                                        int* __restrict__ status) {
@@ -80,9 +93,7 @@ __global__ void __launch_bounds__(256) rope_f16_kernel(const uint4* __restrict__
       const float x0 = __uint_as_float(w[e] << 16);
       const float x1 = __uint_as_float(w[e] & 0xFFFF0000u);
       const float y0 = x0 * a[e].x - x1 * a[e].y, y1 = x0 * a[e].y + x1 * a[e].x;
-      in_range = in_range && fabsf(y0) <= 65504.f && fabsf(y1) <= 65504.f;
-      const __half2 v = __floats2half2_rn(y0, y1);
-      ow[e] = *reinterpret_cast<const uint32_t*>(&v);
+      ow[e] = pack_operand<BF16>(y0, y1, in_range);
     }
     y[idx] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
   }
@@ -103,7 +114,7 @@ __device__ __forceinline__ void load_cs8(const float2* __restrict__ cs, int pos,
 
 // Half-split layout of rope_f16_kernel: the thread of chunk c < CPR/2 rotates it together
 // with its partner chunk c + CPR/2 (element d pairs with d + D/2); the others have no work.
-template <int CPR>
+template <int CPR, bool BF16>
 __global__ void __launch_bounds__(256) rope_f16_half_kernel(const uint4* __restrict__ x, uint4* __restrict__ y,
                                                             const float2* __restrict__ cs, int heads, int S,
                                                             int* __restrict__ status) {
@@ -127,11 +138,9 @@ __global__ void __launch_bounds__(256) rope_f16_half_kernel(const uint4* __restr
         const float2 cz = a[2 * e + k];
         yl[k] = lo[k] * cz.x - hi[k] * cz.y;
         yh[k] = lo[k] * cz.y + hi[k] * cz.x;
-        in_range = in_range && fabsf(yl[k]) <= 65504.f && fabsf(yh[k]) <= 65504.f;
       }
-      const __half2 vl = __floats2half2_rn(yl[0], yl[1]), vh = __floats2half2_rn(yh[0], yh[1]);
-      ol[e] = *reinterpret_cast<const uint32_t*>(&vl);
-      oh[e] = *reinterpret_cast<const uint32_t*>(&vh);
+      ol[e] = pack_operand<BF16>(yl[0], yl[1], in_range);
+      oh[e] = pack_operand<BF16>(yh[0], yh[1], in_range);
     }
     y[idx] = make_uint4(ol[0], ol[1], ol[2], ol[3]);
     y[idx + CPR / 2] = make_uint4(oh[0], oh[1], oh[2], oh[3]);
@@ -237,18 +246,26 @@ cudaError_t launch_rope_table(float2* cs, int S, int D, double theta, double fre
 }
 
 cudaError_t launch_rope_k_f16(const void* k, void* k_f16, const float2* cs, long long rows, int S, int D,
-                              bool half_split, int* status, cudaStream_t stream) {
+                              bool half_split, int* status, cudaStream_t stream, bool bf16_out) {
   const long long heads = rows / S;
   if (heads * S != rows || heads > 0x7fffffffLL) return cudaErrorInvalidValue;
   const dim3 grid = operand_grid(static_cast<int>(heads), S, D / 8);
   const uint4* x = static_cast<const uint4*>(k);
   uint4* y = static_cast<uint4*>(k_f16);
   const int h = static_cast<int>(heads);
-  if (D == 128 && half_split) rope_f16_half_kernel<16><<<grid, 256, 0, stream>>>(x, y, cs, h, S, status);
-  else if (D == 128) rope_f16_kernel<16><<<grid, 256, 0, stream>>>(x, y, cs, h, S, status);
-  else if (D == 64 && half_split) rope_f16_half_kernel<8><<<grid, 256, 0, stream>>>(x, y, cs, h, S, status);
-  else if (D == 64) rope_f16_kernel<8><<<grid, 256, 0, stream>>>(x, y, cs, h, S, status);
-  else return cudaErrorInvalidValue;
+  if (bf16_out) {
+    if (D == 128 && half_split) rope_f16_half_kernel<16, true><<<grid, 256, 0, stream>>>(x, y, cs, h, S, status);
+    else if (D == 128) rope_f16_kernel<16, true><<<grid, 256, 0, stream>>>(x, y, cs, h, S, status);
+    else if (D == 64 && half_split) rope_f16_half_kernel<8, true><<<grid, 256, 0, stream>>>(x, y, cs, h, S, status);
+    else if (D == 64) rope_f16_kernel<8, true><<<grid, 256, 0, stream>>>(x, y, cs, h, S, status);
+    else return cudaErrorInvalidValue;
+  } else {
+    if (D == 128 && half_split) rope_f16_half_kernel<16, false><<<grid, 256, 0, stream>>>(x, y, cs, h, S, status);
+    else if (D == 128) rope_f16_kernel<16, false><<<grid, 256, 0, stream>>>(x, y, cs, h, S, status);
+    else if (D == 64 && half_split) rope_f16_half_kernel<8, false><<<grid, 256, 0, stream>>>(x, y, cs, h, S, status);
+    else if (D == 64) rope_f16_kernel<8, false><<<grid, 256, 0, stream>>>(x, y, cs, h, S, status);
+    else return cudaErrorInvalidValue;
+  }
   return cudaGetLastError();
 }
 

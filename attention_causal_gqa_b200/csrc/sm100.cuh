@@ -288,8 +288,9 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
 // in [-1/2, 1/2], 2^f from a degree-3 polynomial, 2^n added to the exponent field.
 // The coefficients are a minimax fit of 2^f on [-1/2, 1/2] in relative error made
 // for this library by a Remez exchange (maximum relative error 7.5e-5, 25x below
-// the bf16 rounding that P receives). z is clamped below at -126 (result tiny but
-// finite); z must stay below 128.
+// the bf16 rounding that P receives) for z >= -125.5, where the result is a normal
+// float. Just above -126 the result can be subnormal (absolute error below
+// 2^-126 * 2e-4); z is clamped below at -126; z must stay below 128.
 __device__ __forceinline__ float2 exp2_fma2(float2 z) {
   z.x = fmaxf(z.x, -126.f);
   z.y = fmaxf(z.y, -126.f);

@@ -207,6 +207,78 @@ def oracle_prefill_sample(q, k, v, p, budget_s):
     return flops / dt / 1e12, heads, dt
 
 
+def oracle_prefill_rows(q, k, v, p, budget_s):
+    """Times the float64 oracle on the last query rows of head 0 of the workload (the rows
+    that see the most keys), 32 rows per call, until ~budget_s elapsed."""
+    from oracle import prefill_ref
+    qn, kn, vn = (x[0:1, 0:1].float().cpu().numpy() for x in (q, k, v))
+    S, D = p["S"], p["D"]
+    flops, rows, hi, t0 = 0.0, 0, S, time.perf_counter()
+    while hi > 0 and time.perf_counter() - t0 < budget_s:
+        chunk = list(range(max(0, hi - 32), hi))
+        prefill_ref(qn, kn, vn, causal=True, rope_theta=p["theta"], scale=p["scale"],
+                    rows=[(0, 0, i) for i in chunk])
+        flops += sum(4.0 * D * (i + 1) for i in chunk)
+        rows += len(chunk)
+        hi -= 32
+    dt = time.perf_counter() - t0
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"the last {rows} query rows of head (0, 0) ({rows} of {S} rows, each against all "
+                      f"earlier keys), float64, {dt:.1f} s"}
+
+
+def oracle_decode_seqs(d, dp, budget_s):
+    """Times the float64 paged-decode oracle on whole sequences (all Hq heads), one at a
+    time in order, until ~budget_s of oracle time; the pages a sequence uses are copied to
+    the host first (outside the timed part)."""
+    import numpy as np
+    import torch
+    from oracle import decode_paged_ref
+    lens = d["seq_lens"].cpu().tolist()
+    dt, nbytes, nseq = 0.0, 0, 0
+    for b, L in enumerate(lens):
+        if dt > budget_s:
+            break
+        n = (L + 15) // 16
+        pages = d["block_table"][b, :n].long()
+        kp = d["k_pages"][pages].float().cpu().numpy()
+        vp = d["v_pages"][pages].float().cpu().numpy()
+        qb = d["q"][b:b + 1].float().cpu().numpy()
+        t0 = time.perf_counter()
+        decode_paged_ref(qb, kp, vp, np.arange(n, dtype=np.int64)[None, :], [L], dp["scale"])
+        dt += time.perf_counter() - t0
+        nbytes += L * dp["Hkv"] * dp["D"] * 2 * 2
+        nseq += 1
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{nseq} whole sequences of {len(lens)} ({sum(lens[:nseq])} cached tokens, all heads), "
+                      f"float64, {dt:.2f} s of oracle time"}
+
+
+def oracle_mla_seqs(m, mp, budget_s):
+    """Times the float64 MLA oracle on whole sequences (all heads) until ~budget_s."""
+    from oracle import mla_decode_ref
+    lens = m["seq_lens"].cpu().tolist()
+    dt, nbytes, nseq = 0.0, 0, 0
+    for b, L in enumerate(lens):
+        if dt > budget_s:
+            break
+        kv = m["kv_cache"][b:b + 1, :L].float().cpu().numpy()
+        pe = m["pe_cache"][b:b + 1, :L].float().cpu().numpy()
+        qn, qp = m["q_nope"][b:b + 1].float().cpu().numpy(), m["q_pe"][b:b + 1].float().cpu().numpy()
+        t0 = time.perf_counter()
+        mla_decode_ref(qn, qp, kv, pe, [L], mp["scale"])
+        dt += time.perf_counter() - t0
+        nbytes += L * (mp["Dc"] + mp["Dr"]) * 2
+        nseq += 1
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{nseq} whole sequences of {len(lens)} ({sum(lens[:nseq])} cached tokens, all 128 heads), "
+                      f"float64, {dt:.2f} s of oracle time"}
+
+
+def want_cpu(args, world, rank):
+    return rank == 0 and world == 1 and not args.no_cpu_baseline
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -388,6 +460,8 @@ def bench_decode(args, world, dev, seed, pk, pk_kind, fp):
                         "frac": ach / pk["hbm_gbs"], "traffic": traffic_for("decode_kernel"),
                         "kernel": "decode_kernel", "kernel_ms": k_avg, "peak_kind": f"{pk_kind} HBM copy",
                         "algorithmic": "4096 B per cached token (K+V, 8 heads x 128 x bf16)"}}
+    if want_cpu(args, world, int(os.environ.get("RANK", "0"))):
+        res["cpu_baseline"] = oracle_decode_seqs(d, dp, args.cpu_budget * 0.75)
     del d, out, lse, ws
     torch.cuda.empty_cache()
     return res
@@ -477,6 +551,8 @@ def bench_mla(args, world, dev, seed, pk, pk_kind, fp):
                         "algorithmic": "1152 B per cached token (kv 512 + pe 64, bf16)",
                         "tensor_tflops": flops / (k_avg * 1e-3) / 1e12,
                         "tensor_frac": flops / (k_avg * 1e-3) / 1e12 / pk["bf16_tflops"]}}
+    if want_cpu(args, world, int(os.environ.get("RANK", "0"))):
+        res["cpu_baseline"] = oracle_mla_seqs(m, mp, args.cpu_budget * 0.75)
     del m, out, lse, ws
     torch.cuda.empty_cache()
     return res
@@ -591,6 +667,8 @@ def run_ours(args):
         sub["prefill_long"] = {"workload": PREFILL_LONG, "value": lp["value"], "unit": "TFLOP/s",
                                "ms_per_step": lp["ms"] / args.steps, "roofline": lp["roofline"],
                                "gpu_launches": 4 * args.steps}
+        if want_cpu(args, world, rank):
+            sub["prefill_long"]["cpu_baseline"] = oracle_prefill_rows(*lp["inputs"], lp["p"], args.cpu_budget * 0.75)
         del lp
     if do("prefill") and not args.small:
         sub["prefill_chunk"] = bench_chunk(args, world, dev, seed, pk, pk_kind)
@@ -632,6 +710,20 @@ def run_ours(args):
     line["clocks"] = clk
     line["source_fingerprint"] = fp
     line.update(sub)
+    # one compact entry per workload, last in the line: rate, kernel time, roofline fraction
+    # and the oracle's rate on the host cores where it was measured
+    summ = {}
+    if pre is not None:
+        summ["prefill"] = {"value": round(pre["value"], 2), "unit": "TFLOP/s",
+                           "kernel_ms": round(pre["roofline"]["kernel_ms"], 4),
+                           "frac": round(pre["roofline"]["frac"], 3),
+                           "cpu": round(cpu["value"], 5) if cpu else None}
+    for name, w in sub.items():
+        cb = w.get("cpu_baseline")
+        summ[name] = {"value": round(w["value"], 2), "unit": w["unit"],
+                      "kernel_ms": round(w["roofline"]["kernel_ms"], 4), "frac": round(w["roofline"]["frac"], 3),
+                      "cpu": round(cb["value"], 5) if cb else None}
+    line["summary"] = summ
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -42,6 +42,9 @@ enum { ATTN_DTYPE_F32 = 0, ATTN_DTYPE_BF16 = 1 };
 
 /* RoPE pair layouts (attn_prefill_ex). */
 enum { ATTN_ROPE_INTERLEAVED = 0, ATTN_ROPE_HALF_SPLIT = 1 };
+/* OR-ed into attn_prefill_ex's rope_layout: rotated q and k become bf16 operands instead
+ * of fp16 (for bf16 inputs whose rotated values exceed the fp16 range). */
+enum { ATTN_ROPE_BF16_OPERANDS = 4 };
 
 /* Device status flags (attn_read_status). */
 enum { ATTN_DEV_TIMEOUT = 1, ATTN_DEV_BAD_PAGE = 2, ATTN_DEV_BAD_LENGTH = 4, ATTN_DEV_RANGE = 8, ATTN_DEV_BAD_INDEX = 16 };
@@ -86,7 +89,11 @@ int attn_prefill(const void* q, const void* k, const void* v, void* out, float* 
  *   rope_freq_scale  f > 0: the angle of pair i at position p is p * f * rope_theta^(-2i/D)
  *                    (1 = plain RoPE; 1/s interpolates positions by s)
  *   rope_layout      ATTN_ROPE_INTERLEAVED: pairs (2i, 2i+1) (attn_prefill's layout);
- *                    ATTN_ROPE_HALF_SPLIT: pairs (i, i + D/2), i < D/2
+ *                    ATTN_ROPE_HALF_SPLIT: pairs (i, i + D/2), i < D/2;
+ *                    either OR ATTN_ROPE_BF16_OPERANDS (bf16 input only): the rotated q and k
+ *                    are rounded to bf16 instead of fp16, so any bf16 input is served (no
+ *                    ATTN_DEV_RANGE) at 8x the rounding of the fp16 operands; the fallback
+ *                    for calls that reported ATTN_DEV_RANGE
  * Everything else as attn_prefill, which equals attn_prefill_ex(..., rope_freq_scale = 1,
  * ATTN_ROPE_INTERLEAVED, ...). Invalid layout or non-positive scale: ATTN_ERR_INVALID_ARG.
  */
@@ -272,13 +279,17 @@ int dsa_mla_decode_fp8(const void* q_nope, const void* q_pe, const void* kv_code
  * buffers they already own). Same arguments, layouts and results as
  * attn_decode_paged, minus the workspace: the split partials and the status
  * word live in one file-scope device array of ATTN_DECODE_NOALLOC_MAX_BYTES,
- * created when the library is loaded and held by every GPU that loads it until
- * the process exits. The call allocates nothing.
+ * held by every GPU that loads the library until the process exits. The call
+ * allocates nothing (the first call on a device: see below). Device-side flags
+ * (bad block-table entries, lengths beyond the table, timeouts) are read with
+ * attn_decode_paged_noalloc_status.
  *  - Problems whose attn_decode_paged_workspace_size() exceeds the array are
  *    rejected with ATTN_ERR_WORKSPACE and a message naming both sizes.
  *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call before
- *    any stream capture.
+ *    (cudaGetSymbolAddress) with that device current. With CUDA's lazy module
+ *    loading (the default since CUDA 12.2) that first call may also load this
+ *    library's device code and reserve the array, so make it outside any region
+ *    where the caller cannot allocate, and before any stream capture.
  *  - Every call on a device shares the one array and leaves its contents behind;
  *    calls whose GPU work overlaps (different streams, or host threads) race on it
  *    and must be serialised by the caller.
@@ -290,6 +301,16 @@ int attn_decode_paged_noalloc(const void* q, const void* k_pages, const void* v_
                               int page_size, int max_pages_per_seq, int num_pages, float scale, int dtype,
                               void* stream);
 
+/*
+ * Status word of the last attn_decode_paged_noalloc call on the current device (the
+ * call has no workspace for attn_read_status to read): waits for `stream`, then copies
+ * the word at the start of the fixed array into *flags (ATTN_DEV_BAD_PAGE,
+ * ATTN_DEV_BAD_LENGTH, ATTN_DEV_TIMEOUT). Returns ATTN_OK when no flag is set,
+ * ATTN_ERR_DEVICE when one is, ATTN_ERR_CUDA when the lookup or the copy fails.
+ * Allocates nothing; like the entry point, it has no counterpart on the method's pages.
+ */
+int attn_decode_paged_noalloc_status(int* flags, void* stream);
+
 /* Thread-local description of the last error returned on this thread ("" if none). */
 const char* attn_last_error(void);
 
@@ -299,6 +320,52 @@ const char* attn_last_error(void);
  * ATTN_ERR_DEVICE when one is, ATTN_ERR_CUDA when the copy fails.
  */
 int attn_read_status(const void* workspace, int* flags, void* stream);
+
+/*
+ * Combines partial results of the same query rows over disjoint key sets: the slices
+ * of every sequence's KV cache that the GPUs of a sequence-parallel group hold, each
+ * attended with attn_decode_paged or mla_decode on its own GPU and gathered. The
+ * block-level form of the online-softmax recurrence ("attention study note",
+ * section "online-softmax 分块计算原理"): M = max_s lse_s, w_s = exp(lse_s - M),
+ * lse = M + ln(sum_s w_s), out = sum_s w_s o_s / sum_s w_s, in part order
+ * (deterministic); parts with lse = -inf (empty slices) carry no weight, and a row
+ * whose parts are all empty gets out = 0, lse = -inf.
+ *   o_parts   [n_parts, rows, D] bf16 (read)     lse_parts [n_parts, rows] fp32 (read)
+ *   out       [rows, D] bf16 (written)            lse       [rows] fp32 (written)
+ * rows = B * H of the decode (H = Hq, or the 128 MLA heads); D in {64, 128, 256, 512};
+ * 1 <= n_parts <= 65536. Pointers 4-byte aligned. Asynchronous on `stream`; no workspace.
+ */
+int attn_lse_merge(const void* o_parts, const float* lse_parts, int n_parts, long long rows, int D, void* out,
+                   float* lse, void* stream);
+
+/*
+ * RoPE base rescaling for long contexts, the values to pass as rope_theta.
+ * attn_rope_ntk_theta: the NTK-aware base for a context stretched by `scale` (>= 1):
+ *   theta * scale^(D / (D - 2)), which leaves the highest rotary frequency (pair 0)
+ *   unchanged and divides the lowest one, theta^(-(D-2)/D), by `scale`
+ *   ("From 32K to 256K: DeepSeek long-context" (tqpw.cn), section 2.2, names NTK-aware
+ *   scaling; the rule is the published one).
+ * attn_rope_length_scaled_theta: theta * (length / base_length)^alpha (same page,
+ *   section 2.4, the length-aware base).
+ * Host functions (no GPU). Invalid arguments or a non-finite result: return 0 and set
+ * attn_last_error().
+ */
+double attn_rope_ntk_theta(double theta, double scale, int head_dim);
+double attn_rope_length_scaled_theta(double theta, int length, int base_length, double alpha);
+
+/*
+ * Self-test of the exponential that part of the prefill softmax evaluates on the FMA
+ * pipe instead of the MUFU (the score rate of the tensor core at head dim 128 equals
+ * the MUFU rate, so 2 of every 8 exponentials of an unmasked block take this path).
+ * Writes y[i] = 2^z[i] as that routine computes it: Cody-Waite reduction z = n + f with
+ * n = round(z), f in [-1/2, 1/2], 2^f from a degree-3 minimax polynomial fitted for this
+ * library, 2^n added to the exponent field: relative error <= 7.5e-5 for z >= -125.5
+ * (normal results); just above -126 the result can be subnormal (absolute error below
+ * 2^-126 * 2e-4); arguments below -126 are clamped to -126. Valid for z < 128. z, y: device arrays of n fp32 values,
+ * 1 <= n <= 2^30. Asynchronous on `stream`. No counterpart on the pages: the softmax
+ * they describe uses exp(); this only checks the library's own exponential.
+ */
+int attn_selftest_exp2(const float* z, float* y, int n, void* stream);
 
 /*
  * Self-test of the bounded-wait mechanism every kernel uses: launches one CTA that

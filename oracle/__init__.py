@@ -15,9 +15,11 @@ from .attention import (  # noqa: F401
     dsa_topk_ref,
     e4m3_to_float,
     gather_pages,
+    length_scaled_theta_ref,
     lse_merge,
     mla_decode_ref,
     mla_naive_ref,
+    ntk_aware_theta_ref,
     online_softmax_merge,
     prefill_ref,
     rope_cache,

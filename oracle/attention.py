@@ -67,6 +67,19 @@ def rope_cache(seq_len: int, head_dim: int, theta: float, freq_scale: float = 1.
     return np.stack([np.cos(ang), np.sin(ang)], axis=-1)
 
 
+def ntk_aware_theta_ref(theta: float, scale: float, head_dim: int) -> float:
+    """NTK-aware RoPE base for a context stretched by ``scale`` ("From 32K to 256K:
+    DeepSeek long-context", section 2.2 names NTK-aware scaling; the rule is the published
+    one): rescale the base so that the lowest rotary frequency theta^(-(D-2)/D) is divided
+    by ``scale`` while the highest (pair 0, frequency 1) stays: theta' = theta * scale^(D/(D-2))."""
+    return float(theta) * float(scale) ** (float(head_dim) / (head_dim - 2.0))
+
+
+def length_scaled_theta_ref(theta: float, length: int, base_length: int, alpha: float) -> float:
+    """Length-aware RoPE base of the same page, section 2.4: theta * (L / L0)^alpha."""
+    return float(theta) * (float(length) / float(base_length)) ** float(alpha)
+
+
 def _pair_slices(d: int, layout: str):
     """The two members of each rotated pair: adjacent (2i, 2i+1) ("interleaved", the
     long-context page's section 2.1) or the two halves (i, i + d/2) ("half", the

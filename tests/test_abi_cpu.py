@@ -211,3 +211,54 @@ def test_dsa_gather_grid_limit(lib):
     P = ctypes.c_void_p(FAKE)
     g = lib.dsa_mla_decode
     assert g(P, P, P, P, P, P, 1 << 21, 0.07, P, P, 1024, 128, 512, 64, 1 << 22, P, 1 << 62, None) == 2
+
+
+def test_noalloc_array_holds_the_stated_example_and_rejects_past_it(lib):
+    """The fixed array of attn_decode_paged_noalloc holds 8 sequences of 32K tokens at
+    Hq = 32, D = 128 (2048 pages of 16 tokens); with that table width 31 sequences fit
+    and 32 do not. The size check runs before any CUDA call, so the rejection is
+    visible without a GPU."""
+    cap = 32 << 20
+    ws = lib.attn_decode_paged_workspace_size
+    ws.restype = ctypes.c_size_t
+    assert ws(8, 32, 128, 2048, 16) <= cap
+    assert ws(31, 32, 128, 2048, 16) <= cap < ws(32, 32, 128, 2048, 16)
+    f = lib.attn_decode_paged_noalloc
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p] * 7 + [ctypes.c_int] * 7 + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p]
+    P = ctypes.c_void_p(FAKE)
+    assert f(P, P, P, P, P, P, P, 32, 32, 8, 128, 16, 2048, 100, 0.0, 1, None) == 3
+    assert "scratch" in _err(lib)
+    g = lib.attn_decode_paged_noalloc_status
+    g.restype = ctypes.c_int
+    assert g(None, None) == 1 and "null" in _err(lib)
+
+
+def test_rope_base_helpers_match_the_oracle(lib):
+    """The library's NTK-aware and length-scaled RoPE bases (host functions, no GPU)
+    against the oracle's, and their argument checks."""
+    from oracle import length_scaled_theta_ref, ntk_aware_theta_ref
+    from attention_causal_gqa_b200.binding import length_scaled_theta, ntk_aware_theta
+    for D, s, th in ((64, 8.0, 1e4), (128, 4.0, 5e5), (128, 1.0, 1e4), (192, 32.0, 1e6)):
+        assert abs(ntk_aware_theta(th, s, D) - ntk_aware_theta_ref(th, s, D)) <= 1e-12 * ntk_aware_theta_ref(th, s, D)
+    for L, L0, a in ((4096, 4096, 0.2), (131072, 4096, 0.5), (8192, 4096, 1.0), (1024, 4096, 0.3)):
+        r = length_scaled_theta_ref(1e4, L, L0, a)
+        assert abs(length_scaled_theta(1e4, L, L0, a) - r) <= 1e-12 * r
+    lib.attn_rope_ntk_theta.restype = ctypes.c_double
+    lib.attn_rope_ntk_theta.argtypes = [ctypes.c_double, ctypes.c_double, ctypes.c_int]
+    assert lib.attn_rope_ntk_theta(1e4, 0.5, 128) == 0.0 and "scale" in _err(lib)   # shrinking is not a stretch
+    assert lib.attn_rope_ntk_theta(1e4, 2.0, 3) == 0.0                               # odd head dim
+    assert lib.attn_rope_ntk_theta(-1.0, 2.0, 128) == 0.0
+
+
+def test_lse_merge_validation_codes(lib):
+    f = lib.attn_lse_merge
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_int,
+                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    P = ctypes.c_void_p(FAKE)
+    assert f(None, P, 2, 64, 128, P, P, None) == 1 and "null" in _err(lib)
+    assert f(P, P, 0, 64, 128, P, P, None) == 1       # no parts
+    assert f(P, P, 2, 0, 128, P, P, None) == 1        # no rows
+    assert f(P, P, 2, 64, 96, P, P, None) == 2        # D = 96
+    assert f(ctypes.c_void_p(FAKE + 2), P, 2, 64, 128, P, P, None) == 1  # misaligned

@@ -659,16 +659,21 @@ def test_prefill_half_split_equals_interleaved_on_permuted_q_k():
 
 
 def test_ntk_aware_and_length_scaled_bases():
-    """NTK-aware: the lowest frequency is divided by the stretch, the highest stays 1.
-    Length-aware base of the long-context page (section 2.4): theta at L = L0."""
-    from attention_causal_gqa_b200.binding import length_scaled_theta, ntk_aware_theta
-    D, s, th = 128, 8.0, 1e4
-    t2 = ntk_aware_theta(th, s, D)
-    lowest = lambda t: t ** (-2.0 * (D // 2 - 1) / D)  # noqa: E731
-    assert abs(lowest(t2) - lowest(th) / s) < 1e-12 * lowest(th)
-    assert ntk_aware_theta(th, 1.0, D) == th
-    assert length_scaled_theta(th, 4096, 4096, 0.2) == th
-    assert length_scaled_theta(th, 8192, 4096, 1.0) == 2 * th
+    """NTK-aware: the lowest frequency is divided by the stretch, the highest (pair 0)
+    stays 1, for several head dims and stretches. Length-aware base of the long-context
+    page (section 2.4): theta at L = L0 or alpha = 0, linear in L / L0 at alpha = 1."""
+    from oracle import length_scaled_theta_ref, ntk_aware_theta_ref
+    for D in (64, 128, 192):
+        for s, th in ((8.0, 1e4), (4.0, 5e5), (32.0, 1e6)):
+            t2 = ntk_aware_theta_ref(th, s, D)
+            lowest = lambda t: t ** (-2.0 * (D // 2 - 1) / D)  # noqa: E731
+            assert abs(lowest(t2) - lowest(th) / s) < 1e-12 * lowest(th)
+            assert t2 ** 0.0 == 1.0  # pair 0 rotates at frequency 1 whatever the base
+        assert ntk_aware_theta_ref(1e4, 1.0, D) == 1e4
+    assert length_scaled_theta_ref(1e4, 4096, 4096, 0.2) == 1e4
+    assert length_scaled_theta_ref(1e4, 65536, 4096, 0.0) == 1e4
+    assert length_scaled_theta_ref(1e4, 8192, 4096, 1.0) == 2e4
+    assert abs(length_scaled_theta_ref(1e4, 16384, 4096, 0.5) - 2e4) < 1e-9
 
 
 def test_chunk_prefill_half_split_equals_interleaved_on_permuted_dims():
