@@ -429,8 +429,7 @@ int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, c
   if (dtype != ATTN_DTYPE_BF16) return fail(ATTN_ERR_UNSUPPORTED, "paged decode supports bf16 only");
   if (page_size != 16) return fail(ATTN_ERR_UNSUPPORTED, "page_size %d (only 16)", page_size);
   if (D != 64 && D != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d", D);
-  if (Hkv > 8) return fail(ATTN_ERR_UNSUPPORTED, "Hkv %d > 8", Hkv);
-  if (Hq / Hkv > 16) return fail(ATTN_ERR_UNSUPPORTED, "group size %d > 16", Hq / Hkv);
+  if (Hq > 4096 || B > (1 << 20)) return fail(ATTN_ERR_UNSUPPORTED, "problem too large (Hq %d, B %d)", Hq, B);
   if (!aligned(q, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(out, 16) ||
       !aligned(block_table, 4) || !aligned(seq_lens, 4) || !aligned(lse, 4) || !aligned(workspace, 256))
     return fail(ATTN_ERR_INVALID_ARG, "misaligned pointer");
@@ -455,7 +454,9 @@ int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, c
   const cuuint64_t dims[5] = {64, 16, static_cast<cuuint64_t>(D / 64), static_cast<cuuint64_t>(Hkv),
                               static_cast<cuuint64_t>(num_pages)};
   const cuuint64_t strides[4] = {row, 128, static_cast<cuuint64_t>(D) * 2, 16 * row};
-  const cuuint32_t box[5] = {64, 16, static_cast<cuuint32_t>(D / 64), static_cast<cuuint32_t>(Hkv), 1};
+  // one box holds up to 8 KV heads of a page (a head group); a group past Hkv reads zeros
+  const int HG = Hkv < 8 ? Hkv : 8;
+  const cuuint32_t box[5] = {64, 16, static_cast<cuuint32_t>(D / 64), static_cast<cuuint32_t>(HG), 1};
   CUtensorMap tmK, tmV;
   if ((rc = make_map(&tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, k_pages, dims, strides, box, "k_pages"))) return rc;
   if ((rc = make_map(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, v_pages, dims, strides, box, "v_pages"))) return rc;
@@ -476,6 +477,11 @@ int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, c
   p.max_pages = max_pages_per_seq;
   p.num_pages = num_pages;
   p.n_splits = ns;
+  p.HG = HG;
+  p.n_hg = (Hkv + 7) / 8;
+  p.n_qt = (Hq / Hkv + 15) / 16;
+  if (static_cast<long long>(B) * ns * p.n_hg * p.n_qt > 0x7fffffffLL)
+    return fail(ATTN_ERR_UNSUPPORTED, "too many decode work items");
   p.scale_log2 = scale * 1.4426950408889634f;
   p.status = reinterpret_cast<int*>(ws);
   prof_before(st);

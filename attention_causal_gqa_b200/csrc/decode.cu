@@ -11,9 +11,14 @@
 // D=128) with one TMA per page and tensor into a shared-memory ring. The tensor
 // map is 5-D so the shared-memory image is [head][d/64][token][64] with 128-byte
 // swizzle, i.e. tokens on consecutive rows, which makes the ldmatrix reads below
-// bank-conflict free. Warp w handles KV head w and its G query heads; the two
-// tiny products (G x 16 tokens x D) run as warp-level mma.sync m16n8k16 with
-// fp32 accumulation so instruction issue stays far below the HBM rate.
+// bank-conflict free. Warp w handles KV head w of the page's head group and up to
+// 16 of its query heads (one m16 row tile); the two tiny products (16 x 16 tokens
+// x D) run as warp-level mma.sync m16n8k16 with fp32 accumulation so instruction
+// issue stays far below the HBM rate.
+// A work item is (sequence, split, head group, query tile): KV heads are taken 8 at
+// a time (one TMA box of up to 8 heads per page), so any Hkv is served without
+// reading a page twice; a group size G > 16 takes ceil(G / 16) query tiles, each of
+// which reads the pages again (GQA shapes with G <= 16 read every byte once).
 #include <cuda_bf16.h>
 
 #include "kernels.h"
@@ -23,7 +28,7 @@ namespace attn {
 
 namespace {
 
-constexpr int kDecWarps = 8;           // compute warps, one per KV head (Hkv <= 8)
+constexpr int kDecWarps = 8;           // compute warps, one per KV head of a head group
 constexpr int kDecThreads = (kDecWarps + 1) * 32;
 constexpr int kDecStages = 3;
 
@@ -58,7 +63,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   constexpr int PPS = kDecodePagesPerSplit;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int page_bytes = 16 * p.Hkv * D * 2;  // one page of K (or V), all heads
+  const int page_bytes = 16 * p.HG * D * 2;  // one page of K (or V), the heads of one group
   const int stage_bytes = 2 * page_bytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kDecStages * stage_bytes);
   uint64_t* empty = full + kDecStages;
@@ -76,7 +81,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   }
   __syncthreads();
 
-  const int n_items = p.B * p.n_splits;  // item k: split k / B of sequence k % B
+  // item k: sequence k % B; then query tile, head group and split (outermost)
+  const int n_items = p.B * p.n_qt * p.n_hg * p.n_splits;
 
   if (warp == kDecWarps) {
     // ---------------------------------------------------------------- producer
@@ -84,7 +90,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     prefetch_tmap(&tmV);
     int it = 0;  // ring position
     for (int k = blockIdx.x; k < n_items; k += gridDim.x) {
-      const int b = k % p.B, split = k / p.B;
+      const int b = k % p.B, hg = (k / (p.B * p.n_qt)) % p.n_hg, split = k / (p.B * p.n_qt * p.n_hg);
       int L = __ldg(p.seq_lens + b);
       if (L > p.max_pages * 16) {
         if (lane == 0) atomicOr(p.status, kDevErrBadLength);
@@ -114,8 +120,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         if (lane == 0) {
           uint8_t* dst = smem + s * stage_bytes;
           mbar_arrive_expect_tx(&full[s], stage_bytes);
-          tma_load_5d(dst, &tmK, &full[s], 0, 0, 0, 0, phys);
-          tma_load_5d(dst + page_bytes, &tmV, &full[s], 0, 0, 0, 0, phys);
+          tma_load_5d(dst, &tmK, &full[s], 0, 0, 0, hg * kDecWarps, phys);
+          tma_load_5d(dst + page_bytes, &tmV, &full[s], 0, 0, 0, hg * kDecWarps, phys);
         }
       }
     }
@@ -124,13 +130,16 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
   // ------------------------------------------------------------------ consumers
   const int g = lane >> 2, c = lane & 3;
-  const int h = warp;                         // KV head of this warp
-  const bool busy = h < p.Hkv;
   const int G = p.G;
   const float sl2 = p.scale_log2;
   int it = 0;
   for (int k = blockIdx.x; k < n_items; k += gridDim.x) {
-    const int b = k % p.B, split = k / p.B;
+    const int b = k % p.B, qt = (k / p.B) % p.n_qt, hg = (k / (p.B * p.n_qt)) % p.n_hg;
+    const int split = k / (p.B * p.n_qt * p.n_hg);
+    const int h = hg * kDecWarps + warp;        // KV head of this warp
+    const bool busy = warp < p.HG && h < p.Hkv;
+    const int q0 = qt * 16;                     // first query head of this tile within the group
+    const int rows = min(16, G - q0);           // query heads of the tile
     int L = __ldg(p.seq_lens + b);
     L = min(L, p.max_pages * 16);
     const int npages = (L + 15) >> 4;
@@ -138,18 +147,18 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     if (pg0 >= npages) continue;
     const int pg1 = min(npages, pg0 + PPS);
 
-    // Q fragments (A operand, rows = the G query heads of this KV head).
+    // Q fragments (A operand, rows = query heads q0 .. q0 + rows - 1 of this KV head).
     uint32_t qa[KT][4];
     {
       const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(p.q) +
-                                (static_cast<size_t>(b) * p.Hq + (busy ? h : 0) * G) * D;
+                                (static_cast<size_t>(b) * p.Hq + (busy ? h * G + q0 : 0)) * D;
 #pragma unroll
       for (int kt = 0; kt < KT; ++kt) {
         const int d0 = kt * 16 + 2 * c;
-        qa[kt][0] = (busy && g < G) ? *reinterpret_cast<const uint32_t*>(qb + g * D + d0) : 0u;
-        qa[kt][1] = (busy && g + 8 < G) ? *reinterpret_cast<const uint32_t*>(qb + (g + 8) * D + d0) : 0u;
-        qa[kt][2] = (busy && g < G) ? *reinterpret_cast<const uint32_t*>(qb + g * D + d0 + 8) : 0u;
-        qa[kt][3] = (busy && g + 8 < G) ? *reinterpret_cast<const uint32_t*>(qb + (g + 8) * D + d0 + 8) : 0u;
+        qa[kt][0] = (busy && g < rows) ? *reinterpret_cast<const uint32_t*>(qb + g * D + d0) : 0u;
+        qa[kt][1] = (busy && g + 8 < rows) ? *reinterpret_cast<const uint32_t*>(qb + (g + 8) * D + d0) : 0u;
+        qa[kt][2] = (busy && g < rows) ? *reinterpret_cast<const uint32_t*>(qb + g * D + d0 + 8) : 0u;
+        qa[kt][3] = (busy && g + 8 < rows) ? *reinterpret_cast<const uint32_t*>(qb + (g + 8) * D + d0 + 8) : 0u;
       }
     }
     float o[NT][4];
@@ -170,12 +179,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           // tokens past the end: zero their V rows so 0 * garbage cannot poison O
           for (int idx = lane; idx < DH * 16 * 8; idx += 32) {
             const int dh = idx / 128, t = (idx / 8) % 16, ch = idx % 8;
-            if (t >= rem) *reinterpret_cast<uint4*>(vp + ((h * DH + dh) * 16 + t) * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+            if (t >= rem) *reinterpret_cast<uint4*>(vp + ((warp * DH + dh) * 16 + t) * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
           }
           __syncwarp();
         }
-        const uint32_t kbase = smem_u32(kp) + h * DH * 16 * 128;
-        const uint32_t vbase = smem_u32(vp) + h * DH * 16 * 128;
+        const uint32_t kbase = smem_u32(kp) + warp * DH * 16 * 128;
+        const uint32_t vbase = smem_u32(vp) + warp * DH * 16 * 128;
         // S = Q K^T over 16 tokens (two n-tiles of 8 tokens)
         float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         const int mi = lane >> 3, r8 = lane & 7;  // ldmatrix: matrix index and row within it
@@ -256,19 +265,19 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
       l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
       l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-      const size_t base = (static_cast<size_t>(b) * p.n_splits + split) * p.Hq + h * G;
+      const size_t base = (static_cast<size_t>(b) * p.n_splits + split) * p.Hq + h * G + q0;
       const float i0 = 1.f / l0, i1 = 1.f / l1;
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
         const int dim = n * 8 + 2 * c;
-        if (g < G)
+        if (g < rows)
           *reinterpret_cast<float2*>(p.part_o + (base + g) * D + dim) = make_float2(o[n][0] * i0, o[n][1] * i0);
-        if (g + 8 < G)
+        if (g + 8 < rows)
           *reinterpret_cast<float2*>(p.part_o + (base + g + 8) * D + dim) = make_float2(o[n][2] * i1, o[n][3] * i1);
       }
       if (c == 0) {
-        if (g < G) p.part_lse[base + g] = (m0 + log2f(l0)) * 0.69314718055994531f;
-        if (g + 8 < G) p.part_lse[base + g + 8] = (m1 + log2f(l1)) * 0.69314718055994531f;
+        if (g < rows) p.part_lse[base + g] = (m0 + log2f(l0)) * 0.69314718055994531f;
+        if (g + 8 < rows) p.part_lse[base + g + 8] = (m1 + log2f(l1)) * 0.69314718055994531f;
       }
     }
   }
@@ -277,15 +286,15 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 template <int D>
 static cudaError_t launch_decode_t(const DecodeParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
                                    cudaStream_t stream) {
-  const int smem = 1024 + kDecStages * 2 * 16 * p.Hkv * D * 2 + 2 * kDecStages * 8 + 16;
+  const int smem = 1024 + kDecStages * 2 * 16 * p.HG * D * 2 + 2 * kDecStages * 8 + 16;
   auto kern = decode_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int items = p.B * p.n_splits;
-  const int grid = items < sms ? items : sms;
+  const long long items = static_cast<long long>(p.B) * p.n_splits * p.n_hg * p.n_qt;
+  const int grid = items < sms ? static_cast<int>(items) : sms;
   kern<<<grid, kDecThreads, smem, stream>>>(p, tmK, tmV);
   return cudaGetLastError();
 }

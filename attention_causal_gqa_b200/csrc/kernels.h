@@ -39,6 +39,7 @@ struct DecodeParams {
   float* lse;               // [B, Hq]
   int B, Hq, Hkv, D, G;
   int max_pages, num_pages, n_splits;
+  int HG, n_hg, n_qt;       // bf16 kernel: KV heads per TMA box (min(Hkv, 8)), head groups, 16-row query tiles
   float scale_log2;
   int* status;
   const float* k_scale;     // FP8 cache only: [num_pages, Hkv] scales (nullptr: bf16 cache)

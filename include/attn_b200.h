@@ -115,7 +115,9 @@ int attn_prefill_ex(const void* q, const void* k, const void* v, void* out, floa
  *                entries at or past ceil(seq_lens[b]/page_size) are never read
  *   seq_lens     [B] int32, 0 <= seq_lens[b] <= max_pages_per_seq * page_size
  *   out          [B, Hq, D] bf16 (written);  lse [B, Hq] fp32 (written)
- * Supported: dtype BF16, page_size 16, D in {64, 128}, Hkv <= 8, Hq/Hkv <= 16.
+ * Supported: dtype BF16, page_size 16, D in {64, 128}, any Hkv and group size
+ * G = Hq/Hkv (Hq <= 4096). KV heads are read 8 per page load; G > 16 reads each page
+ * once per 16 query heads of a KV head (G <= 16 reads every cached byte once).
  * scale <= 0 selects 1/sqrt(D). Out-of-range table entries or lengths are clamped
  * (no fault) and flagged in the status word.
  */

@@ -94,7 +94,7 @@ def test_decode_validation_codes(lib):
     assert call(Hq=30) == 1
     assert call(ps=32) == 2
     assert call(D=256) == 2
-    assert call(Hkv=16, Hq=32) == 2
+    assert call(Hkv=8, Hq=8192) == 2               # beyond 4096 query heads
     assert call(dt=0) == 2
     assert call(ws=need - 1) == 3
     assert call(npg=0) == 1

@@ -50,6 +50,10 @@ def _oracle(d, pairs=None, scale=None):
         ([700, 33], 4, 1, 128),          # MQA
         ([1200, 64, 9], 16, 2, 64),      # G = 8, D = 64
         ([257, 4096], 32, 2, 128),       # G = 16
+        ([3000, 1, 64], 32, 32, 128),    # MHA with 32 KV heads: four 8-head TMA groups
+        ([900, 17], 12, 12, 64),         # 12 KV heads: the second group is half past the end
+        ([1500, 40], 32, 1, 128),        # MQA with 32 query heads: two 16-row query tiles
+        ([2000, 100], 40, 2, 128),       # G = 20: a full and a partial query tile
     ],
 )
 def test_decode_matches_oracle_small(lens, Hq, Hkv, D):
