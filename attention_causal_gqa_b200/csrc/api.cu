@@ -196,7 +196,7 @@ int attn_prefill_ex(const void* q, const void* k, const void* v, void* out, floa
   if (rc) return rc;
 
   const bool rope = rope_theta > 0.f;
-  if (rope) {
+  if (rope && f32) {  // the fp32 operand split reads a cos/sin table
     cudaError_t e = attn::launch_rope_table(cs, S, D, static_cast<double>(rope_theta),
                                             static_cast<double>(rope_freq_scale), st);
     if (e != cudaSuccess) return cuda_fail(e, "rope table launch");
@@ -215,8 +215,11 @@ int attn_prefill_ex(const void* q, const void* k, const void* v, void* out, floa
     vbase = vop;
     zdim *= 2;
   } else if (rope) {
-    cudaError_t e = attn::launch_rope_k_f16(k, kop, cs, rows, S, D, half_split, status, st, bf16_ops);
-    if (e != cudaSuccess) return cuda_fail(e, "rope K launch");
+    // one launch rotates K into the workspace and Q into `out` (see the Q operand below)
+    cudaError_t e = attn::launch_rope_qk(q, out, static_cast<long long>(B) * Hq, k, kop, static_cast<long long>(B) * Hkv,
+                                         S, D, static_cast<double>(rope_theta), static_cast<double>(rope_freq_scale),
+                                         half_split, status, st, bf16_ops);
+    if (e != cudaSuccess) return cuda_fail(e, "rope launch");
     kbase = kop;
     kdt = bf16_ops ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   }
@@ -234,9 +237,7 @@ int attn_prefill_ex(const void* q, const void* k, const void* v, void* out, floa
     if (e != cudaSuccess) return cuda_fail(e, "Q operand split launch");
     qbase = out;
     zq *= 2;
-  } else if (rope) {
-    cudaError_t e = attn::launch_rope_k_f16(q, out, cs, rows_q, S, D, half_split, status, st, bf16_ops);
-    if (e != cudaSuccess) return cuda_fail(e, "rope Q launch");
+  } else if (rope) {  // rotated by the launch above
     qbase = out;
     qdt = bf16_ops ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   }

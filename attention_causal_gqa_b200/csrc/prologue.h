@@ -11,11 +11,11 @@ namespace attn {
 // RoPE prologue: cos/sin table of pos * freq_scale * theta^(-2i/D) (angles in fp64), then
 // the operands. half_split: element d pairs with d + D/2 instead of 2i with 2i + 1.
 cudaError_t launch_rope_table(float2* cs, int S, int D, double theta, double freq_scale, cudaStream_t stream);
-// bf16 X [rows, D] -> rotated fp16 X (row r at position r % S); flags values outside fp16 range.
-// Used for K and for Q.
-cudaError_t launch_rope_k_f16(const void* k, void* k_f16, const float2* cs, long long rows, int S, int D,
-                              bool half_split, int* status, cudaStream_t stream,
-                              bool bf16_out = false);
+// One launch rotating bf16 Q [q_heads, S, D] into q_op and K [k_heads, S, D] into k_op (fp16,
+// or bf16 when bf16_out), computing each pair's cos/sin from its fp64 angle in the kernel.
+cudaError_t launch_rope_qk(const void* q, void* q_op, long long q_heads, const void* k, void* k_op, long long k_heads,
+                           int S, int D, double theta, double freq_scale, bool half_split, int* status,
+                           cudaStream_t stream, bool bf16_out);
 // fp32 X [rows, D] -> bf16 hi parts at out[0, rows) and lo parts at out[rows, 2 rows), rotating
 // first when cs is non-null.
 cudaError_t launch_split_f32(const float* x, void* out, const float2* cs, long long rows, int S, int D,

@@ -1,11 +1,14 @@
 // RoPE prologue ("From 32K to 256K: DeepSeek long-context", section 2.1 for the
 // rotation, section 2.5 for the cos/sin cache [max_len, head_dim/2, 2]).
 //
-// The table stores cos and sin of pos * f * theta^(-2i/D) for every integer position
-// and pair (f: a frequency scale, 1 for plain RoPE; section 2.2 scales the frequencies
-// by a factor, section 2.4 rescales the base theta, which callers pass as theta); each
-// angle is formed in fp64 straight from the integer position (no running phase), then
-// rounded to fp32. Pairs are adjacent elements (2i, 2i+1) by default:
+// The angle of pair i at position pos is pos * f * theta^(-2i/D) (f: a frequency scale,
+// 1 for plain RoPE; section 2.2 scales the frequencies by a factor, section 2.4 rescales
+// the base theta, which callers pass as theta), always formed in fp64 straight from the
+// integer position (no running phase). The table (for the fp32-input and chunked paths)
+// stores its cos and sin rounded to fp32; the bf16 prefill prologue reduces the fp64
+// angle to [-pi, pi] and takes cos and sin in fp32 inside the rotation kernel, so Q and K
+// are rotated by one launch with no table pass. Pairs are adjacent elements (2i, 2i+1)
+// by default:
 //   y[2i]   = x[2i] cos - x[2i+1] sin
 //   y[2i+1] = x[2i] sin + x[2i+1] cos
 // and (i, i + D/2) in the half-split layout (the concatenated-halves form of section 2.4).
@@ -36,11 +39,11 @@ __global__ void rope_table_kernel(float2* __restrict__ cs, int S, int half, cons
   }
 }
 
-// The two operand-preparation kernels share one layout: a block of 256 threads
-// covers 256 / CPR consecutive positions (CPR = D / 8 chunks of 8 elements per
-// row), and blockIdx.y strides over the heads. Each thread loads the cos/sin of
-// its chunk once and reuses them for every head it visits, and all index
-// arithmetic is 32-bit except the final element offset.
+// The operand-preparation kernels share one layout: a block of 256 threads covers
+// 256 / CPR consecutive positions (CPR = D / 8 chunks of 8 elements per row), and
+// blockIdx.y strides over the heads. Each thread obtains the cos/sin of its chunk
+// once (computed, or from the table) and reuses them for every head it visits, and
+// all index arithmetic is 32-bit except the final element offset.
 template <int CPR>
 __device__ __forceinline__ bool chunk_position(int S, int& pos, int& c) {
   constexpr int RPB = 256 / CPR;
@@ -71,35 +74,6 @@ __device__ __forceinline__ uint32_t pack_operand(float a, float b, bool& in_rang
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// bf16 X [heads, S, D] -> rotated fp16 X (used for K and for Q), or rotated bf16 X for
-// inputs beyond the fp16 range (BF16). fp16 values beyond its range set the range flag
-// of the status word.
-template <int CPR, bool BF16>
-__global__ void __launch_bounds__(256) rope_f16_kernel(const uint4* __restrict__ x, uint4* __restrict__ y,
-                                                       const float2* __restrict__ cs, int heads, int S,
-                                                       int* __restrict__ status) {
-  int pos, c;
-  if (!chunk_position<CPR>(S, pos, c)) return;
-  float2 a[4];
-  load_cs4<CPR>(cs, pos, c, a);
-  bool in_range = true;
-  for (int hd = blockIdx.y; hd < heads; hd += gridDim.y) {
-    const size_t idx = (static_cast<size_t>(hd) * S + pos) * CPR + c;
-    const uint4 raw = x[idx];
-    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-    uint32_t ow[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float x0 = __uint_as_float(w[e] << 16);
-      const float x1 = __uint_as_float(w[e] & 0xFFFF0000u);
-      const float y0 = x0 * a[e].x - x1 * a[e].y, y1 = x0 * a[e].y + x1 * a[e].x;
-      ow[e] = pack_operand<BF16>(y0, y1, in_range);
-    }
-    y[idx] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-  }
-  if (!in_range) atomicOr(status, 8);
-}
-
 // The cos/sin of pairs 8c .. 8c+7 (half-split layout: chunk c of the first half).
 template <int CPR>
 __device__ __forceinline__ void load_cs8(const float2* __restrict__ cs, int pos, int c, float2 (&a)[8]) {
@@ -112,45 +86,6 @@ __device__ __forceinline__ void load_cs8(const float2* __restrict__ cs, int pos,
   }
 }
 
-// Half-split layout of rope_f16_kernel: the thread of chunk c < CPR/2 rotates it together
-// with its partner chunk c + CPR/2 (element d pairs with d + D/2); the others have no work.
-template <int CPR, bool BF16>
-__global__ void __launch_bounds__(256) rope_f16_half_kernel(const uint4* __restrict__ x, uint4* __restrict__ y,
-                                                            const float2* __restrict__ cs, int heads, int S,
-                                                            int* __restrict__ status) {
-  int pos, c;
-  if (!chunk_position<CPR>(S, pos, c) || c >= CPR / 2) return;
-  float2 a[8];
-  load_cs8<CPR>(cs, pos, c, a);
-  bool in_range = true;
-  for (int hd = blockIdx.y; hd < heads; hd += gridDim.y) {
-    const size_t idx = (static_cast<size_t>(hd) * S + pos) * CPR + c;
-    const uint4 rl = x[idx], rh = x[idx + CPR / 2];
-    const uint32_t wl[4] = {rl.x, rl.y, rl.z, rl.w}, wh[4] = {rh.x, rh.y, rh.z, rh.w};
-    uint32_t ol[4], oh[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      float lo[2] = {__uint_as_float(wl[e] << 16), __uint_as_float(wl[e] & 0xFFFF0000u)};
-      float hi[2] = {__uint_as_float(wh[e] << 16), __uint_as_float(wh[e] & 0xFFFF0000u)};
-      float yl[2], yh[2];
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const float2 cz = a[2 * e + k];
-        yl[k] = lo[k] * cz.x - hi[k] * cz.y;
-        yh[k] = lo[k] * cz.y + hi[k] * cz.x;
-      }
-      ol[e] = pack_operand<BF16>(yl[0], yl[1], in_range);
-      oh[e] = pack_operand<BF16>(yh[0], yh[1], in_range);
-    }
-    y[idx] = make_uint4(ol[0], ol[1], ol[2], ol[3]);
-    y[idx + CPR / 2] = make_uint4(oh[0], oh[1], oh[2], oh[3]);
-  }
-  if (!in_range) atomicOr(status, 8);
-}
-
-// fp32 X [heads, S, D] -> hi = bf16(x) in out[0, heads), lo = bf16(x - hi) in
-// out[heads, 2 heads), rotating first when cs is non-null. HALF: half-split pairs (the
-// thread of chunk c < CPR/2 handles chunks c and c + CPR/2).
 template <int CPR, bool HALF>
 __global__ void __launch_bounds__(256) split_f32_kernel(const float4* __restrict__ x, uint4* __restrict__ out,
                                                         const float2* __restrict__ cs, int heads, int S) {
@@ -217,6 +152,72 @@ __global__ void __launch_bounds__(256) split_f32_kernel(const float4* __restrict
 
 // Grid of the operand-preparation kernels: position blocks in x, enough head
 // slices in y for about 32 blocks per SM.
+// cos/sin of pos * inv[i]: the angle is formed and reduced to [-pi, pi] in fp64 (no
+// running phase, exact to ~1e-12 rad however large pos * inv[i] grows), then its cosine
+// and sine come from the fp32 routine (about 1e-7 absolute error, a thousand times below
+// the 16-bit rounding of the rotated operand).
+__device__ __forceinline__ float2 cos_sin_of(int pos, double inv) {
+  constexpr double kTwoPi = 6.283185307179586476925286766559;
+  const double th = static_cast<double>(pos) * inv;
+  const double r = th - kTwoPi * rint(th / kTwoPi);
+  float sn, cs;
+  sincosf(static_cast<float>(r), &sn, &cs);
+  return make_float2(cs, sn);
+}
+
+// One launch for both operands of a bf16 prefill: rotates Q rows [0, hq) and K rows
+// [0, hk) of [heads, S, D] into 16-bit operands (fp16, or bf16 for BF16), computing the
+// cos/sin of its own pairs instead of reading a table (so no table kernel runs first).
+// Interleaved pairs (2i, 2i+1), or the half-split layout (HALF: element d with d + D/2,
+// handled by the threads of the first half's chunks). fp16 values beyond its range set
+// the range flag of the status word.
+template <int CPR, bool HALF, bool BF16>
+__global__ void __launch_bounds__(256) rope_qk_kernel(const uint4* __restrict__ q, uint4* __restrict__ qo, int hq,
+                                                      const uint4* __restrict__ k, uint4* __restrict__ ko, int hk,
+                                                      int S, const __grid_constant__ RopeFreqs f,
+                                                      int* __restrict__ status) {
+  int pos, c;
+  if (!chunk_position<CPR>(S, pos, c)) return;
+  if (HALF && c >= CPR / 2) return;
+  constexpr int NPAIR = HALF ? 8 : 4;  // pairs whose cos/sin this thread needs
+  float2 a[NPAIR];
+#pragma unroll
+  for (int e = 0; e < NPAIR; ++e) a[e] = cos_sin_of(pos, f.inv[NPAIR * c + e]);
+  bool in_range = true;
+  for (int hd = blockIdx.y; hd < hq + hk; hd += gridDim.y) {
+    const bool isq = hd < hq;
+    const uint4* x = isq ? q : k;
+    uint4* y = isq ? qo : ko;
+    const size_t idx = (static_cast<size_t>(isq ? hd : hd - hq) * S + pos) * CPR + c;
+    if (!HALF) {
+      const uint4 raw = x[idx];
+      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+      uint32_t ow[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float x0 = __uint_as_float(w[e] << 16), x1 = __uint_as_float(w[e] & 0xFFFF0000u);
+        ow[e] = pack_operand<BF16>(x0 * a[e].x - x1 * a[e].y, x0 * a[e].y + x1 * a[e].x, in_range);
+      }
+      y[idx] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+    } else {
+      const uint4 rl = x[idx], rh = x[idx + CPR / 2];
+      const uint32_t wl[4] = {rl.x, rl.y, rl.z, rl.w}, wh[4] = {rh.x, rh.y, rh.z, rh.w};
+      uint32_t ol[4], oh[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float l0 = __uint_as_float(wl[e] << 16), l1 = __uint_as_float(wl[e] & 0xFFFF0000u);
+        const float h0 = __uint_as_float(wh[e] << 16), h1 = __uint_as_float(wh[e] & 0xFFFF0000u);
+        const float2 c0 = a[2 * e], c1 = a[2 * e + 1];
+        ol[e] = pack_operand<BF16>(l0 * c0.x - h0 * c0.y, l1 * c1.x - h1 * c1.y, in_range);
+        oh[e] = pack_operand<BF16>(l0 * c0.y + h0 * c0.x, l1 * c1.y + h1 * c1.x, in_range);
+      }
+      y[idx] = make_uint4(ol[0], ol[1], ol[2], ol[3]);
+      y[idx + CPR / 2] = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+    }
+  }
+  if (!in_range) atomicOr(status, 8);
+}
+
 static dim3 operand_grid(int heads, int S, int cpr) {
   const int rpb = 256 / cpr;
   const int gx = (S + rpb - 1) / rpb;
@@ -245,27 +246,31 @@ cudaError_t launch_rope_table(float2* cs, int S, int D, double theta, double fre
   return cudaGetLastError();
 }
 
-cudaError_t launch_rope_k_f16(const void* k, void* k_f16, const float2* cs, long long rows, int S, int D,
-                              bool half_split, int* status, cudaStream_t stream, bool bf16_out) {
-  const long long heads = rows / S;
-  if (heads * S != rows || heads > 0x7fffffffLL) return cudaErrorInvalidValue;
-  const dim3 grid = operand_grid(static_cast<int>(heads), S, D / 8);
-  const uint4* x = static_cast<const uint4*>(k);
-  uint4* y = static_cast<uint4*>(k_f16);
-  const int h = static_cast<int>(heads);
-  if (bf16_out) {
-    if (D == 128 && half_split) rope_f16_half_kernel<16, true><<<grid, 256, 0, stream>>>(x, y, cs, h, S, status);
-    else if (D == 128) rope_f16_kernel<16, true><<<grid, 256, 0, stream>>>(x, y, cs, h, S, status);
-    else if (D == 64 && half_split) rope_f16_half_kernel<8, true><<<grid, 256, 0, stream>>>(x, y, cs, h, S, status);
-    else if (D == 64) rope_f16_kernel<8, true><<<grid, 256, 0, stream>>>(x, y, cs, h, S, status);
-    else return cudaErrorInvalidValue;
+cudaError_t launch_rope_qk(const void* q, void* q_op, long long q_heads, const void* k, void* k_op, long long k_heads,
+                           int S, int D, double theta, double freq_scale, bool half_split, int* status,
+                           cudaStream_t stream, bool bf16_out) {
+  const int half = D / 2;
+  if (half < 1 || half > 64 || q_heads + k_heads > 0x7fffffffLL) return cudaErrorInvalidValue;
+  RopeFreqs f{};
+  for (int i = 0; i < half; ++i) f.inv[i] = freq_scale * std::pow(theta, -2.0 * i / D);
+  const int hq = static_cast<int>(q_heads), hk = static_cast<int>(k_heads);
+  const dim3 grid = operand_grid(hq + hk, S, D / 8);
+  const auto* xq = static_cast<const uint4*>(q);
+  const auto* xk = static_cast<const uint4*>(k);
+  auto* yq = static_cast<uint4*>(q_op);
+  auto* yk = static_cast<uint4*>(k_op);
+#define ATTN_ROPE_QK(CPR, HALF, BF)                                                                      \
+  rope_qk_kernel<CPR, HALF, BF><<<grid, 256, 0, stream>>>(xq, yq, hq, xk, yk, hk, S, f, status)
+  if (D == 128) {
+    if (half_split) { if (bf16_out) ATTN_ROPE_QK(16, true, true); else ATTN_ROPE_QK(16, true, false); }
+    else { if (bf16_out) ATTN_ROPE_QK(16, false, true); else ATTN_ROPE_QK(16, false, false); }
+  } else if (D == 64) {
+    if (half_split) { if (bf16_out) ATTN_ROPE_QK(8, true, true); else ATTN_ROPE_QK(8, true, false); }
+    else { if (bf16_out) ATTN_ROPE_QK(8, false, true); else ATTN_ROPE_QK(8, false, false); }
   } else {
-    if (D == 128 && half_split) rope_f16_half_kernel<16, false><<<grid, 256, 0, stream>>>(x, y, cs, h, S, status);
-    else if (D == 128) rope_f16_kernel<16, false><<<grid, 256, 0, stream>>>(x, y, cs, h, S, status);
-    else if (D == 64 && half_split) rope_f16_half_kernel<8, false><<<grid, 256, 0, stream>>>(x, y, cs, h, S, status);
-    else if (D == 64) rope_f16_kernel<8, false><<<grid, 256, 0, stream>>>(x, y, cs, h, S, status);
-    else return cudaErrorInvalidValue;
+    return cudaErrorInvalidValue;
   }
+#undef ATTN_ROPE_QK
   return cudaGetLastError();
 }
 
