@@ -731,17 +731,24 @@ size_t dsa_mla_decode_workspace_size(int B, int H, int Dc, int Dr, int top_k) {
   return mla + round_up(rows * Dc * 2, 256) + round_up(rows * Dr * 2, 256) + round_up(static_cast<size_t>(B) * 4, 256);
 }
 
-int dsa_mla_decode(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
-                   const int32_t* seq_lens, const int32_t* topk_idx, int top_k, float scale, void* out, float* lse,
-                   int B, int H, int Dc, int Dr, int T_max, void* workspace, size_t workspace_bytes, void* stream) {
-  if (!q_nope || !q_pe || !kv_cache || !pe_cache || !seq_lens || !topk_idx || !out || !lse || !workspace)
+// Shared by both sparse MLA entry points: the argument checks, the workspace layout
+// [MLA workspace | selected latent rows bf16 | selected rotary rows bf16 | counts] and,
+// after the gather `gather(kv_sel, pe_sel, n_sel, status, stream)` has filled the
+// selected rows, the MLA decode over them (T_max = top_k).
+extern "C++" {
+template <typename Gather>
+static int dsa_mla_run(const void* q_nope, const void* q_pe, const void* latent, const void* pe_cache,
+                       const int32_t* seq_lens, const int32_t* topk_idx, int top_k, float scale, void* out, float* lse,
+                       int B, int H, int Dc, int Dr, int T_max, void* workspace, size_t workspace_bytes, void* stream,
+                       Gather&& gather) {
+  if (!q_nope || !q_pe || !latent || !pe_cache || !seq_lens || !topk_idx || !out || !lse || !workspace)
     return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
   if (B <= 0 || H <= 0 || Dc <= 0 || Dr <= 0 || T_max <= 0 || top_k <= 0)
     return fail(ATTN_ERR_INVALID_ARG, "sizes must be positive");
   if (H != 128 || Dc != 512 || Dr != 64)
     return fail(ATTN_ERR_UNSUPPORTED, "MLA decode supports H=128, Dc=512, Dr=64 (got %d, %d, %d)", H, Dc, Dr);
   if (!(scale > 0.f) || !std::isfinite(scale)) return fail(ATTN_ERR_INVALID_ARG, "scale must be positive");
-  if (!aligned(q_nope, 16) || !aligned(q_pe, 16) || !aligned(kv_cache, 16) || !aligned(pe_cache, 16) ||
+  if (!aligned(q_nope, 16) || !aligned(q_pe, 16) || !aligned(latent, 16) || !aligned(pe_cache, 16) ||
       !aligned(out, 16) || !aligned(seq_lens, 4) || !aligned(topk_idx, 4) || !aligned(lse, 4) ||
       !aligned(workspace, 256))
     return fail(ATTN_ERR_INVALID_ARG, "misaligned pointer");
@@ -759,45 +766,35 @@ int dsa_mla_decode(const void* q_nope, const void* q_pe, const void* kv_cache, c
   int* status = reinterpret_cast<int*>(ws);
   int rc = clear_status(ws, st);
   if (rc) return rc;
-  cudaError_t e = attn::launch_dsa_gather(kv_cache, pe_cache, topk_idx, seq_lens, kv_sel, pe_sel, n_sel, B, T_max,
-                                          top_k, Dc, Dr, status, st);
+  cudaError_t e = gather(kv_sel, pe_sel, n_sel, status, st);
   if (e != cudaSuccess) return cuda_fail(e, "gather launch");
   return mla_run(q_nope, q_pe, kv_sel, pe_sel, n_sel, scale, out, lse, B, H, Dc, Dr, top_k, ws + kHeader, status, st);
+}
+}  // extern "C++"
+
+int dsa_mla_decode(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
+                   const int32_t* seq_lens, const int32_t* topk_idx, int top_k, float scale, void* out, float* lse,
+                   int B, int H, int Dc, int Dr, int T_max, void* workspace, size_t workspace_bytes, void* stream) {
+  return dsa_mla_run(q_nope, q_pe, kv_cache, pe_cache, seq_lens, topk_idx, top_k, scale, out, lse, B, H, Dc, Dr, T_max,
+                     workspace, workspace_bytes, stream,
+                     [&](void* kv_sel, void* pe_sel, int32_t* n_sel, int* status, cudaStream_t st) {
+                       return attn::launch_dsa_gather(kv_cache, pe_cache, topk_idx, seq_lens, kv_sel, pe_sel, n_sel, B,
+                                                      T_max, top_k, Dc, Dr, status, st);
+                     });
 }
 
 int dsa_mla_decode_fp8(const void* q_nope, const void* q_pe, const void* kv_codes, const float* kv_scale,
                        const void* pe_cache, const int32_t* seq_lens, const int32_t* topk_idx, int top_k, float scale,
                        void* out, float* lse, int B, int H, int Dc, int Dr, int T_max, void* workspace,
                        size_t workspace_bytes, void* stream) {
-  if (!q_nope || !q_pe || !kv_codes || !kv_scale || !pe_cache || !seq_lens || !topk_idx || !out || !lse || !workspace)
-    return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
-  if (B <= 0 || H <= 0 || Dc <= 0 || Dr <= 0 || T_max <= 0 || top_k <= 0)
-    return fail(ATTN_ERR_INVALID_ARG, "sizes must be positive");
-  if (H != 128 || Dc != 512 || Dr != 64)
-    return fail(ATTN_ERR_UNSUPPORTED, "MLA decode supports H=128, Dc=512, Dr=64 (got %d, %d, %d)", H, Dc, Dr);
-  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(ATTN_ERR_INVALID_ARG, "scale must be positive");
-  if (!aligned(q_nope, 16) || !aligned(q_pe, 16) || !aligned(kv_codes, 16) || !aligned(kv_scale, 4) ||
-      !aligned(pe_cache, 16) || !aligned(out, 16) || !aligned(seq_lens, 4) || !aligned(topk_idx, 4) ||
-      !aligned(lse, 4) || !aligned(workspace, 256))
-    return fail(ATTN_ERR_INVALID_ARG, "misaligned pointer");
-  if (T_max > (1 << 26) || B > (1 << 20) || top_k > (1 << 26) || static_cast<long long>(B) * top_k > (1LL << 30))
-    return fail(ATTN_ERR_UNSUPPORTED, "problem too large");
-  const size_t need = dsa_mla_decode_workspace_size(B, H, Dc, Dr, top_k);
-  if (workspace_bytes < need)
-    return fail(ATTN_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace_bytes, need);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const size_t rows = static_cast<size_t>(B) * top_k;
-  uint8_t* kv_sel = ws + mla_decode_workspace_size(B, H, Dc, Dr, top_k);
-  uint8_t* pe_sel = kv_sel + round_up(rows * Dc * 2, 256);
-  int32_t* n_sel = reinterpret_cast<int32_t*>(pe_sel + round_up(rows * Dr * 2, 256));
-  int* status = reinterpret_cast<int*>(ws);
-  int rc = clear_status(ws, st);
-  if (rc) return rc;
-  cudaError_t e = attn::launch_dsa_gather_fp8(kv_codes, kv_scale, pe_cache, topk_idx, seq_lens, kv_sel, pe_sel, n_sel,
-                                              B, T_max, top_k, Dc, Dr, status, st);
-  if (e != cudaSuccess) return cuda_fail(e, "gather launch");
-  return mla_run(q_nope, q_pe, kv_sel, pe_sel, n_sel, scale, out, lse, B, H, Dc, Dr, top_k, ws + kHeader, status, st);
+  if (!kv_scale) return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned(kv_scale, 4)) return fail(ATTN_ERR_INVALID_ARG, "misaligned pointer");
+  return dsa_mla_run(q_nope, q_pe, kv_codes, pe_cache, seq_lens, topk_idx, top_k, scale, out, lse, B, H, Dc, Dr, T_max,
+                     workspace, workspace_bytes, stream,
+                     [&](void* kv_sel, void* pe_sel, int32_t* n_sel, int* status, cudaStream_t st) {
+                       return attn::launch_dsa_gather_fp8(kv_codes, kv_scale, pe_cache, topk_idx, seq_lens, kv_sel,
+                                                          pe_sel, n_sel, B, T_max, top_k, Dc, Dr, status, st);
+                     });
 }
 
 int attn_read_status(const void* workspace, int* flags, void* stream) {
