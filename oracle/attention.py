@@ -333,7 +333,7 @@ def to_bf16(x):
 
 def chunk_prefill_ref(q, k_new, v_new, k_pages, v_pages, block_table, cache_lens, rope_theta: float = 10000.0,
                       scale: float | None = None, page_size: int = 16, store=to_bf16, rope_freq_scale: float = 1.0,
-                      rope_layout: str = "interleaved"):
+                      rope_layout: str = "interleaved", new_lens=None):
     """Append a chunk of new tokens to a paged KV cache and attend over the whole cache.
 
     "From 32K to 256K: DeepSeek long-context", chapter 1 (key architecture path: a
@@ -352,6 +352,9 @@ def chunk_prefill_ref(q, k_new, v_new, k_pages, v_pages, block_table, cache_lens
     (the causal mask aligned to the end of the cache), two-pass softmax, O = P V.
     rope_freq_scale and rope_layout as ``apply_rope`` (the cached keys are taken as
     rotated the same way).
+    new_lens: optional [B] chunk lengths (0 <= new_lens[b] <= S_new, a batch of chunks of
+    different lengths padded to S_new): sequence b appends and attends only its first
+    new_lens[b] new tokens; its rows past them are o = 0, lse = -inf.
     Returns (k_pages', v_pages', o [B, Hq, S_new, D], lse [B, Hq, S_new]).
     """
     q = np.asarray(q, dtype=F64)
@@ -366,28 +369,31 @@ def chunk_prefill_ref(q, k_new, v_new, k_pages, v_pages, block_table, cache_lens
         scale = 1.0 / math.sqrt(D)
     use_rope = rope_theta and rope_theta > 0
     o = np.zeros((B, Hq, S_new, D))
-    lse = np.zeros((B, Hq, S_new))
+    lse = np.full((B, Hq, S_new), -np.inf)
     for b in range(B):
         L = int(cache_lens[b])
-        pos = L + np.arange(S_new)
+        n = S_new if new_lens is None else int(new_lens[b])
+        if n == 0:
+            continue
+        pos = L + np.arange(n)
         table = np.asarray(block_table[b])
         for kvh in range(Hkv):
-            kr = (apply_rope(k_new[b, kvh], rope_theta, positions=pos, freq_scale=rope_freq_scale, layout=rope_layout)
-                  if use_rope else k_new[b, kvh])
+            kr = (apply_rope(k_new[b, kvh, :n], rope_theta, positions=pos, freq_scale=rope_freq_scale,
+                             layout=rope_layout) if use_rope else k_new[b, kvh, :n])
             kp[table[pos // page_size], pos % page_size, kvh] = store(kr)
-            vp[table[pos // page_size], pos % page_size, kvh] = store(v_new[b, kvh])
-        kk = gather_pages(kp, table, L + S_new, page_size)
-        vv = gather_pages(vp, table, L + S_new, page_size)
+            vp[table[pos // page_size], pos % page_size, kvh] = store(v_new[b, kvh, :n])
+        kk = gather_pages(kp, table, L + n, page_size)
+        vv = gather_pages(vp, table, L + n, page_size)
         for h in range(Hq):
             kvh = h // G
-            qr = (apply_rope(q[b, h], rope_theta, positions=pos, freq_scale=rope_freq_scale, layout=rope_layout)
-                  if use_rope else q[b, h])
+            qr = (apply_rope(q[b, h, :n], rope_theta, positions=pos, freq_scale=rope_freq_scale, layout=rope_layout)
+                  if use_rope else q[b, h, :n])
             s = scale * (qr @ kk[:, kvh, :].T)
-            jj = np.arange(L + S_new)[None, :]
+            jj = np.arange(L + n)[None, :]
             s = np.where(jj > pos[:, None], -np.inf, s)
             p, l_ = two_pass_softmax_rows(s)
-            o[b, h] = p @ vv[:, kvh, :]
-            lse[b, h] = l_
+            o[b, h, :n] = p @ vv[:, kvh, :]
+            lse[b, h, :n] = l_
     return kp, vp, o, lse
 
 

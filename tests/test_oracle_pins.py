@@ -712,3 +712,42 @@ def test_dsa_fp8_latent_equals_dsa_over_the_dequantised_cache():
     sc2[:, :, 1] *= 2.0
     o2, _ = dsa_mla_decode_fp8_ref(qn, qp, codes, sc2, pe, sel, 0.2)
     assert not np.allclose(o2, o)
+
+
+def test_chunk_prefill_varlen_pins():
+    """Per-sequence chunk lengths: (a) all lengths S_new is the uniform call; (b) each
+    sequence equals that sequence alone with its own S_new (brute force per sequence);
+    (c) a zero length appends nothing and leaves its rows at o = 0, lse = -inf;
+    (d) appending n1 then n2 tokens gives the second chunk's rows of one n1 + n2 chunk
+    (chunking does not change the attention)."""
+    from oracle import chunk_prefill_ref
+    rng = np.random.default_rng(75)
+    B, Hq, Hkv, D, S_new = 3, 4, 2, 16, 9
+    cache = [0, 20, 5]
+    q = rng.standard_normal((B, Hq, S_new, D))
+    k = rng.standard_normal((B, Hkv, S_new, D))
+    v = rng.standard_normal((B, Hkv, S_new, D))
+    kp, vp, table = _paged_setup(rng, B, Hkv, D, cache, S_new)
+    ku, vu, ou, lu = chunk_prefill_ref(q, k, v, kp, vp, table, cache, rope_theta=30.0)
+    kf, vf, of, lf = chunk_prefill_ref(q, k, v, kp, vp, table, cache, rope_theta=30.0, new_lens=[S_new] * B)
+    assert np.array_equal(ou, of) and np.array_equal(lu, lf) and np.array_equal(ku, kf)
+    lens = [4, 0, 9]
+    kv_, vv_, o, l = chunk_prefill_ref(q, k, v, kp, vp, table, cache, rope_theta=30.0, new_lens=lens)
+    for b, n in enumerate(lens):
+        if n == 0:
+            assert np.all(o[b] == 0) and np.all(np.isneginf(l[b]))
+            continue
+        _, _, ob, lb = chunk_prefill_ref(q[b:b + 1, :, :n], k[b:b + 1, :, :n], v[b:b + 1, :, :n], kp, vp,
+                                         table[b:b + 1], cache[b:b + 1], rope_theta=30.0)
+        assert np.allclose(o[b, :, :n], ob[0], atol=1e-12) and np.allclose(l[b, :, :n], lb[0], atol=1e-12)
+        assert np.all(o[b, :, n:] == 0) and np.all(np.isneginf(l[b, :, n:]))
+    # sequence 1 appended nothing: its pages are untouched
+    assert np.array_equal(kv_[table[1]], kp[table[1]])
+    # two chunks (3 then 6 tokens) equal one chunk of 9 for the second chunk's rows
+    b = 2
+    qb, kb, vb = q[b:b + 1], k[b:b + 1], v[b:b + 1]
+    k1, v1, _, _ = chunk_prefill_ref(qb, kb, vb, kp, vp, table[b:b + 1], [cache[b]], rope_theta=30.0, new_lens=[3])
+    _, _, o2, l2 = chunk_prefill_ref(qb[:, :, 3:], kb[:, :, 3:], vb[:, :, 3:], k1, v1, table[b:b + 1], [cache[b] + 3],
+                                     rope_theta=30.0)
+    _, _, o9, l9 = chunk_prefill_ref(qb, kb, vb, kp, vp, table[b:b + 1], [cache[b]], rope_theta=30.0)
+    assert np.allclose(o2[0], o9[0, :, 3:], atol=1e-12) and np.allclose(l2[0], l9[0, :, 3:], atol=1e-12)
