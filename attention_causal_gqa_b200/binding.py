@@ -31,6 +31,7 @@ ATTN_DEV_BAD_INDEX = 16
 
 EXPORTED = (
     "attn_prefill_workspace_size", "attn_prefill", "attn_prefill_ex", "attn_prefill_chunk_ex",
+    "attn_prefill_chunk_varlen",
     "attn_decode_paged_workspace_size", "attn_decode_paged",
     "attn_decode_paged_fp8_workspace_size", "mla_decode_workspace_size", "mla_decode",
     "dsa_index_topk_workspace_size", "dsa_index_topk", "dsa_mla_decode_workspace_size", "dsa_mla_decode",
@@ -70,6 +71,8 @@ def _load() -> ctypes.CDLL:
     lib.attn_prefill_chunk.argtypes = [vp] * 9 + [i32] * 9 + [f32, f32, vp, sz, vp]
     lib.attn_prefill_chunk_ex.restype = i32
     lib.attn_prefill_chunk_ex.argtypes = [vp] * 9 + [i32] * 9 + [f32, f32, i32, f32, vp, sz, vp]
+    lib.attn_prefill_chunk_varlen.restype = i32
+    lib.attn_prefill_chunk_varlen.argtypes = [vp] * 10 + [i32] * 9 + [f32, f32, i32, f32, vp, sz, vp]
     lib.attn_decode_paged_fp8_workspace_size.restype = sz
     lib.attn_decode_paged_fp8_workspace_size.argtypes = [i32] * 5
     lib.mla_decode_workspace_size.restype = sz
@@ -288,12 +291,16 @@ def prefill_chunk_workspace_size(B, Hkv, S_new, max_cache_len, D) -> int:
 
 def attn_prefill_chunk(q, k, v, k_pages, v_pages, block_table, cache_lens, max_cache_len, rope_theta=10000.0,
                        scale=None, out=None, lse=None, workspace=None, stream=None, rope_freq_scale=1.0,
-                       rope_layout="interleaved", check=False):
+                       rope_layout="interleaved", check=False, new_lens=None):
     """Append a chunk of new tokens to the paged KV cache and attend over the whole cache.
     q [B,Hq,S_new,D], k/v [B,Hkv,S_new,D] bf16 (not rotated); k/v_pages [P,16,Hkv,D] bf16, updated in
     place; block_table [B,maxp] int32; cache_lens [B] int32 (tokens already cached, each <= max_cache_len).
+    new_lens [B] int32 (optional): chunks of different lengths padded to S_new; sequence b takes only its
+    first new_lens[b] tokens and its rows past them come back as out = 0, lse = -inf.
     Returns (out [B,Hq,S_new,D] bf16, lse [B,Hq,S_new] fp32)."""
     _need_cuda(q, k, v, k_pages, v_pages, block_table, cache_lens)
+    if new_lens is not None:
+        _need_cuda(new_lens)
     B, Hq, S_new, D = q.shape
     Hkv = k.shape[1]
     P, ps, _, _ = k_pages.shape
@@ -305,7 +312,13 @@ def attn_prefill_chunk(q, k, v, k_pages, v_pages, block_table, cache_lens, max_c
     ws = _workspace(prefill_chunk_workspace_size(B, Hkv, S_new, int(max_cache_len), D), q.device, workspace)
     if rope_layout not in ROPE_LAYOUTS:
         raise ValueError(f"rope_layout must be one of {sorted(ROPE_LAYOUTS)}")
-    if float(rope_freq_scale) == 1.0 and rope_layout == "interleaved":
+    if new_lens is not None:
+        rc = lib.attn_prefill_chunk_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(k_pages), _ptr(v_pages), _ptr(block_table),
+                                           _ptr(cache_lens), _ptr(new_lens), _ptr(out), _ptr(lse), B, Hq, Hkv, S_new,
+                                           D, ps, maxp, P, int(max_cache_len), float(rope_theta if rope_theta else 0.0),
+                                           float(rope_freq_scale), ROPE_LAYOUTS[rope_layout], float(scale or 0.0),
+                                           _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    elif float(rope_freq_scale) == 1.0 and rope_layout == "interleaved":
         rc = lib.attn_prefill_chunk(_ptr(q), _ptr(k), _ptr(v), _ptr(k_pages), _ptr(v_pages), _ptr(block_table),
                                     _ptr(cache_lens), _ptr(out), _ptr(lse), B, Hq, Hkv, S_new, D, ps, maxp, P,
                                     int(max_cache_len), float(rope_theta if rope_theta else 0.0), float(scale or 0.0),

@@ -298,13 +298,15 @@ size_t attn_prefill_chunk_workspace_size(int B, int Hkv, int S_new, int max_cach
   return kHeader + table + 2 * op;
 }
 
-int attn_prefill_chunk_ex(const void* q, const void* k, const void* v, void* k_pages, void* v_pages,
-                          const int32_t* block_table, const int32_t* cache_lens, void* out, float* lse, int B, int Hq,
-                          int Hkv, int S_new, int D, int page_size, int max_pages_per_seq, int num_pages,
-                          int max_cache_len, float rope_theta, float rope_freq_scale, int rope_layout, float scale,
-                          void* workspace, size_t workspace_bytes, void* stream) {
+int attn_prefill_chunk_varlen(const void* q, const void* k, const void* v, void* k_pages, void* v_pages,
+                              const int32_t* block_table, const int32_t* cache_lens, const int32_t* new_lens, void* out,
+                              float* lse, int B, int Hq, int Hkv, int S_new, int D, int page_size,
+                              int max_pages_per_seq, int num_pages, int max_cache_len, float rope_theta,
+                              float rope_freq_scale, int rope_layout, float scale, void* workspace,
+                              size_t workspace_bytes, void* stream) {
   if (!q || !k || !v || !k_pages || !v_pages || !block_table || !cache_lens || !out || !lse || !workspace)
     return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
+  if (new_lens && !aligned(new_lens, 4)) return fail(ATTN_ERR_INVALID_ARG, "misaligned new_lens");
   if (rope_layout != ATTN_ROPE_INTERLEAVED && rope_layout != ATTN_ROPE_HALF_SPLIT)
     return fail(ATTN_ERR_INVALID_ARG, "rope_layout %d", rope_layout);
   if (!(rope_freq_scale > 0.f) || !std::isfinite(rope_freq_scale))
@@ -347,14 +349,14 @@ int attn_prefill_chunk_ex(const void* q, const void* k, const void* v, void* k_p
                                             static_cast<double>(rope_freq_scale), st);
     if (e != cudaSuccess) return cuda_fail(e, "rope table launch");
   }
-  attn::ChunkGeometry g{cache_lens, block_table, B, Hkv, S_new, D, page_size, max_pages_per_seq, num_pages,
-                        max_cache_len, rope_layout == ATTN_ROPE_HALF_SPLIT ? 1 : 0};
+  attn::ChunkGeometry g{cache_lens, new_lens, block_table, B, Hkv, S_new, D, page_size, max_pages_per_seq,
+                        num_pages, max_cache_len, rope_layout == ATTN_ROPE_HALF_SPLIT ? 1 : 0};
   const float2* rcs = rope ? cs : nullptr;
   cudaError_t e = attn::launch_kv_append(k, v, k_pages, v_pages, rcs, g, status, st);
   if (e == cudaSuccess) e = attn::launch_kv_gather(k_pages, v_pages, k_op, v_op, g, static_cast<int>(sk), status, st);
   // the prepared Q operand goes into `out` (same byte size; each tile is loaded and
   // later overwritten by the same CTA)
-  if (e == cudaSuccess) e = attn::launch_rope_rows_f16(q, out, rcs, g, Hq, status, st);
+  if (e == cudaSuccess) e = attn::launch_rope_rows_f16(q, out, rcs, g, Hq, lse, status, st);
   if (e != cudaSuccess) return cuda_fail(e, "chunk operand launch");
 
   const int BN = attn::prefill_block_n(D, false);
@@ -385,6 +387,7 @@ int attn_prefill_chunk_ex(const void* q, const void* k, const void* v, void* k_p
   p.status = status;
   p.q_off = cache_lens;
   p.max_off = max_cache_len;
+  p.q_len = new_lens;
   const long long items = p.pair_heads ? static_cast<long long>(B) * (Hq / 2) * p.n_row_blocks
                                        : static_cast<long long>(B) * Hq * ((p.n_row_blocks + 1) / 2);
   if (items > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "too many work items");
@@ -398,6 +401,16 @@ int attn_prefill_chunk_ex(const void* q, const void* k, const void* v, void* k_p
   prof_after(st);
   if (e != cudaSuccess) return cuda_fail(e, "chunk prefill launch");
   return ok();
+}
+
+int attn_prefill_chunk_ex(const void* q, const void* k, const void* v, void* k_pages, void* v_pages,
+                          const int32_t* block_table, const int32_t* cache_lens, void* out, float* lse, int B, int Hq,
+                          int Hkv, int S_new, int D, int page_size, int max_pages_per_seq, int num_pages,
+                          int max_cache_len, float rope_theta, float rope_freq_scale, int rope_layout, float scale,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+  return attn_prefill_chunk_varlen(q, k, v, k_pages, v_pages, block_table, cache_lens, nullptr, out, lse, B, Hq, Hkv,
+                                   S_new, D, page_size, max_pages_per_seq, num_pages, max_cache_len, rope_theta,
+                                   rope_freq_scale, rope_layout, scale, workspace, workspace_bytes, stream);
 }
 
 int attn_prefill_chunk(const void* q, const void* k, const void* v, void* k_pages, void* v_pages,

@@ -14,7 +14,9 @@
 //                        in range), values as bf16, zeros past the sequence;
 //   rope_rows_f16_kernel rotates the new queries at their positions into fp16.
 // The prefill kernel then runs on those operands with each sequence's query
-// offset, so query i sees keys t <= cache_lens[b] + i.
+// offset, so query i sees keys t <= cache_lens[b] + i. Chunks may differ in length
+// (new_lens[b] <= S_new, padded to S_new): only the first new_lens[b] tokens of a
+// sequence are appended and attend; its other rows come out as zeros with LSE -inf.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -90,6 +92,11 @@ __device__ __forceinline__ uint4 pack8_f16_checked(const float (&f)[8], bool& in
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// New tokens of sequence b (all S_new unless chunks differ in length).
+__device__ __forceinline__ int new_len(const ChunkGeometry& g, int b, int* status) {
+  return g.new_lens ? clamp_len(g.new_lens, b, g.S_new, status) : g.S_new;
+}
+
 // Physical page of logical page lp of sequence b, or -1 (flagged) when the table
 // has no valid entry for it.
 __device__ __forceinline__ int page_of(const int32_t* __restrict__ table, int b, int lp, int max_pages, int num_pages,
@@ -115,6 +122,7 @@ __global__ void kv_append_kernel(const uint4* __restrict__ k_new, const uint4* _
   for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < n; idx += gridDim.x * blockDim.x) {
     const int c = idx % cpr, r = idx / cpr;
     const int i = r % g.S_new, kvh = (r / g.S_new) % g.Hkv, b = r / (g.S_new * g.Hkv);
+    if (i >= new_len(g, b, status)) continue;  // past this sequence's chunk
     const int pos = clamp_len(g.cache_lens, b, g.max_cache_len, status) + i;
     const int page = page_of(g.block_table, b, pos / g.page_size, g.max_pages, g.num_pages, status);
     if (page < 0) continue;
@@ -149,7 +157,7 @@ __global__ void kv_gather_kernel(const uint4* __restrict__ k_pages, const uint4*
     const long long r = idx / cpr;
     const int j = static_cast<int>(r % Sk_max);
     const int z = static_cast<int>(r / Sk_max), b = z / g.Hkv, kvh = z % g.Hkv;
-    const int Sk_b = clamp_len(g.cache_lens, b, g.max_cache_len, status) + g.S_new;
+    const int Sk_b = clamp_len(g.cache_lens, b, g.max_cache_len, status) + new_len(g, b, status);
     uint4 kq = make_uint4(0, 0, 0, 0), vq = make_uint4(0, 0, 0, 0);
     if (j < Sk_b) {
       const int page = page_of(g.block_table, b, j / g.page_size, g.max_pages, g.num_pages, status);
@@ -169,13 +177,18 @@ __global__ void kv_gather_kernel(const uint4* __restrict__ k_pages, const uint4*
 
 // Rows [B * Hq, S_new, D] of new queries, rotated at cache_lens[b] + i into fp16.
 __global__ void rope_rows_f16_kernel(const uint4* __restrict__ x, uint4* __restrict__ y, const float2* __restrict__ cs,
-                                     ChunkGeometry g, int Hq, int* __restrict__ status) {
+                                     ChunkGeometry g, int Hq, float* __restrict__ lse, int* __restrict__ status) {
   const int cpr = g.D / 8;
   const int n = g.B * Hq * g.S_new * cpr;
   bool in_range = true;
   for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < n; idx += gridDim.x * blockDim.x) {
     const int c = idx % cpr, r = idx / cpr;
     const int i = r % g.S_new, b = r / (g.S_new * Hq);
+    if (i >= new_len(g, b, status)) {  // a row past this sequence's chunk: its final output
+      y[idx] = make_uint4(0, 0, 0, 0);
+      if (c == 0) lse[r] = -INFINITY;
+      continue;
+    }
     const int pos = clamp_len(g.cache_lens, b, g.max_cache_len, status) + i;
     if (g.half_split && cs) {  // the thread of chunk c < cpr/2 writes chunks c and c + cpr/2
       if (c >= cpr / 2) continue;
@@ -219,10 +232,10 @@ cudaError_t launch_kv_gather(const void* k_pages, const void* v_pages, void* k_o
 }
 
 cudaError_t launch_rope_rows_f16(const void* q, void* q_f16, const float2* cs, const ChunkGeometry& g, int Hq,
-                                 int* status, cudaStream_t stream) {
+                                 float* lse, int* status, cudaStream_t stream) {
   const long long n = static_cast<long long>(g.B) * Hq * g.S_new * (g.D / 8);
   rope_rows_f16_kernel<<<grid_for(n, 256), 256, 0, stream>>>(static_cast<const uint4*>(q), static_cast<uint4*>(q_f16),
-                                                             cs, g, Hq, status);
+                                                             cs, g, Hq, lse, status);
   return cudaGetLastError();
 }
 

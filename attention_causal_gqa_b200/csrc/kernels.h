@@ -18,6 +18,8 @@ struct PrefillParams {
   int n_items;            // work items (pairs of query tiles); the grid walks them persistently
   const int32_t* q_off;   // [B] position of query row 0 among the keys (chunked prefill), or nullptr (0)
   int max_off;            // q_off values are clamped to [0, max_off]
+  const int32_t* q_len;   // [B] valid query rows of each sequence (chunks of different lengths), or nullptr (S);
+                          // rows past them are not written
   int* status;            // device status word
 };
 

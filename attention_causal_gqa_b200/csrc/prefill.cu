@@ -102,6 +102,7 @@ constexpr int kPolyPer8 = 2;
 struct PrefillItem {
   int b, h0, h1, r0_0, r0_1, n_kv0, n_kv1;
   int off;  // position of query row 0 among the keys (0 for a plain prefill)
+  int len;  // valid query rows of the sequence (S unless chunks differ in length)
 };
 
 // Item w of the list ordered heaviest (last row blocks) first.
@@ -132,11 +133,16 @@ __device__ __forceinline__ PrefillItem prefill_item(const PrefillParams& p, int 
     const int o = __ldg(p.q_off + it.b);
     it.off = o < 0 ? 0 : (o > p.max_off ? p.max_off : o);
   }
-  // keys 0 .. off + S - 1; with the causal mask query row r sees keys <= off + r
+  it.len = p.S;
+  if (p.q_len) {
+    const int n = __ldg(p.q_len + it.b);
+    it.len = n < 0 ? 0 : (n > p.S ? p.S : n);
+  }
+  // keys 0 .. off + len - 1; with the causal mask query row r sees keys <= off + r
   auto n_kv_for = [&](int r0) -> int {
-    if (r0 >= p.S) return 0;
-    if (!p.causal) return (it.off + p.S + BN - 1) / BN;
-    return (it.off + min(p.S, r0 + BM) - 1) / BN + 1;
+    if (r0 >= it.len) return 0;
+    if (!p.causal) return (it.off + it.len + BN - 1) / BN;
+    return (it.off + min(it.len, r0 + BM) - 1) / BN + 1;
   };
   it.n_kv0 = n_kv_for(it.r0_0);
   it.n_kv1 = n_kv_for(it.r0_1);
@@ -179,11 +185,16 @@ __global__ void __launch_bounds__(320, 1)
 
   const int G = gridDim.x;
   const int n_rounds = (p.n_items + G - 1) / G;
-  // Calls fn(item) for this CTA's items in order; every role walks the same list.
+  // Calls fn(item) for this CTA's items in order; every role walks the same list. An
+  // item whose two tiles have no rows to compute (past the end of a shorter chunk) is
+  // skipped by every role alike.
   auto for_each_item = [&](auto&& fn) {
     for (int r = 0; r < n_rounds; ++r) {
       const int w = prefill_item_index(r, blockIdx.x, G);
-      if (w < p.n_items && !fn(prefill_item<BN>(p, w))) return;
+      if (w >= p.n_items) continue;
+      const PrefillItem it = prefill_item<BN>(p, w);
+      if (it.n_kv0 == 0 && it.n_kv1 == 0) continue;
+      if (!fn(it)) return;
     }
   };
 
@@ -377,10 +388,10 @@ __global__ void __launch_bounds__(320, 1)
     const int b = it.b;
     if (n_kv == 0) return true;
     const int grow = r0 + row;
-    const bool row_valid = grow < p.S;
+    const bool row_valid = grow < it.len;
     float m_run = -INFINITY;
     float l_run = 0.f;
-    const int limit = it.off + (p.causal ? min(grow, p.S - 1) : p.S - 1);  // last key this row may see
+    const int limit = it.off + (p.causal ? min(grow, it.len - 1) : it.len - 1);  // last key this row may see
 
     for (int j = 0; j < n_kv && alive; ++j) {
       bool ok = mbar_wait(&s_full[t], (g + j) & 1, abort_flag, p.status);

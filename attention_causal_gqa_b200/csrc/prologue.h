@@ -24,6 +24,7 @@ cudaError_t launch_split_f32(const float* x, void* out, const float2* cs, long l
 // --------------------------------------------- chunked prefill into the paged cache
 struct ChunkGeometry {
   const int32_t* cache_lens;   // [B] tokens already cached (new token i sits at cache_lens[b] + i)
+  const int32_t* new_lens;     // [B] new tokens of each sequence (<= S_new), or nullptr (all S_new)
   const int32_t* block_table;  // [B, max_pages]
   int B, Hkv, S_new, D, page_size, max_pages, num_pages, max_cache_len;
   int half_split;              // RoPE pairs (i, i + D/2) instead of (2i, 2i + 1)
@@ -34,8 +35,9 @@ cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* k_pages
 // each sequence's cache into contiguous operands [B*Hkv, Sk_max, D]: keys fp16, values bf16, zeros past it
 cudaError_t launch_kv_gather(const void* k_pages, const void* v_pages, void* k_op, void* v_op, const ChunkGeometry& g,
                              int Sk_max, int* status, cudaStream_t stream);
-// new queries [B*Hq, S_new, D] rotated at their positions into fp16
+// new queries [B*Hq, S_new, D] rotated at their positions into fp16; rows past a sequence's
+// chunk are written as zeros, and their LSE as -inf
 cudaError_t launch_rope_rows_f16(const void* q, void* q_f16, const float2* cs, const ChunkGeometry& g, int Hq,
-                                 int* status, cudaStream_t stream);
+                                 float* lse, int* status, cudaStream_t stream);
 
 }  // namespace attn

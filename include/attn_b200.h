@@ -203,6 +203,26 @@ int attn_prefill_chunk_ex(const void* q, const void* k, const void* v, void* k_p
                           void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * attn_prefill_chunk_ex for a batch of chunks of different lengths ("From 32K to 256K:
+ * DeepSeek long-context", chapter 1: long inputs are cut into chunks streamed into the
+ * KV cache; sequences of a batch reach the end of their input at different points).
+ *   new_lens  [B] int32 (device, read), 0 <= new_lens[b] <= S_new: sequence b appends
+ *             only its first new_lens[b] tokens (rows of k, v padded to S_new) at
+ *             positions cache_lens[b] .. cache_lens[b] + new_lens[b] - 1, and only those
+ *             query rows attend; its rows past them are written as out = 0, lse = -inf.
+ *             nullptr: every sequence takes S_new (attn_prefill_chunk_ex).
+ * Lengths outside [0, S_new] are clamped and flagged (ATTN_DEV_BAD_LENGTH). Query row
+ * blocks past a sequence's chunk cost no tensor-core work. Everything else as
+ * attn_prefill_chunk_ex (same workspace size).
+ */
+int attn_prefill_chunk_varlen(const void* q, const void* k, const void* v, void* k_pages, void* v_pages,
+                              const int32_t* block_table, const int32_t* cache_lens, const int32_t* new_lens, void* out,
+                              float* lse, int B, int Hq, int Hkv, int S_new, int D, int page_size,
+                              int max_pages_per_seq, int num_pages, int max_cache_len, float rope_theta,
+                              float rope_freq_scale, int rope_layout, float scale, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/*
  * DeepSeek MLA absorbed decode (one query token per sequence).
  * Defined by: "DeepSeek-V3 attention: einsum vs hand-optimised" (dksg.cn), absorbed
  * form: scores = (q_nope . kv_cache^T + q_pe . pe_cache^T) * scale,

@@ -262,3 +262,26 @@ def test_lse_merge_validation_codes(lib):
     assert f(P, P, 2, 0, 128, P, P, None) == 1        # no rows
     assert f(P, P, 2, 64, 96, P, P, None) == 2        # D = 96
     assert f(ctypes.c_void_p(FAKE + 2), P, 2, 64, 128, P, P, None) == 1  # misaligned
+
+
+def test_prefill_chunk_varlen_validation_codes(lib):
+    f = lib.attn_prefill_chunk_varlen
+    f.restype = ctypes.c_int
+    P = ctypes.c_void_p(FAKE)
+    need = lib.attn_prefill_chunk_workspace_size(2, 2, 64, 64, 128)
+    #     q  k  v  kp vp bt cl nl out lse  B Hq Hkv S_new D ps maxp np maxc theta fscale layout scale ws bytes stream
+    args = [P, P, P, P, P, P, P, P, P, P, 2, 8, 2, 64, 128, 16, 8, 20, 64, 1e4, 1.0, 0, 0.0, P, need, None]
+    f.argtypes = [ctypes.c_void_p] * 10 + [ctypes.c_int] * 9 + [ctypes.c_float, ctypes.c_float, ctypes.c_int,
+                                                                 ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t,
+                                                                 ctypes.c_void_p]
+
+    def call(**over):
+        a = list(args)
+        for k, v in over.items():
+            a[int(k[1:])] = v
+        return f(*a)
+
+    assert call(_0=None) == 1 and "null" in _err(lib)
+    assert call(_7=ctypes.c_void_p(FAKE + 2)) == 1 and "new_lens" in _err(lib)   # misaligned lengths
+    assert call(_14=96) == 2                                                       # D = 96
+    assert call(_24=need - 1) == 3

@@ -120,3 +120,37 @@ def test_chunk_prefill_rope_variants(B, Hq, Hkv, D, cache_lens, S_new, fscale, l
     assert binding.read_status(ws) == 0
     assert np.array_equal(to_np(dev["v_pages"]), vp)
     assert _within_one_bf16_step(to_np(dev["k_pages"]), kp)
+
+
+@cuda
+@pytest.mark.parametrize("B,Hq,Hkv,D,cache_lens,S_new,new_lens,theta", [
+    (4, 8, 2, 128, [0, 100, 1000, 37], 300, [300, 0, 129, 1], 1e4),   # full, empty, ragged, one token
+    (3, 4, 4, 64, [33, 0, 500], 200, [128, 200, 127], 1e6),            # G = 1 items, tile edges
+    (2, 6, 2, 128, [64, 5], 130, [65, 130], 0.0),                      # no RoPE, G = 3
+])
+def test_chunk_prefill_varlen_matches_oracle(B, Hq, Hkv, D, cache_lens, S_new, new_lens, theta):
+    """Chunks of different lengths padded to S_new (attn_prefill_chunk_varlen): appended
+    pages, outputs and LSE against the oracle; rows past a chunk are exactly 0 / -inf and
+    pages a sequence does not reach stay as they were (the padding rows are poisoned)."""
+    from attention_causal_gqa_b200 import binding
+    d = _setup(B, Hq, Hkv, D, cache_lens, S_new, seed=S_new * 13 + B)
+    for b, n in enumerate(new_lens):  # padding rows hold NaN: they must never be read
+        d["q"][b, :, n:] = float("nan")
+        d["k"][b, :, n:] = float("nan")
+        d["v"][b, :, n:] = float("nan")
+    dev = {k: v.cuda() for k, v in d.items()}
+    nl = torch.tensor(new_lens, dtype=torch.int32, device="cuda")
+    mcl = max(cache_lens)
+    ws = torch.empty(binding.prefill_chunk_workspace_size(B, Hkv, S_new, mcl, D), dtype=torch.uint8, device="cuda")
+    out, lse = binding.attn_prefill_chunk(dev["q"], dev["k"], dev["v"], dev["k_pages"], dev["v_pages"], dev["table"],
+                                          dev["cache_lens"], mcl, rope_theta=theta, workspace=ws, new_lens=nl)
+    torch.cuda.synchronize()
+    kp, vp, ro, rl = chunk_prefill_ref(to_np(d["q"]), to_np(d["k"]), to_np(d["v"]), to_np(d["k_pages"]),
+                                       to_np(d["v_pages"]), d["table"].numpy(), cache_lens, rope_theta=theta,
+                                       new_lens=new_lens)
+    check(out, ro, lse, rl, what=f"chunk varlen {new_lens}")
+    for b, n in enumerate(new_lens):
+        assert torch.all(out[b, :, n:] == 0) and torch.all(torch.isneginf(lse[b, :, n:]))
+    assert binding.read_status(ws) == 0
+    assert np.array_equal(to_np(dev["v_pages"]), vp)
+    assert _within_one_bf16_step(to_np(dev["k_pages"]), kp)
