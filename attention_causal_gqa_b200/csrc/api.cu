@@ -7,6 +7,8 @@
 #include <mutex>
 #include <string>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/attn_b200.h"
 #include "dsa.h"
 #include "dsa_fp8.h"
@@ -33,6 +35,15 @@ int ok() {
   g_last_error.clear();
   return ATTN_OK;
 }
+
+// One NVTX range per public call (named after the call), so a timeline tool shows the
+// host-side span of each entry point around its kernels; free when no tool listens.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 int cuda_fail(cudaError_t e, const char* what) {
   return fail(ATTN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
@@ -159,6 +170,7 @@ size_t attn_prefill_workspace_size(int B, int Hkv, int S, int D, int dtype) {
 int attn_prefill_ex(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv, int S,
                     int D, int causal, float rope_theta, float rope_freq_scale, int rope_layout, float scale, int dtype,
                     void* workspace, size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx_range("attn_prefill_ex");
   if (!q || !k || !v || !out || !lse || !workspace) return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || S <= 0 || D <= 0)
     return fail(ATTN_ERR_INVALID_ARG, "sizes must be positive (B=%d Hq=%d Hkv=%d S=%d D=%d)", B, Hq, Hkv, S, D);
@@ -304,6 +316,7 @@ int attn_prefill_chunk_varlen(const void* q, const void* k, const void* v, void*
                               int max_pages_per_seq, int num_pages, int max_cache_len, float rope_theta,
                               float rope_freq_scale, int rope_layout, float scale, void* workspace,
                               size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx_range("attn_prefill_chunk_varlen");
   if (!q || !k || !v || !k_pages || !v_pages || !block_table || !cache_lens || !out || !lse || !workspace)
     return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
   if (new_lens && !aligned(new_lens, 4)) return fail(ATTN_ERR_INVALID_ARG, "misaligned new_lens");
@@ -435,6 +448,7 @@ int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, c
                       const int32_t* seq_lens, void* out, float* lse, int B, int Hq, int Hkv, int D, int page_size,
                       int max_pages_per_seq, int num_pages, float scale, int dtype, void* workspace,
                       size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx_range("attn_decode_paged");
   if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !out || !lse || !workspace)
     return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || max_pages_per_seq <= 0 || num_pages <= 0 || page_size <= 0)
@@ -519,6 +533,7 @@ int attn_decode_paged_fp8(const void* q, const void* k_pages, const void* v_page
                           const float* v_scale, const int32_t* block_table, const int32_t* seq_lens, void* out,
                           float* lse, int B, int Hq, int Hkv, int D, int page_size, int max_pages_per_seq,
                           int num_pages, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx_range("attn_decode_paged_fp8");
   if (!q || !k_pages || !v_pages || !k_scale || !v_scale || !block_table || !seq_lens || !out || !lse || !workspace)
     return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || max_pages_per_seq <= 0 || num_pages <= 0 || page_size <= 0)
@@ -649,6 +664,7 @@ static int mla_run(const void* q_nope, const void* q_pe, const void* kv_cache, c
 int mla_decode(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
                const int32_t* seq_lens, float scale, void* out, float* lse, int B, int H, int Dc, int Dr, int T_max,
                void* workspace, size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx_range("mla_decode");
   if (!q_nope || !q_pe || !kv_cache || !pe_cache || !seq_lens || !out || !lse || !workspace)
     return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
   if (B <= 0 || H <= 0 || Dc <= 0 || Dr <= 0 || T_max <= 0) return fail(ATTN_ERR_INVALID_ARG, "sizes must be positive");
@@ -684,6 +700,7 @@ size_t dsa_index_topk_workspace_size(int B, int H_I, int d_I, int T_max, int top
 int dsa_index_topk(const void* q_idx, const float* w_idx, const void* k_idx, const int32_t* seq_lens, float* scores,
                    int32_t* topk_idx, int B, int H_I, int d_I, int T_max, int top_k, void* workspace,
                    size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx_range("dsa_index_topk");
   if (!q_idx || !w_idx || !k_idx || !seq_lens || !scores || !topk_idx || !workspace)
     return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
   if (B <= 0 || H_I <= 0 || d_I <= 0 || T_max <= 0 || top_k <= 0)
@@ -788,6 +805,7 @@ static int dsa_mla_run(const void* q_nope, const void* q_pe, const void* latent,
 int dsa_mla_decode(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
                    const int32_t* seq_lens, const int32_t* topk_idx, int top_k, float scale, void* out, float* lse,
                    int B, int H, int Dc, int Dr, int T_max, void* workspace, size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx_range("dsa_mla_decode");
   return dsa_mla_run(q_nope, q_pe, kv_cache, pe_cache, seq_lens, topk_idx, top_k, scale, out, lse, B, H, Dc, Dr, T_max,
                      workspace, workspace_bytes, stream,
                      [&](void* kv_sel, void* pe_sel, int32_t* n_sel, int* status, cudaStream_t st) {
@@ -800,6 +818,7 @@ int dsa_mla_decode_fp8(const void* q_nope, const void* q_pe, const void* kv_code
                        const void* pe_cache, const int32_t* seq_lens, const int32_t* topk_idx, int top_k, float scale,
                        void* out, float* lse, int B, int H, int Dc, int Dr, int T_max, void* workspace,
                        size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx_range("dsa_mla_decode_fp8");
   if (!kv_scale) return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
   if (!aligned(kv_scale, 4)) return fail(ATTN_ERR_INVALID_ARG, "misaligned pointer");
   return dsa_mla_run(q_nope, q_pe, kv_codes, pe_cache, seq_lens, topk_idx, top_k, scale, out, lse, B, H, Dc, Dr, T_max,
@@ -825,6 +844,7 @@ int attn_read_status(const void* workspace, int* flags, void* stream) {
 
 int attn_lse_merge(const void* o_parts, const float* lse_parts, int n_parts, long long rows, int D, void* out,
                    float* lse, void* stream) {
+  NvtxRange nvtx_range("attn_lse_merge");
   if (!o_parts || !lse_parts || !out || !lse) return fail(ATTN_ERR_INVALID_ARG, "null pointer argument");
   if (n_parts < 1 || n_parts > (1 << 16) || rows < 1 || rows > (1LL << 36))
     return fail(ATTN_ERR_INVALID_ARG, "n_parts (%d) or rows (%lld) out of range", n_parts, rows);
