@@ -617,6 +617,10 @@ size_t mla_decode_workspace_size(int B, int H, int Dc, int Dr, int T_max) {
 static int mla_run(const void* q_nope, const void* q_pe, const void* kv_cache, const void* pe_cache,
                    const int32_t* seq_lens, float scale, void* out, float* lse, int B, int H, int Dc, int Dr,
                    int T_max, uint8_t* parts, int* status, cudaStream_t st) {
+  // the kernel's work split counts positions (tiles plus a per-sequence weight) in 32 bits
+  const long long positions =
+      static_cast<long long>(B) * ((T_max + attn::kMlaTile - 1) / attn::kMlaTile + attn::kMlaSegCost);
+  if (positions >= (1ll << 31)) return fail(ATTN_ERR_UNSUPPORTED, "problem too large");
   const size_t slots = static_cast<size_t>(attn::kMlaMaxPairs) + B;
   float* part_o = reinterpret_cast<float*>(parts);
   float* part_lse = reinterpret_cast<float*>(parts + round_up(slots * H * Dc * sizeof(float), 256));

@@ -63,6 +63,10 @@ cudaError_t launch_decode_range_merge(const float* part_o, const float* part_lse
 // ------------------------------------------------------------------ MLA
 constexpr int kMlaTile = 64;        // tokens per tile
 constexpr int kMlaMaxPairs = 74;    // two-CTA clusters in the persistent grid (148 SMs)
+// Weight, in tiles, that the MLA work split gives each non-empty sequence on top of its
+// tiles: a cluster pays a fixed cost per segment (its Q load, the drained pipeline and
+// the partial-result write), so ranges are cut in units of tiles + this per sequence.
+constexpr int kMlaSegCost = 8;
 
 struct MlaParams {
   const void* q_nope;       // [B, 1, H, Dc] bf16

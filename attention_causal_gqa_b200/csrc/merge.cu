@@ -166,14 +166,16 @@ __device__ __forceinline__ int units_of(const int32_t* lens, int b, int T_max) {
 }
 
 // One warp per (b, head). The partial-result kernels that balance work by ranges
-// (the MLA decode with 32-token tiles as units, the FP8 paged decode with 16-token
-// pages) cut the N units of all sequences into n_ranges contiguous ranges
-// [N c / n_ranges, N (c + 1) / n_ranges); range c writes one partial result per
-// sequence it meets, at slot c + b. The ranges meeting sequence b (units [s_b, e_b))
-// are those from the one holding unit s_b to the one holding unit e_b - 1: range c
-// holds unit x iff floor(N c / P) <= x < floor(N (c + 1) / P), i.e.
+// (the MLA decode with 64-token tiles as units, the FP8 paged decode with 16-token
+// pages) lay the units of all sequences out in one position space, a non-empty
+// sequence of n units taking SEG + n positions (its unit u at position SEG + u; SEG
+// weighs the fixed cost of a segment), and cut its N positions into n_ranges contiguous
+// ranges [N c / n_ranges, N (c + 1) / n_ranges); range c writes one partial result per
+// sequence it meets, at slot c + b. The ranges meeting sequence b (units at positions
+// [f_b, e_b)) are those from the one holding position f_b to the one holding e_b - 1:
+// range c holds position x iff floor(N c / P) <= x < floor(N (c + 1) / P), i.e.
 // c = floor(((x + 1) P - 1) / N). They are combined in range order (deterministic).
-template <int DIM, int UNIT>
+template <int DIM, int UNIT, int SEG>
 __global__ void range_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
                                    const int32_t* __restrict__ seq_lens, __nv_bfloat16* __restrict__ out,
                                    float* __restrict__ lse, int B, int H, int T_max, int n_ranges) {
@@ -186,19 +188,21 @@ __global__ void range_merge_kernel(const float* __restrict__ part_o, const float
   long long N = 0, s_b = 0;
   for (int i = lane; i < B; i += 32) {
     const int n = units_of<UNIT>(seq_lens, i, T_max);
-    N += n;
-    if (i < b) s_b += n;
+    const int u = n > 0 ? n + SEG : 0;
+    N += u;
+    if (i < b) s_b += u;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     N += __shfl_xor_sync(0xffffffffu, N, o);
     s_b += __shfl_xor_sync(0xffffffffu, s_b, o);
   }
-  const long long e_b = s_b + units_of<UNIT>(seq_lens, b, T_max);
+  const int n_b = units_of<UNIT>(seq_lens, b, T_max);
+  const long long f_b = s_b + SEG, e_b = f_b + n_b;
   const long long P = n_ranges;
   int c0 = 0, c1 = -1;  // contributing ranges (none for an empty sequence)
-  if (e_b > s_b) {
-    c0 = static_cast<int>(((s_b + 1) * P - 1) / N);
+  if (n_b > 0) {
+    c0 = static_cast<int>(((f_b + 1) * P - 1) / N);
     c1 = static_cast<int>((e_b * P - 1) / N);
   }
   __nv_bfloat16* orow = out + static_cast<size_t>(gw) * DIM + lane * VEC;
@@ -248,25 +252,25 @@ __global__ void range_merge_kernel(const float* __restrict__ part_o, const float
   }
 }
 
-template <int DIM, int UNIT>
+template <int DIM, int UNIT, int SEG>
 static cudaError_t launch_range_merge(const float* part_o, const float* part_lse, const int32_t* seq_lens, void* out,
                                       float* lse, int B, int H, int T_max, int n_ranges, cudaStream_t stream) {
   const long long warps = static_cast<long long>(B) * H;
   const int threads = 256;
   const long long blocks = (warps * 32 + threads - 1) / threads;
-  range_merge_kernel<DIM, UNIT><<<static_cast<int>(blocks), threads, 0, stream>>>(
+  range_merge_kernel<DIM, UNIT, SEG><<<static_cast<int>(blocks), threads, 0, stream>>>(
       part_o, part_lse, seq_lens, static_cast<__nv_bfloat16*>(out), lse, B, H, T_max, n_ranges);
   return cudaGetLastError();
 }
 
 cudaError_t launch_mla_merge(const float* part_o, const float* part_lse, const int32_t* seq_lens, void* out,
                              float* lse, int B, int H, int T_max, int n_pairs, cudaStream_t stream) {
-  return launch_range_merge<512, kMlaTile>(part_o, part_lse, seq_lens, out, lse, B, H, T_max, n_pairs, stream);
+  return launch_range_merge<512, kMlaTile, kMlaSegCost>(part_o, part_lse, seq_lens, out, lse, B, H, T_max, n_pairs, stream);
 }
 
 cudaError_t launch_decode_range_merge(const float* part_o, const float* part_lse, const int32_t* seq_lens, void* out,
                                       float* lse, int B, int H, int T_max, int n_ranges, cudaStream_t stream) {
-  return launch_range_merge<128, 16>(part_o, part_lse, seq_lens, out, lse, B, H, T_max, n_ranges, stream);
+  return launch_range_merge<128, 16, 0>(part_o, part_lse, seq_lens, out, lse, B, H, T_max, n_ranges, stream);
 }
 
 }  // namespace attn

@@ -89,8 +89,10 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t
                "r"(src_cta), "r"(bytes), "r"(bar_cluster)
                : "memory");
 }
-// Remote arrive without release semantics: used only to say "these bytes were read",
-// after the values read have been used (no write needs publishing).
+// Remote arrive that says "these bytes were read". It is relaxed (a release at cluster
+// scope measured 25-40% slower per launch); callers issue it only under a branch on a
+// value computed from every lane's loaded data, so the reads have returned before the
+// peer can learn that the block may be overwritten.
 __device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t bar_cluster_addr) {
   asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
 }
@@ -103,24 +105,52 @@ __device__ __forceinline__ int tiles_of(const int32_t* lens, int b, int T_max) {
   return (L + TN - 1) / TN;
 }
 
-// Calls fn(b, first_tile, end_tile, global_tile_offset_before) for every segment of
-// cluster `pair` in order. Every role enumerates the same segments.
+// Calls fn(b, first_tile, end_tile, global_tile_offset_before, b_next) for every segment
+// of cluster `pair` in order; b_next is b + 1 when the cluster's range reaches past this
+// segment (a hint for prefetching), else -1. The ranges are cut in a position space where
+// a non-empty sequence of n tiles takes kMlaSegCost + n positions, its tile t at position
+// kMlaSegCost + t; the cluster holding a tile's position computes it. The host keeps the
+// position count below 2^31. Whole warps call this (the scan takes 32 sequences per
+// step); every role enumerates the same segments.
 template <typename F>
 __device__ __forceinline__ void for_each_segment(const MlaParams& p, int pair, F&& fn) {
-  long long N = 0;
-  for (int b = 0; b < p.B; ++b) N += tiles_of(p.seq_lens, b, p.T_max);
-  const long long lo = N * pair / p.n_pairs, hi = N * (pair + 1) / p.n_pairs;
-  long long s = 0;
-  int done = 0;
-  for (int b = 0; b < p.B && s < hi; ++b) {
-    const int n = tiles_of(p.seq_lens, b, p.T_max);
-    const long long e = s + n;
-    const long long a0 = s > lo ? s : lo, a1 = e < hi ? e : hi;
-    if (a1 > a0) {
-      fn(b, static_cast<int>(a0 - s), static_cast<int>(a1 - s), done);
-      done += static_cast<int>(a1 - a0);
+  const int lane = threadIdx.x & 31;
+  constexpr unsigned kAll = 0xffffffffu;
+  unsigned N = 0;
+  for (int b0 = 0; b0 < p.B; b0 += 32) {
+    const int n = b0 + lane < p.B ? tiles_of(p.seq_lens, b0 + lane, p.T_max) : 0;
+    N += __reduce_add_sync(kAll, static_cast<unsigned>(n > 0 ? n + kMlaSegCost : 0));
+  }
+  const int lo = static_cast<int>(static_cast<long long>(N) * pair / p.n_pairs);
+  const int hi = static_cast<int>(static_cast<long long>(N) * (pair + 1) / p.n_pairs);
+  // cursor: next sequence to examine (cb) and its first position (cs); only these and
+  // the tile count stay live while a segment runs
+  int cb = 0, cs = 0, done = 0;
+  while (cb < p.B && cs < hi) {
+    const int n = cb + lane < p.B ? tiles_of(p.seq_lens, cb + lane, p.T_max) : 0;
+    const int u = n > 0 ? n + kMlaSegCost : 0;
+    int incl = u;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(kAll, incl, o);
+      if (lane >= o) incl += t;
     }
-    s = e;
+    const int first = cs + (incl - u) + kMlaSegCost;  // position of this lane's tile 0
+    const int a = max(lo - first, 0), e = min(hi - first, n);
+    const unsigned m = __ballot_sync(kAll, n > 0 && e > a);
+    if (!m) {  // nothing of this range among these 32 sequences
+      cs += __shfl_sync(kAll, incl, 31);
+      cb += 32;
+      continue;
+    }
+    const int j = __ffs(m) - 1;
+    const int t0 = __shfl_sync(kAll, a, j), t1 = __shfl_sync(kAll, e, j);
+    const int more = __shfl_sync(kAll, static_cast<int>(hi > first + e), j);
+    const int b = cb + j;
+    cs += __shfl_sync(kAll, incl, j);
+    cb = b + 1;
+    fn(b, t0, t1, done, more && cb < p.B ? cb : -1);
+    done += t1 - t0;
   }
 }
 
@@ -206,20 +236,26 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
     if (lane == 0) {
       prefetch_tmap(tmKV);
       prefetch_tmap(tmPE);
-      int g = 0;
-      bool ok = true;
-      for_each_segment(p, pair, [&](int b, int t0, int t1, int) {
-        for (int t = t0; t < t1 && ok; ++t, ++g) {
-          const int s = g % NST;
-          if (!mbar_wait(&kv_empty[s], ((g / NST) & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
-          uint8_t* dst = sKV + s * STAGE;
-          mbar_arrive_expect_tx(&kv_full[s], STAGE);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) tma_load_3d(dst + c * KV_BOX, tmKV, &kv_full[s], R * 256 + c * 64, t * TN, b);
-          tma_load_3d(dst + 4 * KV_BOX, tmPE, &kv_full[s], R * 32, t * TN, b);
-        }
-      });
     }
+    int g = 0;
+    bool ok = true;
+    for_each_segment(p, pair, [&](int b, int t0, int t1, int, int) {
+      for (int t = t0; t < t1 && ok; ++t, ++g) {
+        if (lane == 0) {
+          const int s = g % NST;
+          if (!mbar_wait(&kv_empty[s], ((g / NST) & 1) ^ 1, abort_flag, p.status)) {
+            ok = false;
+          } else {
+            uint8_t* dst = sKV + s * STAGE;
+            mbar_arrive_expect_tx(&kv_full[s], STAGE);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tma_load_3d(dst + c * KV_BOX, tmKV, &kv_full[s], R * 256 + c * 64, t * TN, b);
+            tma_load_3d(dst + 4 * KV_BOX, tmPE, &kv_full[s], R * 32, t * TN, b);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+      }
+    });
   } else if (warp == 9 || warp == 10) {
     // ------------------------------ MMA issuers (whole warps): 9 = scores, 10 = P V
     constexpr uint32_t HI128 = sdesc_hi_sw128(1024);
@@ -229,7 +265,7 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
       constexpr uint32_t HI64 = sdesc_hi_sw64(512);
       constexpr uint32_t idesc_s = idesc_f32acc(1, 128, TN, false, false);
       const uint32_t kv_lo_k = sdesc_lo(smem_u32(sKV), 16);
-      for_each_segment(p, pair, [&](int, int t0, int t1, int g0) {
+      for_each_segment(p, pair, [&](int, int t0, int t1, int g0, int) {
         if (!ok) return;
         if (!(ok = mbar_wait_warp(q_ready, seg & 1, abort_flag, p.status))) return;
         ++seg;
@@ -258,7 +294,7 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
     } else {
       constexpr uint32_t idesc_o = idesc_f32acc(1, 128, 256, false, true);
       const uint32_t kv_lo_v = sdesc_lo(smem_u32(sKV), KV_BOX);  // MN-major: 64-column blocks KV_BOX apart
-      for_each_segment(p, pair, [&](int, int t0, int t1, int g0) {
+      for_each_segment(p, pair, [&](int, int t0, int t1, int g0, int) {
         if (!ok) return;
         for (int i = 0; ok && i < t1 - t0; ++i) {
           const int k = g0 + i;
@@ -289,7 +325,7 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
     const uint32_t peer_full = mapa_peer(smem_u32(&x_full[q]), PEER);
     const uint32_t send_src = smem_u32(xsend + q * 2 * 32 * HALF);
     bool ok = true;
-    for_each_segment(p, pair, [&](int, int t0, int t1, int g0) {
+    for_each_segment(p, pair, [&](int, int t0, int t1, int g0, int) {
       for (int i = 0; ok && i < t1 - t0; ++i) {
         const int k = g0 + i;
         // S(k) out of TMEM; the buffer may then take S(k + 1)
@@ -305,7 +341,6 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
         // what it received of tile k - 1 (its copy had landed, so the staging block was read)
         if (!(ok = mbar_wait_warp(&own_free[q], (k & 1) ^ 1, abort_flag, p.status))) break;
         if (!(ok = mbar_wait_warp(&x_empty[q], (k & 1) ^ 1, abort_flag, p.status))) break;
-        if (lane == 0) mbar_arrive_expect_tx(&x_full[q], XCHUNK);  // receive tile k from the peer
 #pragma unroll
         for (int c = 0; c < HALF / 4; ++c) {
           const int cc = 4 * ((c + lane) & (HALF / 4 - 1));
@@ -313,9 +348,16 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
           *reinterpret_cast<uint4*>(stage + 32 * HALF + cc) =
               make_uint4(r1[4 * c], r1[4 * c + 1], r1[4 * c + 2], r1[4 * c + 3]);
         }
-        fence_proxy_async_smem();
+        fence_proxy_async_smem();  // the bulk copy reads the staged block through the async proxy
+        __threadfence_block();     // and this CTA's softmax warps read it once x_full completes
         __syncwarp();
-        if (lane == 0) bulk_copy_to_peer(peer_recv, send_src, XCHUNK, peer_full);
+        if (lane == 0) {
+          // x_full(k) completes on this arrive and the peer's bytes, in either order; the
+          // arrive comes after the own block is staged, since the softmax warps read both
+          // parts as soon as the phase completes
+          mbar_arrive_expect_tx(&x_full[q], XCHUNK);
+          bulk_copy_to_peer(peer_recv, send_src, XCHUNK, peer_full);
+        }
       }
     });
   } else {
@@ -335,7 +377,7 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
       return !alive;
     };
     int seg = 0;
-    for_each_segment(p, pair, [&](int b, int t0, int t1, int g0) {
+    for_each_segment(p, pair, [&](int b, int t0, int t1, int g0, int b_next) {
       if (!alive) return;
       const int n = t1 - t0;
       // Q_r of sequence b into TMEM (bf16 pairs are already in the operand layout). Every
@@ -366,6 +408,15 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(q_ready);
+        if (b_next >= 0) {  // the next segment's Q rows into L2 while this one runs
+          const char* nx = reinterpret_cast<const char*>(reinterpret_cast<const __nv_bfloat16*>(p.q_nope) +
+                                                         (static_cast<size_t>(b_next) * kH + h) * kDc + R * 256 + w * 128);
+          prefetch_l2(nx);
+          prefetch_l2(nx + 128);
+          if (w == 1)
+            prefetch_l2(reinterpret_cast<const __nv_bfloat16*>(p.q_pe) + (static_cast<size_t>(b_next) * kH + h) * kDr +
+                        R * 32);
+        }
       }
       const int L = min(max(__ldg(p.seq_lens + b), 0), p.T_max);
       float m_run = -INFINITY, l_run = 0.f;
@@ -384,11 +435,6 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
           s[4 * c + 2] = R == 0 ? o.z + v.z : v.z + o.z;
           s[4 * c + 3] = R == 0 ? o.w + v.w : v.w + o.w;
         }
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&own_free[q]);
-          mbar_arrive_remote_relaxed(peer_empty);
-        }
         const int valid = L - (t0 + i) * TN - w * HALF;  // tokens of this half inside the sequence
         if (valid < HALF) {
 #pragma unroll
@@ -403,9 +449,18 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
         }
         mx0 = fmaxf(mx0, s[HALF - 2]);
         mx1 = fmaxf(mx1, s[HALF - 1]);
+        const float mxh = fmaxf(mx0, mx1);
+        // The half maximum depends on every value this lane read from both blocks, and the
+        // ballot on it on every lane's: past it, the whole warp's reads have returned and
+        // both blocks may be given back (the predicate is always true: fmaxf never yields
+        // that NaN payload).
+        if (__ballot_sync(0xffffffffu, __float_as_uint(mxh) != 0x7fc00001u) != 0u && lane == 0) {
+          mbar_arrive(&own_free[q]);
+          mbar_arrive_remote_relaxed(peer_empty);
+        }
         // the other half's maximum (warp q + 4 or q - 4 holds the same heads)
         float* mslot = mx_sh + (k & 1) * 2 * kH;
-        mslot[w * kH + h] = fmaxf(mx0, mx1);
+        mslot[w * kH + h] = mxh;
         mbar_arrive(&mx_bar[q]);
         if (fail(mbar_wait(&mx_bar[q], k & 1, abort_flag, p.status))) return;
         const float m_tile = fmaxf(mslot[h], mslot[kH + h]) * sl2;
@@ -484,17 +539,31 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
       const float l_tot = lslot[h] + lslot[kH + h];
       const int slot = pair + b;
       const float inv_l = 1.f / l_tot;
-      float* orow = p.part_o + (static_cast<size_t>(slot) * kH + h) * kDc + R * 256 + w * 128;
+      // O / l leaves through this warp's 4 KB block of the staging area, transposed so that
+      // each store instruction writes four whole 128-byte row pieces. The block is idle
+      // from here to the next segment's first score tile, once the peer has consumed the
+      // last tile (the copy out of it has completed).
+      if (fail(mbar_wait(&x_empty[q], k_last & 1, abort_flag, p.status))) return;
+      float* stg = xsend + (q * 2 + w) * 32 * HALF;
+      float* obase = p.part_o + (static_cast<size_t>(slot) * kH + q * 32) * kDc + R * 256 + w * 128;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t r[32];
         tmem_ld32(t_lane + O_COL + w * 128 + c * 32, r);
         tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(orow + c * 32 + e) =
-              make_float4(__uint_as_float(r[e]) * inv_l, __uint_as_float(r[e + 1]) * inv_l,
-                          __uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
+        for (int j = 0; j < 8; ++j)  // row `lane`, 16-byte chunk j at slot j ^ (lane & 7)
+          *reinterpret_cast<float4*>(stg + lane * 32 + 4 * (j ^ (lane & 7))) =
+              make_float4(__uint_as_float(r[4 * j]) * inv_l, __uint_as_float(r[4 * j + 1]) * inv_l,
+                          __uint_as_float(r[4 * j + 2]) * inv_l, __uint_as_float(r[4 * j + 3]) * inv_l);
+        __syncwarp();
+#pragma unroll 1
+        for (int i = 0; i < 8; ++i) {  // rows 4i .. 4i + 3, eight lanes per row
+          const int rr = 4 * i + (lane >> 3), j = lane & 7;
+          *reinterpret_cast<float4*>(obase + static_cast<size_t>(rr) * kDc + c * 32 + 4 * j) =
+              *reinterpret_cast<const float4*>(stg + rr * 32 + 4 * (j ^ (rr & 7)));
+        }
+        __syncwarp();
       }
       if (R == 0 && w == 0) p.part_lse[static_cast<size_t>(slot) * kH + h] = (m_run + log2f(l_tot)) * 0.69314718055994531f;
       tc_fence_before();  // O reads are complete before the next segment's P V overwrites O

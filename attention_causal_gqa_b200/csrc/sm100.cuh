@@ -248,6 +248,9 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, v
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, status));
 }
 
+// Fetch the 128-byte line holding p into L2 (no register result, no completion to wait for).
+__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
 // ------------------------------------------------------------------ math bits
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
