@@ -70,16 +70,6 @@ static_assert(Q_COL + 144 <= S_COL && S_COL + TN <= P_COL && P_COL + TN / 2 <= T
 static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ uint32_t mapa_peer(uint32_t saddr, uint32_t peer) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(peer));
-  return r;
-}
 // One bulk copy of a staged block from this CTA's shared memory into the peer's,
 // completing its bytes on the peer's mbarrier.
 __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
@@ -95,9 +85,6 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t
 // peer can learn that the block may be overwritten.
 __device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t bar_cluster_addr) {
   asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
-}
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ int tiles_of(const int32_t* lens, int b, int T_max) {

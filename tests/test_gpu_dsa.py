@@ -101,6 +101,19 @@ def test_index_scores_and_selection(lens, T, HI, top_k):
 
 
 @cuda
+def test_many_short_sequences():
+    """300 sequences of 0-700 tokens: the indexer's CTAs each walk many sequences (a new
+    Q and head weights per segment) and the top-k clusters meet every short-sequence case."""
+    from attention_causal_gqa_b200.synthetic import dsa_inputs
+    rng = np.random.default_rng(12)
+    lens = rng.integers(0, 701, 300).tolist()
+    d = dsa_inputs(len(lens), 128, 512, 64, 32, 128, seq_lens=lens, T_max=704, seed=12, device="cuda")
+    scores, idx = _index(d, 64)
+    _check_scores(d, scores)
+    _check_selection(scores, idx, lens, 64)
+
+
+@cuda
 def test_selection_ties_take_the_smaller_index():
     """Identical key rows give bit-identical scores; the kept ones must be the earliest."""
     from attention_causal_gqa_b200.synthetic import dsa_inputs
@@ -177,11 +190,11 @@ def test_dsa_full_size_sampled():
 
 @cuda
 def test_selection_past_the_shared_memory_staging_limit():
-    """Sequences longer than the top-k kernel stages in shared memory (48K tokens) take the
-    path that re-reads the scores on every pass."""
+    """A cache longer than the top-k kernel stages in shared memory (four slices of at most
+    48,128 tokens per sequence) takes the path that re-reads the scores on every pass."""
     from attention_causal_gqa_b200.synthetic import dsa_inputs
-    lens = [50000, 7000]
-    d = dsa_inputs(2, 128, 512, 64, 64, 128, seq_lens=lens, T_max=50000, seed=99, device="cuda")
+    lens = [200000, 7000]
+    d = dsa_inputs(2, 128, 512, 64, 64, 128, seq_lens=lens, T_max=200000, seed=99, device="cuda")
     scores, idx = _index(d, 2048)
     _check_scores(d, scores, rows=[0])
     _check_selection(scores, idx, lens, 2048)
