@@ -148,6 +148,7 @@ __global__ void kv_append_kernel(const uint4* __restrict__ k_new, const uint4* _
 __global__ void kv_gather_kernel(const uint4* __restrict__ k_pages, const uint4* __restrict__ v_pages,
                                  uint4* __restrict__ k_op, uint4* __restrict__ v_op, ChunkGeometry g, int Sk_max,
                                  int* __restrict__ status) {
+  griddep_wait();  // launched as a dependent of the cache append
   const int cpr = g.D / 8;
   const long long n = static_cast<long long>(g.B) * g.Hkv * Sk_max * cpr;
   bool in_range = true;
@@ -178,6 +179,7 @@ __global__ void kv_gather_kernel(const uint4* __restrict__ k_pages, const uint4*
 // Rows [B * Hq, S_new, D] of new queries, rotated at cache_lens[b] + i into fp16.
 __global__ void rope_rows_f16_kernel(const uint4* __restrict__ x, uint4* __restrict__ y, const float2* __restrict__ cs,
                                      ChunkGeometry g, int Hq, float* __restrict__ lse, int* __restrict__ status) {
+  griddep_wait();  // launched as a dependent of the cache gather
   const int cpr = g.D / 8;
   const int n = g.B * Hq * g.S_new * cpr;
   bool in_range = true;
@@ -225,18 +227,16 @@ cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* k_pages
 cudaError_t launch_kv_gather(const void* k_pages, const void* v_pages, void* k_op, void* v_op, const ChunkGeometry& g,
                              int Sk_max, int* status, cudaStream_t stream) {
   const long long n = static_cast<long long>(g.B) * g.Hkv * Sk_max * (g.D / 8);
-  kv_gather_kernel<<<grid_for(n, 256), 256, 0, stream>>>(static_cast<const uint4*>(k_pages),
-                                                         static_cast<const uint4*>(v_pages), static_cast<uint4*>(k_op),
-                                                         static_cast<uint4*>(v_op), g, Sk_max, status);
-  return cudaGetLastError();
+  return launch_pdl(kv_gather_kernel, dim3(grid_for(n, 256)), dim3(256), 0, stream, static_cast<const uint4*>(k_pages),
+                    static_cast<const uint4*>(v_pages), static_cast<uint4*>(k_op), static_cast<uint4*>(v_op), g, Sk_max,
+                    status);
 }
 
 cudaError_t launch_rope_rows_f16(const void* q, void* q_f16, const float2* cs, const ChunkGeometry& g, int Hq,
                                  float* lse, int* status, cudaStream_t stream) {
   const long long n = static_cast<long long>(g.B) * Hq * g.S_new * (g.D / 8);
-  rope_rows_f16_kernel<<<grid_for(n, 256), 256, 0, stream>>>(static_cast<const uint4*>(q), static_cast<uint4*>(q_f16),
-                                                             cs, g, Hq, lse, status);
-  return cudaGetLastError();
+  return launch_pdl(rope_rows_f16_kernel, dim3(grid_for(n, 256)), dim3(256), 0, stream, static_cast<const uint4*>(q),
+                    static_cast<uint4*>(q_f16), cs, g, Hq, lse, status);
 }
 
 }  // namespace attn

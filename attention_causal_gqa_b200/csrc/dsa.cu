@@ -282,6 +282,7 @@ template <bool SMEM>
 __global__ void __cluster_dims__(kTopkCluster, 1, 1) __launch_bounds__(kTopkThreads)
     dsa_topk_kernel(const float* __restrict__ scores, const int32_t* __restrict__ seq_lens, int32_t* __restrict__ idx,
                     int T_max, int top_k) {
+  griddep_wait();  // launched as a dependent of the indexer
   extern __shared__ uint32_t skeys[];
   __shared__ unsigned whist[kTopkThreads / 32][256];  // one histogram per warp, summed into hist
   __shared__ unsigned hist[2][256];                   // this CTA's histogram of a pass (pass parity), read by the cluster
@@ -555,11 +556,9 @@ cudaError_t launch_dsa_topk(const float* scores, const int32_t* seq_lens, int32_
     const int smem = slice * static_cast<int>(sizeof(uint32_t));
     cudaError_t e = cudaFuncSetAttribute(dsa_topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    dsa_topk_kernel<true><<<grid, kTopkThreads, smem, stream>>>(scores, seq_lens, idx, T_max, top_k);
-  } else {
-    dsa_topk_kernel<false><<<grid, kTopkThreads, 0, stream>>>(scores, seq_lens, idx, T_max, top_k);
+    return launch_pdl(dsa_topk_kernel<true>, grid, dim3(kTopkThreads), smem, stream, scores, seq_lens, idx, T_max, top_k);
   }
-  return cudaGetLastError();
+  return launch_pdl(dsa_topk_kernel<false>, grid, dim3(kTopkThreads), 0, stream, scores, seq_lens, idx, T_max, top_k);
 }
 
 cudaError_t launch_dsa_gather(const void* kv, const void* pe, const int32_t* idx, const int32_t* seq_lens,

@@ -5,7 +5,30 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <utility>
+
 namespace attn {
+
+// Launches kernel with programmatic dependent launch allowed: its launch overlaps the end
+// of the previous kernel on the stream, so every kernel launched this way calls
+// griddep_wait() before its first memory access. No kernel here triggers its dependents
+// early: a dependent is scheduled only once every CTA of its predecessor has exited, so
+// it can never hold resources that a not-yet-running CTA of the predecessor needs.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 struct PrefillParams {
   void* out;              // [B, Hq, S, D] (T)

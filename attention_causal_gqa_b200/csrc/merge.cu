@@ -9,6 +9,7 @@
 #include <cuda_bf16.h>
 
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace attn {
 
@@ -16,6 +17,7 @@ namespace attn {
 __global__ void merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
                              const int32_t* __restrict__ seq_lens, __nv_bfloat16* __restrict__ out,
                              float* __restrict__ lse, int B, int H, int D, int n_splits, int tokens_per_split) {
+  griddep_wait();  // launched as a dependent of the kernel that wrote the partials
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (gw >= B * H) return;
@@ -88,10 +90,8 @@ cudaError_t launch_merge(const float* part_o, const float* part_lse, const int32
   const long long warps = static_cast<long long>(B) * H;
   const int threads = 256;
   const long long blocks = (warps * 32 + threads - 1) / threads;
-  merge_kernel<<<static_cast<int>(blocks), threads, 0, stream>>>(part_o, part_lse, seq_lens,
-                                                                 static_cast<__nv_bfloat16*>(out), lse, B, H, D,
-                                                                 n_splits, tokens_per_split);
-  return cudaGetLastError();
+  return launch_pdl(merge_kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, stream, part_o, part_lse,
+                    seq_lens, static_cast<__nv_bfloat16*>(out), lse, B, H, D, n_splits, tokens_per_split);
 }
 
 // ------------------------------------------------------------ parts merge
@@ -179,6 +179,7 @@ template <int DIM, int UNIT, int SEG>
 __global__ void range_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
                                    const int32_t* __restrict__ seq_lens, __nv_bfloat16* __restrict__ out,
                                    float* __restrict__ lse, int B, int H, int T_max, int n_ranges) {
+  griddep_wait();  // launched as a dependent of the kernel that wrote the partials
   constexpr int VEC = DIM / 32;  // contiguous columns per lane
   static_assert(VEC % 4 == 0, "whole float4 columns per lane");
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -258,9 +259,8 @@ static cudaError_t launch_range_merge(const float* part_o, const float* part_lse
   const long long warps = static_cast<long long>(B) * H;
   const int threads = 256;
   const long long blocks = (warps * 32 + threads - 1) / threads;
-  range_merge_kernel<DIM, UNIT, SEG><<<static_cast<int>(blocks), threads, 0, stream>>>(
-      part_o, part_lse, seq_lens, static_cast<__nv_bfloat16*>(out), lse, B, H, T_max, n_ranges);
-  return cudaGetLastError();
+  return launch_pdl(range_merge_kernel<DIM, UNIT, SEG>, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, stream,
+                    part_o, part_lse, seq_lens, static_cast<__nv_bfloat16*>(out), lse, B, H, T_max, n_ranges);
 }
 
 cudaError_t launch_mla_merge(const float* part_o, const float* part_lse, const int32_t* seq_lens, void* out,

@@ -572,6 +572,7 @@ __device__ __forceinline__ void mla_body(const MlaParams& p, const CUtensorMap* 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMlaThreads, 1)
     mla_kernel(const __grid_constant__ MlaParams p, const __grid_constant__ CUtensorMap tmKV,
                const __grid_constant__ CUtensorMap tmPE) {
+  griddep_wait();  // (a dependent of the row gather in the sparse form)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   mla_body(p, &tmKV, &tmPE, smem, static_cast<int>(cluster_ctarank()));
@@ -588,8 +589,7 @@ int mla_pairs_for_device() {
 cudaError_t launch_mla(const MlaParams& p, const CUtensorMap& tmKV, const CUtensorMap& tmPE, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  mla_kernel<<<2 * p.n_pairs, kMlaThreads, SMEM_BYTES, stream>>>(p, tmKV, tmPE);
-  return cudaGetLastError();
+  return launch_pdl(mla_kernel, dim3(2 * p.n_pairs), dim3(kMlaThreads), SMEM_BYTES, stream, p, tmKV, tmPE);
 }
 
 }  // namespace attn

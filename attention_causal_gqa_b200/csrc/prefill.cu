@@ -160,6 +160,7 @@ template <int D, int BN, int MODE>
 __global__ void __launch_bounds__(320, 1)
     prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
                    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
+  griddep_wait();  // launched as a dependent of the operand prologue
   using Sh = PrefillShape<D, BN, MODE>;
   using TIn = typename std::conditional<MODE == kModeSplit, float, __nv_bfloat16>::type;
   constexpr int NP = Sh::NPART;
@@ -554,8 +555,7 @@ static cudaError_t launch_prefill_t(const PrefillParams& p, const CUtensorMap& t
   auto kern = prefill_kernel<D, BN, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sh::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  kern<<<grid, 320, Sh::SMEM_BYTES, stream>>>(p, tmQ, tmK, tmV);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(320), Sh::SMEM_BYTES, stream, p, tmQ, tmK, tmV);
 }
 
 int prefill_block_n(int D, bool f32) {

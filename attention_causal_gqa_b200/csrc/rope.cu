@@ -19,6 +19,7 @@
 
 #include "kernels.h"
 #include "prologue.h"
+#include "sm100.cuh"
 
 namespace attn {
 
@@ -89,6 +90,7 @@ __device__ __forceinline__ void load_cs8(const float2* __restrict__ cs, int pos,
 template <int CPR, bool HALF>
 __global__ void __launch_bounds__(256) split_f32_kernel(const float4* __restrict__ x, uint4* __restrict__ out,
                                                         const float2* __restrict__ cs, int heads, int S) {
+  griddep_wait();  // launched as a dependent of the cos/sin table
   int pos, c;
   if (!chunk_position<CPR>(S, pos, c)) return;
   if (HALF && c >= CPR / 2) return;
@@ -282,12 +284,11 @@ cudaError_t launch_split_f32(const float* x, void* out, const float2* cs, long l
   const float4* xx = reinterpret_cast<const float4*>(x);
   uint4* o = static_cast<uint4*>(out);
   const int h = static_cast<int>(heads);
-  if (D == 64 && half_split) split_f32_kernel<8, true><<<grid, 256, 0, stream>>>(xx, o, cs, h, S);
-  else if (D == 64) split_f32_kernel<8, false><<<grid, 256, 0, stream>>>(xx, o, cs, h, S);
-  else if (D == 128 && half_split) split_f32_kernel<16, true><<<grid, 256, 0, stream>>>(xx, o, cs, h, S);
-  else if (D == 128) split_f32_kernel<16, false><<<grid, 256, 0, stream>>>(xx, o, cs, h, S);
-  else return cudaErrorInvalidValue;
-  return cudaGetLastError();
+  if (D == 64 && half_split) return launch_pdl(split_f32_kernel<8, true>, grid, dim3(256), 0, stream, xx, o, cs, h, S);
+  if (D == 64) return launch_pdl(split_f32_kernel<8, false>, grid, dim3(256), 0, stream, xx, o, cs, h, S);
+  if (D == 128 && half_split) return launch_pdl(split_f32_kernel<16, true>, grid, dim3(256), 0, stream, xx, o, cs, h, S);
+  if (D == 128) return launch_pdl(split_f32_kernel<16, false>, grid, dim3(256), 0, stream, xx, o, cs, h, S);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace attn
