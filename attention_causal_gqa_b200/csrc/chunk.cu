@@ -144,7 +144,11 @@ __global__ void kv_append_kernel(const uint4* __restrict__ k_new, const uint4* _
   }
 }
 
-// One thread per 8-element chunk of the contiguous operands [B * Hkv, Sk_max, D].
+constexpr int kChunkKeyBlock = 128;  // key rows per block of the prefill kernel in the chunk path
+
+// One thread per 8-element chunk of the contiguous operands [B * Hkv, Sk_max, D]; rows of a
+// sequence past its last 128-key block are left as they are (the prefill kernel never
+// loads them), rows between its length and that block's end become zeros.
 __global__ void kv_gather_kernel(const uint4* __restrict__ k_pages, const uint4* __restrict__ v_pages,
                                  uint4* __restrict__ k_op, uint4* __restrict__ v_op, ChunkGeometry g, int Sk_max,
                                  int* __restrict__ status) {
@@ -152,26 +156,49 @@ __global__ void kv_gather_kernel(const uint4* __restrict__ k_pages, const uint4*
   const int cpr = g.D / 8;
   const long long n = static_cast<long long>(g.B) * g.Hkv * Sk_max * cpr;
   bool in_range = true;
-  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < n;
-       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int c = static_cast<int>(idx % cpr);
-    const long long r = idx / cpr;
-    const int j = static_cast<int>(r % Sk_max);
-    const int z = static_cast<int>(r / Sk_max), b = z / g.Hkv, kvh = z % g.Hkv;
-    const int Sk_b = clamp_len(g.cache_lens, b, g.max_cache_len, status) + new_len(g, b, status);
-    uint4 kq = make_uint4(0, 0, 0, 0), vq = make_uint4(0, 0, 0, 0);
-    if (j < Sk_b) {
-      const int page = page_of(g.block_table, b, j / g.page_size, g.max_pages, g.num_pages, status);
-      if (page >= 0) {
-        const size_t src = ((static_cast<size_t>(page) * g.page_size + j % g.page_size) * g.Hkv + kvh) * cpr + c;
-        float f[8];
-        rotate8(k_pages[src], nullptr, 0, c, g.D, f);
-        kq = pack8_f16_checked(f, in_range);
-        vq = v_pages[src];
+  // four chunks per step, all page loads issued before any store (more bytes in flight)
+  constexpr int kUnroll = 4;
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long base = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; base < n;
+       base += kUnroll * stride) {
+    uint4 kr[kUnroll], vr[kUnroll];
+    bool have[kUnroll], wr[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const long long idx = base + u * stride;
+      have[u] = wr[u] = false;
+      if (idx >= n) continue;
+      const int c = static_cast<int>(idx % cpr);
+      const long long r = idx / cpr;
+      const int j = static_cast<int>(r % Sk_max);
+      const int z = static_cast<int>(r / Sk_max), b = z / g.Hkv, kvh = z % g.Hkv;
+      const int Sk_b = clamp_len(g.cache_lens, b, g.max_cache_len, status) + new_len(g, b, status);
+      // rows past the sequence's last 128-key block are never loaded by the prefill kernel
+      wr[u] = j < ((Sk_b + kChunkKeyBlock - 1) / kChunkKeyBlock) * kChunkKeyBlock;
+      if (j < Sk_b) {
+        const int page = page_of(g.block_table, b, j / g.page_size, g.max_pages, g.num_pages, status);
+        if (page >= 0) {
+          const size_t src = ((static_cast<size_t>(page) * g.page_size + j % g.page_size) * g.Hkv + kvh) * cpr + c;
+          kr[u] = k_pages[src];
+          vr[u] = v_pages[src];
+          have[u] = true;
+        }
       }
     }
-    k_op[idx] = kq;
-    v_op[idx] = vq;
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const long long idx = base + u * stride;
+      if (!wr[u]) continue;
+      uint4 kq = make_uint4(0, 0, 0, 0), vq = make_uint4(0, 0, 0, 0);
+      if (have[u]) {
+        float f[8];
+        rotate8(kr[u], nullptr, 0, static_cast<int>(idx % cpr), g.D, f);
+        kq = pack8_f16_checked(f, in_range);
+        vq = vr[u];
+      }
+      k_op[idx] = kq;
+      v_op[idx] = vq;
+    }
   }
   if (!in_range) atomicOr(status, kDevErrRange);
 }

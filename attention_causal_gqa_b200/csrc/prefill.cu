@@ -571,6 +571,7 @@ cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmQ, const
     return cudaErrorInvalidValue;
   }
   if (rope) {
+    // (the chunk path leaves its operand rows past a sequence's last 128-key block unwritten)
     if (D == 128) return launch_prefill_t<128, 128, kModeF16QK>(p, tmQ, tmK, tmV, grid, stream);
     if (D == 64) return launch_prefill_t<64, 128, kModeF16QK>(p, tmQ, tmK, tmV, grid, stream);
   } else {

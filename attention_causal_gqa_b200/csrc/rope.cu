@@ -186,35 +186,51 @@ __global__ void __launch_bounds__(256) rope_qk_kernel(const uint4* __restrict__ 
 #pragma unroll
   for (int e = 0; e < NPAIR; ++e) a[e] = cos_sin_of(pos, f.inv[NPAIR * c + e]);
   bool in_range = true;
-  for (int hd = blockIdx.y; hd < hq + hk; hd += gridDim.y) {
-    const bool isq = hd < hq;
-    const uint4* x = isq ? q : k;
-    uint4* y = isq ? qo : ko;
-    const size_t idx = (static_cast<size_t>(isq ? hd : hd - hq) * S + pos) * CPR + c;
-    if (!HALF) {
-      const uint4 raw = x[idx];
-      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-      uint32_t ow[4];
+  // kUnroll heads per step, all loads issued before any store, so each thread keeps
+  // kUnroll (x2 for HALF) 16-byte loads in flight
+  constexpr int kUnroll = 4;
+  const int H = hq + hk;
+  for (int hd0 = blockIdx.y; hd0 < H; hd0 += kUnroll * gridDim.y) {
+    uint4 rl[kUnroll], rh[kUnroll];
+    size_t ix[kUnroll];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float x0 = __uint_as_float(w[e] << 16), x1 = __uint_as_float(w[e] & 0xFFFF0000u);
-        ow[e] = pack_operand<BF16>(x0 * a[e].x - x1 * a[e].y, x0 * a[e].y + x1 * a[e].x, in_range);
-      }
-      y[idx] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-    } else {
-      const uint4 rl = x[idx], rh = x[idx + CPR / 2];
-      const uint32_t wl[4] = {rl.x, rl.y, rl.z, rl.w}, wh[4] = {rh.x, rh.y, rh.z, rh.w};
-      uint32_t ol[4], oh[4];
+    for (int u = 0; u < kUnroll; ++u) {
+      const int hd = hd0 + u * gridDim.y;
+      if (hd >= H) continue;
+      const bool isq = hd < hq;
+      ix[u] = (static_cast<size_t>(isq ? hd : hd - hq) * S + pos) * CPR + c;
+      const uint4* x = isq ? q : k;
+      rl[u] = x[ix[u]];
+      if (HALF) rh[u] = x[ix[u] + CPR / 2];
+    }
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float l0 = __uint_as_float(wl[e] << 16), l1 = __uint_as_float(wl[e] & 0xFFFF0000u);
-        const float h0 = __uint_as_float(wh[e] << 16), h1 = __uint_as_float(wh[e] & 0xFFFF0000u);
-        const float2 c0 = a[2 * e], c1 = a[2 * e + 1];
-        ol[e] = pack_operand<BF16>(l0 * c0.x - h0 * c0.y, l1 * c1.x - h1 * c1.y, in_range);
-        oh[e] = pack_operand<BF16>(l0 * c0.y + h0 * c0.x, l1 * c1.y + h1 * c1.x, in_range);
+    for (int u = 0; u < kUnroll; ++u) {
+      const int hd = hd0 + u * gridDim.y;
+      if (hd >= H) continue;
+      uint4* y = hd < hq ? qo : ko;
+      if (!HALF) {
+        const uint32_t w[4] = {rl[u].x, rl[u].y, rl[u].z, rl[u].w};
+        uint32_t ow[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float x0 = __uint_as_float(w[e] << 16), x1 = __uint_as_float(w[e] & 0xFFFF0000u);
+          ow[e] = pack_operand<BF16>(x0 * a[e].x - x1 * a[e].y, x0 * a[e].y + x1 * a[e].x, in_range);
+        }
+        y[ix[u]] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+      } else {
+        const uint32_t wl[4] = {rl[u].x, rl[u].y, rl[u].z, rl[u].w}, wh[4] = {rh[u].x, rh[u].y, rh[u].z, rh[u].w};
+        uint32_t ol[4], oh[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float l0 = __uint_as_float(wl[e] << 16), l1 = __uint_as_float(wl[e] & 0xFFFF0000u);
+          const float h0 = __uint_as_float(wh[e] << 16), h1 = __uint_as_float(wh[e] & 0xFFFF0000u);
+          const float2 c0 = a[2 * e], c1 = a[2 * e + 1];
+          ol[e] = pack_operand<BF16>(l0 * c0.x - h0 * c0.y, l1 * c1.x - h1 * c1.y, in_range);
+          oh[e] = pack_operand<BF16>(l0 * c0.y + h0 * c0.x, l1 * c1.y + h1 * c1.x, in_range);
+        }
+        y[ix[u]] = make_uint4(ol[0], ol[1], ol[2], ol[3]);
+        y[ix[u] + CPR / 2] = make_uint4(oh[0], oh[1], oh[2], oh[3]);
       }
-      y[idx] = make_uint4(ol[0], ol[1], ol[2], ol[3]);
-      y[idx + CPR / 2] = make_uint4(oh[0], oh[1], oh[2], oh[3]);
     }
   }
   if (!in_range) atomicOr(status, 8);
@@ -256,7 +272,9 @@ cudaError_t launch_rope_qk(const void* q, void* q_op, long long q_heads, const v
   RopeFreqs f{};
   for (int i = 0; i < half; ++i) f.inv[i] = freq_scale * std::pow(theta, -2.0 * i / D);
   const int hq = static_cast<int>(q_heads), hk = static_cast<int>(k_heads);
-  const dim3 grid = operand_grid(hq + hk, S, D / 8);
+  // every thread rotates up to four heads of its chunk in one step
+  const int rpb = 256 / (D / 8);
+  const dim3 grid(static_cast<unsigned>((S + rpb - 1) / rpb), static_cast<unsigned>(std::min(65535, (hq + hk + 3) / 4)));
   const auto* xq = static_cast<const uint4*>(q);
   const auto* xk = static_cast<const uint4*>(k);
   auto* yq = static_cast<uint4*>(q_op);
