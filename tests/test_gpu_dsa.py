@@ -236,3 +236,21 @@ def test_sparse_mla_fp8_bad_index_is_flagged():
                                         d["seq_lens"], idx, SCALE, workspace=ws)
     assert binding.read_status(ws) & binding.ATTN_DEV_BAD_INDEX
     assert torch.isfinite(out.float()).all()
+
+
+@cuda
+@pytest.mark.parametrize("B,lo,hi,T_max,HI,top_k,seed", [(1, 3000, 3000, 3000, 64, 512, 51),
+                                                         (40, 0, 2500, 2600, 32, 300, 52),
+                                                         (160, 100, 400, 400, 16, 128, 53)])
+def test_index_random_layouts(B, lo, hi, T_max, HI, top_k, seed):
+    """Random batches for the persistent indexer (one sequence; some and many sequences per
+    CTA; T_max not a multiple of the 128-token tile) and the cluster top-k: sampled scores
+    against the oracle, every selection exactly the top-k of the kernel's scores."""
+    from attention_causal_gqa_b200.synthetic import dsa_inputs
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(lo, hi + 1, B).tolist()
+    d = dsa_inputs(B, 128, 512, 64, HI, 128, seq_lens=lens, T_max=T_max, seed=seed, device="cuda")
+    scores, idx = _index(d, top_k)
+    rows = sorted(set(rng.integers(0, B, 6).tolist()) | {0, B - 1})
+    _check_scores(d, scores, rows=rows)
+    _check_selection(scores, idx, lens, top_k)

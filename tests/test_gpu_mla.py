@@ -132,3 +132,30 @@ def test_mla_many_segments_deterministic_and_exact():
                                 to_np(d["kv_cache"][b:b + 1, :max(L, 1)]), to_np(d["pe_cache"][b:b + 1, :max(L, 1)]),
                                 sl[b:b + 1], SCALE)
         check(out[b:b + 1], ro, lse[b:b + 1], rl, what=f"mla segments b={b} L={L}")
+
+
+@cuda
+@pytest.mark.parametrize("B,lo,hi,T_max,seed", [(1, 1, 5000, 5000, 31), (3, 0, 200, 257, 32), (74, 0, 1500, 1500, 33),
+                                                 (150, 1, 130, 130, 34)])
+def test_mla_random_layouts(B, lo, hi, T_max, seed):
+    """Random batches (one sequence; fewer, as many as, and twice as many sequences as
+    clusters; cache lengths that are not tile multiples): sampled sequences against the
+    oracle, every output finite, empty sequences exactly 0 / -inf."""
+    from attention_causal_gqa_b200.synthetic import mla_inputs
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(lo, hi + 1, B).tolist()
+    d = mla_inputs(B, 128, 512, 64, seq_lens=lens, T_max=T_max, seed=seed, device="cuda")
+    out, lse = _run(d)
+    assert torch.isfinite(out).all()
+    for b, L in enumerate(lens):
+        if L == 0:
+            assert torch.all(out[b] == 0) and torch.all(torch.isneginf(lse[b]))
+    sl = d["seq_lens"].cpu().numpy()
+    picks = sorted(set(rng.integers(0, B, 5).tolist()) | {0, B - 1})
+    for b in picks:
+        L = int(sl[b])
+        if L == 0:
+            continue
+        ro, rl = mla_decode_ref(to_np(d["q_nope"][b:b + 1]), to_np(d["q_pe"][b:b + 1]),
+                                to_np(d["kv_cache"][b:b + 1, :L]), to_np(d["pe_cache"][b:b + 1, :L]), sl[b:b + 1], SCALE)
+        check(out[b:b + 1], ro, lse[b:b + 1], rl, what=f"mla random B={B} b={b} L={L}")
