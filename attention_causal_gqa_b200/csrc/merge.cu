@@ -13,84 +13,96 @@
 
 namespace attn {
 
-// One warp per (b, head); lanes own interleaved 4-column groups.
-__global__ void merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
-                             const int32_t* __restrict__ seq_lens, __nv_bfloat16* __restrict__ out,
-                             float* __restrict__ lse, int B, int H, int D, int n_splits, int tokens_per_split) {
+// One CTA per (sequence b, group of kMergeHeads heads); the partials of split s of b
+// are one contiguous [H, D] fp32 block, so a CTA reads a contiguous kMergeHeads x D slab
+// per split (every thread 4 consecutive columns, all splits' loads in flight in batches).
+// The split weights w = e^(lse_s - max) and their sums are formed once per head in
+// shared memory; the result is o = sum_s w_s o_s / sum_s w_s in split order
+// (deterministic), lse = max + ln sum_s w_s.
+constexpr int kMergeHeads = 8;
+constexpr int kMergeMaxSplits = 256;  // splits whose weights fit the CTA's table; the rest in a second pass
+
+__global__ void __launch_bounds__(256) merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
+                                                    const int32_t* __restrict__ seq_lens, __nv_bfloat16* __restrict__ out,
+                                                    float* __restrict__ lse, int B, int H, int D, int n_splits,
+                                                    int tokens_per_split) {
   griddep_wait();  // launched as a dependent of the kernel that wrote the partials
-  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (gw >= B * H) return;
-  const int b = gw / H, h = gw % H;
+  __shared__ float s_w[kMergeMaxSplits][kMergeHeads];
+  __shared__ float s_m[kMergeHeads], s_sum[kMergeHeads];
+  const int groups = (H + kMergeHeads - 1) / kMergeHeads;
+  const int b = blockIdx.x / groups, h0 = (blockIdx.x % groups) * kMergeHeads;
+  const int nh = min(kMergeHeads, H - h0);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int L = max(0, __ldg(seq_lens + b));
-  int ns = (L + tokens_per_split - 1) / tokens_per_split;
-  ns = min(ns, n_splits);
-  __nv_bfloat16* orow = out + static_cast<size_t>(gw) * D;
+  const int ns = min((L + tokens_per_split - 1) / tokens_per_split, n_splits);
+  // this thread's 4 columns of the slab: head h0 + hh, column d
+  const int per_head = D / 4;  // 4-column groups per head
+  const int hh = tid / per_head, d = (tid % per_head) * 4;
+  const bool active = hh < nh && tid < kMergeHeads * per_head;
   if (ns == 0) {
-    for (int d = lane * 4; d < D; d += 128) {
-      reinterpret_cast<uint2*>(orow + d)[0] = make_uint2(0u, 0u);
-    }
-    if (lane == 0) lse[gw] = -INFINITY;
+    if (active) *reinterpret_cast<uint2*>(out + (static_cast<size_t>(b) * H + h0 + hh) * D + d) = make_uint2(0u, 0u);
+    if (tid < nh) lse[static_cast<size_t>(b) * H + h0 + tid] = -INFINITY;
     return;
   }
-  const float* pl = part_lse + static_cast<size_t>(b) * n_splits * H + h;
-  float M = -INFINITY;
-  for (int s = lane; s < ns; s += 32) M = fmaxf(M, pl[static_cast<size_t>(s) * H]);
+  const float* pl = part_lse + static_cast<size_t>(b) * n_splits * H + h0;
+  // warp w < nh: the maximum and the weights of head h0 + w over the splits
+  if (warp < nh) {
+    float M = -INFINITY;
+    for (int s = lane; s < ns; s += 32) M = fmaxf(M, __ldg(pl + static_cast<size_t>(s) * H + warp));
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  float acc[16];
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float sum = 0.f;
+    for (int s = lane; s < ns; s += 32) {
+      const float w = __expf(__ldg(pl + static_cast<size_t>(s) * H + warp) - M);
+      if (s < kMergeMaxSplits) s_w[s][warp] = w;
+      sum += w;
+    }
 #pragma unroll
-  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-  // Weights first, one split per lane, then broadcast: the partial loads of the
-  // accumulation loop depend on nothing but their address and can all be in flight.
-  float wpart = 0.f;
-  for (int s0 = 0; s0 < ns; s0 += 32) {
-    const int cnt = min(32, ns - s0);
-    const float w_lane = lane < cnt ? __expf(pl[static_cast<size_t>(s0 + lane) * H] - M) : 0.f;
-    wpart += w_lane;
-    const float* po0 = part_o + ((static_cast<size_t>(b) * n_splits + s0) * H + h) * D;
-#pragma unroll 8
-    for (int i = 0; i < cnt; ++i) {
-      const float w = __shfl_sync(0xffffffffu, w_lane, i);
-      const float* po = po0 + static_cast<size_t>(i) * H * D;
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane == 0) {
+      s_m[warp] = M;
+      s_sum[warp] = sum;
+    }
+  }
+  __syncthreads();
+  if (!active) return;
+  const float* po = part_o + (static_cast<size_t>(b) * n_splits * H + h0 + hh) * D + d;
+  const size_t stride = static_cast<size_t>(H) * D;  // from one split's block to the next
+  const float Mh = s_m[hh];
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  constexpr int kBatch = 8;
+  for (int s0 = 0; s0 < ns; s0 += kBatch) {
+    float4 v[kBatch];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int d = lane * 4 + q * 128;
-        if (d < D) {
-          const float4 v = *reinterpret_cast<const float4*>(po + d);
-          acc[4 * q] += w * v.x;
-          acc[4 * q + 1] += w * v.y;
-          acc[4 * q + 2] += w * v.z;
-          acc[4 * q + 3] += w * v.w;
-        }
+    for (int u = 0; u < kBatch; ++u)
+      if (s0 + u < ns) v[u] = *reinterpret_cast<const float4*>(po + (s0 + u) * stride);
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int s = s0 + u;
+      if (s < ns) {
+        const float w = s < kMergeMaxSplits ? s_w[s][hh] : __expf(__ldg(pl + static_cast<size_t>(s) * H + hh) - Mh);
+        acc.x += w * v[u].x;
+        acc.y += w * v[u].y;
+        acc.z += w * v[u].z;
+        acc.w += w * v[u].w;
       }
     }
   }
-  float wsum = wpart;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
-  const float inv = 1.f / wsum;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int d = lane * 4 + i * 128;
-    if (d < D) {
-      const __nv_bfloat162 a = __floats2bfloat162_rn(acc[4 * i] * inv, acc[4 * i + 1] * inv);
-      const __nv_bfloat162 c = __floats2bfloat162_rn(acc[4 * i + 2] * inv, acc[4 * i + 3] * inv);
-      uint2 u;
-      u.x = *reinterpret_cast<const uint32_t*>(&a);
-      u.y = *reinterpret_cast<const uint32_t*>(&c);
-      *reinterpret_cast<uint2*>(orow + d) = u;
-    }
-  }
-  if (lane == 0) lse[gw] = M + logf(wsum);
+  const float inv = 1.f / s_sum[hh];
+  const __nv_bfloat162 a = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+  const __nv_bfloat162 c = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+  uint2 u;
+  u.x = *reinterpret_cast<const uint32_t*>(&a);
+  u.y = *reinterpret_cast<const uint32_t*>(&c);
+  *reinterpret_cast<uint2*>(out + (static_cast<size_t>(b) * H + h0 + hh) * D + d) = u;
+  if (d == 0) lse[static_cast<size_t>(b) * H + h0 + hh] = Mh + logf(s_sum[hh]);
 }
 
 cudaError_t launch_merge(const float* part_o, const float* part_lse, const int32_t* seq_lens, void* out, float* lse,
                          int B, int H, int D, int n_splits, int tokens_per_split, cudaStream_t stream) {
-  const long long warps = static_cast<long long>(B) * H;
-  const int threads = 256;
-  const long long blocks = (warps * 32 + threads - 1) / threads;
-  return launch_pdl(merge_kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, stream, part_o, part_lse,
+  if (D % 4 != 0 || kMergeHeads * (D / 4) > 256) return cudaErrorInvalidValue;
+  const long long blocks = static_cast<long long>(B) * ((H + kMergeHeads - 1) / kMergeHeads);
+  return launch_pdl(merge_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream, part_o, part_lse,
                     seq_lens, static_cast<__nv_bfloat16*>(out), lse, B, H, D, n_splits, tokens_per_split);
 }
 
