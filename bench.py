@@ -275,6 +275,89 @@ def oracle_mla_seqs(m, mp, budget_s):
                       f"float64, {dt:.2f} s of oracle time"}
 
 
+def oracle_decode_fp8_seqs(d, dp, budget_s):
+    """Times the float64 FP8 paged-decode oracle (E4M3 codes times their page scales, then
+    the decode) on whole sequences, one at a time, until ~budget_s of oracle time."""
+    import numpy as np
+    from oracle import decode_paged_fp8_ref
+    lens = d["seq_lens"].cpu().tolist()
+    dt, nbytes, nseq = 0.0, 0, 0
+    for b, L in enumerate(lens):
+        if dt > budget_s:
+            break
+        n = (L + 15) // 16
+        pages = d["block_table"][b, :n].long()
+        kc, vc = d["k_pages"][pages].cpu().numpy(), d["v_pages"][pages].cpu().numpy()
+        ks, vs = d["k_scale"][pages].cpu().numpy(), d["v_scale"][pages].cpu().numpy()
+        qb = d["q"][b:b + 1].float().cpu().numpy()
+        t0 = time.perf_counter()
+        decode_paged_fp8_ref(qb, kc, vc, ks, vs, np.arange(n, dtype=np.int64)[None, :], [L], dp["scale"])
+        dt += time.perf_counter() - t0
+        nbytes += L * dp["Hkv"] * dp["D"] * 2 + n * dp["Hkv"] * 8
+        nseq += 1
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{nseq} whole sequences of {len(lens)} ({sum(lens[:nseq])} cached tokens, all heads), "
+                      f"float64, {dt:.2f} s of oracle time"}
+
+
+def oracle_chunk_sample(d, p, budget_s):
+    """Times the float64 chunked-prefill oracle on the first sequences of the workload, one
+    KV head group at a time (its G query heads, all new rows, the whole cache), until
+    ~budget_s of oracle time; the group's pages are copied to the host first."""
+    import numpy as np
+    from oracle import chunk_prefill_ref
+    G = p["Hq"] // p["Hkv"]
+    S, D = p["S_new"], p["D"]
+    lens = d["cache_lens"].cpu().tolist()
+    dt, flops, done = 0.0, 0.0, 0
+    for b, L in enumerate(lens):
+        for kvh in range(p["Hkv"]):
+            if dt > budget_s:
+                break
+            n = (L + S + 15) // 16
+            pages = d["block_table"][b, :n].long()
+            kp = d["k_pages"][pages][:, :, kvh:kvh + 1].float().cpu().numpy()
+            vp = d["v_pages"][pages][:, :, kvh:kvh + 1].float().cpu().numpy()
+            qb = d["q"][b:b + 1, kvh * G:(kvh + 1) * G].float().cpu().numpy()
+            kb = d["k"][b:b + 1, kvh:kvh + 1].float().cpu().numpy()
+            vb = d["v"][b:b + 1, kvh:kvh + 1].float().cpu().numpy()
+            t0 = time.perf_counter()
+            chunk_prefill_ref(qb, kb, vb, kp, vp, np.arange(n, dtype=np.int64)[None, :], [L], rope_theta=p["theta"],
+                              scale=p["scale"])
+            dt += time.perf_counter() - t0
+            flops += G * 4 * D * (S * L + S * (S + 1) / 2)
+            done += 1
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{done} (sequence, kv head) groups of {len(lens) * p['Hkv']} ({G} query heads x {S} new rows "
+                      f"over the whole cache each), float64, {dt:.2f} s of oracle time"}
+
+
+def oracle_dsa_seqs(d, p, top_k, budget_s):
+    """Times the float64 oracle of the whole sparse step (indexer scores, top-k, MLA over the
+    selected tokens) on whole sequences, until ~budget_s of oracle time."""
+    from oracle import dsa_index_scores_ref, dsa_mla_decode_ref, dsa_topk_ref
+    lens = d["seq_lens"].cpu().tolist()
+    dt, tokens, nseq = 0.0, 0, 0
+    for b, L in enumerate(lens):
+        if dt > budget_s:
+            break
+        qi, wi = d["q_idx"][b:b + 1].float().cpu().numpy(), d["w_idx"][b:b + 1].float().cpu().numpy()
+        ki = d["k_idx"][b:b + 1, :L].float().cpu().numpy()
+        kv = d["kv_cache"][b:b + 1, :L].float().cpu().numpy()
+        pe = d["pe_cache"][b:b + 1, :L].float().cpu().numpy()
+        qn, qp = d["q_nope"][b:b + 1].float().cpu().numpy(), d["q_pe"][b:b + 1].float().cpu().numpy()
+        t0 = time.perf_counter()
+        sc = dsa_index_scores_ref(qi, wi, ki, [L])
+        sel = dsa_topk_ref(sc, [L], top_k)
+        dsa_mla_decode_ref(qn, qp, kv, pe, sel, p["scale"])
+        dt += time.perf_counter() - t0
+        tokens += L
+        nseq += 1
+    return {"value": tokens / dt, "unit": "cached tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{nseq} whole sequences of {len(lens)} ({tokens} cached tokens: indexer, top-{top_k}, MLA over "
+                      f"the selection, all heads), float64, {dt:.2f} s of oracle time"}
+
+
 def want_cpu(args, world, rank):
     return rank == 0 and world == 1 and not args.no_cpu_baseline
 
@@ -468,7 +551,10 @@ def bench_chunk(args, world, dev, seed, pk, pk_kind):
     flops = float(np.sum(Hq * 4 * D * (S * lens + S * (S + 1) / 2)))
     kern_avg = max_over_ranks(kern_ms / max(n_launch, 1), world)
     achieved = flops / (kern_avg * 1e-3) / 1e12
-    return {"workload": CHUNK, "value": world * flops * args.steps / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+    cpu = None
+    if want_cpu(args, world, int(os.environ.get("RANK", "0"))):
+        cpu = oracle_chunk_sample(d, p, args.cpu_budget * 0.75)
+    return {"workload": CHUNK, "cpu_baseline": cpu, "value": world * flops * args.steps / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
             "ms_per_step": ms / args.steps, "cached_tokens": int(lens.sum()), "gpu_launches": 5 * args.steps,
             "l2": "cache (1.2 GB of pages) larger than L2",
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
@@ -559,6 +645,8 @@ def bench_decode_fp8(args, world, dev, seed, pk, pk_kind):
                         "kernel": "decode_fp8_kernel",
                         "kernel_ms": k_avg, "peak_kind": f"{pk_kind} HBM copy",
                         "algorithmic": "2048 B of codes per cached token + 64 B of scales per 16-token page"}}
+    if want_cpu(args, world, int(os.environ.get("RANK", "0"))):
+        res["cpu_baseline"] = oracle_decode_fp8_seqs(d, dp, args.cpu_budget * 0.75)
     del d, out, lse, ws
     torch.cuda.empty_cache()
     return res
@@ -684,6 +772,8 @@ def bench_dsa(args, world, dev, seed, pk, pk_kind, dense_ms=None):
                         "frac": ach / pk["hbm_gbs"], "traffic": traffic_for("dsa_index_kernel"),
                         "kernel": "dsa_index_kernel", "kernel_ms": k_idx, "peak_kind": f"{pk_kind} HBM copy",
                         "algorithmic": "260 B per cached token (128 bf16 indexer key + fp32 score)"}}
+    if want_cpu(args, world, int(os.environ.get("RANK", "0"))):
+        res["cpu_baseline"] = oracle_dsa_seqs(d, p, K, args.cpu_budget * 0.75)
     del d, scores, idx, out, lse, ws1, ws2
     torch.cuda.empty_cache()
     return res
