@@ -1,5 +1,5 @@
 // Hand-written inline-PTX helpers for sm_100a: mbarriers with bounded waits,
-// TMA tensor loads (no cluster multicast anywhere in this library), tcgen05
+// TMA tensor loads (each into the issuing CTA's own shared memory only), tcgen05
 // tensor-core MMAs with TMEM accumulators, TMEM loads/stores and allocation.
 #pragma once
 #include <cstdint>

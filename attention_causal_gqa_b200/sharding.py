@@ -6,8 +6,9 @@ the ranks' partial results (outputs and LSEs) are all-gathered and combined by t
 LSE merge (attn_lse_merge) — the block-level form of the online-softmax recurrence
 ("attention study note", section "online-softmax 分块计算原理"). Prefill needs no
 exchange: its (batch, kv-head) units are independent and are dealt out in contiguous
-ranges. The only collective is one all-gather of the partials per decode step; no TMA
-multicast and no library kernel ever reads another GPU's memory.
+ranges. The only collective is one all-gather of the partials per decode step; every
+TMA load of the library reads this GPU's own memory into the issuing CTA, and no library
+kernel ever reads another GPU's memory.
 
 The partition functions are plain host code; ``split_and_merge`` runs any
 (attend, merge) pair over a torch.distributed group, so the same orchestration serves
