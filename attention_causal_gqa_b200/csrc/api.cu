@@ -73,7 +73,7 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Tiled tensor map with 128-byte swizzle; dims/strides innermost first, strides in bytes for dims 1..rank-1.
+// Tiled tensor map (128-byte swizzle unless told otherwise); dims/strides innermost first, strides in bytes for dims 1..rank-1.
 int make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const cuuint64_t* dims,
              const cuuint64_t* strides, const cuuint32_t* box, const char* what,
              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
@@ -540,7 +540,7 @@ int attn_decode_paged_fp8(const void* q, const void* k_pages, const void* v_page
     return fail(ATTN_ERR_INVALID_ARG, "sizes must be positive");
   if (Hq % Hkv != 0) return fail(ATTN_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
   if (page_size != 16) return fail(ATTN_ERR_UNSUPPORTED, "page_size %d (only 16)", page_size);
-  if (D != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d (the FP8 cache supports 128)", D);
+  if (D != 128 && D != 64) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d (the FP8 cache supports 64 and 128)", D);
   if (Hkv > 8) return fail(ATTN_ERR_UNSUPPORTED, "Hkv %d > 8", Hkv);
   if (Hq / Hkv > 16) return fail(ATTN_ERR_UNSUPPORTED, "group size %d > 16", Hq / Hkv);
   if (!aligned(q, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(out, 16) ||
@@ -569,8 +569,10 @@ int attn_decode_paged_fp8(const void* q, const void* k_pages, const void* v_page
   const cuuint64_t strides[3] = {row, static_cast<cuuint64_t>(D), 16 * row};
   const cuuint32_t box[4] = {static_cast<cuuint32_t>(D), 16, static_cast<cuuint32_t>(Hkv), 1};
   CUtensorMap tmK, tmV;
-  if ((rc = make_map(&tmK, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, k_pages, dims, strides, box, "k_pages"))) return rc;
-  if ((rc = make_map(&tmV, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, v_pages, dims, strides, box, "v_pages"))) return rc;
+  // 128-byte rows (D = 128) under the 128-byte swizzle, 64-byte rows (D = 64) under the 64-byte one
+  const CUtensorMapSwizzle swz = D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  if ((rc = make_map(&tmK, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, k_pages, dims, strides, box, "k_pages", swz))) return rc;
+  if ((rc = make_map(&tmV, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, v_pages, dims, strides, box, "v_pages", swz))) return rc;
 
   attn::DecodeParams p{};
   p.q = q;
@@ -597,8 +599,8 @@ int attn_decode_paged_fp8(const void* q, const void* k_pages, const void* v_page
   cudaError_t e = attn::launch_decode_fp8(p, tmK, tmV, &n_ranges, st);
   prof_after(st);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-  e = attn::launch_decode_range_merge(part_o, part_lse, seq_lens, out, lse, B, Hq, max_pages_per_seq * 16, n_ranges,
-                                      st);
+  e = attn::launch_decode_range_merge(part_o, part_lse, seq_lens, out, lse, B, Hq, D, max_pages_per_seq * 16,
+                                      n_ranges, st);
   if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   return ok();
 }

@@ -116,13 +116,19 @@ __device__ __forceinline__ int f8_pages_of(const DecodeParams& p, int b) {
 // ranges [N c / P, N (c + 1) / P): every CTA streams the same number of pages (+-1),
 // whatever the length mix. The producer walks its range and hands each page's
 // sequence, position and scales to the consumers with the page itself.
-template <int NH>  // 8-head column tiles: G <= 8 * NH
+// D = 128: one 128-byte swizzle row per token and head (the fragment orders above);
+// D = 64: 64-byte rows under the 64-byte swizzle (chunk x of token t stored at chunk
+// x ^ ((t >> 1) & 3)), the same orders with d = 16c + 4kt + e for the scores (one 16-byte
+// chunk per lane and token) and m-row g of m-tile t standing for d = 8g + t, row g + 8 for
+// d = 8g + 4 + t (8 code bytes per lane and token) for the output.
+template <int NH, int D>  // 8-head column tiles: G <= 8 * NH
 __global__ void __launch_bounds__(kF8Threads, 1)
     decode_fp8_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV) {
-  constexpr int D = 128;   // one 128-byte swizzle row per token and head
-  constexpr int KT = 8;    // k-steps of the score product
-  constexpr int MT = 8;    // m-tiles (16 dims each) of the output product
+  static_assert(D == 64 || D == 128, "code rows of 64 or 128 bytes");
+  constexpr int KT = D / 16;  // k-steps of the score product
+  constexpr int MT = D / 16;  // m-tiles of the output product
+  constexpr int QU = D / 32;  // 16-byte pieces of a lane's share of a query row
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int page_bytes = 16 * p.Hkv * D;  // one page of K (or V) codes, all heads
@@ -252,7 +258,7 @@ __global__ void __launch_bounds__(kF8Threads, 1)
   const int G = p.G;
   const float sl2 = p.scale_log2;
   uint32_t qf[NH][KT][2];  // Q^T (B operand of S^T) of the current sequence
-  float o[NH][MT][4];      // O^T: rows d = 16g + t (elements 0, 1) and 16g + 8 + t (2, 3),
+  float o[NH][MT][4];      // O^T: rows d = (D/8)g + t (elements 0, 1) and (D/8)g + D/16 + t (2, 3),
                            // columns heads 8j + 2c (elements 0, 2) and 8j + 2c + 1 (1, 3)
   float m[NH][2], l[NH][2];  // heads 8j + 2c + x; l sums this lane's tokens only
   for (int it = 0;; ++it) {
@@ -275,11 +281,11 @@ __global__ void __launch_bounds__(kF8Threads, 1)
 #pragma unroll
       for (int j = 0; j < NH; ++j) {
         const int row = 8 * j + g;
-        const __nv_bfloat16* qb =
-            reinterpret_cast<const __nv_bfloat16*>(p.q) + (static_cast<size_t>(b) * p.Hq + h * G + row) * D + 32 * c;
-        uint4 r[4];
+        const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(p.q) +
+                                  (static_cast<size_t>(b) * p.Hq + h * G + row) * D + (D / 4) * c;
+        uint4 r[QU];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < QU; ++i)
           r[i] = row < G ? *reinterpret_cast<const uint4*>(qb + 8 * i) : make_uint4(0, 0, 0, 0);
 #pragma unroll
         for (int kt = 0; kt < KT; ++kt) {  // words 2kt, 2kt + 1: d = 32c + 4kt + {0,1} and {2,3}
@@ -299,12 +305,21 @@ __global__ void __launch_bounds__(kF8Threads, 1)
     const int rem = L - pg * 16;  // valid tokens in this page (>= 1)
     const uint8_t* kpg = smem + s * stage_bytes + h * 16 * D;  // this head's 16 token rows
     const int g7 = g & 7;
-    // keys: d = 32c .. 32c+31 (logical 16-byte chunks 2c, 2c+1) of tokens g and g + 8
     uint4 kc[4];
-    kc[0] = *reinterpret_cast<const uint4*>(kpg + g * D + (((2 * c) ^ g7) << 4));
-    kc[1] = *reinterpret_cast<const uint4*>(kpg + g * D + (((2 * c + 1) ^ g7) << 4));
-    kc[2] = *reinterpret_cast<const uint4*>(kpg + (g + 8) * D + (((2 * c) ^ g7) << 4));
-    kc[3] = *reinterpret_cast<const uint4*>(kpg + (g + 8) * D + (((2 * c + 1) ^ g7) << 4));
+    if constexpr (D == 128) {
+      // keys: d = 32c .. 32c+31 (logical 16-byte chunks 2c, 2c+1) of tokens g and g + 8
+      kc[0] = *reinterpret_cast<const uint4*>(kpg + g * D + (((2 * c) ^ g7) << 4));
+      kc[1] = *reinterpret_cast<const uint4*>(kpg + g * D + (((2 * c + 1) ^ g7) << 4));
+      kc[2] = *reinterpret_cast<const uint4*>(kpg + (g + 8) * D + (((2 * c) ^ g7) << 4));
+      kc[3] = *reinterpret_cast<const uint4*>(kpg + (g + 8) * D + (((2 * c + 1) ^ g7) << 4));
+    } else {
+      // keys: d = 16c .. 16c+15 (logical chunk c) of tokens g and g + 8 (the same swizzle
+      // phase: (g + 8) >> 1 and g >> 1 agree in their low two bits)
+      const int sw = (g >> 1) & 3;
+      kc[0] = *reinterpret_cast<const uint4*>(kpg + g * D + ((c ^ sw) << 4));
+      kc[2] = *reinterpret_cast<const uint4*>(kpg + (g + 8) * D + ((c ^ sw) << 4));
+      kc[1] = kc[3] = make_uint4(0, 0, 0, 0);
+    }
 
     // S^T = K Q^T: rows g, g + 8 = tokens; columns 2c, 2c + 1 = heads 8j + 2c + x
     float sc[NH][4];
@@ -357,16 +372,24 @@ __global__ void __launch_bounds__(kF8Threads, 1)
           o[j][t][3] *= al[j][1];
         }
     }
-    // values: d = 16g .. 16g+15 (logical chunk g) of tokens 2c, 2c+1, 2c+8, 2c+9;
-    // tokens past the end become zeros so 0 * garbage cannot poison O
+    // values: d = 16g .. 16g+15 (D = 128: logical chunk g) or 8g .. 8g+7 (D = 64: half
+    // g & 1 of chunk g >> 1) of tokens 2c, 2c+1, 2c+8, 2c+9; tokens past the end become
+    // zeros so 0 * garbage cannot poison O
     uint4 vc[4];
     {
       const uint8_t* vpg = kpg + page_bytes;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int t = 2 * c + (i & 1) + 8 * (i >> 1);
-        vc[i] = t < rem ? *reinterpret_cast<const uint4*>(vpg + t * D + ((g ^ (t & 7)) << 4))
-                        : make_uint4(0, 0, 0, 0);
+        if constexpr (D == 128) {
+          vc[i] = t < rem ? *reinterpret_cast<const uint4*>(vpg + t * D + ((g ^ (t & 7)) << 4))
+                          : make_uint4(0, 0, 0, 0);
+        } else {
+          const uint2 w = t < rem ? *reinterpret_cast<const uint2*>(vpg + t * D + (((g >> 1) ^ ((t >> 1) & 3)) << 4) +
+                                                                    (g & 1) * 8)
+                                  : make_uint2(0, 0);
+          vc[i] = make_uint4(w.x, w.y, 0, 0);
+        }
       }
     }
     __syncwarp();
@@ -378,7 +401,7 @@ __global__ void __launch_bounds__(kF8Threads, 1)
       // bytes t, t + 1 of the two tokens interleaved: the low half pairs d = 16g + t,
       // the high half d = 16g + t + 1 (and + 8 for rows g + 8)
       const uint32_t sel = (t & 3) | ((4 + (t & 3)) << 4) | ((1 + (t & 3)) << 8) | ((5 + (t & 3)) << 12);
-      const int wl = t >> 2, wh = 2 + (t >> 2);
+      const int wl = t >> 2, wh = (D == 128 ? 2 : 1) + (t >> 2);  // words of rows g and g + 8
       const uint32_t u0 = __byte_perm(word_of(vc[0], wl), word_of(vc[1], wl), sel);
       const uint32_t u1 = __byte_perm(word_of(vc[0], wh), word_of(vc[1], wh), sel);
       const uint32_t u2 = __byte_perm(word_of(vc[2], wl), word_of(vc[3], wl), sel);
@@ -403,14 +426,15 @@ __global__ void __launch_bounds__(kF8Threads, 1)
           const int head = 8 * j + 2 * c + x;
           if (head >= G) continue;
           const float inv = 0.00390625f / lx;
-          float* r = p.part_o + (base + head) * D + 16 * g;
+          float* r = p.part_o + (base + head) * D + (D / 8) * g;  // rows g: d = (D/8)g + t; rows g + 8: + D/16
 #pragma unroll
-          for (int q4 = 0; q4 < 2; ++q4) {
+          for (int q4 = 0; q4 < MT / 4; ++q4) {
             const int t = 4 * q4;
             *reinterpret_cast<float4*>(r + t) = make_float4(o[j][t][x] * inv, o[j][t + 1][x] * inv,
                                                             o[j][t + 2][x] * inv, o[j][t + 3][x] * inv);
-            *reinterpret_cast<float4*>(r + 8 + t) = make_float4(o[j][t][2 + x] * inv, o[j][t + 1][2 + x] * inv,
-                                                                o[j][t + 2][2 + x] * inv, o[j][t + 3][2 + x] * inv);
+            *reinterpret_cast<float4*>(r + D / 16 + t) =
+                make_float4(o[j][t][2 + x] * inv, o[j][t + 1][2 + x] * inv, o[j][t + 2][2 + x] * inv,
+                            o[j][t + 3][2 + x] * inv);
           }
           if (g == 0) p.part_lse[base + head] = (m[j][x] + log2f(lx)) * 0.69314718055994531f;
         }
@@ -420,9 +444,11 @@ __global__ void __launch_bounds__(kF8Threads, 1)
 
 cudaError_t launch_decode_fp8(const DecodeParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV, int* n_ranges,
                               cudaStream_t stream) {
-  if (p.D != 128 || p.Hkv > kF8Warps || p.Hkv < 1 || p.G < 1 || p.G > 16) return cudaErrorInvalidValue;
+  if ((p.D != 128 && p.D != 64) || p.Hkv > kF8Warps || p.Hkv < 1 || p.G < 1 || p.G > 16)
+    return cudaErrorInvalidValue;
   const int smem = 1024 + kF8Stages * 2 * 16 * p.Hkv * p.D + 256 + kF8Stages * static_cast<int>(sizeof(F8StageMeta));
-  auto kern = p.G <= 8 ? decode_fp8_kernel<1> : decode_fp8_kernel<2>;
+  auto kern = p.D == 128 ? (p.G <= 8 ? decode_fp8_kernel<1, 128> : decode_fp8_kernel<2, 128>)
+                         : (p.G <= 8 ? decode_fp8_kernel<1, 64> : decode_fp8_kernel<2, 64>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;

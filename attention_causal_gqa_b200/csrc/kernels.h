@@ -81,7 +81,7 @@ constexpr int kDecodeFp8MaxRanges = 148;
 cudaError_t launch_decode_fp8(const DecodeParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV, int* n_ranges,
                               cudaStream_t stream);
 cudaError_t launch_decode_range_merge(const float* part_o, const float* part_lse, const int32_t* seq_lens, void* out,
-                                      float* lse, int B, int H, int T_max, int n_ranges, cudaStream_t stream);
+                                      float* lse, int B, int H, int D, int T_max, int n_ranges, cudaStream_t stream);
 
 // ------------------------------------------------------------------ MLA
 constexpr int kMlaTile = 64;        // tokens per tile

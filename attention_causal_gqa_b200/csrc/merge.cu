@@ -193,7 +193,7 @@ __global__ void range_merge_kernel(const float* __restrict__ part_o, const float
                                    float* __restrict__ lse, int B, int H, int T_max, int n_ranges) {
   griddep_wait();  // launched as a dependent of the kernel that wrote the partials
   constexpr int VEC = DIM / 32;  // contiguous columns per lane
-  static_assert(VEC % 4 == 0, "whole float4 columns per lane");
+  static_assert(VEC == 2 || VEC % 4 == 0, "whole float2 or float4 columns per lane");
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (gw >= B * H) return;
@@ -239,13 +239,19 @@ __global__ void range_merge_kernel(const float* __restrict__ part_o, const float
       const float w = __expf(part_lse[slot * H + h] - M);
       wsum += w;
       const float* po = part_o + (slot * H + h) * DIM + lane * VEC;
+      if constexpr (VEC == 2) {
+        const float2 v = *reinterpret_cast<const float2*>(po);
+        acc[0] += w * v.x;
+        acc[1] += w * v.y;
+      } else {
 #pragma unroll
-      for (int q = 0; q < VEC / 4; ++q) {
-        const float4 v = *reinterpret_cast<const float4*>(po + 4 * q);
-        acc[4 * q] += w * v.x;
-        acc[4 * q + 1] += w * v.y;
-        acc[4 * q + 2] += w * v.z;
-        acc[4 * q + 3] += w * v.w;
+        for (int q = 0; q < VEC / 4; ++q) {
+          const float4 v = *reinterpret_cast<const float4*>(po + 4 * q);
+          acc[4 * q] += w * v.x;
+          acc[4 * q + 1] += w * v.y;
+          acc[4 * q + 2] += w * v.z;
+          acc[4 * q + 3] += w * v.w;
+        }
       }
     }
     const float inv = 1.f / wsum;
@@ -260,8 +266,10 @@ __global__ void range_merge_kernel(const float* __restrict__ part_o, const float
 #pragma unroll
     for (int i = 0; i < VEC / 8; ++i)
       reinterpret_cast<uint4*>(orow)[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
-  } else {
+  } else if constexpr (VEC == 4) {
     reinterpret_cast<uint2*>(orow)[0] = make_uint2(packed[0], packed[1]);
+  } else {
+    reinterpret_cast<uint32_t*>(orow)[0] = packed[0];
   }
 }
 
@@ -281,8 +289,10 @@ cudaError_t launch_mla_merge(const float* part_o, const float* part_lse, const i
 }
 
 cudaError_t launch_decode_range_merge(const float* part_o, const float* part_lse, const int32_t* seq_lens, void* out,
-                                      float* lse, int B, int H, int T_max, int n_ranges, cudaStream_t stream) {
-  return launch_range_merge<128, 16, 0>(part_o, part_lse, seq_lens, out, lse, B, H, T_max, n_ranges, stream);
+                                      float* lse, int B, int H, int D, int T_max, int n_ranges, cudaStream_t stream) {
+  if (D == 64) return launch_range_merge<64, 16, 0>(part_o, part_lse, seq_lens, out, lse, B, H, T_max, n_ranges, stream);
+  if (D == 128) return launch_range_merge<128, 16, 0>(part_o, part_lse, seq_lens, out, lse, B, H, T_max, n_ranges, stream);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace attn

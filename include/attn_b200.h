@@ -139,7 +139,7 @@ int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, c
  *   v_pages      [num_pages, page_size, Hkv, D] uint8 E4M3 codes
  *   k_scale      [num_pages, Hkv] fp32;  v_scale [num_pages, Hkv] fp32
  *   block_table, seq_lens, out, lse: as attn_decode_paged.
- * Supported: D = 128, page_size 16, Hkv <= 8, Hq/Hkv <= 16. NaN codes are out of
+ * Supported: D in {64, 128}, page_size 16, Hkv <= 8, Hq/Hkv <= 16. NaN codes are out of
  * contract. Products run in fp16: codes convert exactly, q converts exactly within
  * +-65504 (else ATTN_DEV_RANGE), P carries the value scale (times 2^8) in fp16, so
  * 256 * v_scale must stay below about 6.5e4.

@@ -144,7 +144,8 @@ def test_decode_fp8_validation_codes(lib):
 
     def call(D=128, Hkv=8, Hq=32, ps=16, ws=need, ks=P):
         return f(P, P, P, ks, P, P, P, P, P, 2, Hq, Hkv, D, ps, 64, 100, 0.0, P, ws, None)
-    assert call(D=64) == 2
+    assert call(D=96) == 2
+    assert call(D=256) == 2
     assert call(Hkv=16, Hq=32) == 2
     assert call(ps=32) == 2
     assert call(Hq=30) == 1

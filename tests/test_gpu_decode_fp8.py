@@ -34,20 +34,22 @@ def _oracle(d, pairs=None):
     ([33, 800, 1601], 48, 8),    # G = 6: a lane's second head column past the group
     ([100, 1500], 12, 1),        # G = 12: the second 8-head tile half used
 ])
-def test_fp8_decode_matches_oracle(lens, Hq, Hkv):
+@pytest.mark.parametrize("D", [128, 64])
+def test_fp8_decode_matches_oracle(lens, Hq, Hkv, D):
     from attention_causal_gqa_b200.synthetic import decode_inputs_fp8
-    d = decode_inputs_fp8(len(lens), Hq, Hkv, 128, seq_lens=lens, seed=len(lens) * 31 + Hq, device="cuda",
+    d = decode_inputs_fp8(len(lens), Hq, Hkv, D, seq_lens=lens, seed=len(lens) * 31 + Hq + D, device="cuda",
                           extra_pages=3)
     out, lse = _run(d)
     ro, rl = _oracle(d)
-    check(out, ro, lse, rl, what=f"fp8 decode {lens},{Hq},{Hkv}")
+    check(out, ro, lse, rl, what=f"fp8 decode {lens},{Hq},{Hkv},D={D}")
 
 
 @cuda
-def test_fp8_decode_empty_sequence_and_poisoned_tail():
+@pytest.mark.parametrize("D", [128, 64])
+def test_fp8_decode_empty_sequence_and_poisoned_tail(D):
     from attention_causal_gqa_b200.synthetic import decode_inputs_fp8
     lens = [0, 37, 70]
-    d = decode_inputs_fp8(3, 16, 4, 128, seq_lens=lens, seed=12, device="cuda")
+    d = decode_inputs_fp8(3, 16, 4, D, seq_lens=lens, seed=12, device="cuda")
     ro, rl = _oracle(d)
     # slots past each length hold the largest finite code: they must not reach the result
     bt = d["block_table"].cpu().numpy()
@@ -62,13 +64,14 @@ def test_fp8_decode_empty_sequence_and_poisoned_tail():
 
 
 @cuda
-def test_fp8_decode_full_size_sampled():
+@pytest.mark.parametrize("D", [128, 64])
+def test_fp8_decode_full_size_sampled(D):
     from attention_causal_gqa_b200.synthetic import decode_inputs_fp8
-    d = decode_inputs_fp8(64, 32, 8, 128, seed=20261202, device="cuda")
+    d = decode_inputs_fp8(64, 32, 8, D, seed=20261202, device="cuda")
     out, lse = _run(d)
     rng = np.random.default_rng(4)
     bs = sorted({int(x) for x in rng.integers(0, 64, size=6)} | {0, 63})
     pairs = [(b, h) for b in bs for h in (0, 5, 31)]
     ro, rl = _oracle(d, pairs)
     idx = torch.tensor(pairs, device="cuda")
-    check(out[idx[:, 0], idx[:, 1]], ro, lse[idx[:, 0], idx[:, 1]], rl, what="fp8 decode full")
+    check(out[idx[:, 0], idx[:, 1]], ro, lse[idx[:, 0], idx[:, 1]], rl, what=f"fp8 decode full D={D}")
