@@ -451,10 +451,15 @@ cudaError_t launch_decode_fp8(const DecodeParams& p, const CUtensorMap& tmK, con
                          : (p.G <= 8 ? decode_fp8_kernel<1, 64> : decode_fp8_kernel<2, 64>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
+  int dev = 0, sms = 148, per_sm = 1;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = sms < kDecodeFp8MaxRanges ? sms : kDecodeFp8MaxRanges;
+  // D = 64 with one head tile fits two CTAs per SM (half the stage bytes, fewer registers):
+  // twice the warps to hide the per-page softmax and hand-off latency
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kF8Threads, smem);
+  if (e != cudaSuccess) return e;
+  per_sm = per_sm < 1 ? 1 : (per_sm > 2 ? 2 : per_sm);
+  const int grid = sms * per_sm < kDecodeFp8MaxRanges ? sms * per_sm : kDecodeFp8MaxRanges;
   *n_ranges = grid;
   kern<<<grid, kF8Threads, smem, stream>>>(p, tmK, tmV);
   return cudaGetLastError();

@@ -72,12 +72,12 @@ struct DecodeParams {
 };
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
                           cudaStream_t stream);
-// FP8 (E4M3) pages: tmK / tmV are 4-D uint8 maps (d, token, head, page); D = 128.
+// FP8 (E4M3) pages: tmK / tmV are 4-D uint8 maps (d, token, head, page); D = 64 or 128.
 // The persistent grid (at most kDecodeFp8MaxRanges CTAs) cuts the pages of all
 // sequences into one contiguous range per CTA; range c writes the partial result of
 // each sequence b it meets at slot c + b of part_o / part_lse (launch_decode_range_merge
 // combines them). Returns the number of ranges through *n_ranges.
-constexpr int kDecodeFp8MaxRanges = 148;
+constexpr int kDecodeFp8MaxRanges = 2 * 148;  // up to two CTAs per SM (D = 64)
 cudaError_t launch_decode_fp8(const DecodeParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV, int* n_ranges,
                               cudaStream_t stream);
 cudaError_t launch_decode_range_merge(const float* part_o, const float* part_lse, const int32_t* seq_lens, void* out,

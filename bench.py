@@ -182,6 +182,25 @@ def timed_region(fn, steps, warmup, world, flush=None):
     return max_over_ranks(ms, world)
 
 
+def hooked_kernel_ms(fn, steps, world, flush=None):
+    """Average device time per launch of a call's main kernel, from the library's timing
+    hook (CUDA events recorded around that kernel on its launch stream). Taken on steps of
+    their own: while a call is timed the hook is off, so no event sits between the call's
+    dependent launches and the programmatic launch overlap stays as a caller gets it."""
+    import torch
+    from attention_causal_gqa_b200 import binding as B_
+    B_.profile_enable(True)
+    B_.profile_collect()
+    for _ in range(steps):
+        if flush is not None:
+            flush()
+        fn()
+    torch.cuda.synchronize()
+    k_ms, n = B_.profile_collect()
+    B_.profile_enable(False)
+    return max_over_ranks(k_ms / max(n, 1), world)
+
+
 # ----------------------------------------------------------- CPU oracle leg
 def oracle_prefill_sample(q, k, v, p, budget_s):
     """Times the float64 oracle on whole heads of the workload until ~budget_s elapsed."""
@@ -502,12 +521,10 @@ def bench_prefill(args, world, dev, seed, flush, pk, pk_kind, fp, name=None, wit
         flush()
         step()
     torch.cuda.synchronize()
-    B_.profile_collect()
     ms = timed_region(step, args.steps, 0, world, flush=flush)
-    kern_ms, n_launch = B_.profile_collect()
+    kern_avg = hooked_kernel_ms(step, args.steps, world, flush=flush)
     flops = prefill_flops(p)
     value = world * flops * args.steps / (ms * 1e-3) / 1e12
-    kern_avg = max_over_ranks(kern_ms / max(n_launch, 1), world)
     achieved = flops / (kern_avg * 1e-3) / 1e12
     roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
             "frac": achieved / pk["bf16_tflops"], "traffic": traffic_for("prefill_kernel"),
@@ -543,13 +560,11 @@ def bench_chunk(args, world, dev, seed, pk, pk_kind):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    B_.profile_collect()
     ms = timed_region(step, args.steps, 0, world)
-    kern_ms, n_launch = B_.profile_collect()
+    kern_avg = hooked_kernel_ms(step, args.steps, world)
     lens = d["cache_lens"].cpu().numpy().astype(np.float64)
     # exact causal work: query i of sequence b sees cache_lens[b] + i + 1 keys; QK^T and P V
     flops = float(np.sum(Hq * 4 * D * (S * lens + S * (S + 1) / 2)))
-    kern_avg = max_over_ranks(kern_ms / max(n_launch, 1), world)
     achieved = flops / (kern_avg * 1e-3) / 1e12
     cpu = None
     if want_cpu(args, world, int(os.environ.get("RANK", "0"))):
@@ -588,10 +603,8 @@ def bench_decode(args, world, dev, seed, pk, pk_kind, fp):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    B_.profile_collect()
     ms = timed_region(step, args.steps, 0, world)
-    k_ms, n = B_.profile_collect()
-    k_avg = max_over_ranks(k_ms / max(n, 1), world)
+    k_avg = hooked_kernel_ms(step, args.steps, world)
     ach = kv_bytes / (k_avg * 1e-3) / 1e9
     res = {"workload": DECODE + ("_small_b8" if args.small else ""), "value": world * kv_bytes * args.steps / (ms * 1e-3) / 1e9, "unit": "GB/s",
            "ms_per_step": ms / args.steps, "kv_tokens": tokens, "kv_bytes_per_step": kv_bytes,
@@ -631,10 +644,8 @@ def bench_decode_fp8(args, world, dev, seed, pk, pk_kind):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    B_.profile_collect()
     ms = timed_region(step, args.steps, 0, world)
-    k_ms, n = B_.profile_collect()
-    k_avg = max_over_ranks(k_ms / max(n, 1), world)
+    k_avg = hooked_kernel_ms(step, args.steps, world)
     ach = kv_bytes / (k_avg * 1e-3) / 1e9
     res = {"workload": DECODE + "_fp8_e4m3" + ("_small_b8" if args.small else ""),
            "value": world * kv_bytes * args.steps / (ms * 1e-3) / 1e9, "unit": "GB/s",
@@ -678,10 +689,8 @@ def bench_mla(args, world, dev, seed, pk, pk_kind, fp):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    B_.profile_collect()
     ms = timed_region(step, args.steps, 0, world)
-    k_ms, n = B_.profile_collect()
-    k_avg = max_over_ranks(k_ms / max(n, 1), world)
+    k_avg = hooked_kernel_ms(step, args.steps, world)
     ach = nbytes / (k_avg * 1e-3) / 1e9
     res = {"workload": MLA + ("_small_b8" if args.small else ""), "value": world * nbytes * args.steps / (ms * 1e-3) / 1e9, "unit": "GB/s",
            "ms_per_step": ms / args.steps, "kv_tokens": tokens, "kv_bytes_per_step": nbytes,
@@ -738,15 +747,11 @@ def bench_dsa(args, world, dev, seed, pk, pk_kind, dense_ms=None):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    B_.profile_collect()
     ms = timed_region(step, args.steps, 0, world)
-    B_.profile_collect()  # (the step's two brackets; kernel times are taken one call at a time below)
     ms_index = timed_region(index, args.steps, 0, world)
-    k_ms, n = B_.profile_collect()
-    k_idx = max_over_ranks(k_ms / max(n, 1), world)
+    k_idx = hooked_kernel_ms(index, args.steps, world)
     ms_attend = timed_region(attend, args.steps, 0, world)
-    m_ms, mn = B_.profile_collect()
-    k_mla = max_over_ranks(m_ms / max(mn, 1), world)
+    k_mla = hooked_kernel_ms(attend, args.steps, world)
     # the same selection attended over an E4M3 latent cache (one scale per token and 128-wide block)
     from attention_causal_gqa_b200.synthetic import quantize_e4m3_rows
     kv_codes, kv_scale = quantize_e4m3_rows(d["kv_cache"])
@@ -758,7 +763,6 @@ def bench_dsa(args, world, dev, seed, pk, pk_kind, dense_ms=None):
     for _ in range(args.warmup):
         attend_fp8()
     ms_attend_fp8 = timed_region(attend_fp8, args.steps, 0, world)
-    B_.profile_collect()
     del kv_codes, kv_scale
     ach = idx_bytes / (k_idx * 1e-3) / 1e9
     res = {"workload": DSA + ("_small_b8" if args.small else ""), "value": world * tokens * args.steps / (ms * 1e-3),
@@ -799,8 +803,7 @@ def run_ours(args):
 
     smi_index = local if world > 1 else int((os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0] or "0"))
     clocks = Clocks(smi_index)
-    B_.profile_enable(True)
-    B_.profile_collect()
+    B_.profile_enable(False)  # on only inside hooked_kernel_ms
     clocks.start()
     pre = bench_prefill(args, world, dev, seed, flush, pk, pk_kind, fp) if do("prefill") else None
     sub = {}
